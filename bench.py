@@ -1,0 +1,385 @@
+"""Benchmark of the NVFP4 W4A4 hot path on B200.
+
+One step = the whole path on one batch: tensor amax -> Four-Over-Six (MSE,
+fp8_max 256) quantization of X -> NVFP4 GEMM against a pre-quantized weight
+(scale-6, fp8_max 448) -> bf16 Y, on the long-prefill MLP shape
+(X 32768 x 5120, W 17408 x 5120).  `value` is whole-job GEMM-equivalent
+throughput, 2*M*N*K per step per GPU summed over ranks / step time (TFLOP/s);
+the JSON line also carries the quantizer's GB/s and the GEMM's TFLOP/s with
+their roofline fractions.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+With N > 1 (torchrun) every rank runs an independent replica on its own X
+(weak scaling: the path shards by tokens with W replicated and needs no
+collective); times are the max over ranks.  `--impl reference` times the CPU
+oracle (the plain, slow definition) on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+L2_FLUSH_BYTES = 256 << 20
+METRIC = "quantize GB/s (% HBM peak); W4A4 GEMM TFLOPS (% dense NVFP4 peak)"
+QUANT_BYTES_PER_ELEM = 2.5625   # read bf16 + write 0.5 B codes + 1/16 B scale
+AMAX_BYTES_PER_ELEM = 2.0
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return dict(hbm=float(p["hbm_gbs"]), bf16=float(p["bf16_tflops"]),
+                    bf16_sus=float(p["bf16_tflops_sustained"]), source="measured")
+    except (OSError, KeyError, ValueError):
+        return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, source="fallback")
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle samples taken while the timed region runs."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.file = None
+
+    def __enter__(self):
+        try:
+            self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=self.file, stderr=subprocess.DEVNULL)
+        except (OSError, ValueError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None or self.file is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.file.seek(0)
+        rows = [ln.strip().split(",") for ln in self.file.read().splitlines() if ln.strip()]
+        os.unlink(self.file.name)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            try:
+                sm.append(float(r[1]))
+                smax.append(float(r[2]))
+                for name, v in zip(names, r[5:9]):
+                    if v.strip().lower() == "active":
+                        reasons.add(name)
+            except (ValueError, IndexError):
+                continue
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        busy = [s for s in sm if s > 0.5 * max(sm)] or sm
+        return {"sm_mhz": statistics.median(busy), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def _dist():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def _barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def _max_over_ranks(world, value: float, device) -> float:
+    if world == 1:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------- ours --
+
+def run_ours(args, world, rank, local):
+    import w4a4_gemm_nvfp4_b200 as nv
+
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    wl = workloads.WORKLOADS[args.workload]
+    xm, xr, xF = args.x_recipe
+    wm, wr, wF = wl.w_recipe
+    M, N, K = wl.M, wl.N, wl.K
+    # each rank gets its own activations (weak scaling), same weights
+    xop = workloads.Operand(**{**wl.x.__dict__, "seed": wl.x.seed + 101 * rank})
+    x_host = xop.make().pin_memory()
+    x = x_host.to(device)
+    w = wl.w.make().to(device)
+    qw = nv.quantize(w, wm, wr, wF)               # offline weight quantization
+    del w
+    qx = nv.quantize(x, xm, xr, xF)
+    q6 = nv.quantize(x, "six", "max", 448.0)      # scale-6 comparison buffers
+    y = torch.empty(M, N, dtype=torch.bfloat16, device=device)
+    gws = torch.zeros(nv.nvfp4_gemm_workspace_bytes(), dtype=torch.uint8, device=device)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream(device)
+
+    def step(qbuf, mode, rule, F, ev=None):
+        if ev:
+            ev[0].record(stream)
+        nv.quantize(x, mode, rule, F, out=qbuf)
+        if ev:
+            ev[1].record(stream)
+        nv.gemm(qbuf, qw, out_dtype=torch.bfloat16, out=y, workspace=gws)
+        if ev:
+            ev[2].record(stream)
+
+    for _ in range(args.warmup):
+        step(qx, xm, xr, xF)
+        step(q6, "six", "max", 448.0)
+    torch.cuda.synchronize()
+    assert nv.device_status(qx.workspace) == nv.OK and nv.device_status(gws) == nv.OK
+
+    def timed(qbuf, mode, rule, F, steps):
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+        for i in range(steps):
+            flush.fill_(i & 0xFF)                   # L2 flush between steps (untimed)
+            step(qbuf, mode, rule, F, evs[i])
+        torch.cuda.synchronize()
+        tq = [e[0].elapsed_time(e[1]) for e in evs]
+        tg = [e[1].elapsed_time(e[2]) for e in evs]
+        return tq, tg
+
+    _barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clocks:
+        tq, tg = timed(qx, xm, xr, xF, args.steps)
+    _barrier(world)
+    torch.cuda.synchronize()
+    tq6, tg6 = timed(q6, "six", "max", 448.0, args.steps)
+    assert nv.device_status(qx.workspace) == nv.OK and nv.device_status(gws) == nv.OK
+
+    ms_step = _max_over_ranks(world, statistics.mean(a + b for a, b in zip(tq, tg)), device)
+    ms_quant = _max_over_ranks(world, statistics.mean(tq), device)
+    ms_gemm = _max_over_ranks(world, statistics.mean(tg), device)
+    ms_quant6 = _max_over_ranks(world, statistics.mean(tq6), device)
+
+    # end to end through the public API with host buffers: pinned X in, Y out
+    y_host = torch.empty(M, N, dtype=torch.bfloat16, pin_memory=True)
+    e2e_steps = max(1, min(args.steps, 5))
+    _barrier(world)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        x.copy_(x_host, non_blocking=True)
+        nv.quantize(x, xm, xr, xF, out=qx)
+        nv.gemm(qx, qw, out_dtype=torch.bfloat16, out=y, workspace=gws)
+        y_host.copy_(y, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms_e2e = _max_over_ranks(world, e0.elapsed_time(e1) / e2e_steps, device)
+
+    flops = 2.0 * M * N * K
+    peaks = _peaks()
+    fp4_peak = 4.0 * peaks["bf16"]
+    gemm_tflops = flops / (ms_gemm * 1e-3) / 1e12
+    quant_gbs = (QUANT_BYTES_PER_ELEM + AMAX_BYTES_PER_ELEM) * M * K / (ms_quant * 1e-3) / 1e9
+    value = world * flops / (ms_step * 1e-3) / 1e12
+    result = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_step, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "nvfp4",
+        "data": "synthetic (seeded; shapes of the pages' long-prefill MLP workload)",
+        "config": {
+            "workload": f"{args.workload}: X {M}x{K} bf16 (4/6-{xr}, fp8_max {xF:g}) -> GEMM with "
+                        f"W {N}x{K} pre-quantized ({wm}, fp8_max {wF:g}) -> Y bf16",
+            "M": M, "N": N, "K": K, "per_gpu_batch_tokens": M,
+            "parallelism": f"replicas x{world}",
+            "l2": "flushed between steps (256 MiB write, untimed)",
+        },
+        "roofline": {
+            "bound": "tensor",
+            "kernel": "gemm_kernel",
+            "achieved": round(gemm_tflops, 1),
+            "peak": round(fp4_peak, 1),
+            "unit": "TFLOP/s",
+            "frac": round(gemm_tflops / fp4_peak, 4),
+            "peak_source": f"4 x {peaks['source']} bf16 burst ({peaks['bf16']} TF/s)",
+            "traffic": None,
+        },
+        "breakdown": {
+            "ms_quantize_46": round(ms_quant, 4),
+            "ms_quantize_six": round(ms_quant6, 4),
+            "overhead_46_vs_six": round(ms_quant / ms_quant6 - 1.0, 4),
+            "quantize_end_to_end_GBps": round(quant_gbs, 1),
+            "quantize_frac_hbm": round(quant_gbs / peaks["hbm"], 4),
+            "hbm_peak_GBps": peaks["hbm"],
+            "ms_gemm": round(ms_gemm, 4),
+            "gemm_TFLOPs": round(gemm_tflops, 1),
+            "ms_gemm_after_six": round(_max_over_ranks(world, statistics.mean(tg6), device), 4),
+        },
+        "e2e": {
+            "value": round(world * flops / (ms_e2e * 1e-3) / 1e12, 2),
+            "unit": "TFLOP/s",
+            "h2d_bytes_per_step": M * K * 2,
+            "d2h_bytes_per_step": M * N * 2,
+            "ms_per_step": round(ms_e2e, 3),
+        },
+        "gpu_launches": 3 * args.steps,
+        "clocks": clocks.summary(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        result["cpu_baseline"] = cpu_baseline(args, sample_rows=1024)
+    return result
+
+
+# ------------------------------------------------------------ oracle (CPU) --
+
+def _oracle_sample(wl, xr_recipe, rows, w_deq=None):
+    """One bounded oracle pass: quantize `rows` rows of X (4/6 rule) and
+    their fp64 GEMM against the oracle-quantized W.  Returns flops done."""
+    import numpy as np
+
+    import oracle
+
+    mode = {"six": oracle.MODE_SIX, "four_over_six": oracle.MODE_FOUR_OVER_SIX}
+    rule = {"max": oracle.RULE_MAX, "mae": oracle.RULE_MAE, "mse": oracle.RULE_MSE}
+    xm, xr, xF = xr_recipe
+    x = workloads.Operand(**{**wl.x.__dict__, "rows": rows}).make()
+    xc, xs, xa = oracle.quantize(x, mode[xm], rule[xr], xF)
+    xd = oracle.dequantize(xc, xs, xa)
+    _ = xd @ w_deq.T
+    return 2.0 * rows * w_deq.shape[0] * wl.K
+
+
+def _w_dequant(wl):
+    import oracle
+
+    mode = {"six": oracle.MODE_SIX, "four_over_six": oracle.MODE_FOUR_OVER_SIX}
+    rule = {"max": oracle.RULE_MAX, "mae": oracle.RULE_MAE, "mse": oracle.RULE_MSE}
+    wm, wr, wF = wl.w_recipe
+    wc, ws, wa = oracle.quantize(wl.w.make(), mode[wm], rule[wr], wF)
+    return oracle.dequantize(wc, ws, wa)
+
+
+def _cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count()
+
+
+def cpu_baseline(args, sample_rows=64):
+    wl = workloads.WORKLOADS[args.workload]
+    w_deq = _w_dequant(wl)
+    t0 = time.perf_counter()
+    flops = _oracle_sample(wl, args.x_recipe, sample_rows, w_deq)
+    dt = time.perf_counter() - t0
+    return {"value": round(flops / dt / 1e12, 6), "unit": "TFLOP/s", "cores": _cores(),
+            "kind": "oracle",
+            "sample": f"{sample_rows} rows of X ({wl.K} wide) quantized by the C oracle (1 thread) + "
+                      f"fp64 numpy GEMM against the oracle-dequantized W {wl.N}x{wl.K} "
+                      f"(BLAS threads); W quantization untimed; {dt:.1f} s"}
+
+
+def run_reference(args, world, rank):
+    wl = workloads.WORKLOADS[args.workload]
+    w_deq = _w_dequant(wl)
+    rows = args.cpu_rows
+    for _ in range(args.warmup):
+        _oracle_sample(wl, args.x_recipe, max(1, rows // 8), w_deq)
+    t0 = time.perf_counter()
+    flops = 0.0
+    for _ in range(args.steps):
+        flops += _oracle_sample(wl, args.x_recipe, rows, w_deq)
+    dt = time.perf_counter() - t0
+    value = flops / dt / 1e12
+    sample = (f"each step: {rows} rows of X quantized by the C oracle (1 thread) + fp64 numpy "
+              f"GEMM against the oracle-dequantized W {wl.N}x{wl.K}")
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(dt / args.steps * 1e3, 2), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32 quantize + f64 GEMM",
+        "data": "synthetic (seeded)",
+        "config": {"workload": f"{args.workload} (oracle sample of {rows} X rows per step)",
+                   "M": wl.M, "N": wl.N, "K": wl.K},
+        "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": _cores(),
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="prefill", choices=["prefill", "mlp8b", "attn27b", "pr1"])
+    ap.add_argument("--x-recipe", default="four_over_six,mse,256",
+                    help="mode,rule,fp8_max for X (default four_over_six,mse,256)")
+    ap.add_argument("--cpu-rows", type=int, default=256, help="X rows per oracle step (reference arm)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    m, r, f = args.x_recipe.split(",")
+    args.x_recipe = (m, r, float(f))
+    if args.warmup < 3 and args.impl == "ours":
+        ap.error("--warmup must be >= 3")
+
+    world, rank, local = _dist()
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args, world, rank)), flush=True)
+        return
+    if world > 1:
+        import datetime
+
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                             device_id=torch.device("cuda", local))
+    try:
+        res = run_ours(args, world, rank, local)
+        if rank == 0:
+            print(json.dumps(res), flush=True)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

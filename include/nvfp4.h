@@ -1,0 +1,161 @@
+/*
+ * nvfp4.h -- C ABI of libnvfp4.so: NVFP4 W4A4 linear-layer kernels for
+ * NVIDIA B200 (sm_100a).
+ *
+ * Two operations, both asynchronous on a caller-supplied CUDA stream:
+ *
+ *  nvfp4_quantize  16-element block-scaled NVFP4 quantization of a bf16
+ *                  matrix: E2M1 codes, one FP8 E4M3 scale per 16 elements
+ *                  along K, one FP32 global scale per tensor.  Two modes:
+ *                  scale-to-6 and the adaptive Four-Over-Six (4/6), which
+ *                  quantizes every block with scale targets 6 and 4 and keeps
+ *                  the one with the smaller error under a max / MAE / MSE rule.
+ *                  Source: "Four Over Six (4/6)" technical summary,
+ *                  gist.science/ko/paper/2512.02010 -- sections "문제 제기"
+ *                  (E2M1 grid 0,.5,1,1.5,2,3,4,6), "적응형 블록 스케일링
+ *                  알고리즘" (double quantization, three selection rules) and
+ *                  "구현 세부 사항" (E4M3 block scales; FP8 max 256 instead of
+ *                  448 in the global scale for 4/6).
+ *
+ *  nvfp4_gemm      Y = alpha_A * alpha_B * sum_kb sA[m,kb] sB[n,kb] *
+ *                      sum_{k in kb} qA[m,k] qB[n,k]
+ *                  i.e. Y = A_hat . B_hat^T for two NVFP4 operands stored as
+ *                  nvfp4_quantize writes them, both K-major, with an fp32
+ *                  accumulator and a bf16 or fp32 output.  Source: "ARCQuant"
+ *                  technical summary, gist.science/ko/paper/2601.07475,
+ *                  section "방법론" (one uniform NVFP4 GEMM along K on the
+ *                  Blackwell tensor cores), and the Minima page, section
+ *                  "심층 분석" (global scales applied around one fused GEMM).
+ *
+ * Exact arithmetic of nvfp4_quantize (every step one IEEE binary32 operation,
+ * round-to-nearest-even, in this order):
+ *   amax  = max |x| over the tensor
+ *   alpha = amax / (fp8_max * 6)            (alpha = 1 when amax == 0)
+ *   per block of 16 along K, b = max |x_i|, for Q in {6} or {6, 4}:
+ *     s = E4M3_RNE_satfinite(b / (alpha * Q));  d = s * alpha
+ *     r = 1 / d, or 0 when that is infinite;    v_i = x_i * r
+ *     q_i = E2M1_RNE_satfinite(v_i) (sign kept); e_i = fma(-q_i, d, x_i)
+ *     E_Q = max|e_i| (MAX), sum |e_i| (MAE) or sum e_i*e_i (MSE), sums as
+ *           the contiguous pairwise tree ((e0+e1)+(e2+e3))+...
+ *   keep Q = 4 only when E_4 < E_6.
+ *
+ * Memory layouts (all buffers are device memory owned by the caller; the
+ * library allocates nothing and keeps no pointer after a call returns):
+ *   x       bf16 [rows, K], row stride ldx elements (ldx >= K, ldx % 8 == 0,
+ *           base 16-byte aligned).
+ *   codes   uint8 [rows, K/2], row-major, two E2M1 codes per byte, element 2j
+ *           in the low nibble (nvfp4_codes_bytes).  16-byte aligned.
+ *   scales  E4M3 bytes in the block-scaled MMA's scale-factor layout: atoms
+ *           of 128 rows x 4 K-blocks (64 elements), 512 bytes each, atom
+ *           (r/128)*(K/64) + (k/64), byte (r%32)*16 + ((r/32)%4)*4 + (k/16)%4
+ *           inside the atom; rows padded to a multiple of 128 with zero bytes
+ *           (nvfp4_scales_bytes).  16-byte aligned.
+ *   global_scale  one fp32 in device memory (alpha).
+ *   Y       bf16 or fp32 [M, N], row-major, row stride ldy >= N elements,
+ *           aligned to its element size (rows that start 16-byte aligned get
+ *           vector stores).
+ *
+ * Errors: every call validates its arguments on the host and returns a status
+ * without launching anything when they are invalid.  Conditions only the GPU
+ * can see (non-finite input to nvfp4_quantize, a bounded wait that ran out in
+ * nvfp4_gemm) are written to a status word in the call's workspace and read
+ * by nvfp4_get_device_status.  Launch failures return NVFP4_ERR_CUDA with
+ * the CUDA message available from nvfp4_last_error_message.
+ *
+ * Streams are passed as void* and must be a cudaStream_t of the current
+ * device (NULL = the legacy default stream).  All calls use the current CUDA
+ * device of the calling thread.
+ */
+#ifndef NVFP4_H
+#define NVFP4_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define NVFP4_API __attribute__((visibility("default")))
+#else
+#define NVFP4_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  NVFP4_OK = 0,
+  NVFP4_ERR_INVALID_ARG = 1,        /* null pointer, bad size, alignment, enum value */
+  NVFP4_ERR_UNSUPPORTED_DEVICE = 2, /* current device is not compute capability 10.0 */
+  NVFP4_ERR_NONFINITE = 3,          /* input tensor holds Inf or NaN (device status) */
+  NVFP4_ERR_TIMEOUT = 4,            /* a bounded device wait ran out (device status) */
+  NVFP4_ERR_CUDA = 5                /* a CUDA runtime / driver call failed */
+} nvfp4_status;
+
+typedef enum { NVFP4_MODE_SIX = 0, NVFP4_MODE_FOUR_OVER_SIX = 1 } nvfp4_mode;
+typedef enum { NVFP4_RULE_MAX = 0, NVFP4_RULE_MAE = 1, NVFP4_RULE_MSE = 2 } nvfp4_rule;
+typedef enum { NVFP4_OUT_BF16 = 0, NVFP4_OUT_FP32 = 1 } nvfp4_out_dtype;
+
+/* Bytes of the packed code buffer: rows * K / 2. */
+NVFP4_API size_t nvfp4_codes_bytes(int64_t rows, int64_t K);
+
+/* Bytes of the swizzled scale buffer: ceil(rows/128)*128 * K/16. */
+NVFP4_API size_t nvfp4_scales_bytes(int64_t rows, int64_t K);
+
+/* Bytes of device workspace nvfp4_quantize needs (a status word and the
+ * per-CTA partial maxima of the tensor-amax pass).  Any size-independent
+ * workspace of at least this many bytes, 16-byte aligned, may be reused
+ * across calls on one stream; calls that run concurrently need their own. */
+NVFP4_API size_t nvfp4_quantize_workspace_bytes(int64_t rows, int64_t K);
+
+/* Bytes of device workspace nvfp4_gemm needs (its status word). */
+NVFP4_API size_t nvfp4_gemm_workspace_bytes(void);
+
+/* Quantize x [rows, K] (bf16) to NVFP4.
+ *   mode     NVFP4_MODE_SIX or NVFP4_MODE_FOUR_OVER_SIX.
+ *   rule     selection rule for 4/6 (NVFP4_RULE_*); ignored for SIX but must
+ *            still be a valid value.
+ *   fp8_max  448 or 256: the FP8 maximum used in alpha = amax/(fp8_max*6).
+ *            The pages use 448 for scale-6 and 256 for 4/6; any pairing is
+ *            accepted.
+ * Requirements: rows >= 1, K >= 64, K % 64 == 0, ldx >= K, ldx % 8 == 0,
+ * x / codes / scales / workspace 16-byte aligned, global_scale 4-byte
+ * aligned, workspace_bytes >= nvfp4_quantize_workspace_bytes(rows, K).
+ * Writes codes, every byte of scales (padding = 0), *global_scale and the
+ * workspace status word.  When x holds Inf or NaN the status word becomes
+ * NVFP4_ERR_NONFINITE, *global_scale becomes NaN, and codes/scales are left
+ * unwritten.  Returns once both kernels are enqueued (two launches). */
+NVFP4_API nvfp4_status nvfp4_quantize(const void* x, int64_t rows, int64_t K, int64_t ldx, int mode,
+                            int rule, float fp8_max, void* codes, void* scales,
+                            float* global_scale, void* workspace, size_t workspace_bytes,
+                            void* stream);
+
+/* Y [M, N] = (alpha_A * alpha_B) * (A_hat . B_hat^T) with an fp32 accumulator.
+ *   a_codes/a_scales/a_global  operand A (M rows), as nvfp4_quantize wrote it
+ *   b_codes/b_scales/b_global  operand B (N rows, e.g. a weight [N, K])
+ *   out_dtype  NVFP4_OUT_BF16 (round-to-nearest-even) or NVFP4_OUT_FP32.
+ * Requirements: M, N >= 1, K >= 64, K % 64 == 0, ldy >= N, code and scale
+ * buffers 16-byte aligned, Y aligned to its element size, workspace
+ * (>= nvfp4_gemm_workspace_bytes(), 16-byte aligned) for the status word.
+ * Enqueues a 64-byte memset of the status word and one kernel launch. */
+NVFP4_API nvfp4_status nvfp4_gemm(const void* a_codes, const void* a_scales, const float* a_global,
+                        const void* b_codes, const void* b_scales, const float* b_global,
+                        int64_t M, int64_t N, int64_t K, void* y, int64_t ldy, int out_dtype,
+                        void* workspace, size_t workspace_bytes, void* stream);
+
+/* Synchronizes `stream`, then returns the status word the last call that used
+ * `workspace` wrote (NVFP4_OK, NVFP4_ERR_NONFINITE or NVFP4_ERR_TIMEOUT), or
+ * NVFP4_ERR_CUDA if the synchronization or the read failed. */
+NVFP4_API nvfp4_status nvfp4_get_device_status(const void* workspace, void* stream);
+
+/* Static text for a status code. */
+NVFP4_API const char* nvfp4_status_string(nvfp4_status status);
+
+/* Text of the last NVFP4_ERR_CUDA / NVFP4_ERR_INVALID_ARG on this host
+ * thread (empty string when none); valid until the next call on the thread. */
+NVFP4_API const char* nvfp4_last_error_message(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* NVFP4_H */

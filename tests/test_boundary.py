@@ -1,0 +1,101 @@
+"""The C-ABI boundary on a machine without a GPU: libnvfp4.so loads, exports
+every function include/*.h declares, computes buffer sizes, and rejects bad
+arguments on the host before touching any device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import w4a4_gemm_nvfp4_b200 as nv
+from w4a4_gemm_nvfp4_b200 import _lib
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_functions():
+    names = set()
+    for h in os.listdir(os.path.join(ROOT, "include")):
+        if h.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", h)).read()
+            names |= set(re.findall(r"NVFP4_API\s+[\w\s\*]+?\b(nvfp4_\w+)\s*\(", text))
+    return sorted(names)
+
+
+def test_headers_declare_the_boundary():
+    names = _declared_functions()
+    for required in ("nvfp4_quantize", "nvfp4_gemm", "nvfp4_get_device_status",
+                     "nvfp4_codes_bytes", "nvfp4_scales_bytes", "nvfp4_status_string"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = nv.load()
+    for name in _declared_functions():
+        assert hasattr(lib, name), name
+        assert name in _lib._SIGNATURES, f"binding lacks {name}"
+
+
+def test_sizes():
+    assert nv.nvfp4_codes_bytes(64, 512) == 64 * 256
+    assert nv.nvfp4_scales_bytes(64, 512) == 128 * 32
+    assert nv.nvfp4_scales_bytes(129, 128) == 256 * 8
+    assert nv.nvfp4_scales_bytes(32768, 5120) == 32768 * 320
+    assert nv.nvfp4_gemm_workspace_bytes() >= 8
+    assert nv.nvfp4_quantize_workspace_bytes(1, 64) >= 64
+    assert nv.nvfp4_codes_bytes(0, 64) == 0
+
+
+def test_status_strings():
+    assert nv.status_string(nv.OK) == "NVFP4_OK"
+    assert nv.status_string(nv.ERR_TIMEOUT) == "NVFP4_ERR_TIMEOUT"
+    assert nv.status_string(99) == "NVFP4_ERR_UNKNOWN"
+
+
+FAKE = 0x10000  # 16-byte aligned, never dereferenced: validation fails first
+
+
+def _q(**kw):
+    args = dict(x=FAKE, rows=64, K=512, ldx=512, mode=0, rule=0, fp8_max=448.0, codes=FAKE,
+                scales=FAKE, global_scale=FAKE, workspace=FAKE, workspace_bytes=1 << 20, stream=None)
+    args.update(kw)
+    return nv.nvfp4_quantize(*args.values())
+
+
+@pytest.mark.parametrize("bad", [
+    dict(x=None), dict(codes=None), dict(scales=None), dict(global_scale=None), dict(workspace=None),
+    dict(rows=0), dict(K=0), dict(K=48), dict(K=96), dict(ldx=256), dict(ldx=516),
+    dict(mode=2), dict(rule=3), dict(rule=-1), dict(fp8_max=300.0), dict(fp8_max=0.0),
+    dict(x=FAKE + 8), dict(codes=FAKE + 4), dict(global_scale=FAKE + 2), dict(workspace_bytes=16),
+])
+def test_quantize_rejects_bad_arguments(bad):
+    assert _q(**bad) == nv.ERR_INVALID_ARG
+    assert nv.last_error_message()
+
+
+def _g(**kw):
+    args = dict(a_codes=FAKE, a_scales=FAKE, a_global=FAKE, b_codes=FAKE, b_scales=FAKE,
+                b_global=FAKE, M=64, N=256, K=512, y=FAKE, ldy=256, out_dtype=0, workspace=FAKE,
+                workspace_bytes=64, stream=None)
+    args.update(kw)
+    return nv.nvfp4_gemm(*args.values())
+
+
+@pytest.mark.parametrize("bad", [
+    dict(a_codes=None), dict(b_scales=None), dict(y=None), dict(workspace=None), dict(M=0),
+    dict(N=-1), dict(K=32), dict(K=100), dict(ldy=128), dict(ldy=255), dict(out_dtype=2),
+    dict(y=FAKE + 1), dict(a_global=FAKE + 1), dict(workspace_bytes=4),
+])
+def test_gemm_rejects_bad_arguments(bad):
+    assert _g(**bad) == nv.ERR_INVALID_ARG
+
+
+def test_no_gpu_fails_loudly():
+    """Valid arguments without a usable sm_100 device: an error status, never a
+    silent fallback."""
+    import torch
+
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    assert _q() in (nv.ERR_CUDA, nv.ERR_UNSUPPORTED_DEVICE)
+    assert _g() in (nv.ERR_CUDA, nv.ERR_UNSUPPORTED_DEVICE)

@@ -1,0 +1,149 @@
+"""Parity of the CUDA W4A4 GEMM (nvfp4_gemm through the C ABI) with the fp64
+oracle product of the dequantized operands.  Operands are made by the oracle
+(quantizer output or arbitrary codes/scales) and uploaded, so these tests
+exercise the GEMM alone; the full-size cases run the quantize -> GEMM
+pipeline as the benchmark does and check sampled output rows."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+import w4a4_gemm_nvfp4_b200 as nv
+from gpu_util import MODE, RULE, assert_gemm_close, gpu_quantize, to_np, upload_operand
+
+pytestmark = pytest.mark.gpu
+
+
+def _run(a, b, out_dtype):
+    y = nv.gemm(a, b, out_dtype=out_dtype)
+    ws = torch.zeros(nv.nvfp4_gemm_workspace_bytes(), dtype=torch.uint8, device="cuda")
+    y = nv.gemm(a, b, out_dtype=out_dtype, out=y, workspace=ws)
+    assert nv.device_status(ws) == nv.OK
+    return to_np(y.float()) if out_dtype == torch.bfloat16 else to_np(y)
+
+
+def _quantized(rows, K, seed, recipe, kind="t"):
+    x = workloads.small_operand(rows, K, seed, kind=kind).make()
+    mode, rule, F = recipe
+    c, s, a = oracle.quantize(x, MODE[mode], RULE[rule], F)
+    return c, s, a
+
+
+def _random_operand(rows, K, rng, max_scale_code=0x60):
+    codes = rng.integers(0, 256, size=(rows, K // 2), dtype=np.uint8)
+    scales = rng.integers(0, max_scale_code, size=(rows, K // 16), dtype=np.uint8)
+    return codes, scales
+
+
+def _check(ac, as_, aa, bc, bs, ba):
+    ref, guard = oracle.gemm_reference(ac, as_, aa, bc, bs, ba)
+    A, B = upload_operand(ac, as_, aa), upload_operand(bc, bs, ba)
+    rel32 = assert_gemm_close(_run(A, B, torch.float32), ref, guard)
+    assert_gemm_close(_run(A, B, torch.bfloat16), ref, guard, bf16=True)
+    return rel32
+
+
+SHAPES = [(64, 256, 512), (1, 1, 64), (3, 5, 128), (127, 129, 192), (128, 256, 256),
+          (200, 300, 320), (257, 513, 1024), (130, 1000, 2048), (1024, 768, 64)]
+
+
+@pytest.mark.parametrize("M,N,K", SHAPES)
+def test_gemm_quantized_operands(M, N, K):
+    ac, as_, aa = _quantized(M, K, 1, ("four_over_six", "mse", 256.0))
+    bc, bs, ba = _quantized(N, K, 2, ("six", "max", 448.0), kind="normal")
+    _check(ac, as_, aa, bc, bs, ba)
+
+
+@pytest.mark.parametrize("M,N,K", [(64, 256, 512), (130, 260, 576), (256, 512, 4096)])
+def test_gemm_random_codes_and_scales(M, N, K):
+    rng = np.random.default_rng(M + N + K)
+    ac, as_ = _random_operand(M, K, rng)
+    bc, bs = _random_operand(N, K, rng)
+    _check(ac, as_, 0.75, bc, bs, 1.25)
+
+
+def test_pr1():
+    wl = workloads.WORKLOADS["pr1"]
+    x, w = wl.x.make(), wl.w.make()
+    for mode, rule, F in wl.x_recipes:
+        xc, xs, xa = oracle.quantize(x, MODE[mode], RULE[rule], F)
+        wc, ws, wa = oracle.quantize(w, MODE[mode], RULE[rule], F)
+        _check(xc, xs, xa, wc, ws, wa)
+
+
+def test_closed_form_all_half():
+    """All codes +1 (0.5), constant scales: every output equals
+    K * 0.25 * sA * sB * alphaA * alphaB exactly."""
+    M, N, K = 200, 300, 1024
+    ac = np.full((M, K // 2), 0x11, np.uint8)
+    bc = np.full((N, K // 2), 0x11, np.uint8)
+    as_ = np.full((M, K // 16), 0x38, np.uint8)   # 1.0
+    bs = np.full((N, K // 16), 0x41, np.uint8)    # 2.25
+    A, B = upload_operand(ac, as_, 0.5), upload_operand(bc, bs, 0.25)
+    y = _run(A, B, torch.float32)
+    assert np.all(y == K * 0.25 * 2.25 * 0.5 * 0.25)
+
+
+@pytest.mark.parametrize("kb", [0, 1, 2, 3, 4, 7, 13, 31])
+def test_one_hot_k_block_pins_scale_layout(kb):
+    """Only K block kb is nonzero and every row/column gets its own scale:
+    Y[m,n] = sA[m,kb] sB[n,kb] * sum_k qA qB exactly, which fails for any
+    misplaced scale byte (row, K group or atom order)."""
+    M, N, K = 256, 256, 512
+    rng = np.random.default_rng(kb)
+    ac, as_ = _random_operand(M, K, rng)
+    bc, bs = _random_operand(N, K, rng)
+    mask = np.zeros((1, K // 2), np.uint8)
+    mask[0, kb * 8:(kb + 1) * 8] = 0xFF
+    ac &= mask
+    bc &= mask
+    as_ = rng.integers(0x30, 0x50, size=as_.shape, dtype=np.uint8)
+    bs = rng.integers(0x30, 0x50, size=bs.shape, dtype=np.uint8)
+    ref, _ = oracle.gemm_reference(ac, as_, 1.0, bc, bs, 1.0)
+    y = _run(upload_operand(ac, as_, 1.0), upload_operand(bc, bs, 1.0), torch.float32)
+    assert np.array_equal(y.astype(np.float64), ref)
+
+
+# ------------------------------------------------ full sizes, sampled rows --
+
+@pytest.mark.slow
+@pytest.mark.parametrize("name", ["mlp8b", "attn27b", "prefill"])
+def test_pipeline_full_size_sampled(name):
+    """quantize X (each recipe) and W on the GPU, GEMM, and compare sampled
+    rows of Y with the oracle's fp64 product of its own quantized operands."""
+    wl = workloads.WORKLOADS[name]
+    x, w = wl.x.make(), wl.w.make()
+    wm, wr, wF = wl.w_recipe
+    qw, st = gpu_quantize(w, wm, wr, wF, canary=0)
+    assert st == nv.OK
+    wc, ws, wa = oracle.quantize(w, MODE[wm], RULE[wr], wF)
+    assert np.array_equal(to_np(qw.codes), wc)
+    xamax, _ = oracle.amax(x)
+    idx = workloads.sample_rows(wl.M, 64, 1).numpy()
+    for xm, xr, xF in wl.x_recipes:
+        qx, st = gpu_quantize(x, xm, xr, xF, canary=0)
+        assert st == nv.OK
+        y = nv.gemm(qx, qw, out_dtype=torch.bfloat16)
+        y32 = nv.gemm(qx, qw, out_dtype=torch.float32)
+        xa = oracle.global_scale(xamax, xF)
+        xc, xs = oracle.quantize_rows(x[idx], xa, MODE[xm], RULE[xr])
+        ref, guard = oracle.gemm_reference(xc, xs, xa, wc, ws, wa)
+        rows = torch.from_numpy(idx).cuda()
+        assert_gemm_close(to_np(y32[rows]), ref, guard)
+        assert_gemm_close(to_np(y[rows].float()), ref, guard, bf16=True)
+
+
+@pytest.mark.parametrize("ldy_pad", [3, 8, 130])
+def test_strided_output(ldy_pad):
+    M, N, K = 150, 200, 256
+    ac, as_, aa = _quantized(M, K, 3, ("four_over_six", "max", 256.0))
+    bc, bs, ba = _quantized(N, K, 4, ("six", "max", 448.0))
+    ref, guard = oracle.gemm_reference(ac, as_, aa, bc, bs, ba)
+    A, B = upload_operand(ac, as_, aa), upload_operand(bc, bs, ba)
+    for dt in (torch.float32, torch.bfloat16):
+        big = torch.full((M, N + ldy_pad), 7.0, dtype=dt, device="cuda")
+        nv.gemm(A, B, out_dtype=dt, out=big[:, :N])
+        got = to_np(big.float())
+        assert_gemm_close(got[:, :N], ref, guard, bf16=dt == torch.bfloat16)
+        assert (got[:, N:] == 7.0).all()  # nothing written past N

@@ -1,0 +1,17 @@
+"""NVFP4 W4A4 linear-layer kernels for NVIDIA B200 (sm_100a).
+
+``quantize`` -- 16-element block-scaled NVFP4 quantization (scale-to-6 or
+Four-Over-Six with a max / MAE / MSE selection rule) of a bf16 CUDA matrix,
+writing codes and scales in the layout the block-scaled tensor-core MMA reads.
+``gemm`` -- Y = A_hat @ B_hat^T on two such operands (tcgen05 block-scaled FP4
+MMA, fp32 accumulation, bf16 or fp32 output).
+
+Both run in libnvfp4.so (CUDA, built in-tree by ``build.py``); this package is
+a ctypes binding around its C ABI (``include/nvfp4.h``).
+"""
+from ._lib import (  # noqa: F401
+    DEFAULT_FP8_MAX, ERR_CUDA, ERR_INVALID_ARG, ERR_NONFINITE, ERR_TIMEOUT, ERR_UNSUPPORTED_DEVICE,
+    LIB_PATH, MODES, OK, OUT_BF16, OUT_FP32, RULES, NVFP4Error, NVFP4Tensor, device_status, gemm,
+    last_error_message, load, nvfp4_codes_bytes, nvfp4_gemm, nvfp4_gemm_workspace_bytes,
+    nvfp4_get_device_status, nvfp4_quantize, nvfp4_quantize_workspace_bytes, nvfp4_scales_bytes,
+    quantize, status_string, testing_set_gemm_wait)

@@ -1,0 +1,194 @@
+"""ctypes binding of libnvfp4.so (argument marshalling only).
+
+The functions named like the C ABI (``nvfp4_quantize``, ``nvfp4_gemm``, ...)
+take raw integers (device pointers, sizes, a cudaStream_t handle) and return
+the C status.  ``quantize`` / ``gemm`` wrap them for torch CUDA tensors:
+they allocate outputs with torch, pass pointers and the current stream, and
+raise ``NVFP4Error`` on a non-OK status.  Every step of the computation runs
+in the library's kernels; there is no CPU or PyTorch fallback, and importing
+this module on a machine without the built library raises at first use.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+from dataclasses import dataclass
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libnvfp4.so")
+
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED_DEVICE, ERR_NONFINITE, ERR_TIMEOUT, ERR_CUDA = range(6)
+MODES = {"six": 0, "four_over_six": 1}
+RULES = {"max": 0, "mae": 1, "mse": 2}
+OUT_BF16, OUT_FP32 = 0, 1
+DEFAULT_FP8_MAX = {"six": 448.0, "four_over_six": 256.0}
+
+# name -> (restype, argtypes); every function declared in include/nvfp4.h and
+# include/nvfp4_testing.h
+_P = ctypes.c_void_p
+_I64 = ctypes.c_int64
+_SIGNATURES = {
+    "nvfp4_codes_bytes": (ctypes.c_size_t, [_I64, _I64]),
+    "nvfp4_scales_bytes": (ctypes.c_size_t, [_I64, _I64]),
+    "nvfp4_quantize_workspace_bytes": (ctypes.c_size_t, [_I64, _I64]),
+    "nvfp4_gemm_workspace_bytes": (ctypes.c_size_t, []),
+    "nvfp4_quantize": (ctypes.c_int, [_P, _I64, _I64, _I64, ctypes.c_int, ctypes.c_int,
+                                      ctypes.c_float, _P, _P, _P, _P, ctypes.c_size_t, _P]),
+    "nvfp4_gemm": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _I64,
+                                  ctypes.c_int, _P, ctypes.c_size_t, _P]),
+    "nvfp4_get_device_status": (ctypes.c_int, [_P, _P]),
+    "nvfp4_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "nvfp4_last_error_message": (ctypes.c_char_p, []),
+    "nvfp4_testing_set_gemm_wait": (None, [ctypes.c_uint64, ctypes.c_int]),
+}
+
+_lock = threading.Lock()
+_lib = None
+
+
+class NVFP4Error(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {status_string(status)}: {last_error_message()}")
+
+
+def load() -> ctypes.CDLL:
+    """Load libnvfp4.so (raises if it has not been built)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                raise ImportError(
+                    f"{LIB_PATH} is missing: build it with `python -m w4a4_gemm_nvfp4_b200.build`")
+            lib = ctypes.CDLL(LIB_PATH)
+            for name, (res, args) in _SIGNATURES.items():
+                fn = getattr(lib, name)
+                fn.restype = res
+                fn.argtypes = args
+            _lib = lib
+    return _lib
+
+
+# ------------------------------------------------------- raw C functions --
+
+def nvfp4_codes_bytes(rows: int, K: int) -> int:
+    return load().nvfp4_codes_bytes(rows, K)
+
+
+def nvfp4_scales_bytes(rows: int, K: int) -> int:
+    return load().nvfp4_scales_bytes(rows, K)
+
+
+def nvfp4_quantize_workspace_bytes(rows: int, K: int) -> int:
+    return load().nvfp4_quantize_workspace_bytes(rows, K)
+
+
+def nvfp4_gemm_workspace_bytes() -> int:
+    return load().nvfp4_gemm_workspace_bytes()
+
+
+def nvfp4_quantize(x, rows, K, ldx, mode, rule, fp8_max, codes, scales, global_scale, workspace,
+                   workspace_bytes, stream) -> int:
+    return load().nvfp4_quantize(x, rows, K, ldx, mode, rule, fp8_max, codes, scales, global_scale,
+                                 workspace, workspace_bytes, stream)
+
+
+def nvfp4_gemm(a_codes, a_scales, a_global, b_codes, b_scales, b_global, M, N, K, y, ldy,
+               out_dtype, workspace, workspace_bytes, stream) -> int:
+    return load().nvfp4_gemm(a_codes, a_scales, a_global, b_codes, b_scales, b_global, M, N, K, y,
+                             ldy, out_dtype, workspace, workspace_bytes, stream)
+
+
+def nvfp4_get_device_status(workspace, stream) -> int:
+    return load().nvfp4_get_device_status(workspace, stream)
+
+
+def status_string(status: int) -> str:
+    return load().nvfp4_status_string(status).decode()
+
+
+def last_error_message() -> str:
+    return load().nvfp4_last_error_message().decode()
+
+
+def testing_set_gemm_wait(timeout_ns: int = 0, debug_flags: int = 0) -> None:
+    load().nvfp4_testing_set_gemm_wait(timeout_ns, debug_flags)
+
+
+# --------------------------------------------------- torch-level helpers --
+
+@dataclass
+class NVFP4Tensor:
+    """A quantized [rows, K] operand as the C ABI lays it out."""
+    codes: "torch.Tensor"         # uint8 [rows, K/2]
+    scales: "torch.Tensor"        # uint8 [nvfp4_scales_bytes(rows, K)], swizzled
+    global_scale: "torch.Tensor"  # float32 [1]
+    workspace: "torch.Tensor"     # uint8, holds the status word of the call
+    rows: int
+    K: int
+
+
+def _stream_handle(stream) -> int:
+    import torch
+
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return int(s.cuda_stream)
+
+
+def _check(status: int, what: str) -> None:
+    if status != OK:
+        raise NVFP4Error(status, what)
+
+
+def quantize(x, mode: str = "six", rule: str = "max", fp8_max: float | None = None,
+             out: NVFP4Tensor | None = None, stream=None) -> NVFP4Tensor:
+    """NVFP4-quantize a CUDA bf16 matrix [rows, K] (K % 64 == 0)."""
+    import torch
+
+    if x.dtype != torch.bfloat16 or x.dim() != 2 or not x.is_cuda:
+        raise ValueError("x must be a 2-D bfloat16 CUDA tensor")
+    if x.stride(1) != 1:
+        raise ValueError("x must have unit stride along K")
+    rows, K = x.shape
+    F = DEFAULT_FP8_MAX[mode] if fp8_max is None else float(fp8_max)
+    if out is None:
+        dev = x.device
+        out = NVFP4Tensor(
+            codes=torch.empty(rows, K // 2, dtype=torch.uint8, device=dev),
+            scales=torch.empty(max(1, nvfp4_scales_bytes(rows, K)), dtype=torch.uint8, device=dev),
+            global_scale=torch.empty(1, dtype=torch.float32, device=dev),
+            workspace=torch.empty(nvfp4_quantize_workspace_bytes(rows, K), dtype=torch.uint8, device=dev),
+            rows=rows, K=K)
+    st = nvfp4_quantize(x.data_ptr(), rows, K, x.stride(0), MODES[mode], RULES[rule], F,
+                        out.codes.data_ptr(), out.scales.data_ptr(), out.global_scale.data_ptr(),
+                        out.workspace.data_ptr(), out.workspace.numel(), _stream_handle(stream))
+    _check(st, "nvfp4_quantize")
+    return out
+
+
+def gemm(a: NVFP4Tensor, b: NVFP4Tensor, out_dtype=None, out=None, workspace=None,
+         stream=None):
+    """Y[M, N] = A_hat @ B_hat^T for two NVFP4 operands with the same K."""
+    import torch
+
+    if a.K != b.K:
+        raise ValueError("operands disagree on K")
+    out_dtype = torch.bfloat16 if out_dtype is None else out_dtype
+    code = {torch.bfloat16: OUT_BF16, torch.float32: OUT_FP32}[out_dtype]
+    M, N, K = a.rows, b.rows, a.K
+    if out is None:
+        out = torch.empty(M, N, dtype=out_dtype, device=a.codes.device)
+    if workspace is None:
+        workspace = torch.empty(nvfp4_gemm_workspace_bytes(), dtype=torch.uint8, device=a.codes.device)
+    st = nvfp4_gemm(a.codes.data_ptr(), a.scales.data_ptr(), a.global_scale.data_ptr(),
+                    b.codes.data_ptr(), b.scales.data_ptr(), b.global_scale.data_ptr(), M, N, K,
+                    out.data_ptr(), out.stride(0), code, workspace.data_ptr(), workspace.numel(),
+                    _stream_handle(stream))
+    _check(st, "nvfp4_gemm")
+    return out
+
+
+def device_status(workspace, stream=None) -> int:
+    """Synchronize the stream and read a call's device status word."""
+    return nvfp4_get_device_status(workspace.data_ptr(), _stream_handle(stream))

@@ -1,0 +1,431 @@
+// gemm.cu -- NVFP4 x NVFP4 GEMM (W4A4 linear layer) on the sm_100a fifth-
+// generation tensor cores.
+//
+// Y[m, n] = (alpha_A * alpha_B) * sum_kb sA[m,kb] sB[n,kb] sum_{k in kb} qA[m,k] qB[n,k]
+// for operands quantized as in nvfp4_quantize: E2M1 codes (two per byte,
+// K-major) and one E4M3 scale per 16 elements along K (ARCQuant summary,
+// gist.science/ko/paper/2601.07475, "방법론": one uniform NVFP4 GEMM along K;
+// Minima page "심층 분석": per-tensor global scales applied around the fused
+// GEMM).
+//
+// Kernel shape: one 128 x 256 output tile per CTA, K consumed 256 elements
+// (128 bytes per row) per pipeline stage, 4 stages in shared memory.
+//   warp 0       TMA producer: A tile 128x128 B and B tile 256x128 B (128-byte
+//                swizzle, out-of-range rows/columns zero-filled by the tensor
+//                map) plus the matching scale atoms (plain bulk copies: the
+//                atoms of one 128-row block and 4 K-groups are contiguous).
+//   warp 1       allocates TMEM (512 columns: accumulator 0..255, A scales
+//                256..271, B scales 272..303) and, from one lane, copies each
+//                stage's scale atoms into TMEM (tcgen05.cp 32x128b.warpx4)
+//                and issues four tcgen05.mma kind::mxf4nvf4 block16 (M=128,
+//                N=256, K=64) per stage; tcgen05.commit frees the stage.
+//   warps 2..5   epilogue: tcgen05.ld 32 lanes x 32 columns at a time,
+//                multiply by alpha_A*alpha_B, convert, store.
+// Every wait is bounded by a deadline on %globaltimer; a wait that runs out
+// records NVFP4_ERR_TIMEOUT in the workspace, raises a CTA-wide abort flag,
+// and every role drains what it has in flight before TMEM is freed.
+#include <cuda_bf16.h>
+
+#include <algorithm>
+#include <mutex>
+
+#include "common.cuh"
+#include "nvfp4_testing.h"
+
+namespace nvfp4 {
+namespace {
+
+constexpr int BM = 128;
+constexpr int BN = 256;
+constexpr int BK_BYTES = 128;  // 256 FP4 elements per row per stage
+constexpr int STAGES = 4;
+constexpr int kThreads = 192;
+constexpr uint32_t A_STAGE = BM * BK_BYTES;    // 16 KB
+constexpr uint32_t B_STAGE = BN * BK_BYTES;    // 32 KB
+constexpr uint32_t SFA_STAGE = 4 * 512;        // 4 atoms (4 K-groups x 128 rows)
+constexpr uint32_t SFB_STAGE = 2 * 4 * 512;    // [row block 0..1][K-group 0..3]
+constexpr uint32_t OFF_A = 0;
+constexpr uint32_t OFF_B = OFF_A + STAGES * A_STAGE;
+constexpr uint32_t OFF_SFA = OFF_B + STAGES * B_STAGE;
+constexpr uint32_t OFF_SFB = OFF_SFA + STAGES * SFA_STAGE;
+constexpr uint32_t OFF_BAR = OFF_SFB + STAGES * SFB_STAGE;
+constexpr uint32_t NUM_BARS = 2 * STAGES + 2;  // full[], empty[], acc_full, drain
+constexpr uint32_t OFF_MISC = OFF_BAR + NUM_BARS * 8;
+constexpr uint32_t SMEM_BYTES = OFF_MISC + 16 + 1024;  // + alignment slack
+constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t TM_ACC = 0, TM_SFA = 256, TM_SFB = 272;
+
+// Instruction descriptor, kind::mxf4nvf4: A/B format E2M1 (1) at bits 7-9 and
+// 10-12, K-major A and B, N>>3 at bits 17-22, scale format UE4M3 (0) at bit
+// 23, M>>4 at bits 24-28, dense K = 64.
+constexpr uint32_t kIdesc = (1u << 7) | (1u << 10) | (uint32_t(BN >> 3) << 17) | (uint32_t(BM >> 4) << 24);
+
+// Shared-memory matrix descriptor for a K-major operand tile written by TMA
+// with the 128-byte swizzle: rows of 128 bytes, 8-row groups 1024 bytes apart
+// (SBO), descriptor version 1, layout type 2 (SWIZZLE_128B).
+__device__ __forceinline__ uint64_t operand_desc(uint32_t saddr) {
+  return static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4) | (static_cast<uint64_t>(1) << 16) |
+         (static_cast<uint64_t>(1024 >> 4) << 32) | (static_cast<uint64_t>(1) << 46) |
+         (static_cast<uint64_t>(2) << 61);
+}
+// Descriptor of one 512-byte scale atom for tcgen05.cp 32x128b: 32 rows of
+// 16 bytes, no swizzle, 8-row core matrices 128 bytes apart (SBO).
+__device__ __forceinline__ uint64_t scale_desc(uint32_t saddr) {
+  return static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4) | (static_cast<uint64_t>(128 >> 4) << 32) |
+         (static_cast<uint64_t>(1) << 46);
+}
+
+__device__ __forceinline__ void tmem_copy_scales(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc)
+               : "memory");
+}
+
+__device__ __forceinline__ void mma_nvf4(uint32_t tacc, uint64_t adesc, uint64_t bdesc,
+                                         uint32_t tsfa, uint32_t tsfb, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(
+          tacc),
+      "l"(adesc), "l"(bdesc), "r"(kIdesc), "r"(accumulate), "r"(tsfa), "r"(tsfb)
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
+      "%12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, "
+      "%30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]),
+        "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]),
+        "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&v);
+}
+
+struct GemmParams {
+  const uint8_t* a_scales;
+  const uint8_t* b_scales;
+  const float* a_global;
+  const float* b_global;
+  void* y;
+  WorkspaceHeader* ws;
+  int64_t ldy;
+  int M, N;
+  uint32_t kgroups;       // K / 64
+  uint32_t ktiles;        // ceil(K / 256)
+  uint32_t n_rowblocks;   // ceil(N / 128): scale row blocks that exist for B
+  int out_fp32;
+  int vec_store;          // rows of Y start 16-byte aligned: 32-column vector stores
+  uint64_t timeout_ns;
+  int debug_flags;        // bit 0: never issue the first stage's copies (timeout test)
+};
+
+__device__ __forceinline__ void record_timeout(const GemmParams& p, volatile int* abort,
+                                               uint32_t where) {
+  *abort = 1;
+  p.ws->detail = where;
+  p.ws->status = NVFP4_ERR_TIMEOUT;
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                const GemmParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t bar_full = sbase + OFF_BAR;
+  const uint32_t bar_empty = bar_full + 8 * STAGES;
+  const uint32_t bar_acc = bar_empty + 8 * STAGES;
+  const uint32_t bar_drain = bar_acc + 8;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_MISC);
+  volatile int* abort = reinterpret_cast<volatile int*>(smem + OFF_MISC + 4);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int m0 = blockIdx.y * BM, n0 = blockIdx.x * BN;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(bar_full + 8 * s, 1);
+      mbar_init(bar_empty + 8 * s, 1);
+    }
+    mbar_init(bar_acc, 1);
+    mbar_init(bar_drain, 1);
+    *abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tensormap(&tmA);
+    prefetch_tensormap(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint64_t deadline = global_timer_ns() + p.timeout_ns;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------ TMA producer ----
+      const uint32_t nb_valid = min(2u, p.n_rowblocks - static_cast<uint32_t>(n0 / 128));
+      const uint8_t* sfa_src = p.a_scales + static_cast<size_t>(m0 / 128) * p.kgroups * 512;
+      const uint8_t* sfb_src = p.b_scales + static_cast<size_t>(n0 / 128) * p.kgroups * 512;
+      uint32_t issued = 0;
+      for (uint32_t kt = 0; kt < p.ktiles; ++kt) {
+        const uint32_t s = kt % STAGES, ph = (kt / STAGES) & 1u;
+        if (kt >= STAGES && !mbar_wait_bounded(bar_empty + 8 * s, ph ^ 1u, abort, deadline)) {
+          if (!*abort) record_timeout(p, abort, 1);
+          break;
+        }
+        const uint32_t nk = min(4u, p.kgroups - kt * 4);
+        const uint32_t fb = bar_full + 8 * s;
+        mbar_expect_tx(fb, A_STAGE + B_STAGE + nk * 512 * (1 + nb_valid));
+        ++issued;
+        if ((p.debug_flags & 1) && kt == 0) continue;  // test hook: this stage never fills
+        tma_load_2d(sbase + OFF_A + s * A_STAGE, &tmA, fb, static_cast<int32_t>(kt * BK_BYTES), m0);
+        tma_load_2d(sbase + OFF_B + s * B_STAGE, &tmB, fb, static_cast<int32_t>(kt * BK_BYTES), n0);
+        bulk_load(sbase + OFF_SFA + s * SFA_STAGE, sfa_src + static_cast<size_t>(kt) * 4 * 512, nk * 512, fb);
+        for (uint32_t i = 0; i < nb_valid; ++i)
+          bulk_load(sbase + OFF_SFB + s * SFB_STAGE + i * 2048,
+                    sfb_src + (static_cast<size_t>(i) * p.kgroups + kt * 4) * 512, nk * 512, fb);
+      }
+      if (*abort) {
+        // Drain: wait (briefly) for the copies of the last stages issued so
+        // no bulk copy is still writing shared memory when the CTA exits.
+        const uint64_t dl = global_timer_ns() + 100000000ull;  // 100 ms
+        const volatile int no_abort = 0;
+        const uint32_t first = issued > STAGES ? issued - STAGES : 0;
+        for (uint32_t kt = first; kt < issued; ++kt)
+          mbar_wait_bounded(bar_full + 8 * (kt % STAGES), (kt / STAGES) & 1u, &no_abort, dl);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ------------------------------------------------ MMA issuer ------
+      bool any_mma = false;
+      for (uint32_t kt = 0; kt < p.ktiles; ++kt) {
+        const uint32_t s = kt % STAGES, ph = (kt / STAGES) & 1u;
+        if (!mbar_wait_bounded(bar_full + 8 * s, ph, abort, deadline)) {
+          if (!*abort) record_timeout(p, abort, 2);
+          break;
+        }
+        tc_fence_after();
+        const uint32_t nk = min(4u, p.kgroups - kt * 4);
+        const uint32_t sfa = sbase + OFF_SFA + s * SFA_STAGE;
+        const uint32_t sfb = sbase + OFF_SFB + s * SFB_STAGE;
+        for (uint32_t j = 0; j < nk; ++j) {
+          tmem_copy_scales(tmem + TM_SFA + 4 * j, scale_desc(sfa + 512 * j));
+          tmem_copy_scales(tmem + TM_SFB + 8 * j, scale_desc(sfb + 512 * j));
+          tmem_copy_scales(tmem + TM_SFB + 8 * j + 4, scale_desc(sfb + 2048 + 512 * j));
+        }
+        const uint32_t sa = sbase + OFF_A + s * A_STAGE;
+        const uint32_t sb = sbase + OFF_B + s * B_STAGE;
+        for (uint32_t j = 0; j < nk; ++j) {
+          mma_nvf4(tmem + TM_ACC, operand_desc(sa + 32 * j), operand_desc(sb + 32 * j),
+                   tmem + TM_SFA + 4 * j, tmem + TM_SFB + 8 * j, (kt | j) != 0);
+        }
+        any_mma = true;
+        tc_commit(bar_empty + 8 * s);
+      }
+      if (!*abort) {
+        tc_commit(bar_acc);
+      } else if (any_mma) {
+        // Drain the MMAs already issued before TMEM is released.
+        const volatile int no_abort = 0;
+        tc_commit(bar_drain);
+        mbar_wait_bounded(bar_drain, 0, &no_abort, global_timer_ns() + 100000000ull);
+      }
+    }
+  } else {
+    // -------------------------------------------------- epilogue --------
+    const int quad = warp & 3;  // warps 2,3,4,5 -> TMEM lanes 64,96,0,32
+    const int row = m0 + quad * 32 + lane;
+    bool ok = mbar_wait_bounded(bar_acc, 0, abort, deadline);
+    ok = __all_sync(0xffffffffu, ok);
+    if (!ok) {
+      if (lane == 0 && !*abort) record_timeout(p, abort, 3);
+    } else {
+      tc_fence_after();
+      const float ab = __fmul_rn(__ldg(p.a_global), __ldg(p.b_global));
+      for (int c = 0; c < BN; c += 32) {
+        uint32_t r[32];
+        tmem_ld32(tmem + (static_cast<uint32_t>(quad * 32) << 16) + TM_ACC + c, r);
+        const int col0 = n0 + c;
+        if (row >= p.M || col0 >= p.N) continue;
+        const bool full = p.vec_store && col0 + 32 <= p.N;
+        if (p.out_fp32) {
+          float* dst = static_cast<float*>(p.y) + static_cast<int64_t>(row) * p.ldy + col0;
+          if (full) {
+#pragma unroll
+            for (int i = 0; i < 32; i += 4)
+              *reinterpret_cast<float4*>(dst + i) =
+                  make_float4(__uint_as_float(r[i]) * ab, __uint_as_float(r[i + 1]) * ab,
+                              __uint_as_float(r[i + 2]) * ab, __uint_as_float(r[i + 3]) * ab);
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              if (col0 + i < p.N) dst[i] = __uint_as_float(r[i]) * ab;
+          }
+        } else {
+          __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(p.y) + static_cast<int64_t>(row) * p.ldy + col0;
+          if (full) {
+#pragma unroll
+            for (int i = 0; i < 32; i += 8) {
+              uint4 v;
+              v.x = pack_bf16x2(__uint_as_float(r[i]) * ab, __uint_as_float(r[i + 1]) * ab);
+              v.y = pack_bf16x2(__uint_as_float(r[i + 2]) * ab, __uint_as_float(r[i + 3]) * ab);
+              v.z = pack_bf16x2(__uint_as_float(r[i + 4]) * ab, __uint_as_float(r[i + 5]) * ab);
+              v.w = pack_bf16x2(__uint_as_float(r[i + 6]) * ab, __uint_as_float(r[i + 7]) * ab);
+              *reinterpret_cast<uint4*>(dst + i) = v;
+            }
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              if (col0 + i < p.N) dst[i] = __float2bfloat16_rn(__uint_as_float(r[i]) * ab);
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, TMEM_COLS);
+}
+
+// ------------------------------------------------------------------ host --
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  });
+  return fn;
+}
+
+// 2D uint8 tensor map over a K-major code matrix [rows, K/2] with a
+// 128-byte x box_rows box and the 128-byte swizzle.
+nvfp4_status make_code_map(CUtensorMap* map, const void* base, int64_t rows, int64_t K, uint32_t box_rows) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc) return set_error(NVFP4_ERR_CUDA, "cuTensorMapEncodeTiled entry point not available");
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K / 2), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K / 2)};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(BK_BYTES), box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box,
+                   estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return set_error(NVFP4_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return NVFP4_OK;
+}
+
+}  // namespace
+
+// Test hooks (not part of the public header): bounded-wait deadline and
+// debug flags for the next nvfp4_gemm calls on this process.
+static uint64_t g_timeout_ns = 4000000000ull;  // 4 s
+static int g_debug_flags = 0;
+
+}  // namespace nvfp4
+
+using namespace nvfp4;
+
+extern "C" {
+
+void nvfp4_testing_set_gemm_wait(uint64_t timeout_ns, int debug_flags) {
+  g_timeout_ns = timeout_ns ? timeout_ns : 4000000000ull;
+  g_debug_flags = debug_flags;
+}
+
+nvfp4_status nvfp4_gemm(const void* a_codes, const void* a_scales, const float* a_global,
+                        const void* b_codes, const void* b_scales, const float* b_global,
+                        int64_t M, int64_t N, int64_t K, void* y, int64_t ldy, int out_dtype,
+                        void* workspace, size_t workspace_bytes, void* stream) {
+  if (!a_codes || !a_scales || !a_global || !b_codes || !b_scales || !b_global || !y || !workspace)
+    return set_error(NVFP4_ERR_INVALID_ARG, "nvfp4_gemm: null pointer argument");
+  if (M < 1 || N < 1 || K < 64 || K % 64 != 0)
+    return set_error(NVFP4_ERR_INVALID_ARG,
+                     "nvfp4_gemm: need M, N >= 1 and K a positive multiple of 64 (M=%lld N=%lld K=%lld)",
+                     (long long)M, (long long)N, (long long)K);
+  if (M > (1ll << 30) || N > (1ll << 30) || K > (1ll << 30))
+    return set_error(NVFP4_ERR_INVALID_ARG, "nvfp4_gemm: dimension too large");
+  if (ldy < N) return set_error(NVFP4_ERR_INVALID_ARG, "nvfp4_gemm: need ldy >= N");
+  if (out_dtype != NVFP4_OUT_BF16 && out_dtype != NVFP4_OUT_FP32)
+    return set_error(NVFP4_ERR_INVALID_ARG, "nvfp4_gemm: unknown out_dtype %d", out_dtype);
+  if (!aligned16(a_codes) || !aligned16(b_codes) || !aligned16(a_scales) || !aligned16(b_scales) ||
+      (reinterpret_cast<uintptr_t>(y) & (out_dtype == NVFP4_OUT_FP32 ? 3u : 1u)) ||
+      !aligned16(workspace) || (reinterpret_cast<uintptr_t>(a_global) & 3u) ||
+      (reinterpret_cast<uintptr_t>(b_global) & 3u))
+    return set_error(NVFP4_ERR_INVALID_ARG, "nvfp4_gemm: misaligned buffer");
+  if (workspace_bytes < nvfp4_gemm_workspace_bytes())
+    return set_error(NVFP4_ERR_INVALID_ARG, "nvfp4_gemm: workspace too small");
+  int dev = 0, sms = 0;
+  nvfp4_status st = check_device(&dev, &sms);
+  if (st != NVFP4_OK) return st;
+
+  CUtensorMap ta, tb;
+  if ((st = make_code_map(&ta, a_codes, M, K, BM)) != NVFP4_OK) return st;
+  if ((st = make_code_map(&tb, b_codes, N, K, BN)) != NVFP4_OK) return st;
+
+  static std::once_flag attr_once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(attr_once, [] {
+    attr_err = cudaFuncSetAttribute(gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    static_cast<int>(SMEM_BYTES));
+  });
+  if (attr_err != cudaSuccess) return cuda_status(attr_err, "cudaFuncSetAttribute(gemm_kernel)");
+
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemsetAsync(workspace, 0, sizeof(WorkspaceHeader), s);
+  if (e != cudaSuccess) return cuda_status(e, "cudaMemsetAsync(status)");
+
+  GemmParams p;
+  p.a_scales = static_cast<const uint8_t*>(a_scales);
+  p.b_scales = static_cast<const uint8_t*>(b_scales);
+  p.a_global = a_global;
+  p.b_global = b_global;
+  p.y = y;
+  p.ws = static_cast<WorkspaceHeader*>(workspace);
+  p.ldy = ldy;
+  p.M = static_cast<int>(M);
+  p.N = static_cast<int>(N);
+  p.kgroups = static_cast<uint32_t>(K / 64);
+  p.ktiles = static_cast<uint32_t>((K + 255) / 256);
+  p.n_rowblocks = static_cast<uint32_t>((N + 127) / 128);
+  p.out_fp32 = out_dtype == NVFP4_OUT_FP32;
+  p.vec_store = aligned16(y) && ((ldy * (p.out_fp32 ? 4 : 2)) % 16 == 0);
+  p.timeout_ns = g_timeout_ns;
+  p.debug_flags = g_debug_flags;
+  dim3 grid(static_cast<unsigned>((N + BN - 1) / BN), static_cast<unsigned>((M + BM - 1) / BM));
+  if (grid.y > 65535u) return set_error(NVFP4_ERR_INVALID_ARG, "nvfp4_gemm: M too large");
+  gemm_kernel<<<grid, kThreads, SMEM_BYTES, s>>>(ta, tb, p);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_status(e, "gemm_kernel launch");
+  return NVFP4_OK;
+}
+
+}  // extern "C"
