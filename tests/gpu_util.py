@@ -70,7 +70,7 @@ def upload_operand(codes: np.ndarray, scales_canon: np.ndarray, alpha: float) ->
         rows=rows, K=K)
 
 
-# GEMM tolerance (the benchmark spec: max relative error 1e-3 against the fp64 product
+# GEMM tolerance (max relative error 1e-3 against the fp64 product
 # of the dequantized operands).  Entries whose |ref| is below 1e-3 of the sum
 # of |products| are cancellation-dominated; they must be within 1e-6 of that
 # sum instead.  bf16 output adds its own rounding (2^-9 relative).
