@@ -129,6 +129,29 @@ NVFP4_API nvfp4_status nvfp4_quantize(const void* x, int64_t rows, int64_t K, in
                             float* global_scale, void* workspace, size_t workspace_bytes,
                             void* stream);
 
+/* nvfp4_quantize without a workspace, for callers that cannot allocate device
+ * memory where they quantize: a custom-op or plugin hook inside another
+ * inference runtime that owns every device allocation and passes the op only
+ * its inputs and outputs, or a service whose device-memory footprint is fixed
+ * at start-up and which must not allocate on the request path.  The paper has
+ * no counterpart; this is an interface convenience of this library.
+ * Same arguments, requirements and outputs as nvfp4_quantize, minus the
+ * workspace.  The scratch (status word and amax partial maxima) is a static
+ * device array of 16448 bytes inside this library, held on every GPU that
+ * loads it until the process exits; a launch whose amax pass would need more
+ * than its 4096 partial slots is rejected with NVFP4_ERR_INVALID_ARG (a B200
+ * uses at most 592).  Nothing in the scratch has to start at zero: every call
+ * writes what it later reads.  All calls on a device share the array, so calls
+ * that may overlap on the GPU race and must be ordered by the caller (same
+ * stream, or events).  The first call on each device looks up the array's
+ * device address with cudaGetSymbolAddress (with that device current); make
+ * that first call before any stream capture.  Non-finite input shows as a NaN
+ * *global_scale (there is no workspace status word to read).  Allocates
+ * nothing: no cudaMalloc, cudaFree or allocating library routine. */
+NVFP4_API nvfp4_status nvfp4_quantize_noalloc(const void* x, int64_t rows, int64_t K, int64_t ldx,
+                                              int mode, int rule, float fp8_max, void* codes,
+                                              void* scales, float* global_scale, void* stream);
+
 /* Y [M, N] = (alpha_A * alpha_B) * (A_hat . B_hat^T) with an fp32 accumulator.
  *   a_codes/a_scales/a_global  operand A (M rows), as nvfp4_quantize wrote it
  *   b_codes/b_scales/b_global  operand B (N rows, e.g. a weight [N, K])

@@ -35,6 +35,8 @@ _SIGNATURES = {
     "nvfp4_gemm_workspace_bytes": (ctypes.c_size_t, []),
     "nvfp4_quantize": (ctypes.c_int, [_P, _I64, _I64, _I64, ctypes.c_int, ctypes.c_int,
                                       ctypes.c_float, _P, _P, _P, _P, ctypes.c_size_t, _P]),
+    "nvfp4_quantize_noalloc": (ctypes.c_int, [_P, _I64, _I64, _I64, ctypes.c_int, ctypes.c_int,
+                                              ctypes.c_float, _P, _P, _P, _P]),
     "nvfp4_gemm": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _I64,
                                   ctypes.c_int, _P, ctypes.c_size_t, _P]),
     "nvfp4_get_device_status": (ctypes.c_int, [_P, _P]),
@@ -92,6 +94,14 @@ def nvfp4_quantize(x, rows, K, ldx, mode, rule, fp8_max, codes, scales, global_s
                    workspace_bytes, stream) -> int:
     return load().nvfp4_quantize(x, rows, K, ldx, mode, rule, fp8_max, codes, scales, global_scale,
                                  workspace, workspace_bytes, stream)
+
+
+def nvfp4_quantize_noalloc(x, rows, K, ldx, mode, rule, fp8_max, codes, scales, global_scale,
+                           stream) -> int:
+    """nvfp4_quantize with its scratch in a static device array inside the
+    library: no workspace argument, nothing allocated (see include/nvfp4.h)."""
+    return load().nvfp4_quantize_noalloc(x, rows, K, ldx, mode, rule, fp8_max, codes, scales,
+                                         global_scale, stream)
 
 
 def nvfp4_gemm(a_codes, a_scales, a_global, b_codes, b_scales, b_global, M, N, K, y, ldy,

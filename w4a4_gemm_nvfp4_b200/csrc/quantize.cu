@@ -27,6 +27,7 @@
 #include <cuda_fp16.h>
 
 #include <algorithm>
+#include <mutex>
 
 #include "common.cuh"
 
@@ -391,3 +392,132 @@ nvfp4_status nvfp4_quantize(const void* x, int64_t rows, int64_t K, int64_t ldx,
 }
 
 }  // extern "C"
+
+// ------------------------------------------------ allocation-free variant --
+//
+// nvfp4_quantize needs a caller-provided device workspace for the amax pass's
+// per-CTA partial maxima and the status word.  Some callers cannot provide
+// one: a custom-op or plugin hook running inside another inference runtime
+// that owns every device allocation and hands the op only its inputs and
+// outputs, or a service that fixes its device-memory footprint at start-up
+// and must not allocate on the request path (an allocation there can block,
+// fragment the pool, or fail under memory pressure in the middle of a
+// request).  nvfp4_quantize_noalloc runs the same two kernels with that
+// scratch in a static device array instead, so it allocates nothing.
+//
+// The array below is held by every GPU that loads this library, from module
+// load until process exit.  Its size bounds the amax pass at kMaxPartials
+// CTAs (the launch uses at most 4 per SM, 592 on a B200); a launch that would
+// need more is rejected.  Nothing in it has to start at zero: each call's amax
+// kernel writes every partial slot the following quantize kernel reads, and
+// the quantize kernel writes the status word.  All calls on a device share it,
+// so two calls that may overlap on the GPU (different streams without an
+// ordering between them) race on it and must be serialized by the caller.
+
+namespace nvfp4 {
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = sizeof(WorkspaceHeader) + sizeof(uint32_t) * kMaxPartials;
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+constexpr int kNoAllocMaxDevices = 64;
+static std::mutex g_noalloc_mu;
+static void* g_noalloc_addr[kNoAllocMaxDevices];
+
+// Device address of g_noalloc_scratch on the current device `dev`, looked up
+// once per device (the first call on a device does this set-up).  In host
+// code the array's name is only a host-side stand-in for the symbol, never a
+// device address, so kernels must get this pointer instead.
+nvfp4_status noalloc_scratch(int dev, void** out) {
+  if (dev < 0 || dev >= kNoAllocMaxDevices)
+    return set_error(NVFP4_ERR_UNSUPPORTED_DEVICE, "nvfp4_quantize_noalloc: device %d", dev);
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (!g_noalloc_addr[dev]) {
+    void* p = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return cuda_status(e, "cudaGetSymbolAddress(noalloc scratch)");
+    g_noalloc_addr[dev] = p;
+  }
+  *out = g_noalloc_addr[dev];
+  return NVFP4_OK;
+}
+
+}  // namespace
+}  // namespace nvfp4
+
+extern "C" nvfp4_status nvfp4_quantize_noalloc(const void* x, int64_t rows, int64_t K, int64_t ldx,
+                                               int mode, int rule, float fp8_max, void* codes,
+                                               void* scales, float* global_scale, void* stream) {
+  if (!x || !codes || !scales || !global_scale)
+    return set_error(NVFP4_ERR_INVALID_ARG, "nvfp4_quantize_noalloc: null pointer argument");
+  if (rows < 1 || K < 64 || K % 64 != 0)
+    return set_error(NVFP4_ERR_INVALID_ARG,
+                     "nvfp4_quantize_noalloc: need rows >= 1 and K a positive multiple of 64 (rows=%lld K=%lld)",
+                     (long long)rows, (long long)K);
+  if (ldx < K || ldx % 8 != 0)
+    return set_error(NVFP4_ERR_INVALID_ARG, "nvfp4_quantize_noalloc: need ldx >= K and ldx %% 8 == 0");
+  if (mode != NVFP4_MODE_SIX && mode != NVFP4_MODE_FOUR_OVER_SIX)
+    return set_error(NVFP4_ERR_INVALID_ARG, "nvfp4_quantize_noalloc: unknown mode %d", mode);
+  if (rule != NVFP4_RULE_MAX && rule != NVFP4_RULE_MAE && rule != NVFP4_RULE_MSE)
+    return set_error(NVFP4_ERR_INVALID_ARG, "nvfp4_quantize_noalloc: unknown rule %d", rule);
+  if (!(fp8_max == 448.0f || fp8_max == 256.0f))
+    return set_error(NVFP4_ERR_INVALID_ARG, "nvfp4_quantize_noalloc: fp8_max must be 448 or 256");
+  if (!aligned16(x) || !aligned16(codes) || !aligned16(scales) ||
+      (reinterpret_cast<uintptr_t>(global_scale) & 3u))
+    return set_error(NVFP4_ERR_INVALID_ARG, "nvfp4_quantize_noalloc: misaligned buffer");
+  const int64_t row_blocks = (rows + 127) / 128;
+  const int64_t ntasks = row_blocks * 16 * (K / 64);
+  if (ntasks > 0xFFFFFFFFll || rows * ldx > (1ll << 40))
+    return set_error(NVFP4_ERR_INVALID_ARG, "nvfp4_quantize_noalloc: tensor too large");
+  int dev = 0, sms = 0;
+  nvfp4_status st = check_device(&dev, &sms);
+  if (st != NVFP4_OK) return st;
+
+  int amax_grid;
+  if (ldx == K) {
+    const int64_t nvec = rows * K / 8;
+    amax_grid = static_cast<int>(std::min<int64_t>((nvec + kAmaxThreads * 4 - 1) / (kAmaxThreads * 4),
+                                                   static_cast<int64_t>(sms) * 4));
+  } else {
+    amax_grid = static_cast<int>(std::min<int64_t>(rows, static_cast<int64_t>(sms) * 4));
+  }
+  amax_grid = std::max(1, amax_grid);
+  if (amax_grid > kMaxPartials)
+    return set_error(NVFP4_ERR_INVALID_ARG,
+                     "nvfp4_quantize_noalloc: the amax pass needs %d partial slots but the static "
+                     "scratch holds %d (%zu bytes)", amax_grid, kMaxPartials, kNoAllocScratchBytes);
+
+  void* scratch = nullptr;
+  if ((st = noalloc_scratch(dev, &scratch)) != NVFP4_OK) return st;
+  auto* ws = static_cast<WorkspaceHeader*>(scratch);
+  auto* partials = reinterpret_cast<uint32_t*>(static_cast<char*>(scratch) + sizeof(WorkspaceHeader));
+
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  amax_kernel<<<amax_grid, kAmaxThreads, 0, s>>>(static_cast<const uint16_t*>(x), rows, K, ldx,
+                                                  partials);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_status(e, "amax_kernel launch");
+
+  QuantParams p;
+  p.x = static_cast<const uint16_t*>(x);
+  p.rows = rows;
+  p.K = K;
+  p.ldx = ldx;
+  p.codes = static_cast<uint8_t*>(codes);
+  p.scales = static_cast<uint8_t*>(scales);
+  p.global_scale = global_scale;
+  p.partials = partials;
+  p.ws = ws;
+  p.nparts = amax_grid;
+  p.f6 = fp8_max * 6.0f;
+  p.ntasks = static_cast<uint32_t>(ntasks);
+  p.kgroups = static_cast<uint32_t>(K / 64);
+  const int64_t want = (ntasks + kQuantWarps - 1) / kQuantWarps;
+  const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(want, static_cast<int64_t>(sms) * 8)));
+  if (mode == NVFP4_MODE_SIX) e = launch_quantize<false, kRuleMax>(grid, p, s);
+  else if (rule == NVFP4_RULE_MAX) e = launch_quantize<true, kRuleMax>(grid, p, s);
+  else if (rule == NVFP4_RULE_MAE) e = launch_quantize<true, kRuleMae>(grid, p, s);
+  else e = launch_quantize<true, kRuleMse>(grid, p, s);
+  if (e != cudaSuccess) return cuda_status(e, "quantize_kernel launch");
+  return NVFP4_OK;
+}
