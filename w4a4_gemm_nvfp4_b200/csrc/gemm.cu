@@ -8,19 +8,26 @@
 // Minima page "심층 분석": per-tensor global scales applied around the fused
 // GEMM).
 //
-// Kernel shape: one 128 x 256 output tile per CTA, K consumed 256 elements
-// (128 bytes per row) per pipeline stage, 4 stages in shared memory.
+// Kernel shape: persistent, one CTA per SM walking 128 x 256 output tiles
+// (tile t, t + gridDim.x, ...), K consumed 256 elements (128 bytes per row)
+// per pipeline stage through a 4-stage shared-memory ring that runs on
+// across tile boundaries.
 //   warp 0       TMA producer: A tile 128x128 B and B tile 256x128 B (128-byte
 //                swizzle, out-of-range rows/columns zero-filled by the tensor
 //                map) plus the matching scale atoms (plain bulk copies: the
 //                atoms of one 128-row block and 4 K-groups are contiguous).
-//   warp 1       allocates TMEM (512 columns: accumulator 0..255, A scales
-//                256..271, B scales 272..303) and, from one lane, copies each
-//                stage's scale atoms into TMEM (tcgen05.cp 32x128b.warpx4)
-//                and issues four tcgen05.mma kind::mxf4nvf4 block16 (M=128,
-//                N=256, K=64) per stage; tcgen05.commit frees the stage.
-//   warps 2..5   epilogue: tcgen05.ld 32 lanes x 32 columns at a time,
+//   warp 1       allocates TMEM and, from one lane, copies each stage's scale
+//                atoms into TMEM (tcgen05.cp 32x128b.warpx4) and issues four
+//                tcgen05.mma kind::mxf4nvf4 block16 (M=128, N=256, K=64) per
+//                stage; tcgen05.commit frees the stage.
+//   warps 2..5   epilogue: tcgen05.ld 32 lanes x 64 columns at a time,
 //                multiply by alpha_A*alpha_B, convert, store.
+// TMEM (512 columns): two accumulators that share one 64-column subtile,
+// buffer 0 = columns 0..255 and buffer 1 = columns 192..447, scales at
+// 448..511.  The epilogue drains the shared subtile (columns 192..255) first
+// and then lets the next tile's MMAs start, so storing tile i overlaps the
+// mainloop of tile i+1 although two full 256-column accumulators would not
+// fit next to the scales.
 // Every wait is bounded by a deadline on %globaltimer; a wait that runs out
 // records NVFP4_ERR_TIMEOUT in the workspace, raises a CTA-wide abort flag,
 // and every role drains what it has in flight before TMEM is freed.
@@ -49,11 +56,15 @@ constexpr uint32_t OFF_B = OFF_A + STAGES * A_STAGE;
 constexpr uint32_t OFF_SFA = OFF_B + STAGES * B_STAGE;
 constexpr uint32_t OFF_SFB = OFF_SFA + STAGES * SFA_STAGE;
 constexpr uint32_t OFF_BAR = OFF_SFB + STAGES * SFB_STAGE;
-constexpr uint32_t NUM_BARS = 2 * STAGES + 2;  // full[], empty[], acc_full, drain
+constexpr uint32_t NUM_BARS = 2 * STAGES + 3;  // full[], empty[], acc_full, acc_free, drain
 constexpr uint32_t OFF_MISC = OFF_BAR + NUM_BARS * 8;
 constexpr uint32_t SMEM_BYTES = OFF_MISC + 16 + 1024;  // + alignment slack
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t TM_ACC = 0, TM_SFA = 256, TM_SFB = 272;
+constexpr uint32_t EPI_N = 64;                    // epilogue subtile (columns)
+constexpr uint32_t TM_ACC1 = 256 - EPI_N;         // buffer 1 starts on buffer 0's last subtile
+constexpr uint32_t TM_SFA = TM_ACC1 + 256;        // 448: 4 columns per K-group x 4
+constexpr uint32_t TM_SFB = TM_SFA + 16;          // 464: 8 columns per K-group x 4
+static_assert(TM_SFB + 32 <= TMEM_COLS, "scales must fit after the accumulators");
 
 // Instruction descriptor, kind::mxf4nvf4: A/B format E2M1 (1) at bits 7-9 and
 // 10-12, K-major A and B, N>>3 at bits 17-22, scale format UE4M3 (0) at bit
@@ -122,6 +133,8 @@ struct GemmParams {
   uint32_t kgroups;       // K / 64
   uint32_t ktiles;        // ceil(K / 256)
   uint32_t n_rowblocks;   // ceil(N / 128): scale row blocks that exist for B
+  uint32_t n_tiles;       // ceil(N / 256)
+  uint32_t num_tiles;     // ceil(M / 128) * n_tiles
   int out_fp32;
   int vec_store;          // rows of Y start 16-byte aligned: 32-column vector stores
   uint64_t timeout_ns;
@@ -144,20 +157,21 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t sbase = smem_u32(smem);
   const uint32_t bar_full = sbase + OFF_BAR;
   const uint32_t bar_empty = bar_full + 8 * STAGES;
-  const uint32_t bar_acc = bar_empty + 8 * STAGES;
-  const uint32_t bar_drain = bar_acc + 8;
+  const uint32_t bar_acc_full = bar_empty + 8 * STAGES;
+  const uint32_t bar_acc_free = bar_acc_full + 8;
+  const uint32_t bar_drain = bar_acc_free + 8;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_MISC);
   volatile int* abort = reinterpret_cast<volatile int*>(smem + OFF_MISC + 4);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int m0 = blockIdx.y * BM, n0 = blockIdx.x * BN;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(bar_full + 8 * s, 1);
       mbar_init(bar_empty + 8 * s, 1);
     }
-    mbar_init(bar_acc, 1);
+    mbar_init(bar_acc_full, 1);
+    mbar_init(bar_acc_free, 4);  // one arrive per epilogue warp
     mbar_init(bar_drain, 1);
     *abort = 0;
     fence_barrier_init();
@@ -179,69 +193,86 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     if (lane == 0) {
       // ------------------------------------------------ TMA producer ----
-      const uint32_t nb_valid = min(2u, p.n_rowblocks - static_cast<uint32_t>(n0 / 128));
-      const uint8_t* sfa_src = p.a_scales + static_cast<size_t>(m0 / 128) * p.kgroups * 512;
-      const uint8_t* sfb_src = p.b_scales + static_cast<size_t>(n0 / 128) * p.kgroups * 512;
-      uint32_t issued = 0;
-      for (uint32_t kt = 0; kt < p.ktiles; ++kt) {
-        const uint32_t s = kt % STAGES, ph = (kt / STAGES) & 1u;
-        if (kt >= STAGES && !mbar_wait_bounded(bar_empty + 8 * s, ph ^ 1u, abort, deadline)) {
-          if (!*abort) record_timeout(p, abort, 1);
-          break;
+      uint32_t it = 0;  // global k-tile counter across this CTA's tiles
+      bool stop = false;
+      for (uint32_t tile = blockIdx.x; tile < p.num_tiles && !stop; tile += gridDim.x) {
+        const int m0 = static_cast<int>(tile / p.n_tiles) * BM;
+        const int n0 = static_cast<int>(tile % p.n_tiles) * BN;
+        const uint32_t nb_valid = min(2u, p.n_rowblocks - static_cast<uint32_t>(n0 / 128));
+        const uint8_t* sfa_src = p.a_scales + static_cast<size_t>(m0 / 128) * p.kgroups * 512;
+        const uint8_t* sfb_src = p.b_scales + static_cast<size_t>(n0 / 128) * p.kgroups * 512;
+        for (uint32_t kt = 0; kt < p.ktiles; ++kt, ++it) {
+          const uint32_t s = it % STAGES, ph = (it / STAGES) & 1u;
+          if (it >= STAGES && !mbar_wait_bounded(bar_empty + 8 * s, ph ^ 1u, abort, deadline)) {
+            if (!*abort) record_timeout(p, abort, 1);
+            stop = true;
+            break;
+          }
+          const uint32_t nk = min(4u, p.kgroups - kt * 4);
+          const uint32_t fb = bar_full + 8 * s;
+          mbar_expect_tx(fb, A_STAGE + B_STAGE + nk * 512 * (1 + nb_valid));
+          if ((p.debug_flags & 1) && it == 0) continue;  // test hook: this stage never fills
+          tma_load_2d(sbase + OFF_A + s * A_STAGE, &tmA, fb, static_cast<int32_t>(kt * BK_BYTES), m0);
+          tma_load_2d(sbase + OFF_B + s * B_STAGE, &tmB, fb, static_cast<int32_t>(kt * BK_BYTES), n0);
+          bulk_load(sbase + OFF_SFA + s * SFA_STAGE, sfa_src + static_cast<size_t>(kt) * 4 * 512,
+                    nk * 512, fb);
+          for (uint32_t i = 0; i < nb_valid; ++i)
+            bulk_load(sbase + OFF_SFB + s * SFB_STAGE + i * 2048,
+                      sfb_src + (static_cast<size_t>(i) * p.kgroups + kt * 4) * 512, nk * 512, fb);
         }
-        const uint32_t nk = min(4u, p.kgroups - kt * 4);
-        const uint32_t fb = bar_full + 8 * s;
-        mbar_expect_tx(fb, A_STAGE + B_STAGE + nk * 512 * (1 + nb_valid));
-        ++issued;
-        if ((p.debug_flags & 1) && kt == 0) continue;  // test hook: this stage never fills
-        tma_load_2d(sbase + OFF_A + s * A_STAGE, &tmA, fb, static_cast<int32_t>(kt * BK_BYTES), m0);
-        tma_load_2d(sbase + OFF_B + s * B_STAGE, &tmB, fb, static_cast<int32_t>(kt * BK_BYTES), n0);
-        bulk_load(sbase + OFF_SFA + s * SFA_STAGE, sfa_src + static_cast<size_t>(kt) * 4 * 512, nk * 512, fb);
-        for (uint32_t i = 0; i < nb_valid; ++i)
-          bulk_load(sbase + OFF_SFB + s * SFB_STAGE + i * 2048,
-                    sfb_src + (static_cast<size_t>(i) * p.kgroups + kt * 4) * 512, nk * 512, fb);
       }
       if (*abort) {
         // Drain: wait (briefly) for the copies of the last stages issued so
         // no bulk copy is still writing shared memory when the CTA exits.
         const uint64_t dl = global_timer_ns() + 100000000ull;  // 100 ms
         const volatile int no_abort = 0;
-        const uint32_t first = issued > STAGES ? issued - STAGES : 0;
-        for (uint32_t kt = first; kt < issued; ++kt)
-          mbar_wait_bounded(bar_full + 8 * (kt % STAGES), (kt / STAGES) & 1u, &no_abort, dl);
+        const uint32_t first = it > STAGES ? it - STAGES : 0;
+        for (uint32_t k = first; k < it; ++k)
+          mbar_wait_bounded(bar_full + 8 * (k % STAGES), (k / STAGES) & 1u, &no_abort, dl);
       }
     }
   } else if (warp == 1) {
     if (lane == 0) {
       // ------------------------------------------------ MMA issuer ------
-      bool any_mma = false;
-      for (uint32_t kt = 0; kt < p.ktiles; ++kt) {
-        const uint32_t s = kt % STAGES, ph = (kt / STAGES) & 1u;
-        if (!mbar_wait_bounded(bar_full + 8 * s, ph, abort, deadline)) {
-          if (!*abort) record_timeout(p, abort, 2);
+      bool any_mma = false, stop = false;
+      uint32_t it = 0, local = 0;
+      for (uint32_t tile = blockIdx.x; tile < p.num_tiles && !stop; tile += gridDim.x, ++local) {
+        // The accumulator this tile writes overlaps the previous tile's
+        // last-drained subtile: wait until the epilogue released it.
+        if (local > 0 && !mbar_wait_bounded(bar_acc_free, (local - 1) & 1u, abort, deadline)) {
+          if (!*abort) record_timeout(p, abort, 4);
           break;
         }
         tc_fence_after();
-        const uint32_t nk = min(4u, p.kgroups - kt * 4);
-        const uint32_t sfa = sbase + OFF_SFA + s * SFA_STAGE;
-        const uint32_t sfb = sbase + OFF_SFB + s * SFB_STAGE;
-        for (uint32_t j = 0; j < nk; ++j) {
-          tmem_copy_scales(tmem + TM_SFA + 4 * j, scale_desc(sfa + 512 * j));
-          tmem_copy_scales(tmem + TM_SFB + 8 * j, scale_desc(sfb + 512 * j));
-          tmem_copy_scales(tmem + TM_SFB + 8 * j + 4, scale_desc(sfb + 2048 + 512 * j));
+        const uint32_t acc = tmem + ((local & 1u) ? TM_ACC1 : 0u);
+        for (uint32_t kt = 0; kt < p.ktiles; ++kt, ++it) {
+          const uint32_t s = it % STAGES, ph = (it / STAGES) & 1u;
+          if (!mbar_wait_bounded(bar_full + 8 * s, ph, abort, deadline)) {
+            if (!*abort) record_timeout(p, abort, 2);
+            stop = true;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t nk = min(4u, p.kgroups - kt * 4);
+          const uint32_t sfa = sbase + OFF_SFA + s * SFA_STAGE;
+          const uint32_t sfb = sbase + OFF_SFB + s * SFB_STAGE;
+          for (uint32_t j = 0; j < nk; ++j) {
+            tmem_copy_scales(tmem + TM_SFA + 4 * j, scale_desc(sfa + 512 * j));
+            tmem_copy_scales(tmem + TM_SFB + 8 * j, scale_desc(sfb + 512 * j));
+            tmem_copy_scales(tmem + TM_SFB + 8 * j + 4, scale_desc(sfb + 2048 + 512 * j));
+          }
+          const uint32_t sa = sbase + OFF_A + s * A_STAGE;
+          const uint32_t sb = sbase + OFF_B + s * B_STAGE;
+          for (uint32_t j = 0; j < nk; ++j) {
+            mma_nvf4(acc, operand_desc(sa + 32 * j), operand_desc(sb + 32 * j),
+                     tmem + TM_SFA + 4 * j, tmem + TM_SFB + 8 * j, (kt | j) != 0);
+          }
+          any_mma = true;
+          tc_commit(bar_empty + 8 * s);
         }
-        const uint32_t sa = sbase + OFF_A + s * A_STAGE;
-        const uint32_t sb = sbase + OFF_B + s * B_STAGE;
-        for (uint32_t j = 0; j < nk; ++j) {
-          mma_nvf4(tmem + TM_ACC, operand_desc(sa + 32 * j), operand_desc(sb + 32 * j),
-                   tmem + TM_SFA + 4 * j, tmem + TM_SFB + 8 * j, (kt | j) != 0);
-        }
-        any_mma = true;
-        tc_commit(bar_empty + 8 * s);
+        if (!stop) tc_commit(bar_acc_full);
       }
-      if (!*abort) {
-        tc_commit(bar_acc);
-      } else if (any_mma) {
+      if (*abort && any_mma) {
         // Drain the MMAs already issued before TMEM is released.
         const volatile int no_abort = 0;
         tc_commit(bar_drain);
@@ -251,38 +282,55 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // -------------------------------------------------- epilogue --------
     const int quad = warp & 3;  // warps 2,3,4,5 -> TMEM lanes 64,96,0,32
-    const int row = m0 + quad * 32 + lane;
-    bool ok = mbar_wait_bounded(bar_acc, 0, abort, deadline);
-    ok = __all_sync(0xffffffffu, ok);
-    if (!ok) {
-      if (lane == 0 && !*abort) record_timeout(p, abort, 3);
-    } else {
+    const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
+    const float ab = __fmul_rn(__ldg(p.a_global), __ldg(p.b_global));
+    uint32_t local = 0;
+    for (uint32_t tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++local) {
+      bool ok = mbar_wait_bounded(bar_acc_full, local & 1u, abort, deadline);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) {
+        if (lane == 0 && !*abort) record_timeout(p, abort, 3);
+        break;
+      }
       tc_fence_after();
-      const float ab = __fmul_rn(__ldg(p.a_global), __ldg(p.b_global));
-      for (int c = 0; c < BN; c += 32) {
-        uint32_t r[32];
-        tmem_ld32(tmem + (static_cast<uint32_t>(quad * 32) << 16) + TM_ACC + c, r);
-        const int col0 = n0 + c;
+      const int m0 = static_cast<int>(tile / p.n_tiles) * BM;
+      const int n0 = static_cast<int>(tile % p.n_tiles) * BN;
+      const int row = m0 + quad * 32 + lane;
+      const bool odd = (local & 1u) != 0;
+      const uint32_t acc = tmem + lane_base + (odd ? TM_ACC1 : 0u);
+      // Buffer 0 is drained from its last subtile down, buffer 1 from its
+      // first subtile up: either way the shared columns 192..255 go first.
+      for (int q = 0; q < 4; ++q) {
+        const int sub = odd ? q : 3 - q;
+        uint32_t r[64];
+        tmem_ld32(acc + sub * EPI_N, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+        tmem_ld32(acc + sub * EPI_N + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
+        if (q == 0) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar_acc_free);
+        }
+        const int col0 = n0 + sub * static_cast<int>(EPI_N);
         if (row >= p.M || col0 >= p.N) continue;
-        const bool full = p.vec_store && col0 + 32 <= p.N;
+        const bool full = p.vec_store && col0 + static_cast<int>(EPI_N) <= p.N;
         if (p.out_fp32) {
           float* dst = static_cast<float*>(p.y) + static_cast<int64_t>(row) * p.ldy + col0;
           if (full) {
 #pragma unroll
-            for (int i = 0; i < 32; i += 4)
+            for (int i = 0; i < 64; i += 4)
               *reinterpret_cast<float4*>(dst + i) =
                   make_float4(__uint_as_float(r[i]) * ab, __uint_as_float(r[i + 1]) * ab,
                               __uint_as_float(r[i + 2]) * ab, __uint_as_float(r[i + 3]) * ab);
           } else {
 #pragma unroll
-            for (int i = 0; i < 32; ++i)
+            for (int i = 0; i < 64; ++i)
               if (col0 + i < p.N) dst[i] = __uint_as_float(r[i]) * ab;
           }
         } else {
           __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(p.y) + static_cast<int64_t>(row) * p.ldy + col0;
           if (full) {
 #pragma unroll
-            for (int i = 0; i < 32; i += 8) {
+            for (int i = 0; i < 64; i += 8) {
               uint4 v;
               v.x = pack_bf16x2(__uint_as_float(r[i]) * ab, __uint_as_float(r[i + 1]) * ab);
               v.y = pack_bf16x2(__uint_as_float(r[i + 2]) * ab, __uint_as_float(r[i + 3]) * ab);
@@ -292,7 +340,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           } else {
 #pragma unroll
-            for (int i = 0; i < 32; ++i)
+            for (int i = 0; i < 64; ++i)
               if (col0 + i < p.N) dst[i] = __float2bfloat16_rn(__uint_as_float(r[i]) * ab);
           }
         }
@@ -416,12 +464,15 @@ nvfp4_status nvfp4_gemm(const void* a_codes, const void* a_scales, const float* 
   p.kgroups = static_cast<uint32_t>(K / 64);
   p.ktiles = static_cast<uint32_t>((K + 255) / 256);
   p.n_rowblocks = static_cast<uint32_t>((N + 127) / 128);
+  p.n_tiles = static_cast<uint32_t>((N + BN - 1) / BN);
+  const int64_t num_tiles = ((M + BM - 1) / BM) * static_cast<int64_t>(p.n_tiles);
+  if (num_tiles > 0x7FFFFFFFll) return set_error(NVFP4_ERR_INVALID_ARG, "nvfp4_gemm: too many tiles");
+  p.num_tiles = static_cast<uint32_t>(num_tiles);
   p.out_fp32 = out_dtype == NVFP4_OUT_FP32;
   p.vec_store = aligned16(y) && ((ldy * (p.out_fp32 ? 4 : 2)) % 16 == 0);
   p.timeout_ns = g_timeout_ns;
   p.debug_flags = g_debug_flags;
-  dim3 grid(static_cast<unsigned>((N + BN - 1) / BN), static_cast<unsigned>((M + BM - 1) / BM));
-  if (grid.y > 65535u) return set_error(NVFP4_ERR_INVALID_ARG, "nvfp4_gemm: M too large");
+  const unsigned grid = static_cast<unsigned>(std::min<int64_t>(num_tiles, sms));
   gemm_kernel<<<grid, kThreads, SMEM_BYTES, s>>>(ta, tb, p);
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_status(e, "gemm_kernel launch");
