@@ -8,26 +8,37 @@
 // Minima page "심층 분석": per-tensor global scales applied around the fused
 // GEMM).
 //
-// Kernel shape: persistent, one CTA per SM walking 128 x 256 output tiles
-// (tile t, t + gridDim.x, ...), K consumed 256 elements (128 bytes per row)
-// per pipeline stage through a 4-stage shared-memory ring that runs on
-// across tile boundaries.
-//   warp 0       TMA producer: A tile 128x128 B and B tile 256x128 B (128-byte
-//                swizzle, out-of-range rows/columns zero-filled by the tensor
-//                map) plus the matching scale atoms (plain bulk copies: the
-//                atoms of one 128-row block and 4 K-groups are contiguous).
-//   warp 1       allocates TMEM and, from one lane, copies each stage's scale
-//                atoms into TMEM (tcgen05.cp 32x128b.warpx4) and issues four
-//                tcgen05.mma kind::mxf4nvf4 block16 (M=128, N=256, K=64) per
-//                stage; tcgen05.commit frees the stage.
-//   warps 2..5   epilogue: tcgen05.ld 32 lanes x 64 columns at a time,
-//                multiply by alpha_A*alpha_B, convert, store.
-// TMEM (512 columns): two accumulators that share one 64-column subtile,
-// buffer 0 = columns 0..255 and buffer 1 = columns 192..447, scales at
-// 448..511.  The epilogue drains the shared subtile (columns 192..255) first
-// and then lets the next tile's MMAs start, so storing tile i overlaps the
-// mainloop of tile i+1 although two full 256-column accumulators would not
-// fit next to the scales.
+// Kernel shape: persistent CTA pairs (clusters of 2 on neighbouring SMs), each
+// pair walking 256 x 256 output tiles (tile t, t + pairs, ...).  The pair
+// issues one tcgen05.mma.cta_group::2 (M=256, N=256, K=64) per K step: CTA r
+// holds rows [128r, 128r+128) of the A tile and the same half of the B tile
+// in its shared memory, and the accumulator rows [128r, 128r+128) x 256 in
+// its TMEM, so every operand byte crosses each SM's shared memory once.
+// K is consumed 256 elements (128 bytes per row) per stage through a 5-stage
+// ring that runs on across tile boundaries.
+//   warp 0      TMA producer (both CTAs): A half 128x128 B and B half 128x128 B
+//               (128-byte swizzle) plus the K step's scale atoms (3-D tensor
+//               maps over the swizzled scale buffers: this CTA's 128-row A
+//               atoms, both 128-row B atoms); all of them complete on the
+//               leader CTA's stage barrier.  Out-of-range rows, columns and
+//               K groups are zero-filled by the tensor maps.
+//   warp 1      TMEM allocation (pair) and, in the leader CTA only, the MMA
+//               issuer: per K step one tcgen05.cp.cta_group::2 of the A scale
+//               atom and two of the B atoms into TMEM (replicated over the
+//               four 32-lane subpartitions), then the MMA; commits free the
+//               stage in both CTAs and finally the accumulator.  The whole
+//               warp runs the loop converged and one elected lane issues each
+//               tcgen05 instruction (issuing them from a lone lane of a
+//               diverged warp is several times slower).
+//   warps 2..5  epilogue (both CTAs): tcgen05.ld 32 lanes x 64 columns,
+//               multiply by alpha_A*alpha_B, convert, store.
+// TMEM (512 columns per CTA): two accumulators that share two 64-column
+// subtiles, buffer 0 = columns 0..255 and buffer 1 = columns 128..383, and
+// one stage of scales at 384..431 (per K step: 4 columns of A scales, 8 of B
+// scales); the copies and MMAs of one thread execute in order, so a single
+// buffer suffices.  The epilogue loads the shared columns 128..255 first, releases
+// them to the next tile's MMAs at once, and stores the rest of tile i while
+// the mainloop of tile i+1 runs.
 // Every wait is bounded by a deadline on %globaltimer; a wait that runs out
 // records NVFP4_ERR_TIMEOUT in the workspace, raises a CTA-wide abort flag,
 // and every role drains what it has in flight before TMEM is freed.
@@ -42,33 +53,39 @@
 namespace nvfp4 {
 namespace {
 
-constexpr int BM = 128;
-constexpr int BN = 256;
-constexpr int BK_BYTES = 128;  // 256 FP4 elements per row per stage
-constexpr int STAGES = 4;
-constexpr int kThreads = 192;
-constexpr uint32_t A_STAGE = BM * BK_BYTES;    // 16 KB
-constexpr uint32_t B_STAGE = BN * BK_BYTES;    // 32 KB
+constexpr int BM = 256;                 // rows per pair tile (128 per CTA)
+constexpr int BN = 256;                 // columns per pair tile
+constexpr int HALF = 128;               // rows of A and of B held per CTA
+constexpr int BK_BYTES = 128;           // 256 FP4 elements per row per stage
+constexpr int STAGES = 5;
+constexpr int kThreads = 192;                  // 6 warps
+constexpr uint32_t A_STAGE = HALF * BK_BYTES;  // 16 KB
+constexpr uint32_t B_STAGE = HALF * BK_BYTES;  // 16 KB
 constexpr uint32_t SFA_STAGE = 4 * 512;        // 4 atoms (4 K-groups x 128 rows)
 constexpr uint32_t SFB_STAGE = 2 * 4 * 512;    // [row block 0..1][K-group 0..3]
+constexpr uint32_t STAGE_TX = A_STAGE + B_STAGE + SFA_STAGE + SFB_STAGE;  // per CTA
 constexpr uint32_t OFF_A = 0;
 constexpr uint32_t OFF_B = OFF_A + STAGES * A_STAGE;
 constexpr uint32_t OFF_SFA = OFF_B + STAGES * B_STAGE;
 constexpr uint32_t OFF_SFB = OFF_SFA + STAGES * SFA_STAGE;
 constexpr uint32_t OFF_BAR = OFF_SFB + STAGES * SFB_STAGE;
-constexpr uint32_t NUM_BARS = 2 * STAGES + 3;  // full[], empty[], acc_full, acc_free, drain
+// full[], empty[], acc_full, acc_free, drain
+constexpr uint32_t NUM_BARS = 2 * STAGES + 3;
 constexpr uint32_t OFF_MISC = OFF_BAR + NUM_BARS * 8;
 constexpr uint32_t SMEM_BYTES = OFF_MISC + 16 + 1024;  // + alignment slack
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t EPI_N = 64;                    // epilogue subtile (columns)
-constexpr uint32_t TM_ACC1 = 256 - EPI_N;         // buffer 1 starts on buffer 0's last subtile
-constexpr uint32_t TM_SFA = TM_ACC1 + 256;        // 448: 4 columns per K-group x 4
-constexpr uint32_t TM_SFB = TM_SFA + 16;          // 464: 8 columns per K-group x 4
+constexpr uint32_t TM_ACC1 = 256 - 2 * EPI_N;     // buffer 1 starts on buffer 0's last two subtiles
+constexpr uint32_t TM_SF = TM_ACC1 + 256;         // 384: scale ring
+constexpr uint32_t TM_SFA = TM_SF;                // 4 columns per K step
+constexpr uint32_t TM_SFB = TM_SF + 16;           // 8 columns per K step
 static_assert(TM_SFB + 32 <= TMEM_COLS, "scales must fit after the accumulators");
+static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+static_assert(2 * STAGE_TX < (1u << 20), "transaction count range of an mbarrier phase");
 
 // Instruction descriptor, kind::mxf4nvf4: A/B format E2M1 (1) at bits 7-9 and
 // 10-12, K-major A and B, N>>3 at bits 17-22, scale format UE4M3 (0) at bit
-// 23, M>>4 at bits 24-28, dense K = 64.
+// 23, M>>4 at bits 24-28 (M = 256 across the CTA pair), dense K = 64.
 constexpr uint32_t kIdesc = (1u << 7) | (1u << 10) | (uint32_t(BN >> 3) << 17) | (uint32_t(BM >> 4) << 24);
 
 // Shared-memory matrix descriptor for a K-major operand tile written by TMA
@@ -86,23 +103,25 @@ __device__ __forceinline__ uint64_t scale_desc(uint32_t saddr) {
          (static_cast<uint64_t>(1) << 46);
 }
 
-__device__ __forceinline__ void tmem_copy_scales(uint32_t taddr, uint64_t sdesc) {
-  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc)
+// Copies one 128-row scale atom from each CTA's shared memory (same offset)
+// into each CTA's TMEM, replicated over the four 32-lane subpartitions.
+__device__ __forceinline__ void tmem_copy_scales_pair(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc)
                : "memory");
 }
 
-__device__ __forceinline__ void mma_nvf4(uint32_t tacc, uint64_t adesc, uint64_t bdesc,
-                                         uint32_t tsfa, uint32_t tsfb, uint32_t accumulate) {
+__device__ __forceinline__ void mma_nvf4_pair(uint32_t tacc, uint64_t adesc, uint64_t bdesc,
+                                              uint32_t tsfa, uint32_t tsfb, uint32_t accumulate) {
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(
+      "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(
           tacc),
       "l"(adesc), "l"(bdesc), "r"(kIdesc), "r"(accumulate), "r"(tsfa), "r"(tsfb)
       : "memory");
 }
 
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t* r) {
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
       "%12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, "
@@ -113,6 +132,8 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
         "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]),
         "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
       : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_wait_ld() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
@@ -122,8 +143,6 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 }
 
 struct GemmParams {
-  const uint8_t* a_scales;
-  const uint8_t* b_scales;
   const float* a_global;
   const float* b_global;
   void* y;
@@ -132,11 +151,10 @@ struct GemmParams {
   int M, N;
   uint32_t kgroups;       // K / 64
   uint32_t ktiles;        // ceil(K / 256)
-  uint32_t n_rowblocks;   // ceil(N / 128): scale row blocks that exist for B
   uint32_t n_tiles;       // ceil(N / 256)
-  uint32_t num_tiles;     // ceil(M / 128) * n_tiles
+  uint32_t num_tiles;     // ceil(M / 256) * n_tiles
   int out_fp32;
-  int vec_store;          // rows of Y start 16-byte aligned: 32-column vector stores
+  int vec_store;          // rows of Y start 16-byte aligned: vector stores
   uint64_t timeout_ns;
   int debug_flags;        // bit 0: never issue the first stage's copies (timeout test)
 };
@@ -148,8 +166,9 @@ __device__ __forceinline__ void record_timeout(const GemmParams& p, volatile int
   p.ws->status = NVFP4_ERR_TIMEOUT;
 }
 
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                const __grid_constant__ CUtensorMap tmSFA, const __grid_constant__ CUtensorMap tmSFB,
                 const GemmParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -164,14 +183,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   volatile int* abort = reinterpret_cast<volatile int*>(smem + OFF_MISC + 4);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();          // 0 = leader (issues the MMAs)
+  const uint32_t pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(bar_full + 8 * s, 1);
-      mbar_init(bar_empty + 8 * s, 1);
+      mbar_init(bar_full + 8 * s, 1);   // the leader's expect_tx arrival (+ both CTAs' bytes)
+      mbar_init(bar_empty + 8 * s, 1);  // the leader's MMA commit
     }
     mbar_init(bar_acc_full, 1);
-    mbar_init(bar_acc_free, 4);  // one arrive per epilogue warp
+    mbar_init(bar_acc_free, 8);  // one arrive per epilogue warp of both CTAs
     mbar_init(bar_drain, 1);
     *abort = 0;
     fence_barrier_init();
@@ -179,76 +200,95 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0 && lane == 0) {
     prefetch_tensormap(&tmA);
     prefetch_tensormap(&tmB);
+    prefetch_tensormap(&tmSFA);
+    prefetch_tensormap(&tmSFB);
   }
   if (warp == 1) {
-    tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
-    tmem_relinquish();
+    tmem_alloc_pair(smem_u32(tmem_slot), TMEM_COLS);
+    tmem_relinquish_pair();
   }
   tc_fence_before();
-  __syncthreads();
+  cluster_sync_all();  // both CTAs' barriers exist before anyone signals them
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const uint64_t deadline = global_timer_ns() + p.timeout_ns;
 
   if (warp == 0) {
-    if (lane == 0) {
-      // ------------------------------------------------ TMA producer ----
-      uint32_t it = 0;  // global k-tile counter across this CTA's tiles
-      bool stop = false;
-      for (uint32_t tile = blockIdx.x; tile < p.num_tiles && !stop; tile += gridDim.x) {
-        const int m0 = static_cast<int>(tile / p.n_tiles) * BM;
-        const int n0 = static_cast<int>(tile % p.n_tiles) * BN;
-        const uint32_t nb_valid = min(2u, p.n_rowblocks - static_cast<uint32_t>(n0 / 128));
-        const uint8_t* sfa_src = p.a_scales + static_cast<size_t>(m0 / 128) * p.kgroups * 512;
-        const uint8_t* sfb_src = p.b_scales + static_cast<size_t>(n0 / 128) * p.kgroups * 512;
-        for (uint32_t kt = 0; kt < p.ktiles; ++kt, ++it) {
-          const uint32_t s = it % STAGES, ph = (it / STAGES) & 1u;
-          if (it >= STAGES && !mbar_wait_bounded(bar_empty + 8 * s, ph ^ 1u, abort, deadline)) {
-            if (!*abort) record_timeout(p, abort, 1);
-            stop = true;
-            break;
-          }
-          const uint32_t nk = min(4u, p.kgroups - kt * 4);
-          const uint32_t fb = bar_full + 8 * s;
-          mbar_expect_tx(fb, A_STAGE + B_STAGE + nk * 512 * (1 + nb_valid));
-          if ((p.debug_flags & 1) && it == 0) continue;  // test hook: this stage never fills
-          tma_load_2d(sbase + OFF_A + s * A_STAGE, &tmA, fb, static_cast<int32_t>(kt * BK_BYTES), m0);
-          tma_load_2d(sbase + OFF_B + s * B_STAGE, &tmB, fb, static_cast<int32_t>(kt * BK_BYTES), n0);
-          bulk_load(sbase + OFF_SFA + s * SFA_STAGE, sfa_src + static_cast<size_t>(kt) * 4 * 512,
-                    nk * 512, fb);
-          for (uint32_t i = 0; i < nb_valid; ++i)
-            bulk_load(sbase + OFF_SFB + s * SFB_STAGE + i * 2048,
-                      sfb_src + (static_cast<size_t>(i) * p.kgroups + kt * 4) * 512, nk * 512, fb);
+    // -------------------------------------------------- TMA producer ----
+    // The whole warp walks the loop; one elected lane issues.
+    uint32_t it = 0;  // k-step counter across this pair's tiles
+    bool stop = false;
+    for (uint32_t tile = pair; tile < p.num_tiles && !stop; tile += npairs) {
+      const int m0 = static_cast<int>(tile / p.n_tiles) * BM;
+      const int n0 = static_cast<int>(tile % p.n_tiles) * BN;
+      const int a_row = m0 + static_cast<int>(rank) * HALF;
+      const int b_row = n0 + static_cast<int>(rank) * HALF;
+      for (uint32_t kt = 0; kt < p.ktiles; ++kt, ++it) {
+        const uint32_t s = it % STAGES, ph = (it / STAGES) & 1u;
+        if (it >= STAGES &&
+            !__all_sync(0xffffffffu, mbar_wait_bounded(bar_empty + 8 * s, ph ^ 1u, abort, deadline))) {
+          if (lane == 0 && !*abort) record_timeout(p, abort, 1);
+          stop = true;
+          break;
         }
+        if (elect_one()) {
+          const uint32_t fb = map_to_rank(bar_full + 8 * s, 0);  // the leader's stage barrier
+          if (rank == 0) mbar_expect_tx(bar_full + 8 * s, 2 * STAGE_TX);
+          if (!((p.debug_flags & 1) && it == 0)) {  // test hook: the first stage never fills
+            const int32_t kx = static_cast<int32_t>(kt * BK_BYTES);
+            tma_load_2d_pair(sbase + OFF_A + s * A_STAGE, &tmA, fb, kx, a_row);
+            tma_load_2d_pair(sbase + OFF_B + s * B_STAGE, &tmB, fb, kx, b_row);
+            tma_load_3d_pair(sbase + OFF_SFA + s * SFA_STAGE, &tmSFA, fb, 0,
+                             static_cast<int32_t>(kt * 4), a_row / 128);
+            tma_load_3d_pair(sbase + OFF_SFB + s * SFB_STAGE, &tmSFB, fb, 0,
+                             static_cast<int32_t>(kt * 4), n0 / 128);
+          }
+        }
+        __syncwarp();
       }
-      if (*abort) {
-        // Drain: wait (briefly) for the copies of the last stages issued so
-        // no bulk copy is still writing shared memory when the CTA exits.
-        const uint64_t dl = global_timer_ns() + 100000000ull;  // 100 ms
+    }
+    if (*abort && lane == 0) {
+      // Drain: let the copies this CTA issued for its last stages land
+      // before the CTA can exit.  The leader watches its stage barriers
+      // (they complete once both CTAs' bytes arrived); the other CTA, whose
+      // copies complete on the leader's barriers, waits out a 2 ms grace
+      // period instead -- a bulk copy of a few KB lands in microseconds.
+      const uint64_t now = global_timer_ns();
+      if (rank == 0) {
         const volatile int no_abort = 0;
         const uint32_t first = it > STAGES ? it - STAGES : 0;
         for (uint32_t k = first; k < it; ++k)
-          mbar_wait_bounded(bar_full + 8 * (k % STAGES), (k / STAGES) & 1u, &no_abort, dl);
+          mbar_wait_bounded(bar_full + 8 * (k % STAGES), (k / STAGES) & 1u, &no_abort,
+                            now + 100000000ull);
+      } else {
+        while (global_timer_ns() < now + 2000000ull) {
+        }
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
+    if (rank == 0) {
       // ------------------------------------------------ MMA issuer ------
+      // The whole warp walks the loop; one elected lane issues.
+      const uint32_t own_empty = map_to_rank(bar_empty, 0);
+      const uint32_t peer_empty = map_to_rank(bar_empty, 1);
+      const uint32_t acc_full_0 = map_to_rank(bar_acc_full, 0);
+      const uint32_t acc_full_1 = map_to_rank(bar_acc_full, 1);
       bool any_mma = false, stop = false;
       uint32_t it = 0, local = 0;
-      for (uint32_t tile = blockIdx.x; tile < p.num_tiles && !stop; tile += gridDim.x, ++local) {
+      for (uint32_t tile = pair; tile < p.num_tiles && !stop; tile += npairs, ++local) {
         // The accumulator this tile writes overlaps the previous tile's
-        // last-drained subtile: wait until the epilogue released it.
-        if (local > 0 && !mbar_wait_bounded(bar_acc_free, (local - 1) & 1u, abort, deadline)) {
-          if (!*abort) record_timeout(p, abort, 4);
+        // first-drained subtiles: wait until both CTAs' epilogues released them.
+        if (local > 0 &&
+            !__all_sync(0xffffffffu, mbar_wait_bounded(bar_acc_free, (local - 1) & 1u, abort, deadline))) {
+          if (lane == 0 && !*abort) record_timeout(p, abort, 4);
           break;
         }
         tc_fence_after();
         const uint32_t acc = tmem + ((local & 1u) ? TM_ACC1 : 0u);
         for (uint32_t kt = 0; kt < p.ktiles; ++kt, ++it) {
           const uint32_t s = it % STAGES, ph = (it / STAGES) & 1u;
-          if (!mbar_wait_bounded(bar_full + 8 * s, ph, abort, deadline)) {
-            if (!*abort) record_timeout(p, abort, 2);
+          if (!__all_sync(0xffffffffu, mbar_wait_bounded(bar_full + 8 * s, ph, abort, deadline))) {
+            if (lane == 0 && !*abort) record_timeout(p, abort, 2);
             stop = true;
             break;
           }
@@ -256,36 +296,46 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t nk = min(4u, p.kgroups - kt * 4);
           const uint32_t sfa = sbase + OFF_SFA + s * SFA_STAGE;
           const uint32_t sfb = sbase + OFF_SFB + s * SFB_STAGE;
-          for (uint32_t j = 0; j < nk; ++j) {
-            tmem_copy_scales(tmem + TM_SFA + 4 * j, scale_desc(sfa + 512 * j));
-            tmem_copy_scales(tmem + TM_SFB + 8 * j, scale_desc(sfb + 512 * j));
-            tmem_copy_scales(tmem + TM_SFB + 8 * j + 4, scale_desc(sfb + 2048 + 512 * j));
-          }
           const uint32_t sa = sbase + OFF_A + s * A_STAGE;
           const uint32_t sb = sbase + OFF_B + s * B_STAGE;
-          for (uint32_t j = 0; j < nk; ++j) {
-            mma_nvf4(acc, operand_desc(sa + 32 * j), operand_desc(sb + 32 * j),
-                     tmem + TM_SFA + 4 * j, tmem + TM_SFB + 8 * j, (kt | j) != 0);
+          if (elect_one()) {
+            for (uint32_t j = 0; j < nk; ++j) {
+              tmem_copy_scales_pair(tmem + TM_SFA + 4 * j, scale_desc(sfa + 512 * j));
+              tmem_copy_scales_pair(tmem + TM_SFB + 8 * j, scale_desc(sfb + 512 * j));
+              tmem_copy_scales_pair(tmem + TM_SFB + 8 * j + 4, scale_desc(sfb + 2048 + 512 * j));
+            }
+            for (uint32_t j = 0; j < nk; ++j)
+              mma_nvf4_pair(acc, operand_desc(sa + 32 * j), operand_desc(sb + 32 * j),
+                            tmem + TM_SFA + 4 * j, tmem + TM_SFB + 8 * j, (kt | j) != 0);
+            tc_commit_pair(own_empty + 8 * s);
+            tc_commit_pair(peer_empty + 8 * s);
           }
+          __syncwarp();
           any_mma = true;
-          tc_commit(bar_empty + 8 * s);
         }
-        if (!stop) tc_commit(bar_acc_full);
+        if (!stop && elect_one()) {
+          tc_commit_pair(acc_full_0);
+          tc_commit_pair(acc_full_1);
+        }
+        __syncwarp();
       }
-      if (*abort && any_mma) {
+      const bool drain = __shfl_sync(0xffffffffu, (*abort && any_mma) ? 1 : 0, 0) != 0;
+      if (drain && elect_one()) {
         // Drain the MMAs already issued before TMEM is released.
         const volatile int no_abort = 0;
-        tc_commit(bar_drain);
+        tc_commit_pair(map_to_rank(bar_drain, 0));
         mbar_wait_bounded(bar_drain, 0, &no_abort, global_timer_ns() + 100000000ull);
       }
+      __syncwarp();
     }
   } else {
     // -------------------------------------------------- epilogue --------
     const int quad = warp & 3;  // warps 2,3,4,5 -> TMEM lanes 64,96,0,32
     const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
+    const uint32_t acc_free_leader = map_to_rank(bar_acc_free, 0);
     const float ab = __fmul_rn(__ldg(p.a_global), __ldg(p.b_global));
     uint32_t local = 0;
-    for (uint32_t tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++local) {
+    for (uint32_t tile = pair; tile < p.num_tiles; tile += npairs, ++local) {
       bool ok = mbar_wait_bounded(bar_acc_full, local & 1u, abort, deadline);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) {
@@ -295,42 +345,46 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const int m0 = static_cast<int>(tile / p.n_tiles) * BM;
       const int n0 = static_cast<int>(tile % p.n_tiles) * BN;
-      const int row = m0 + quad * 32 + lane;
+      const int row = m0 + static_cast<int>(rank) * HALF + quad * 32 + lane;
       const bool odd = (local & 1u) != 0;
       const uint32_t acc = tmem + lane_base + (odd ? TM_ACC1 : 0u);
-      // Buffer 0 is drained from its last subtile down, buffer 1 from its
-      // first subtile up: either way the shared columns 192..255 go first.
-      for (int q = 0; q < 4; ++q) {
-        const int sub = odd ? q : 3 - q;
-        uint32_t r[64];
-        tmem_ld32(acc + sub * EPI_N, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
-        tmem_ld32(acc + sub * EPI_N + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
-        if (q == 0) {
+      // Buffer 0 is drained from its last subtiles down, buffer 1 from its
+      // first subtiles up: either way the shared columns 128..255 go first,
+      // loaded together and released before anything is stored.
+      for (int half = 0; half < 2; ++half) {
+        const int sub0 = odd ? 2 * half : 2 - 2 * half;  // first of the two subtiles
+        uint32_t r[128];
+        tmem_ld32(acc + sub0 * EPI_N, r);
+        tmem_ld32(acc + sub0 * EPI_N + 32, r + 32);
+        tmem_ld32(acc + sub0 * EPI_N + 64, r + 64);
+        tmem_ld32(acc + sub0 * EPI_N + 96, r + 96);
+        tmem_wait_ld();
+        if (half == 0) {
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(bar_acc_free);
+          if (lane == 0) mbar_arrive_cluster(acc_free_leader);
         }
-        const int col0 = n0 + sub * static_cast<int>(EPI_N);
+        const int col0 = n0 + sub0 * static_cast<int>(EPI_N);
         if (row >= p.M || col0 >= p.N) continue;
-        const bool full = p.vec_store && col0 + static_cast<int>(EPI_N) <= p.N;
+        const bool full = p.vec_store && col0 + 2 * static_cast<int>(EPI_N) <= p.N;
         if (p.out_fp32) {
           float* dst = static_cast<float*>(p.y) + static_cast<int64_t>(row) * p.ldy + col0;
           if (full) {
 #pragma unroll
-            for (int i = 0; i < 64; i += 4)
+            for (int i = 0; i < 128; i += 4)
               *reinterpret_cast<float4*>(dst + i) =
                   make_float4(__uint_as_float(r[i]) * ab, __uint_as_float(r[i + 1]) * ab,
                               __uint_as_float(r[i + 2]) * ab, __uint_as_float(r[i + 3]) * ab);
           } else {
 #pragma unroll
-            for (int i = 0; i < 64; ++i)
+            for (int i = 0; i < 128; ++i)
               if (col0 + i < p.N) dst[i] = __uint_as_float(r[i]) * ab;
           }
         } else {
           __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(p.y) + static_cast<int64_t>(row) * p.ldy + col0;
           if (full) {
 #pragma unroll
-            for (int i = 0; i < 64; i += 8) {
+            for (int i = 0; i < 128; i += 8) {
               uint4 v;
               v.x = pack_bf16x2(__uint_as_float(r[i]) * ab, __uint_as_float(r[i + 1]) * ab);
               v.y = pack_bf16x2(__uint_as_float(r[i + 2]) * ab, __uint_as_float(r[i + 3]) * ab);
@@ -340,7 +394,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           } else {
 #pragma unroll
-            for (int i = 0; i < 64; ++i)
+            for (int i = 0; i < 128; ++i)
               if (col0 + i < p.N) dst[i] = __float2bfloat16_rn(__uint_as_float(r[i]) * ab);
           }
         }
@@ -349,9 +403,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 
   tc_fence_before();
-  __syncthreads();
+  cluster_sync_all();  // no CTA leaves while its pair may still touch its barriers or TMEM
   tc_fence_after();
-  if (warp == 1) tmem_dealloc(tmem, TMEM_COLS);
+  if (warp == 1) tmem_dealloc_pair(tmem, TMEM_COLS);
 }
 
 // ------------------------------------------------------------------ host --
@@ -375,19 +429,38 @@ EncodeTiledFn get_encode_fn() {
   return fn;
 }
 
-// 2D uint8 tensor map over a K-major code matrix [rows, K/2] with a
-// 128-byte x box_rows box and the 128-byte swizzle.
-nvfp4_status make_code_map(CUtensorMap* map, const void* base, int64_t rows, int64_t K, uint32_t box_rows) {
+// 2D uint8 tensor map over a K-major code matrix [rows, K/2]: 128-byte x
+// 128-row boxes with the 128-byte swizzle.
+nvfp4_status make_code_map(CUtensorMap* map, const void* base, int64_t rows, int64_t K) {
   EncodeTiledFn enc = get_encode_fn();
   if (!enc) return set_error(NVFP4_ERR_CUDA, "cuTensorMapEncodeTiled entry point not available");
   const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K / 2), static_cast<cuuint64_t>(rows)};
   const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K / 2)};
-  const cuuint32_t box[2] = {static_cast<cuuint32_t>(BK_BYTES), box_rows};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(BK_BYTES), static_cast<cuuint32_t>(HALF)};
   const cuuint32_t estr[2] = {1, 1};
   CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box,
                    estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (r != CUDA_SUCCESS) return set_error(NVFP4_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  if (r != CUDA_SUCCESS) return set_error(NVFP4_ERR_CUDA, "cuTensorMapEncodeTiled(codes) failed (%d)", (int)r);
+  return NVFP4_OK;
+}
+
+// 3D uint32 tensor map over a swizzled scale buffer seen as
+// [row blocks][K groups][128 words]: one 512-byte atom per (row block, K
+// group); boxes of 4 K groups x `blocks` row blocks, zero-filled past the end.
+nvfp4_status make_scale_map(CUtensorMap* map, const void* base, int64_t rows, int64_t K,
+                            uint32_t blocks) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc) return set_error(NVFP4_ERR_CUDA, "cuTensorMapEncodeTiled entry point not available");
+  const int64_t kgroups = K / 64, rblocks = (rows + 127) / 128;
+  const cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(kgroups), static_cast<cuuint64_t>(rblocks)};
+  const cuuint64_t strides[2] = {512, static_cast<cuuint64_t>(512 * kgroups)};
+  const cuuint32_t box[3] = {128, 4, blocks};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, const_cast<void*>(base), dims, strides, box,
+                   estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return set_error(NVFP4_ERR_CUDA, "cuTensorMapEncodeTiled(scales) failed (%d)", (int)r);
   return NVFP4_OK;
 }
 
@@ -426,7 +499,8 @@ nvfp4_status nvfp4_gemm(const void* a_codes, const void* a_scales, const float* 
     return set_error(NVFP4_ERR_INVALID_ARG, "nvfp4_gemm: unknown out_dtype %d", out_dtype);
   if (!aligned16(a_codes) || !aligned16(b_codes) || !aligned16(a_scales) || !aligned16(b_scales) ||
       (reinterpret_cast<uintptr_t>(y) & (out_dtype == NVFP4_OUT_FP32 ? 3u : 1u)) ||
-      !aligned16(workspace) || (reinterpret_cast<uintptr_t>(a_global) & 3u) ||
+      !aligned16(workspace) ||
+      (reinterpret_cast<uintptr_t>(a_global) & 3u) ||
       (reinterpret_cast<uintptr_t>(b_global) & 3u))
     return set_error(NVFP4_ERR_INVALID_ARG, "nvfp4_gemm: misaligned buffer");
   if (workspace_bytes < nvfp4_gemm_workspace_bytes())
@@ -435,9 +509,11 @@ nvfp4_status nvfp4_gemm(const void* a_codes, const void* a_scales, const float* 
   nvfp4_status st = check_device(&dev, &sms);
   if (st != NVFP4_OK) return st;
 
-  CUtensorMap ta, tb;
-  if ((st = make_code_map(&ta, a_codes, M, K, BM)) != NVFP4_OK) return st;
-  if ((st = make_code_map(&tb, b_codes, N, K, BN)) != NVFP4_OK) return st;
+  CUtensorMap ta, tb, tsa, tsb;
+  if ((st = make_code_map(&ta, a_codes, M, K)) != NVFP4_OK) return st;
+  if ((st = make_code_map(&tb, b_codes, N, K)) != NVFP4_OK) return st;
+  if ((st = make_scale_map(&tsa, a_scales, M, K, 1)) != NVFP4_OK) return st;
+  if ((st = make_scale_map(&tsb, b_scales, N, K, 2)) != NVFP4_OK) return st;
 
   static std::once_flag attr_once;
   static cudaError_t attr_err = cudaSuccess;
@@ -452,8 +528,6 @@ nvfp4_status nvfp4_gemm(const void* a_codes, const void* a_scales, const float* 
   if (e != cudaSuccess) return cuda_status(e, "cudaMemsetAsync(status)");
 
   GemmParams p;
-  p.a_scales = static_cast<const uint8_t*>(a_scales);
-  p.b_scales = static_cast<const uint8_t*>(b_scales);
   p.a_global = a_global;
   p.b_global = b_global;
   p.y = y;
@@ -463,7 +537,6 @@ nvfp4_status nvfp4_gemm(const void* a_codes, const void* a_scales, const float* 
   p.N = static_cast<int>(N);
   p.kgroups = static_cast<uint32_t>(K / 64);
   p.ktiles = static_cast<uint32_t>((K + 255) / 256);
-  p.n_rowblocks = static_cast<uint32_t>((N + 127) / 128);
   p.n_tiles = static_cast<uint32_t>((N + BN - 1) / BN);
   const int64_t num_tiles = ((M + BM - 1) / BM) * static_cast<int64_t>(p.n_tiles);
   if (num_tiles > 0x7FFFFFFFll) return set_error(NVFP4_ERR_INVALID_ARG, "nvfp4_gemm: too many tiles");
@@ -472,8 +545,9 @@ nvfp4_status nvfp4_gemm(const void* a_codes, const void* a_scales, const float* 
   p.vec_store = aligned16(y) && ((ldy * (p.out_fp32 ? 4 : 2)) % 16 == 0);
   p.timeout_ns = g_timeout_ns;
   p.debug_flags = g_debug_flags;
-  const unsigned grid = static_cast<unsigned>(std::min<int64_t>(num_tiles, sms));
-  gemm_kernel<<<grid, kThreads, SMEM_BYTES, s>>>(ta, tb, p);
+  // one CTA pair per two SMs, never more pairs than tiles
+  const int64_t pairs = std::max<int64_t>(1, std::min<int64_t>(num_tiles, sms / 2));
+  gemm_kernel<<<static_cast<unsigned>(2 * pairs), kThreads, SMEM_BYTES, s>>>(ta, tb, tsa, tsb, p);
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_status(e, "gemm_kernel launch");
   return NVFP4_OK;
