@@ -190,6 +190,31 @@ def run_ours(args, world, rank, local):
     tq6, tg6 = timed(q6, "six", "max", 448.0, args.steps)
     assert nv.device_status(qx.workspace) == nv.OK and nv.device_status(gws) == nv.OK
 
+    # the quantize kernel alone: alpha supplied (static), no amax pass
+    qs = nv.quantize(x, xm, xr, xF)
+    qs6 = nv.quantize(x, "six", "max", 448.0)
+
+    def time_op(fn, steps):
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(steps)]
+        for i in range(steps):
+            flush.fill_(i & 0xFF)
+            evs[i][0].record(stream)
+            fn()
+            evs[i][1].record(stream)
+        torch.cuda.synchronize()
+        return statistics.mean(a.elapsed_time(b) for a, b in evs)
+
+    _barrier(world)
+    torch.cuda.synchronize()
+    ms_qstatic = time_op(lambda: nv.quantize(x, xm, xr, out=qs, global_scale=qx.global_scale),
+                         args.steps)
+    ms_qstatic6 = time_op(lambda: nv.quantize(x, "six", "max", out=qs6, global_scale=q6.global_scale),
+                          args.steps)
+    assert nv.device_status(qs.workspace) == nv.OK and nv.device_status(qs6.workspace) == nv.OK
+    ms_qstatic = _max_over_ranks(world, ms_qstatic, device)
+    ms_qstatic6 = _max_over_ranks(world, ms_qstatic6, device)
+
     ms_step = _max_over_ranks(world, statistics.mean(a + b for a, b in zip(tq, tg)), device)
     ms_quant = _max_over_ranks(world, statistics.mean(tq), device)
     ms_gemm = _max_over_ranks(world, statistics.mean(tg), device)
@@ -253,6 +278,12 @@ def run_ours(args, world, rank, local):
             "overhead_46_vs_six": round(ms_quant / ms_quant6 - 1.0, 4),
             "quantize_end_to_end_GBps": round(quant_gbs, 1),
             "quantize_frac_hbm": round(quant_gbs / peaks["hbm"], 4),
+            "ms_quantize_kernel_46_static_alpha": round(ms_qstatic, 4),
+            "ms_quantize_kernel_six_static_alpha": round(ms_qstatic6, 4),
+            "quantize_kernel_46_GBps": round(QUANT_BYTES_PER_ELEM * M * K / (ms_qstatic * 1e-3) / 1e9, 1),
+            "quantize_kernel_46_frac_hbm": round(
+                QUANT_BYTES_PER_ELEM * M * K / (ms_qstatic * 1e-3) / 1e9 / peaks["hbm"], 4),
+            "overhead_46_vs_six_kernel": round(ms_qstatic / ms_qstatic6 - 1.0, 4),
             "hbm_peak_GBps": peaks["hbm"],
             "ms_gemm": round(ms_gemm, 4),
             "gemm_TFLOPs": round(gemm_tflops, 1),

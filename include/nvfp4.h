@@ -57,8 +57,8 @@
  *
  * Errors: every call validates its arguments on the host and returns a status
  * without launching anything when they are invalid.  Conditions only the GPU
- * can see (non-finite input to nvfp4_quantize, a bounded wait that ran out in
- * nvfp4_gemm) are written to a status word in the call's workspace and read
+ * can see (non-finite input to nvfp4_quantize, a static alpha that is not a
+ * positive finite number, a bounded wait that ran out in nvfp4_gemm) are written to a status word in the call's workspace and read
  * by nvfp4_get_device_status.  Launch failures return NVFP4_ERR_CUDA with
  * the CUDA message available from nvfp4_last_error_message.
  *
@@ -129,6 +129,25 @@ NVFP4_API nvfp4_status nvfp4_quantize(const void* x, int64_t rows, int64_t K, in
                             float* global_scale, void* workspace, size_t workspace_bytes,
                             void* stream);
 
+/* nvfp4_quantize with a caller-supplied tensor scale: alpha is read from
+ * *global_scale (device memory; e.g. calibrated offline, or a previous call's
+ * output), the tensor-amax pass and its read of x are skipped, and every
+ * block is quantized against that alpha (block scales saturate at 448 and
+ * codes at 6 where alpha is smaller than amax / (fp8_max * 6)).  Source: the
+ * Minima page, "심층 분석" (calibrated module-level scales) -- the quantity is
+ * the same alpha the "Four Over Six (4/6)" summary defines in "구현 세부 사항".
+ * Same arguments, requirements and outputs as nvfp4_quantize except that
+ * fp8_max is not needed and *global_scale is read, not written; the workspace
+ * needs only nvfp4_gemm_workspace_bytes() bytes (the status word).  Device
+ * status: NVFP4_ERR_INVALID_ARG when alpha is not a positive finite number
+ * (nothing written), NVFP4_ERR_NONFINITE when a block holds Inf or NaN (that
+ * block's codes and scale are written as zeros).  One 8-byte memset of the
+ * status word, then one kernel launch. */
+NVFP4_API nvfp4_status nvfp4_quantize_with_scale(const void* x, int64_t rows, int64_t K, int64_t ldx,
+                                                 int mode, int rule, const float* global_scale,
+                                                 void* codes, void* scales, void* workspace,
+                                                 size_t workspace_bytes, void* stream);
+
 /* nvfp4_quantize without a workspace, for callers that cannot allocate device
  * memory where they quantize: a custom-op or plugin hook inside another
  * inference runtime that owns every device allocation and passes the op only
@@ -165,8 +184,32 @@ NVFP4_API nvfp4_status nvfp4_gemm(const void* a_codes, const void* a_scales, con
                         int64_t M, int64_t N, int64_t K, void* y, int64_t ldy, int out_dtype,
                         void* workspace, size_t workspace_bytes, void* stream);
 
+/* nvfp4_gemm with one B global scale per output-column segment, for one GEMM
+ * over several weights fused along N (e.g. the Q, K and V projections, or
+ * gate and up), each quantized with its own tensor scale -- for instance
+ * module-level calibrated scales.  Column n of Y belongs to the segment s with
+ * seg_ends[s-1] <= n < seg_ends[s] (seg_ends[-1] = 0) and is scaled by
+ * alpha_A * b_globals[s].  Source: the Minima page, "심층 분석" (the global
+ * scale mismatch met when module-level calibrated checkpoints are fused into
+ * one GEMM kernel).
+ *   b_globals  device array of nseg floats
+ *   seg_ends   host array of nseg exclusive end columns, strictly ascending,
+ *              each a multiple of 64 except the last, which must equal N
+ *   nseg       1 .. 16
+ * Everything else as nvfp4_gemm (B's codes and scales are the fused [N, K]
+ * operand; when its segments are quantized separately with nvfp4_quantize
+ * into one buffer, their row counts must be multiples of 128 so their scale
+ * atoms do not overlap).  nseg == 1 with seg_ends = {N} is nvfp4_gemm. */
+NVFP4_API nvfp4_status nvfp4_gemm_segmented(const void* a_codes, const void* a_scales,
+                                            const float* a_global, const void* b_codes,
+                                            const void* b_scales, const float* b_globals,
+                                            const int64_t* seg_ends, int nseg, int64_t M, int64_t N,
+                                            int64_t K, void* y, int64_t ldy, int out_dtype,
+                                            void* workspace, size_t workspace_bytes, void* stream);
+
 /* Synchronizes `stream`, then returns the status word the last call that used
- * `workspace` wrote (NVFP4_OK, NVFP4_ERR_NONFINITE or NVFP4_ERR_TIMEOUT), or
+ * `workspace` wrote (NVFP4_OK, NVFP4_ERR_INVALID_ARG, NVFP4_ERR_NONFINITE or
+ * NVFP4_ERR_TIMEOUT), or
  * NVFP4_ERR_CUDA if the synchronization or the read failed. */
 NVFP4_API nvfp4_status nvfp4_get_device_status(const void* workspace, void* stream);
 

@@ -91,3 +91,43 @@ def assert_gemm_close(y: np.ndarray, ref: np.ndarray, guard: np.ndarray, bf16: b
     with np.errstate(divide="ignore", invalid="ignore"):
         r = np.where(big, err / np.abs(ref), 0.0)
     return float(r.max()) if r.size else 0.0
+
+
+def hard_block_maxima(alpha: float, Q: float, limit: int = 512) -> np.ndarray:
+    """bf16 block maxima b (as float32) for which b * fl(1/(alpha*Q)) and the
+    correctly rounded quotient b / (alpha*Q) round to different E4M3 scales,
+    plus those whose quotient sits within two units of an E4M3 rounding
+    midpoint: the blocks on which a reciprocal-multiply shortcut for the scale
+    quotient would go wrong."""
+    bits = np.arange(1, 0x7F80, dtype=np.uint32)          # positive finite bf16
+    b = (bits << 16).view(np.float32)
+    a = np.float32(alpha) * np.float32(Q)
+    with np.errstate(over="ignore", divide="ignore", invalid="ignore"):
+        q_true = b / a
+        q_fast = b * (np.float32(1.0) / a)
+    low20 = q_true.view(np.uint32) & np.uint32(0xFFFFF)
+    near_mid = np.abs(low20.astype(np.int64) - 0x80000) <= 2
+    cand = np.nonzero((q_true != q_fast) | near_mid)[0]
+    hard = [i for i in cand
+            if near_mid[i] or oracle.e4m3_encode(float(q_true[i])) != oracle.e4m3_encode(float(q_fast[i]))]
+    return b[np.array(hard[:limit], dtype=np.int64)] if hard else np.zeros(0, np.float32)
+
+
+def blocks_with_maxima(maxima: np.ndarray, K: int, seed: int) -> torch.Tensor:
+    """A bf16 [rows, K] tensor, one 16-element block per entry of `maxima`
+    (row-major over blocks), whose block max |x| is exactly that value: one
+    element is +-max, the rest uniform in (-max, max) and rounded toward zero
+    so they stay below it."""
+    g = np.random.default_rng(seed)
+    nb = len(maxima)
+    per_row = K // 16
+    rows = (nb + per_row - 1) // per_row
+    blocks = np.zeros((rows * per_row, 16), np.float32)
+    m = np.asarray(maxima, np.float32)
+    blocks[:nb] = (g.uniform(-1, 1, (nb, 16)) * m[:, None]).astype(np.float32)
+    # truncate to bf16 (toward zero) so |x| <= max keeps holding
+    blocks = (blocks.view(np.uint32) & np.uint32(0xFFFF0000)).view(np.float32)
+    pos = g.integers(0, 16, nb)
+    sign = np.where(g.random(nb) < 0.5, -1.0, 1.0).astype(np.float32)
+    blocks[np.arange(nb), pos] = sign * m
+    return torch.from_numpy(blocks.reshape(rows, K).copy()).to(torch.bfloat16)

@@ -73,6 +73,23 @@ def test_quantize_rejects_bad_arguments(bad):
     assert nv.last_error_message()
 
 
+def _qs(**kw):
+    args = dict(x=FAKE, rows=64, K=512, ldx=512, mode=1, rule=2, global_scale=FAKE, codes=FAKE,
+                scales=FAKE, workspace=FAKE, workspace_bytes=64, stream=None)
+    args.update(kw)
+    return nv.nvfp4_quantize_with_scale(*args.values())
+
+
+@pytest.mark.parametrize("bad", [
+    dict(x=None), dict(codes=None), dict(scales=None), dict(global_scale=None), dict(workspace=None),
+    dict(rows=0), dict(K=48), dict(ldx=256), dict(ldx=516), dict(mode=2), dict(rule=3),
+    dict(x=FAKE + 8), dict(scales=FAKE + 4), dict(global_scale=FAKE + 2), dict(workspace_bytes=16),
+])
+def test_quantize_with_scale_rejects_bad_arguments(bad):
+    assert _qs(**bad) == nv.ERR_INVALID_ARG
+    assert nv.last_error_message()
+
+
 def _g(**kw):
     args = dict(a_codes=FAKE, a_scales=FAKE, a_global=FAKE, b_codes=FAKE, b_scales=FAKE,
                 b_global=FAKE, M=64, N=256, K=512, y=FAKE, ldy=256, out_dtype=0, workspace=FAKE,
@@ -90,6 +107,27 @@ def test_gemm_rejects_bad_arguments(bad):
     assert _g(**bad) == nv.ERR_INVALID_ARG
 
 
+def _gs(ends=(256,), nseg=None, **kw):
+    import ctypes as C
+    arr = (C.c_int64 * max(1, len(ends)))(*ends)
+    args = dict(a_codes=FAKE, a_scales=FAKE, a_global=FAKE, b_codes=FAKE, b_scales=FAKE,
+                b_globals=FAKE, seg_ends=C.addressof(arr), nseg=len(ends) if nseg is None else nseg,
+                M=64, N=256, K=512, y=FAKE, ldy=256, out_dtype=0, workspace=FAKE,
+                workspace_bytes=64, stream=None)
+    args.update(kw)
+    return nv.nvfp4_gemm_segmented(*args.values())
+
+
+@pytest.mark.parametrize("ends,nseg,kw", [
+    ((256,), 0, {}), (tuple(range(64, 64 * 18, 64)), None, dict(N=64 * 17, ldy=64 * 17)), ((128, 100), None, {}),
+    ((100, 256), None, {}), ((128, 128, 256), None, {}), ((192, 128), None, {}), ((128,), None, {}),
+    ((256,), None, dict(seg_ends=None)), ((256,), None, dict(b_globals=None)),
+    ((256,), None, dict(b_globals=FAKE + 2)),
+])
+def test_gemm_segmented_rejects_bad_arguments(ends, nseg, kw):
+    assert _gs(ends, nseg, **kw) == nv.ERR_INVALID_ARG
+
+
 def test_no_gpu_fails_loudly():
     """Valid arguments without a usable sm_100 device: an error status, never a
     silent fallback."""
@@ -98,4 +136,6 @@ def test_no_gpu_fails_loudly():
     if torch.cuda.is_available():
         pytest.skip("a GPU is present")
     assert _q() in (nv.ERR_CUDA, nv.ERR_UNSUPPORTED_DEVICE)
+    assert _qs() in (nv.ERR_CUDA, nv.ERR_UNSUPPORTED_DEVICE)
+    assert _gs((64, 128, 256)) in (nv.ERR_CUDA, nv.ERR_UNSUPPORTED_DEVICE)
     assert _g() in (nv.ERR_CUDA, nv.ERR_UNSUPPORTED_DEVICE)

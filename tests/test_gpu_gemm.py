@@ -147,3 +147,43 @@ def test_strided_output(ldy_pad):
         got = to_np(big.float())
         assert_gemm_close(got[:, :N], ref, guard, bf16=dt == torch.bfloat16)
         assert (got[:, N:] == 7.0).all()  # nothing written past N
+
+
+# ------------------------------------------- per-segment B global scales --
+
+@pytest.mark.parametrize("M,K,seg_rows", [
+    (200, 512, [128, 64, 192, 80]),            # boundaries inside a 256-column tile and a half
+    (64, 256, [64] * 16),                       # the most segments, 64 columns each
+    (130, 1024, [1024, 640, 320]),              # a fused Q / K / V-like split
+])
+def test_gemm_segmented_matches_oracle(M, K, seg_rows):
+    ac, as_, aa = _quantized(M, K, 5, ("four_over_six", "mse", 256.0))
+    parts = [_quantized(n, K, 40 + i, ("six", "max", 448.0), kind="normal") for i, n in enumerate(seg_rows)]
+    bc = np.concatenate([p[0] for p in parts])
+    bs = np.concatenate([p[1] for p in parts])
+    alphas = np.array([p[2] for p in parts], np.float32)
+    ends = np.cumsum(seg_rows).tolist()
+    A = upload_operand(ac, as_, aa)
+    B = upload_operand(bc, bs, 1.0)
+    bg = torch.from_numpy(alphas).cuda()
+    ws = torch.zeros(nv.nvfp4_gemm_workspace_bytes(), dtype=torch.uint8, device="cuda")
+    refs, guards = [], []
+    for (c, s, a), lo, hi in zip(parts, [0] + ends[:-1], ends):
+        r, g = oracle.gemm_reference(ac, as_, aa, c, s, a)
+        refs.append(r)
+        guards.append(g)
+    ref, guard = np.concatenate(refs, axis=1), np.concatenate(guards, axis=1)
+    for dt, bf16 in ((torch.float32, False), (torch.bfloat16, True)):
+        y = nv.gemm_segmented(A, B, bg, ends, out_dtype=dt, workspace=ws)
+        assert nv.device_status(ws) == nv.OK
+        assert_gemm_close(to_np(y.float()), ref, guard, bf16=bf16)
+
+
+def test_gemm_segmented_one_segment_is_gemm():
+    ac, as_, aa = _quantized(300, 640, 7, ("four_over_six", "mae", 256.0))
+    bc, bs, ba = _quantized(520, 640, 8, ("six", "max", 448.0), kind="normal")
+    A, B = upload_operand(ac, as_, aa), upload_operand(bc, bs, ba)
+    y1 = nv.gemm(A, B, out_dtype=torch.float32)
+    y2 = nv.gemm_segmented(A, B, B.global_scale.clone(), [520], out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    assert torch.equal(y1, y2)

@@ -37,8 +37,12 @@ _SIGNATURES = {
                                       ctypes.c_float, _P, _P, _P, _P, ctypes.c_size_t, _P]),
     "nvfp4_quantize_noalloc": (ctypes.c_int, [_P, _I64, _I64, _I64, ctypes.c_int, ctypes.c_int,
                                               ctypes.c_float, _P, _P, _P, _P]),
+    "nvfp4_quantize_with_scale": (ctypes.c_int, [_P, _I64, _I64, _I64, ctypes.c_int, ctypes.c_int,
+                                                 _P, _P, _P, _P, ctypes.c_size_t, _P]),
     "nvfp4_gemm": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _I64,
                                   ctypes.c_int, _P, ctypes.c_size_t, _P]),
+    "nvfp4_gemm_segmented": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, ctypes.c_int, _I64, _I64,
+                                            _I64, _P, _I64, ctypes.c_int, _P, ctypes.c_size_t, _P]),
     "nvfp4_get_device_status": (ctypes.c_int, [_P, _P]),
     "nvfp4_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "nvfp4_last_error_message": (ctypes.c_char_p, []),
@@ -104,10 +108,27 @@ def nvfp4_quantize_noalloc(x, rows, K, ldx, mode, rule, fp8_max, codes, scales, 
                                          global_scale, stream)
 
 
+def nvfp4_quantize_with_scale(x, rows, K, ldx, mode, rule, global_scale, codes, scales, workspace,
+                              workspace_bytes, stream) -> int:
+    """nvfp4_quantize against a caller-supplied tensor scale read from the
+    device float at ``global_scale`` (no amax pass)."""
+    return load().nvfp4_quantize_with_scale(x, rows, K, ldx, mode, rule, global_scale, codes,
+                                            scales, workspace, workspace_bytes, stream)
+
+
 def nvfp4_gemm(a_codes, a_scales, a_global, b_codes, b_scales, b_global, M, N, K, y, ldy,
                out_dtype, workspace, workspace_bytes, stream) -> int:
     return load().nvfp4_gemm(a_codes, a_scales, a_global, b_codes, b_scales, b_global, M, N, K, y,
                              ldy, out_dtype, workspace, workspace_bytes, stream)
+
+
+def nvfp4_gemm_segmented(a_codes, a_scales, a_global, b_codes, b_scales, b_globals, seg_ends, nseg,
+                         M, N, K, y, ldy, out_dtype, workspace, workspace_bytes, stream) -> int:
+    """nvfp4_gemm with one B global scale per output-column segment;
+    ``seg_ends`` is a host pointer to nseg int64 exclusive end columns."""
+    return load().nvfp4_gemm_segmented(a_codes, a_scales, a_global, b_codes, b_scales, b_globals,
+                                       seg_ends, nseg, M, N, K, y, ldy, out_dtype, workspace,
+                                       workspace_bytes, stream)
 
 
 def nvfp4_get_device_status(workspace, stream) -> int:
@@ -152,14 +173,22 @@ def _check(status: int, what: str) -> None:
 
 
 def quantize(x, mode: str = "six", rule: str = "max", fp8_max: float | None = None,
-             out: NVFP4Tensor | None = None, stream=None) -> NVFP4Tensor:
-    """NVFP4-quantize a CUDA bf16 matrix [rows, K] (K % 64 == 0)."""
+             out: NVFP4Tensor | None = None, stream=None, global_scale=None) -> NVFP4Tensor:
+    """NVFP4-quantize a CUDA bf16 matrix [rows, K] (K % 64 == 0).
+
+    With ``global_scale`` (a float32 CUDA tensor of one element, e.g. a
+    calibrated alpha) the tensor scale is taken from it instead of the
+    tensor's amax; ``fp8_max`` is then unused.
+    """
     import torch
 
     if x.dtype != torch.bfloat16 or x.dim() != 2 or not x.is_cuda:
         raise ValueError("x must be a 2-D bfloat16 CUDA tensor")
     if x.stride(1) != 1:
         raise ValueError("x must have unit stride along K")
+    if global_scale is not None and (global_scale.dtype != torch.float32 or global_scale.numel() != 1
+                                     or global_scale.device != x.device):
+        raise ValueError("global_scale must be a one-element float32 tensor on x's device")
     rows, K = x.shape
     F = DEFAULT_FP8_MAX[mode] if fp8_max is None else float(fp8_max)
     if out is None:
@@ -170,6 +199,14 @@ def quantize(x, mode: str = "six", rule: str = "max", fp8_max: float | None = No
             global_scale=torch.empty(1, dtype=torch.float32, device=dev),
             workspace=torch.empty(nvfp4_quantize_workspace_bytes(rows, K), dtype=torch.uint8, device=dev),
             rows=rows, K=K)
+    if global_scale is not None:
+        out.global_scale.copy_(global_scale.reshape(1))
+        st = nvfp4_quantize_with_scale(x.data_ptr(), rows, K, x.stride(0), MODES[mode], RULES[rule],
+                                       out.global_scale.data_ptr(), out.codes.data_ptr(),
+                                       out.scales.data_ptr(), out.workspace.data_ptr(),
+                                       out.workspace.numel(), _stream_handle(stream))
+        _check(st, "nvfp4_quantize_with_scale")
+        return out
     st = nvfp4_quantize(x.data_ptr(), rows, K, x.stride(0), MODES[mode], RULES[rule], F,
                         out.codes.data_ptr(), out.scales.data_ptr(), out.global_scale.data_ptr(),
                         out.workspace.data_ptr(), out.workspace.numel(), _stream_handle(stream))
@@ -196,6 +233,34 @@ def gemm(a: NVFP4Tensor, b: NVFP4Tensor, out_dtype=None, out=None, workspace=Non
                     out.data_ptr(), out.stride(0), code, workspace.data_ptr(), workspace.numel(),
                     _stream_handle(stream))
     _check(st, "nvfp4_gemm")
+    return out
+
+
+def gemm_segmented(a: NVFP4Tensor, b: NVFP4Tensor, b_globals, seg_ends, out_dtype=None, out=None,
+                   workspace=None, stream=None):
+    """Y = A_hat @ B_hat^T where B is several weights fused along N: columns
+    [seg_ends[s-1], seg_ends[s]) of Y are scaled by alpha_A * b_globals[s]
+    (b_globals: float32 CUDA tensor [nseg]; b.global_scale is not used)."""
+    import torch
+
+    if a.K != b.K:
+        raise ValueError("operands disagree on K")
+    ends = (ctypes.c_int64 * len(seg_ends))(*[int(e) for e in seg_ends])
+    if b_globals.dtype != torch.float32 or b_globals.numel() != len(seg_ends) or not b_globals.is_cuda:
+        raise ValueError("b_globals must be a float32 CUDA tensor with one entry per segment")
+    out_dtype = torch.bfloat16 if out_dtype is None else out_dtype
+    code = {torch.bfloat16: OUT_BF16, torch.float32: OUT_FP32}[out_dtype]
+    M, N, K = a.rows, b.rows, a.K
+    if out is None:
+        out = torch.empty(M, N, dtype=out_dtype, device=a.codes.device)
+    if workspace is None:
+        workspace = torch.empty(nvfp4_gemm_workspace_bytes(), dtype=torch.uint8, device=a.codes.device)
+    st = nvfp4_gemm_segmented(a.codes.data_ptr(), a.scales.data_ptr(), a.global_scale.data_ptr(),
+                              b.codes.data_ptr(), b.scales.data_ptr(), b_globals.data_ptr(),
+                              ctypes.addressof(ends), len(seg_ends), M, N, K, out.data_ptr(),
+                              out.stride(0), code, workspace.data_ptr(), workspace.numel(),
+                              _stream_handle(stream))
+    _check(st, "nvfp4_gemm_segmented")
     return out
 
 

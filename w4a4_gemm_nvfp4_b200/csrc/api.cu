@@ -101,7 +101,7 @@ nvfp4_status nvfp4_get_device_status(const void* workspace, void* stream) {
   e = cudaMemcpy(&h, workspace, sizeof(h), cudaMemcpyDeviceToHost);
   if (e != cudaSuccess) return cuda_status(e, "cudaMemcpy(status)");
   switch (h.status) {
-    case NVFP4_OK: case NVFP4_ERR_NONFINITE: case NVFP4_ERR_TIMEOUT:
+    case NVFP4_OK: case NVFP4_ERR_INVALID_ARG: case NVFP4_ERR_NONFINITE: case NVFP4_ERR_TIMEOUT:
       return static_cast<nvfp4_status>(h.status);
     default:
       return set_error(NVFP4_ERR_CUDA, "workspace status word holds %u (never written?)", h.status);

@@ -142,9 +142,13 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<const uint32_t*>(&v);
 }
 
+constexpr int kMaxSegments = 16;
+
 struct GemmParams {
   const float* a_global;
-  const float* b_global;
+  const float* b_global;  // nseg entries: alpha_B of each output-column segment
+  int nseg;
+  int seg_end[kMaxSegments];  // exclusive end column of each segment; the last is N
   void* y;
   WorkspaceHeader* ws;
   int64_t ldy;
@@ -333,7 +337,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const int quad = warp & 3;  // warps 2,3,4,5 -> TMEM lanes 64,96,0,32
     const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
     const uint32_t acc_free_leader = map_to_rank(bar_acc_free, 0);
-    const float ab = __fmul_rn(__ldg(p.a_global), __ldg(p.b_global));
+    const float alpha_a = __ldg(p.a_global);
+    // alpha_A * alpha_B of the segment holding column `col` (segments are
+    // whole 64-column epilogue subtiles)
+    auto segment_scale = [&](int col) {
+      int sg = 0;
+      while (sg + 1 < p.nseg && col >= p.seg_end[sg]) ++sg;
+      return __fmul_rn(alpha_a, __ldg(p.b_global + sg));
+    };
     uint32_t local = 0;
     for (uint32_t tile = pair; tile < p.num_tiles; tile += npairs, ++local) {
       bool ok = mbar_wait_bounded(bar_acc_full, local & 1u, abort, deadline);
@@ -366,6 +377,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
         const int col0 = n0 + sub0 * static_cast<int>(EPI_N);
         if (row >= p.M || col0 >= p.N) continue;
+        const float ab0 = segment_scale(col0);                                  // r[0..63]
+        const float ab1 = p.nseg == 1 ? ab0 : segment_scale(col0 + static_cast<int>(EPI_N));  // r[64..127]
         const bool full = p.vec_store && col0 + 2 * static_cast<int>(EPI_N) <= p.N;
         if (p.out_fp32) {
           float* dst = static_cast<float*>(p.y) + static_cast<int64_t>(row) * p.ldy + col0;
@@ -373,12 +386,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int i = 0; i < 128; i += 4)
               *reinterpret_cast<float4*>(dst + i) =
-                  make_float4(__uint_as_float(r[i]) * ab, __uint_as_float(r[i + 1]) * ab,
-                              __uint_as_float(r[i + 2]) * ab, __uint_as_float(r[i + 3]) * ab);
+                  make_float4(__uint_as_float(r[i]) * (i < 64 ? ab0 : ab1), __uint_as_float(r[i + 1]) * (i < 64 ? ab0 : ab1),
+                              __uint_as_float(r[i + 2]) * (i < 64 ? ab0 : ab1), __uint_as_float(r[i + 3]) * (i < 64 ? ab0 : ab1));
           } else {
 #pragma unroll
             for (int i = 0; i < 128; ++i)
-              if (col0 + i < p.N) dst[i] = __uint_as_float(r[i]) * ab;
+              if (col0 + i < p.N) dst[i] = __uint_as_float(r[i]) * (i < 64 ? ab0 : ab1);
           }
         } else {
           __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(p.y) + static_cast<int64_t>(row) * p.ldy + col0;
@@ -386,16 +399,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int i = 0; i < 128; i += 8) {
               uint4 v;
-              v.x = pack_bf16x2(__uint_as_float(r[i]) * ab, __uint_as_float(r[i + 1]) * ab);
-              v.y = pack_bf16x2(__uint_as_float(r[i + 2]) * ab, __uint_as_float(r[i + 3]) * ab);
-              v.z = pack_bf16x2(__uint_as_float(r[i + 4]) * ab, __uint_as_float(r[i + 5]) * ab);
-              v.w = pack_bf16x2(__uint_as_float(r[i + 6]) * ab, __uint_as_float(r[i + 7]) * ab);
+              v.x = pack_bf16x2(__uint_as_float(r[i]) * (i < 64 ? ab0 : ab1), __uint_as_float(r[i + 1]) * (i < 64 ? ab0 : ab1));
+              v.y = pack_bf16x2(__uint_as_float(r[i + 2]) * (i < 64 ? ab0 : ab1), __uint_as_float(r[i + 3]) * (i < 64 ? ab0 : ab1));
+              v.z = pack_bf16x2(__uint_as_float(r[i + 4]) * (i < 64 ? ab0 : ab1), __uint_as_float(r[i + 5]) * (i < 64 ? ab0 : ab1));
+              v.w = pack_bf16x2(__uint_as_float(r[i + 6]) * (i < 64 ? ab0 : ab1), __uint_as_float(r[i + 7]) * (i < 64 ? ab0 : ab1));
               *reinterpret_cast<uint4*>(dst + i) = v;
             }
           } else {
 #pragma unroll
             for (int i = 0; i < 128; ++i)
-              if (col0 + i < p.N) dst[i] = __float2bfloat16_rn(__uint_as_float(r[i]) * ab);
+              if (col0 + i < p.N) dst[i] = __float2bfloat16_rn(__uint_as_float(r[i]) * (i < 64 ? ab0 : ab1));
           }
         }
       }
@@ -482,29 +495,41 @@ void nvfp4_testing_set_gemm_wait(uint64_t timeout_ns, int debug_flags) {
   g_debug_flags = debug_flags;
 }
 
-nvfp4_status nvfp4_gemm(const void* a_codes, const void* a_scales, const float* a_global,
-                        const void* b_codes, const void* b_scales, const float* b_global,
-                        int64_t M, int64_t N, int64_t K, void* y, int64_t ldy, int out_dtype,
-                        void* workspace, size_t workspace_bytes, void* stream) {
+}  // extern "C"
+
+namespace {
+
+nvfp4_status gemm_impl(const char* fn, const void* a_codes, const void* a_scales, const float* a_global,
+                       const void* b_codes, const void* b_scales, const float* b_global,
+                       const int64_t* seg_ends, int nseg, int64_t M, int64_t N, int64_t K, void* y,
+                       int64_t ldy, int out_dtype, void* workspace, size_t workspace_bytes,
+                       void* stream) {
   if (!a_codes || !a_scales || !a_global || !b_codes || !b_scales || !b_global || !y || !workspace)
-    return set_error(NVFP4_ERR_INVALID_ARG, "nvfp4_gemm: null pointer argument");
+    return set_error(NVFP4_ERR_INVALID_ARG, "%s: null pointer argument", fn);
   if (M < 1 || N < 1 || K < 64 || K % 64 != 0)
-    return set_error(NVFP4_ERR_INVALID_ARG,
-                     "nvfp4_gemm: need M, N >= 1 and K a positive multiple of 64 (M=%lld N=%lld K=%lld)",
+    return set_error(NVFP4_ERR_INVALID_ARG, "%s: need M, N >= 1 and K a positive multiple of 64 (M=%lld N=%lld K=%lld)", fn,
                      (long long)M, (long long)N, (long long)K);
   if (M > (1ll << 30) || N > (1ll << 30) || K > (1ll << 30))
-    return set_error(NVFP4_ERR_INVALID_ARG, "nvfp4_gemm: dimension too large");
-  if (ldy < N) return set_error(NVFP4_ERR_INVALID_ARG, "nvfp4_gemm: need ldy >= N");
+    return set_error(NVFP4_ERR_INVALID_ARG, "%s: dimension too large", fn);
+  if (ldy < N) return set_error(NVFP4_ERR_INVALID_ARG, "%s: need ldy >= N", fn);
   if (out_dtype != NVFP4_OUT_BF16 && out_dtype != NVFP4_OUT_FP32)
-    return set_error(NVFP4_ERR_INVALID_ARG, "nvfp4_gemm: unknown out_dtype %d", out_dtype);
+    return set_error(NVFP4_ERR_INVALID_ARG, "%s: unknown out_dtype %d", fn, out_dtype);
   if (!aligned16(a_codes) || !aligned16(b_codes) || !aligned16(a_scales) || !aligned16(b_scales) ||
       (reinterpret_cast<uintptr_t>(y) & (out_dtype == NVFP4_OUT_FP32 ? 3u : 1u)) ||
       !aligned16(workspace) ||
       (reinterpret_cast<uintptr_t>(a_global) & 3u) ||
       (reinterpret_cast<uintptr_t>(b_global) & 3u))
-    return set_error(NVFP4_ERR_INVALID_ARG, "nvfp4_gemm: misaligned buffer");
+    return set_error(NVFP4_ERR_INVALID_ARG, "%s: misaligned buffer", fn);
+  if (nseg < 1 || nseg > kMaxSegments)
+    return set_error(NVFP4_ERR_INVALID_ARG, "%s: need 1 <= nseg <= %d", fn, kMaxSegments);
+  for (int i = 0; i < nseg; ++i) {
+    const int64_t lo = i ? seg_ends[i - 1] : 0;
+    if (seg_ends[i] <= lo || (i + 1 < nseg ? seg_ends[i] % 64 != 0 : seg_ends[i] != N))
+      return set_error(NVFP4_ERR_INVALID_ARG,
+                       "%s: segment ends must ascend, be multiples of 64, and end at N", fn);
+  }
   if (workspace_bytes < nvfp4_gemm_workspace_bytes())
-    return set_error(NVFP4_ERR_INVALID_ARG, "nvfp4_gemm: workspace too small");
+    return set_error(NVFP4_ERR_INVALID_ARG, "%s: workspace too small", fn);
   int dev = 0, sms = 0;
   nvfp4_status st = check_device(&dev, &sms);
   if (st != NVFP4_OK) return st;
@@ -530,6 +555,8 @@ nvfp4_status nvfp4_gemm(const void* a_codes, const void* a_scales, const float* 
   GemmParams p;
   p.a_global = a_global;
   p.b_global = b_global;
+  p.nseg = nseg;
+  for (int i = 0; i < kMaxSegments; ++i) p.seg_end[i] = static_cast<int>(i < nseg ? seg_ends[i] : N);
   p.y = y;
   p.ws = static_cast<WorkspaceHeader*>(workspace);
   p.ldy = ldy;
@@ -539,7 +566,7 @@ nvfp4_status nvfp4_gemm(const void* a_codes, const void* a_scales, const float* 
   p.ktiles = static_cast<uint32_t>((K + 255) / 256);
   p.n_tiles = static_cast<uint32_t>((N + BN - 1) / BN);
   const int64_t num_tiles = ((M + BM - 1) / BM) * static_cast<int64_t>(p.n_tiles);
-  if (num_tiles > 0x7FFFFFFFll) return set_error(NVFP4_ERR_INVALID_ARG, "nvfp4_gemm: too many tiles");
+  if (num_tiles > 0x7FFFFFFFll) return set_error(NVFP4_ERR_INVALID_ARG, "%s: too many tiles", fn);
   p.num_tiles = static_cast<uint32_t>(num_tiles);
   p.out_fp32 = out_dtype == NVFP4_OUT_FP32;
   p.vec_store = aligned16(y) && ((ldy * (p.out_fp32 ? 4 : 2)) % 16 == 0);
@@ -551,6 +578,29 @@ nvfp4_status nvfp4_gemm(const void* a_codes, const void* a_scales, const float* 
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_status(e, "gemm_kernel launch");
   return NVFP4_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+nvfp4_status nvfp4_gemm(const void* a_codes, const void* a_scales, const float* a_global,
+                        const void* b_codes, const void* b_scales, const float* b_global,
+                        int64_t M, int64_t N, int64_t K, void* y, int64_t ldy, int out_dtype,
+                        void* workspace, size_t workspace_bytes, void* stream) {
+  const int64_t end = N;
+  return gemm_impl("nvfp4_gemm", a_codes, a_scales, a_global, b_codes, b_scales, b_global, &end, 1,
+                   M, N, K, y, ldy, out_dtype, workspace, workspace_bytes, stream);
+}
+
+nvfp4_status nvfp4_gemm_segmented(const void* a_codes, const void* a_scales, const float* a_global,
+                                  const void* b_codes, const void* b_scales, const float* b_globals,
+                                  const int64_t* seg_ends, int nseg, int64_t M, int64_t N, int64_t K,
+                                  void* y, int64_t ldy, int out_dtype, void* workspace,
+                                  size_t workspace_bytes, void* stream) {
+  if (!seg_ends) return set_error(NVFP4_ERR_INVALID_ARG, "nvfp4_gemm_segmented: null seg_ends");
+  return gemm_impl("nvfp4_gemm_segmented", a_codes, a_scales, a_global, b_codes, b_scales, b_globals,
+                   seg_ends, nseg, M, N, K, y, ldy, out_dtype, workspace, workspace_bytes, stream);
 }
 
 }  // extern "C"

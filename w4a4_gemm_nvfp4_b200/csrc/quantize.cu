@@ -13,6 +13,11 @@
 // Every step is one binary32 operation (explicit __f*_rn intrinsics; the
 // file is also built with -fmad=false) so the result is bit-reproducible.
 //
+// The 16 values of a block are held as binary32 pairs (x_j, x_{j+8}) and the
+// per-element arithmetic uses packed f32x2 instructions (each lane an IEEE RNE
+// operation, like the scalar one); with that pairing the contiguous pairwise
+// error sum is three packed additions and one scalar one.
+//
 // Two kernels per call:
 //   amax_kernel      one HBM read of x; each CTA writes the max |bf16| bit
 //                    pattern it saw to a partials array in the workspace.
@@ -27,6 +32,7 @@
 #include <cuda_fp16.h>
 
 #include <algorithm>
+#include <atomic>
 #include <mutex>
 
 #include "common.cuh"
@@ -34,7 +40,7 @@
 namespace nvfp4 {
 namespace {
 
-constexpr int kAmaxThreads = 256;
+constexpr int kAmaxThreads = 512;
 constexpr int kMaxPartials = 4096;
 constexpr int kQuantThreads = 256;
 constexpr int kQuantWarps = kQuantThreads / 32;
@@ -64,8 +70,9 @@ __device__ __forceinline__ uint32_t absmax4(const uint4& v, uint32_t m) {
 // ------------------------------------------------------------- amax pass --
 // Magnitudes compare like their bit patterns once the sign is cleared, and
 // every NaN pattern (> 0x7F80) compares above Inf (0x7F80) above any finite
-// value, so one unsigned max gives both amax and the non-finite flag.
-__global__ void __launch_bounds__(kAmaxThreads)
+// value, so one unsigned max gives both amax and the non-finite flag.  Each
+// thread keeps eight 16-byte loads in flight; two 512-thread CTAs per SM.
+__global__ void __launch_bounds__(kAmaxThreads, 2)
     amax_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t K, int64_t ldx,
                 uint32_t* __restrict__ partials) {
   uint32_t m = 0;
@@ -74,13 +81,12 @@ __global__ void __launch_bounds__(kAmaxThreads)
     const int64_t n = rows * K / 8;
     const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
     int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-    for (; i + 3 * stride < n; i += 4 * stride) {
-      uint4 a = ld_stream(v + i), b = ld_stream(v + i + stride);
-      uint4 c = ld_stream(v + i + 2 * stride), d = ld_stream(v + i + 3 * stride);
-      m = absmax4(a, m);
-      m = absmax4(b, m);
-      m = absmax4(c, m);
-      m = absmax4(d, m);
+    for (; i + 7 * stride < n; i += 8 * stride) {
+      uint4 a[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) a[u] = ld_stream(v + i + u * stride);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) m = absmax4(a[u], m);
     }
     for (; i < n; i += stride) m = absmax4(ld_stream(v + i), m);
   } else {
@@ -114,32 +120,68 @@ __device__ __forceinline__ uint32_t cvt_e4m3x2(float hi, float lo) {
 }
 // Two E4M3 (byte pair) -> two binary32 (exact, via f16).
 __device__ __forceinline__ void e4m3x2_to_f32(uint32_t pair, float& lo, float& hi) {
-  uint32_t h;
-  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h) : "h"(static_cast<uint16_t>(pair)));
-  lo = __half2float(__ushort_as_half(static_cast<unsigned short>(h & 0xFFFFu)));
-  hi = __half2float(__ushort_as_half(static_cast<unsigned short>(h >> 16)));
+  asm("{\n\t.reg .b32 h2;\n\t.reg .f16 h0, h1;\n\t"
+      "cvt.rn.f16x2.e4m3x2 h2, %2;\n\t"
+      "mov.b32 {h0, h1}, h2;\n\t"
+      "cvt.f32.f16 %0, h0;\n\t"
+      "cvt.f32.f16 %1, h1;\n\t}"
+      : "=f"(lo), "=f"(hi)
+      : "h"(static_cast<uint16_t>(pair)));
 }
-// Two binary32 -> one byte of two E2M1 codes (RNE, saturating to 6, sign kept):
-// low nibble from `lo`.
-__device__ __forceinline__ uint32_t cvt_e2m1x2(float hi, float lo) {
-  uint32_t r;
-  asm("{\n\t.reg .b8 t;\n\t"
-      "cvt.rn.satfinite.e2m1x2.f32 t, %1, %2;\n\t"
-      "cvt.u32.u8 %0, t;\n\t}"
-      : "=r"(r)
+// Two binary32 -> E2M1 codes (RNE, saturating to 6, sign kept); the code byte
+// holds `lo` in its low nibble.
+__device__ __forceinline__ uint32_t e2m1x2_encode(float hi, float lo) {
+  uint32_t byte;
+  asm("{\n\t.reg .b8 c;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 c, %1, %2;\n\t"
+      "cvt.u32.u8 %0, c;\n\t}"
+      : "=r"(byte)
       : "f"(hi), "f"(lo));
+  return byte;
+}
+// e2m1x2_encode, plus the two code values back as binary32 (exact, via f16).
+__device__ __forceinline__ uint32_t e2m1x2_round(float hi, float lo, float& qlo, float& qhi) {
+  uint32_t byte;
+  asm("{\n\t.reg .b8 c;\n\t.reg .b32 h2;\n\t.reg .f16 h0, h1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 c, %3, %4;\n\t"
+      "cvt.rn.f16x2.e2m1x2 h2, c;\n\t"
+      "mov.b32 {h0, h1}, h2;\n\t"
+      "cvt.f32.f16 %1, h0;\n\t"
+      "cvt.f32.f16 %2, h1;\n\t"
+      "cvt.u32.u8 %0, c;\n\t}"
+      : "=r"(byte), "=f"(qlo), "=f"(qhi)
+      : "f"(hi), "f"(lo));
+  return byte;
+}
+
+// Packed binary32 pairs (one IEEE RNE operation per lane, like the scalar
+// instruction on each lane).
+struct f2 {
+  float a, b;
+};
+__device__ __forceinline__ f2 mul2(f2 x, f2 y) {
+  f2 r;
+  asm("{\n\t.reg .b64 p, q, o;\n\tmov.b64 p, {%2, %3};\n\tmov.b64 q, {%4, %5};\n\t"
+      "mul.rn.f32x2 o, p, q;\n\tmov.b64 {%0, %1}, o;\n\t}"
+      : "=f"(r.a), "=f"(r.b)
+      : "f"(x.a), "f"(x.b), "f"(y.a), "f"(y.b));
   return r;
 }
-// One byte of two E2M1 codes -> the two values as binary32 (exact, via f16).
-__device__ __forceinline__ void e2m1x2_to_f32(uint32_t byte, float& lo, float& hi) {
-  uint32_t h;
-  asm("{\n\t.reg .b8 t;\n\t"
-      "cvt.u8.u32 t, %1;\n\t"
-      "cvt.rn.f16x2.e2m1x2 %0, t;\n\t}"
-      : "=r"(h)
-      : "r"(byte));
-  lo = __half2float(__ushort_as_half(static_cast<unsigned short>(h & 0xFFFFu)));
-  hi = __half2float(__ushort_as_half(static_cast<unsigned short>(h >> 16)));
+__device__ __forceinline__ f2 fma2(f2 x, f2 y, f2 z) {
+  f2 r;
+  asm("{\n\t.reg .b64 p, q, s, o;\n\tmov.b64 p, {%2, %3};\n\tmov.b64 q, {%4, %5};\n\t"
+      "mov.b64 s, {%6, %7};\n\tfma.rn.f32x2 o, p, q, s;\n\tmov.b64 {%0, %1}, o;\n\t}"
+      : "=f"(r.a), "=f"(r.b)
+      : "f"(x.a), "f"(x.b), "f"(y.a), "f"(y.b), "f"(z.a), "f"(z.b));
+  return r;
+}
+__device__ __forceinline__ f2 add2(f2 x, f2 y) {
+  f2 r;
+  asm("{\n\t.reg .b64 p, q, o;\n\tmov.b64 p, {%2, %3};\n\tmov.b64 q, {%4, %5};\n\t"
+      "add.rn.f32x2 o, p, q;\n\tmov.b64 {%0, %1}, o;\n\t}"
+      : "=f"(r.a), "=f"(r.b)
+      : "f"(x.a), "f"(x.b), "f"(y.a), "f"(y.b));
+  return r;
 }
 
 __device__ __forceinline__ float safe_recip(float d) {
@@ -147,85 +189,126 @@ __device__ __forceinline__ float safe_recip(float d) {
   return isinf(r) ? 0.0f : r;  // d == 0 or 1/d overflowed
 }
 
-// The 16-term contiguous pairwise tree ((t0+t1)+(t2+t3))+...
-__device__ __forceinline__ float pairwise16(float t[16]) {
-#pragma unroll
-  for (int n = 16; n > 1; n >>= 1) {
-#pragma unroll
-    for (int i = 0; i < n / 2; ++i) t[i] = __fadd_rn(t[2 * i], t[2 * i + 1]);
-  }
-  return t[0];
-}
-
 enum { kRuleMax = 0, kRuleMae = 1, kRuleMse = 2 };
 
-// One candidate: codes (8 bytes, element 2j in the low nibble of byte j) and
-// its block error under RULE.
-template <int RULE>
-__device__ __forceinline__ float candidate(const float x[16], float d, float r, uint2& codes) {
-  float t[16];
+// Codes of one candidate: v = x * r per element, E2M1-rounded.  The block's
+// 16 values are held as pairs p[j] = (x_j, x_{j+8}), j < 8; codes byte j holds
+// elements 2j, 2j+1 (low nibble first).
+__device__ __forceinline__ uint2 candidate_codes(const f2 p[8], float r) {
+  const f2 rr = {r, r};
   uint32_t bytes[8];
-  const float nd = -d;
 #pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    const float v0 = __fmul_rn(x[2 * j], r);
-    const float v1 = __fmul_rn(x[2 * j + 1], r);
-    bytes[j] = cvt_e2m1x2(v1, v0);
-    float q0, q1;
-    e2m1x2_to_f32(bytes[j], q0, q1);
-    const float e0 = __fmaf_rn(q0, nd, x[2 * j]);
-    const float e1 = __fmaf_rn(q1, nd, x[2 * j + 1]);
-    if (RULE == kRuleMse) {
-      t[2 * j] = __fmul_rn(e0, e0);
-      t[2 * j + 1] = __fmul_rn(e1, e1);
-    } else {
-      t[2 * j] = fabsf(e0);
-      t[2 * j + 1] = fabsf(e1);
-    }
+  for (int j = 0; j < 4; ++j) {
+    const f2 v0 = mul2(p[2 * j], rr), v1 = mul2(p[2 * j + 1], rr);
+    bytes[j] = e2m1x2_encode(v1.a, v0.a);
+    bytes[j + 4] = e2m1x2_encode(v1.b, v0.b);
+  }
+  return make_uint2(bytes[0] | (bytes[1] << 8) | (bytes[2] << 16) | (bytes[3] << 24),
+                    bytes[4] | (bytes[5] << 8) | (bytes[6] << 16) | (bytes[7] << 24));
+}
+
+// One candidate with its block error under RULE.  With the (x_j, x_{j+8})
+// pairing the contiguous pairwise tree of the error terms
+// ((t0+t1)+(t2+t3))+... is exactly three packed additions and one scalar one:
+//   (t_2i + t_2i+1, t_2i+8 + t_2i+9)      = (u_i, u_i+4)   i < 4
+//   (u_2i + u_2i+1, u_2i+4 + u_2i+5)      = (w_i, w_i+2)   i < 2
+//   (w_0 + w_1, w_2 + w_3)                = (z_0, z_1),    then z_0 + z_1.
+template <int RULE>
+__device__ __forceinline__ float candidate(const f2 p[8], float d, float r, uint2& codes) {
+  const f2 rr = {r, r};
+  const f2 nd = {-d, -d};
+  f2 v[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) v[j] = mul2(p[j], rr);
+  // element k is v[k % 8].a (k < 8) or v[k % 8].b (k >= 8)
+  float q[16];
+  uint32_t bytes[8];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    // byte j: elements 2j, 2j+1 (first half); byte j+4: elements 2j+8, 2j+9
+    bytes[j] = e2m1x2_round(v[2 * j + 1].a, v[2 * j].a, q[2 * j], q[2 * j + 1]);
+    bytes[j + 4] = e2m1x2_round(v[2 * j + 1].b, v[2 * j].b, q[2 * j + 8], q[2 * j + 9]);
   }
   codes.x = bytes[0] | (bytes[1] << 8) | (bytes[2] << 16) | (bytes[3] << 24);
   codes.y = bytes[4] | (bytes[5] << 8) | (bytes[6] << 16) | (bytes[7] << 24);
-  if (RULE == kRuleMax) {
-    float m = t[0];
+  // e = fma(-q, d, x), paired like p
+  f2 e[8];
 #pragma unroll
-    for (int i = 1; i < 16; ++i) m = fmaxf(m, t[i]);
-    return m;
+  for (int j = 0; j < 8; ++j) e[j] = fma2(f2{q[j], q[j + 8]}, nd, p[j]);
+  if (RULE == kRuleMax) {
+    float m0 = 0.0f, m1 = 0.0f;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      m0 = fmaxf(m0, fabsf(e[j].a));
+      m1 = fmaxf(m1, fabsf(e[j].b));
+    }
+    return fmaxf(m0, m1);
   }
-  return pairwise16(t);
+  f2 t[8];
+  if (RULE == kRuleMse) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) t[j] = mul2(e[j], e[j]);
+  } else {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) t[j] = f2{fabsf(e[j].a), fabsf(e[j].b)};
+  }
+  const f2 u0 = add2(t[0], t[1]), u1 = add2(t[2], t[3]), u2 = add2(t[4], t[5]), u3 = add2(t[6], t[7]);
+  const f2 w0 = add2(u0, u1), w1 = add2(u2, u3);
+  const f2 z = add2(w0, w1);
+  return __fadd_rn(z.a, z.b);
+}
+
+// Per-call constants of the block step.  The scale quotient b / (alpha*Q) must
+// be the correctly rounded binary32 quotient before its E4M3 rounding; it is
+// taken as b * fl(1/(alpha*Q)), which is within 3 units in the last place of
+// the quotient, and recomputed by a true division whenever that distance
+// could change the E4M3 result: below the E4M3 normal range (2^-6), or with
+// the 20 bits under E4M3's 3-bit mantissa within 5 units of the rounding
+// midpoint 0x80000.  Above 448 both saturate to 448.
+struct BlockConsts {
+  float a6, a4;      // alpha * 6, alpha * 4
+  float inv6, inv4;  // fl(1 / a6), fl(1 / a4)
+  bool fast_div;     // both reciprocals finite and normal
+};
+__device__ __forceinline__ bool needs_exact_quotient(float q) {
+  const uint32_t b = __float_as_uint(q);
+  return b < 0x3C800008u || ((b & 0xFFFFFu) - 0x7FFFBu) < 11u;
 }
 
 // Quantize one block held as 8 words of bf16 pairs (element 2j in the low
-// half of word j).
+// half of word j).  dr[c] = (d, r) of E4M3 scale code c: d = val(c) * alpha,
+// r = 1/d (0 if infinite).
 template <bool FOUR_OVER_SIX, int RULE>
-__device__ __forceinline__ void quantize_block(const uint4& lo, const uint4& hi, float alpha,
-                                               float a6, float a4, uint2& codes,
-                                               uint32_t& scale) {
+__device__ __forceinline__ void quantize_block(const uint4& lo, const uint4& hi, const BlockConsts& k,
+                                               const float2* dr, uint2& codes, uint32_t& scale) {
   const uint32_t w[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
   uint32_t m = absmax4(lo, 0u);
   m = absmax4(hi, m);
   const float b = __uint_as_float(max(m & 0xFFFFu, m >> 16) << 16);
-  float x[16];
+  // p[j] = (x_j, x_{j+8}): x_2i is the low half of word i, x_2i+1 the high half
+  f2 p[8];
 #pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    x[2 * j] = __uint_as_float(w[j] << 16);
-    x[2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
+  for (int i = 0; i < 4; ++i) {
+    p[2 * i] = f2{__uint_as_float(w[i] << 16), __uint_as_float(w[i + 4] << 16)};
+    p[2 * i + 1] = f2{__uint_as_float(w[i] & 0xFFFF0000u), __uint_as_float(w[i + 4] & 0xFFFF0000u)};
   }
-  const float s6raw = __fdiv_rn(b, a6);
-  const float s4raw = FOUR_OVER_SIX ? __fdiv_rn(b, a4) : 0.0f;
+  float s6raw = __fmul_rn(b, k.inv6);
+  float s4raw = FOUR_OVER_SIX ? __fmul_rn(b, k.inv4) : 0.0f;
+  if (!k.fast_div || needs_exact_quotient(s6raw) || (FOUR_OVER_SIX && needs_exact_quotient(s4raw))) {
+    s6raw = __fdiv_rn(b, k.a6);
+    if (FOUR_OVER_SIX) s4raw = __fdiv_rn(b, k.a4);
+  }
   const uint32_t sc = cvt_e4m3x2(s4raw, s6raw);  // low byte: scale-6, high byte: scale-4
-  float s6, s4;
-  e4m3x2_to_f32(sc, s6, s4);
-  const float d6 = __fmul_rn(s6, alpha);
-  uint2 c6;
-  const float E6 = candidate<RULE>(x, d6, safe_recip(d6), c6);
+  const float2 dr6 = dr[sc & 0xFFu];
   if (!FOUR_OVER_SIX) {
-    codes = c6;
+    codes = candidate_codes(p, dr6.y);
     scale = sc & 0xFFu;
     return;
   }
-  const float d4 = __fmul_rn(s4, alpha);
-  uint2 c4;
-  const float E4 = candidate<RULE>(x, d4, safe_recip(d4), c4);
+  const float2 dr4 = dr[sc >> 8];
+  uint2 c6, c4;
+  const float E6 = candidate<RULE>(p, dr6.x, dr6.y, c6);
+  const float E4 = candidate<RULE>(p, dr4.x, dr4.y, c4);
   const bool pick4 = E4 < E6;  // ties keep scale 6
   codes = pick4 ? c4 : c6;
   scale = pick4 ? (sc >> 8) : (sc & 0xFFu);
@@ -237,7 +320,8 @@ struct QuantParams {
   uint8_t* codes;
   uint8_t* scales;
   float* global_scale;
-  const uint32_t* partials;
+  const uint32_t* partials;   // amax partials (dynamic alpha) ...
+  const float* alpha_in;      // ... or a caller-supplied alpha (static), else null
   WorkspaceHeader* ws;
   int nparts;
   float f6;            // fp8_max * 6
@@ -248,61 +332,142 @@ struct QuantParams {
 template <bool FOUR_OVER_SIX, int RULE>
 __global__ void __launch_bounds__(kQuantThreads)
     quantize_kernel(const QuantParams p) {
-  // ---- tensor amax -> alpha (every CTA reduces the same partials) ----
-  __shared__ uint32_t s_red[kQuantWarps];
+  // ---- alpha: a caller-supplied static scale, or the tensor amax reduced
+  // from the partials of the amax pass (every CTA reduces the same partials)
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  uint32_t m = 0;
-  for (int i = threadIdx.x; i < p.nparts; i += kQuantThreads) m = max(m, p.partials[i]);
+  float alpha;
+  if (p.alpha_in) {
+    alpha = __ldg(p.alpha_in);
+    if (!(alpha > 0.0f) || isinf(alpha)) {  // not a positive finite number
+      if (blockIdx.x == 0 && threadIdx.x == 0) p.ws->status = NVFP4_ERR_INVALID_ARG;
+      return;
+    }
+    // the status word was cleared to NVFP4_OK before the launch; CTAs only
+    // ever raise it (to NVFP4_ERR_NONFINITE), so their order does not matter
+  } else {
+    __shared__ uint32_t s_red[kQuantWarps];
+    uint32_t m = 0;
+    for (int i = threadIdx.x; i < p.nparts; i += kQuantThreads) m = max(m, p.partials[i]);
 #pragma unroll
-  for (int o = 16; o; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
-  if (lane == 0) s_red[warp] = m;
-  __syncthreads();
-  uint32_t amax_bits = 0;
+    for (int o = 16; o; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if (lane == 0) s_red[warp] = m;
+    __syncthreads();
+    uint32_t amax_bits = 0;
 #pragma unroll
-  for (int w = 0; w < kQuantWarps; ++w) amax_bits = max(amax_bits, s_red[w]);
-  const bool nonfinite = amax_bits >= 0x7F80u;
-  const float alpha =
-      amax_bits == 0 ? 1.0f : __fdiv_rn(__uint_as_float(amax_bits << 16), p.f6);
-  if (blockIdx.x == 0 && threadIdx.x == 0) {
-    p.ws->status = nonfinite ? NVFP4_ERR_NONFINITE : NVFP4_OK;
-    p.ws->detail = amax_bits;
-    *p.global_scale = nonfinite ? __uint_as_float(0x7FC00000u) : alpha;
+    for (int w = 0; w < kQuantWarps; ++w) amax_bits = max(amax_bits, s_red[w]);
+    const bool nonfinite = amax_bits >= 0x7F80u;
+    alpha = amax_bits == 0 ? 1.0f : __fdiv_rn(__uint_as_float(amax_bits << 16), p.f6);
+    if (blockIdx.x == 0 && threadIdx.x == 0) {
+      p.ws->status = nonfinite ? NVFP4_ERR_NONFINITE : NVFP4_OK;
+      p.ws->detail = amax_bits;
+      *p.global_scale = nonfinite ? __uint_as_float(0x7FC00000u) : alpha;
+    }
+    if (nonfinite) return;
   }
-  if (nonfinite) return;
-  const float a6 = __fmul_rn(alpha, 6.0f);
-  const float a4 = __fmul_rn(alpha, 4.0f);
+  BlockConsts k;
+  k.a6 = __fmul_rn(alpha, 6.0f);
+  k.a4 = __fmul_rn(alpha, 4.0f);
+  k.inv6 = __frcp_rn(k.a6);
+  k.inv4 = __frcp_rn(k.a4);
+  k.fast_div = k.inv6 >= 1.17549435e-38f && !isinf(k.inv4);
+
+  // (d, r) of every E4M3 scale code (0x7F is NaN and never produced)
+  __shared__ float2 s_dr[128];
+  if (threadIdx.x < 128) {
+    float s, unused;
+    e4m3x2_to_f32(threadIdx.x, s, unused);
+    const float d = threadIdx.x == 0x7F ? 0.0f : __fmul_rn(s, alpha);
+    s_dr[threadIdx.x] = make_float2(d, safe_recip(d));
+  }
+  __syncthreads();
 
   // ---- lane -> (row, 16-element block) inside a warp task ----
   // task = (row_block * 16 + piece) * kgroups + kgroup; a piece is 32 bytes of
   // a 512-byte scale atom: atom byte o = 32*piece + lane holds the scale of
-  // row (o/16) + 32*((o/4)%4) and K-block o%4 of the atom.
+  // row (o/16) + 32*((o/4)%4) and K-block o%4 of the atom.  Each warp walks
+  // its tasks with a fixed stride, loading the next task's block while it
+  // quantizes the current one.
   const int row_in_atom = ((lane >> 2) & 3) * 32 + (lane >> 4);
   const int kb_in_group = lane & 3;
-  const uint32_t total_warps = gridDim.x * kQuantWarps;
+  const uint32_t stride = gridDim.x * kQuantWarps;
+  const uint32_t stride_hi = stride / p.kgroups, stride_lo = stride % p.kgroups;
   const int64_t half_k = p.K / 2;
-  for (uint32_t task = blockIdx.x * kQuantWarps + warp; task < p.ntasks; task += total_warps) {
-    const uint32_t kg = task % p.kgroups;
-    const uint32_t t2 = task / p.kgroups;
-    const uint32_t piece = t2 & 15u, rb = t2 >> 4;
-    const int64_t row = static_cast<int64_t>(rb) * 128 + row_in_atom + 2 * piece;
-    const int64_t kb = static_cast<int64_t>(kg) * 4 + kb_in_group;
+  uint32_t task = blockIdx.x * kQuantWarps + warp;
+  uint32_t kg = task % p.kgroups, t2 = task / p.kgroups;
+  int64_t row = static_cast<int64_t>(t2 >> 4) * 128 + row_in_atom + 2 * (t2 & 15u);
+  uint4 lo = make_uint4(0, 0, 0, 0), hi = lo;
+  if (task < p.ntasks && row < p.rows) {
+    const uint4* src = reinterpret_cast<const uint4*>(p.x + row * p.ldx + (kg * 4 + kb_in_group) * 16);
+    lo = ld_stream(src);
+    hi = ld_stream(src + 1);
+  }
+  while (task < p.ntasks) {
+    // next task (ntasks < 2^31 and stride < 2^16: no wrap-around)
+    const uint32_t ntask = task + stride;
+    uint32_t nkg = kg + stride_lo, nt2 = t2 + stride_hi;
+    if (nkg >= p.kgroups) {
+      nkg -= p.kgroups;
+      ++nt2;
+    }
+    const int64_t nrow = static_cast<int64_t>(nt2 >> 4) * 128 + row_in_atom + 2 * (nt2 & 15u);
+    uint4 nlo = make_uint4(0, 0, 0, 0), nhi = nlo;
+    if (ntask < p.ntasks && nrow < p.rows) {
+      const uint4* src = reinterpret_cast<const uint4*>(p.x + nrow * p.ldx + (nkg * 4 + kb_in_group) * 16);
+      nlo = ld_stream(src);
+      nhi = ld_stream(src + 1);
+    }
+
     uint32_t scale = 0;
     if (row < p.rows) {
-      const uint4* src = reinterpret_cast<const uint4*>(p.x + row * p.ldx + kb * 16);
-      const uint4 lo = ld_stream(src), hi = ld_stream(src + 1);
       uint2 codes;
-      quantize_block<FOUR_OVER_SIX, RULE>(lo, hi, alpha, a6, a4, codes, scale);
-      *reinterpret_cast<uint2*>(p.codes + row * half_k + kb * 8) = codes;
+      quantize_block<FOUR_OVER_SIX, RULE>(lo, hi, k, s_dr, codes, scale);
+      const uint32_t bmax = p.alpha_in ? absmax4(hi, absmax4(lo, 0u)) : 0u;
+      if (max(bmax & 0xFFFFu, bmax >> 16) >= 0x7F80u) {
+        // Inf/NaN in this block (a static alpha skips the tensor check):
+        // the block is written as zeros and the call reports it
+        codes = make_uint2(0u, 0u);
+        scale = 0u;
+        p.ws->status = NVFP4_ERR_NONFINITE;
+      }
+      *reinterpret_cast<uint2*>(p.codes + row * half_k + (kg * 4 + kb_in_group) * 8) = codes;
     }
-    p.scales[(static_cast<int64_t>(rb) * p.kgroups + kg) * 512 + piece * 32 + lane] =
+    p.scales[(static_cast<int64_t>(t2 >> 4) * p.kgroups + kg) * 512 + (t2 & 15u) * 32 + lane] =
         static_cast<uint8_t>(scale);
+
+    task = ntask;
+    kg = nkg;
+    t2 = nt2;
+    row = nrow;
+    lo = nlo;
+    hi = nhi;
   }
 }
 
+// Grid: one wave of resident CTAs (SMs x CTAs per SM at this kernel's
+// register use), fewer when there are fewer tasks; every warp then walks its
+// tasks with a grid-wide stride.
 template <bool F, int R>
-cudaError_t launch_quantize(int grid, const QuantParams& p, cudaStream_t s) {
+cudaError_t launch_quantize(int sms, const QuantParams& p, cudaStream_t s) {
+  static std::atomic<int> per_sm{0};
+  int occ = per_sm.load(std::memory_order_relaxed);
+  if (occ == 0) {
+    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, quantize_kernel<F, R>,
+                                                                  kQuantThreads, 0);
+    if (e != cudaSuccess) return e;
+    occ = std::max(1, occ);
+    per_sm.store(occ, std::memory_order_relaxed);
+  }
+  const int64_t want = (static_cast<int64_t>(p.ntasks) + kQuantWarps - 1) / kQuantWarps;
+  const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(want, static_cast<int64_t>(sms) * occ)));
   quantize_kernel<F, R><<<grid, kQuantThreads, 0, s>>>(p);
   return cudaGetLastError();
+}
+
+cudaError_t launch_quantize_kernel(int mode, int rule, int sms, const QuantParams& p, cudaStream_t s) {
+  if (mode == NVFP4_MODE_SIX) return launch_quantize<false, kRuleMax>(sms, p, s);
+  if (rule == NVFP4_RULE_MAX) return launch_quantize<true, kRuleMax>(sms, p, s);
+  if (rule == NVFP4_RULE_MAE) return launch_quantize<true, kRuleMae>(sms, p, s);
+  return launch_quantize<true, kRuleMse>(sms, p, s);
 }
 
 }  // namespace
@@ -343,7 +508,7 @@ nvfp4_status nvfp4_quantize(const void* x, int64_t rows, int64_t K, int64_t ldx,
     return set_error(NVFP4_ERR_INVALID_ARG, "nvfp4_quantize: workspace too small");
   const int64_t row_blocks = (rows + 127) / 128;
   const int64_t ntasks = row_blocks * 16 * (K / 64);
-  if (ntasks > 0xFFFFFFFFll || rows * ldx > (1ll << 40))
+  if (ntasks >= 0x80000000ll || rows * ldx > (1ll << 40))
     return set_error(NVFP4_ERR_INVALID_ARG, "nvfp4_quantize: tensor too large");
   int dev = 0, sms = 0;
   nvfp4_status st = check_device(&dev, &sms);
@@ -356,10 +521,10 @@ nvfp4_status nvfp4_quantize(const void* x, int64_t rows, int64_t K, int64_t ldx,
   int amax_grid;
   if (ldx == K) {
     const int64_t nvec = rows * K / 8;
-    amax_grid = static_cast<int>(std::min<int64_t>((nvec + kAmaxThreads * 4 - 1) / (kAmaxThreads * 4),
-                                                   static_cast<int64_t>(sms) * 4));
+    amax_grid = static_cast<int>(std::min<int64_t>((nvec + kAmaxThreads * 8 - 1) / (kAmaxThreads * 8),
+                                                   static_cast<int64_t>(sms) * 2));
   } else {
-    amax_grid = static_cast<int>(std::min<int64_t>(rows, static_cast<int64_t>(sms) * 4));
+    amax_grid = static_cast<int>(std::min<int64_t>(rows, static_cast<int64_t>(sms) * 2));
   }
   amax_grid = std::max(1, std::min(amax_grid, kMaxPartials));
   amax_kernel<<<amax_grid, kAmaxThreads, 0, s>>>(static_cast<const uint16_t*>(x), rows, K, ldx,
@@ -376,17 +541,13 @@ nvfp4_status nvfp4_quantize(const void* x, int64_t rows, int64_t K, int64_t ldx,
   p.scales = static_cast<uint8_t*>(scales);
   p.global_scale = global_scale;
   p.partials = partials;
+  p.alpha_in = nullptr;
   p.ws = ws;
   p.nparts = amax_grid;
   p.f6 = fp8_max * 6.0f;
   p.ntasks = static_cast<uint32_t>(ntasks);
   p.kgroups = static_cast<uint32_t>(K / 64);
-  const int64_t want = (ntasks + kQuantWarps - 1) / kQuantWarps;
-  const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(want, static_cast<int64_t>(sms) * 8)));
-  if (mode == NVFP4_MODE_SIX) e = launch_quantize<false, kRuleMax>(grid, p, s);
-  else if (rule == NVFP4_RULE_MAX) e = launch_quantize<true, kRuleMax>(grid, p, s);
-  else if (rule == NVFP4_RULE_MAE) e = launch_quantize<true, kRuleMae>(grid, p, s);
-  else e = launch_quantize<true, kRuleMse>(grid, p, s);
+  e = launch_quantize_kernel(mode, rule, sms, p, s);
   if (e != cudaSuccess) return cuda_status(e, "quantize_kernel launch");
   return NVFP4_OK;
 }
@@ -467,7 +628,7 @@ extern "C" nvfp4_status nvfp4_quantize_noalloc(const void* x, int64_t rows, int6
     return set_error(NVFP4_ERR_INVALID_ARG, "nvfp4_quantize_noalloc: misaligned buffer");
   const int64_t row_blocks = (rows + 127) / 128;
   const int64_t ntasks = row_blocks * 16 * (K / 64);
-  if (ntasks > 0xFFFFFFFFll || rows * ldx > (1ll << 40))
+  if (ntasks >= 0x80000000ll || rows * ldx > (1ll << 40))
     return set_error(NVFP4_ERR_INVALID_ARG, "nvfp4_quantize_noalloc: tensor too large");
   int dev = 0, sms = 0;
   nvfp4_status st = check_device(&dev, &sms);
@@ -476,10 +637,10 @@ extern "C" nvfp4_status nvfp4_quantize_noalloc(const void* x, int64_t rows, int6
   int amax_grid;
   if (ldx == K) {
     const int64_t nvec = rows * K / 8;
-    amax_grid = static_cast<int>(std::min<int64_t>((nvec + kAmaxThreads * 4 - 1) / (kAmaxThreads * 4),
-                                                   static_cast<int64_t>(sms) * 4));
+    amax_grid = static_cast<int>(std::min<int64_t>((nvec + kAmaxThreads * 8 - 1) / (kAmaxThreads * 8),
+                                                   static_cast<int64_t>(sms) * 2));
   } else {
-    amax_grid = static_cast<int>(std::min<int64_t>(rows, static_cast<int64_t>(sms) * 4));
+    amax_grid = static_cast<int>(std::min<int64_t>(rows, static_cast<int64_t>(sms) * 2));
   }
   amax_grid = std::max(1, amax_grid);
   if (amax_grid > kMaxPartials)
@@ -507,17 +668,67 @@ extern "C" nvfp4_status nvfp4_quantize_noalloc(const void* x, int64_t rows, int6
   p.scales = static_cast<uint8_t*>(scales);
   p.global_scale = global_scale;
   p.partials = partials;
+  p.alpha_in = nullptr;
   p.ws = ws;
   p.nparts = amax_grid;
   p.f6 = fp8_max * 6.0f;
   p.ntasks = static_cast<uint32_t>(ntasks);
   p.kgroups = static_cast<uint32_t>(K / 64);
-  const int64_t want = (ntasks + kQuantWarps - 1) / kQuantWarps;
-  const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(want, static_cast<int64_t>(sms) * 8)));
-  if (mode == NVFP4_MODE_SIX) e = launch_quantize<false, kRuleMax>(grid, p, s);
-  else if (rule == NVFP4_RULE_MAX) e = launch_quantize<true, kRuleMax>(grid, p, s);
-  else if (rule == NVFP4_RULE_MAE) e = launch_quantize<true, kRuleMae>(grid, p, s);
-  else e = launch_quantize<true, kRuleMse>(grid, p, s);
+  e = launch_quantize_kernel(mode, rule, sms, p, s);
+  if (e != cudaSuccess) return cuda_status(e, "quantize_kernel launch");
+  return NVFP4_OK;
+}
+
+// ------------------------------------------------------ static tensor scale --
+// nvfp4_quantize with a caller-supplied alpha (e.g. calibrated offline): the
+// amax pass and its HBM read of x are skipped, one kernel launch.
+
+extern "C" nvfp4_status nvfp4_quantize_with_scale(const void* x, int64_t rows, int64_t K, int64_t ldx,
+                                                  int mode, int rule, const float* global_scale,
+                                                  void* codes, void* scales, void* workspace,
+                                                  size_t workspace_bytes, void* stream) {
+  if (!x || !codes || !scales || !global_scale || !workspace)
+    return set_error(NVFP4_ERR_INVALID_ARG, "nvfp4_quantize_with_scale: null pointer argument");
+  if (rows < 1 || K < 64 || K % 64 != 0)
+    return set_error(NVFP4_ERR_INVALID_ARG,
+                     "nvfp4_quantize_with_scale: need rows >= 1 and K a positive multiple of 64");
+  if (ldx < K || ldx % 8 != 0)
+    return set_error(NVFP4_ERR_INVALID_ARG, "nvfp4_quantize_with_scale: need ldx >= K and ldx %% 8 == 0");
+  if (mode != NVFP4_MODE_SIX && mode != NVFP4_MODE_FOUR_OVER_SIX)
+    return set_error(NVFP4_ERR_INVALID_ARG, "nvfp4_quantize_with_scale: unknown mode %d", mode);
+  if (rule != NVFP4_RULE_MAX && rule != NVFP4_RULE_MAE && rule != NVFP4_RULE_MSE)
+    return set_error(NVFP4_ERR_INVALID_ARG, "nvfp4_quantize_with_scale: unknown rule %d", rule);
+  if (!aligned16(x) || !aligned16(codes) || !aligned16(scales) || !aligned16(workspace) ||
+      (reinterpret_cast<uintptr_t>(global_scale) & 3u))
+    return set_error(NVFP4_ERR_INVALID_ARG, "nvfp4_quantize_with_scale: misaligned buffer");
+  if (workspace_bytes < sizeof(WorkspaceHeader))
+    return set_error(NVFP4_ERR_INVALID_ARG, "nvfp4_quantize_with_scale: workspace too small");
+  const int64_t row_blocks = (rows + 127) / 128;
+  const int64_t ntasks = row_blocks * 16 * (K / 64);
+  if (ntasks >= 0x80000000ll || rows * ldx > (1ll << 40))
+    return set_error(NVFP4_ERR_INVALID_ARG, "nvfp4_quantize_with_scale: tensor too large");
+  int dev = 0, sms = 0;
+  nvfp4_status st = check_device(&dev, &sms);
+  if (st != NVFP4_OK) return st;
+  QuantParams p;
+  p.x = static_cast<const uint16_t*>(x);
+  p.rows = rows;
+  p.K = K;
+  p.ldx = ldx;
+  p.codes = static_cast<uint8_t*>(codes);
+  p.scales = static_cast<uint8_t*>(scales);
+  p.global_scale = nullptr;
+  p.partials = nullptr;
+  p.alpha_in = global_scale;
+  p.ws = static_cast<WorkspaceHeader*>(workspace);
+  p.nparts = 0;
+  p.f6 = 0.0f;
+  p.ntasks = static_cast<uint32_t>(ntasks);
+  p.kgroups = static_cast<uint32_t>(K / 64);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemsetAsync(workspace, 0, 2 * sizeof(uint32_t), s);  // status, detail
+  if (e != cudaSuccess) return cuda_status(e, "nvfp4_quantize_with_scale: status reset");
+  e = launch_quantize_kernel(mode, rule, sms, p, s);
   if (e != cudaSuccess) return cuda_status(e, "quantize_kernel launch");
   return NVFP4_OK;
 }
