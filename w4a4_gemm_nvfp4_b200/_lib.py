@@ -178,7 +178,9 @@ def quantize(x, mode: str = "six", rule: str = "max", fp8_max: float | None = No
 
     With ``global_scale`` (a float32 CUDA tensor of one element, e.g. a
     calibrated alpha) the tensor scale is taken from it instead of the
-    tensor's amax; ``fp8_max`` is then unused.
+    tensor's amax; ``fp8_max`` is then unused.  A new result refers to that
+    tensor as its ``global_scale`` (no copy); into an existing ``out`` it is
+    copied unless it already is ``out.global_scale``.
     """
     import torch
 
@@ -196,11 +198,13 @@ def quantize(x, mode: str = "six", rule: str = "max", fp8_max: float | None = No
         out = NVFP4Tensor(
             codes=torch.empty(rows, K // 2, dtype=torch.uint8, device=dev),
             scales=torch.empty(max(1, nvfp4_scales_bytes(rows, K)), dtype=torch.uint8, device=dev),
-            global_scale=torch.empty(1, dtype=torch.float32, device=dev),
+            global_scale=(torch.empty(1, dtype=torch.float32, device=dev) if global_scale is None
+                          else global_scale.reshape(1)),
             workspace=torch.empty(nvfp4_quantize_workspace_bytes(rows, K), dtype=torch.uint8, device=dev),
             rows=rows, K=K)
     if global_scale is not None:
-        out.global_scale.copy_(global_scale.reshape(1))
+        if out.global_scale.data_ptr() != global_scale.data_ptr():
+            out.global_scale.copy_(global_scale.reshape(1))
         st = nvfp4_quantize_with_scale(x.data_ptr(), rows, K, x.stride(0), MODES[mode], RULES[rule],
                                        out.global_scale.data_ptr(), out.codes.data_ptr(),
                                        out.scales.data_ptr(), out.workspace.data_ptr(),

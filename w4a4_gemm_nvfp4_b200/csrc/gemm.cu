@@ -25,26 +25,31 @@
 //   warp 1      TMEM allocation (pair) and, in the leader CTA only, the MMA
 //               issuer: per K step one tcgen05.cp.cta_group::2 of the A scale
 //               atom and two of the B atoms into TMEM (replicated over the
-//               four 32-lane subpartitions), then the MMA; commits free the
-//               stage in both CTAs and finally the accumulator.  The whole
+//               four 32-lane subpartitions), then that K step's MMA; commits
+//               free the stage in both CTAs and finally the accumulator.  The whole
 //               warp runs the loop converged and one elected lane issues each
 //               tcgen05 instruction (issuing them from a lone lane of a
 //               diverged warp is several times slower).
-//   warps 2..5  epilogue (both CTAs): tcgen05.ld 32 lanes x 64 columns,
-//               multiply by alpha_A*alpha_B, convert, store.
-// TMEM (512 columns per CTA): two accumulators that share two 64-column
-// subtiles, buffer 0 = columns 0..255 and buffer 1 = columns 128..383, and
-// one stage of scales at 384..431 (per K step: 4 columns of A scales, 8 of B
+//   warps 2..5  epilogue (both CTAs): per 64-column subtile, tcgen05.ld of 32
+//               lanes x 64 columns, multiply by alpha_A*alpha_B, convert,
+//               write the 32 x 128-byte block to a staging buffer in shared
+//               memory (128-byte swizzle) and TMA-store it (two buffers per
+//               warp, bulk-group waits before reuse); when Y's base or row
+//               pitch is not 16-byte aligned, direct stores of one row per lane.
+// TMEM (512 columns per CTA): two accumulators that share one 64-column
+// subtile, buffer 0 = columns 0..255 and buffer 1 = columns 192..447, and
+// one stage of scales at 448..495 (per K step: 4 columns of A scales, 8 of B
 // scales); the copies and MMAs of one thread execute in order, so a single
-// buffer suffices.  The epilogue loads the shared columns 128..255 first, releases
-// them to the next tile's MMAs at once, and stores the rest of tile i while
-// the mainloop of tile i+1 runs.
+// buffer suffices.  The epilogue loads the shared columns 192..255 first,
+// releases them to the next tile's MMAs at once, and stores the rest of tile
+// i while the mainloop of tile i+1 runs.
 // Every wait is bounded by a deadline on %globaltimer; a wait that runs out
 // records NVFP4_ERR_TIMEOUT in the workspace, raises a CTA-wide abort flag,
 // and every role drains what it has in flight before TMEM is freed.
 #include <cuda_bf16.h>
 
 #include <algorithm>
+#include <cstring>
 #include <mutex>
 
 #include "common.cuh"
@@ -72,11 +77,15 @@ constexpr uint32_t OFF_BAR = OFF_SFB + STAGES * SFB_STAGE;
 // full[], empty[], acc_full, acc_free, drain
 constexpr uint32_t NUM_BARS = 2 * STAGES + 3;
 constexpr uint32_t OFF_MISC = OFF_BAR + NUM_BARS * 8;
-constexpr uint32_t SMEM_BYTES = OFF_MISC + 16 + 1024;  // + alignment slack
+// epilogue staging for TMA stores: per epilogue warp two 32-row x 128-byte
+// buffers (1024-byte aligned for the 128-byte swizzle)
+constexpr uint32_t STG_BYTES = 32 * 128;
+constexpr uint32_t OFF_STG = (OFF_MISC + 16 + 1023) & ~1023u;
+constexpr uint32_t SMEM_BYTES = OFF_STG + 4 * 2 * STG_BYTES + 1024;  // + alignment slack
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t EPI_N = 64;                    // epilogue subtile (columns)
-constexpr uint32_t TM_ACC1 = 256 - 2 * EPI_N;     // buffer 1 starts on buffer 0's last two subtiles
-constexpr uint32_t TM_SF = TM_ACC1 + 256;         // 384: scale ring
+constexpr uint32_t TM_ACC1 = 256 - EPI_N;         // buffer 1 starts on buffer 0's last subtile
+constexpr uint32_t TM_SF = TM_ACC1 + 256;         // 448: scales
 constexpr uint32_t TM_SFA = TM_SF;                // 4 columns per K step
 constexpr uint32_t TM_SFB = TM_SF + 16;           // 8 columns per K step
 static_assert(TM_SFB + 32 <= TMEM_COLS, "scales must fit after the accumulators");
@@ -137,6 +146,12 @@ __device__ __forceinline__ void tmem_wait_ld() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
+                                             uint32_t d) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d)
+               : "memory");
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<const uint32_t*>(&v);
@@ -159,6 +174,7 @@ struct GemmParams {
   uint32_t num_tiles;     // ceil(M / 256) * n_tiles
   int out_fp32;
   int vec_store;          // rows of Y start 16-byte aligned: vector stores
+  int tma_store;          // Y base and row pitch 16-byte aligned: TMA stores through shared memory
   uint64_t timeout_ns;
   int debug_flags;        // bit 0: never issue the first stage's copies (timeout test)
 };
@@ -173,7 +189,7 @@ __device__ __forceinline__ void record_timeout(const GemmParams& p, volatile int
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const __grid_constant__ CUtensorMap tmSFA, const __grid_constant__ CUtensorMap tmSFB,
-                const GemmParams p) {
+                const __grid_constant__ CUtensorMap tmY, const GemmParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -206,6 +222,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     prefetch_tensormap(&tmB);
     prefetch_tensormap(&tmSFA);
     prefetch_tensormap(&tmSFB);
+    if (p.tma_store) prefetch_tensormap(&tmY);
   }
   if (warp == 1) {
     tmem_alloc_pair(smem_u32(tmem_slot), TMEM_COLS);
@@ -303,14 +320,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           const uint32_t sa = sbase + OFF_A + s * A_STAGE;
           const uint32_t sb = sbase + OFF_B + s * B_STAGE;
           if (elect_one()) {
+            // Each K step's scale copies go right before its MMA: an MMA
+            // waits for the copies issued ahead of it, while copies issued
+            // after an MMA run alongside it.
             for (uint32_t j = 0; j < nk; ++j) {
               tmem_copy_scales_pair(tmem + TM_SFA + 4 * j, scale_desc(sfa + 512 * j));
               tmem_copy_scales_pair(tmem + TM_SFB + 8 * j, scale_desc(sfb + 512 * j));
               tmem_copy_scales_pair(tmem + TM_SFB + 8 * j + 4, scale_desc(sfb + 2048 + 512 * j));
-            }
-            for (uint32_t j = 0; j < nk; ++j)
               mma_nvf4_pair(acc, operand_desc(sa + 32 * j), operand_desc(sb + 32 * j),
                             tmem + TM_SFA + 4 * j, tmem + TM_SFB + 8 * j, (kt | j) != 0);
+            }
             tc_commit_pair(own_empty + 8 * s);
             tc_commit_pair(peer_empty + 8 * s);
           }
@@ -345,6 +364,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       while (sg + 1 < p.nseg && col >= p.seg_end[sg]) ++sg;
       return __fmul_rn(alpha_a, __ldg(p.b_global + sg));
     };
+    // this warp's two staging buffers; lane 0 issues (and waits for) every
+    // TMA store of the warp, so the bulk groups it waits on are its own
+    const uint32_t stg0 = sbase + OFF_STG + static_cast<uint32_t>(quad) * 2 * STG_BYTES;
+    uint32_t nstore = 0;
     uint32_t local = 0;
     for (uint32_t tile = pair; tile < p.num_tiles; tile += npairs, ++local) {
       bool ok = mbar_wait_bounded(bar_acc_full, local & 1u, abort, deadline);
@@ -356,63 +379,116 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const int m0 = static_cast<int>(tile / p.n_tiles) * BM;
       const int n0 = static_cast<int>(tile % p.n_tiles) * BN;
-      const int row = m0 + static_cast<int>(rank) * HALF + quad * 32 + lane;
+      const int row0 = m0 + static_cast<int>(rank) * HALF + quad * 32;  // this warp's first row
+      const int row = row0 + lane;
       const bool odd = (local & 1u) != 0;
       const uint32_t acc = tmem + lane_base + (odd ? TM_ACC1 : 0u);
-      // Buffer 0 is drained from its last subtiles down, buffer 1 from its
-      // first subtiles up: either way the shared columns 128..255 go first,
-      // loaded together and released before anything is stored.
-      for (int half = 0; half < 2; ++half) {
-        const int sub0 = odd ? 2 * half : 2 - 2 * half;  // first of the two subtiles
-        uint32_t r[128];
-        tmem_ld32(acc + sub0 * EPI_N, r);
-        tmem_ld32(acc + sub0 * EPI_N + 32, r + 32);
-        tmem_ld32(acc + sub0 * EPI_N + 64, r + 64);
-        tmem_ld32(acc + sub0 * EPI_N + 96, r + 96);
+      // Buffer 0 is drained from its last subtile, buffer 1 from its first:
+      // either way the shared columns 192..255 go first and are released
+      // before anything is stored.
+      for (int si = 0; si < 4; ++si) {
+        const int sub = odd ? si : (si == 0 ? 3 : si - 1);
+        uint32_t r[64];
+        tmem_ld32(acc + sub * EPI_N, r);
+        tmem_ld32(acc + sub * EPI_N + 32, r + 32);
         tmem_wait_ld();
-        if (half == 0) {
+        if (si == 0) {
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive_cluster(acc_free_leader);
         }
-        const int col0 = n0 + sub0 * static_cast<int>(EPI_N);
-        if (row >= p.M || col0 >= p.N) continue;
-        const float ab0 = segment_scale(col0);                                  // r[0..63]
-        const float ab1 = p.nseg == 1 ? ab0 : segment_scale(col0 + static_cast<int>(EPI_N));  // r[64..127]
-        const bool full = p.vec_store && col0 + 2 * static_cast<int>(EPI_N) <= p.N;
+        const int col0 = n0 + sub * static_cast<int>(EPI_N);
+        if (row0 >= p.M || col0 >= p.N) continue;  // warp-uniform
+        const float ab = segment_scale(col0);
+        if (p.tma_store) {
+          if (p.out_fp32) {
+            // 64 fp32 columns = two 32-column boxes, one per staging buffer
+            if (lane == 0) bulk_wait_group_read<0>();
+            __syncwarp();
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const uint32_t buf = stg0 + h * STG_BYTES + lane * 128;
+#pragma unroll
+              for (int c = 0; c < 8; ++c) {
+                const int i = h * 32 + c * 4;
+                st_shared_v4(buf + ((c ^ (lane & 7)) << 4),
+                             __float_as_uint(__uint_as_float(r[i]) * ab),
+                             __float_as_uint(__uint_as_float(r[i + 1]) * ab),
+                             __float_as_uint(__uint_as_float(r[i + 2]) * ab),
+                             __float_as_uint(__uint_as_float(r[i + 3]) * ab));
+              }
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              tma_store_2d(&tmY, stg0, col0, row0);
+              tma_store_2d(&tmY, stg0 + STG_BYTES, col0 + 32, row0);
+              bulk_commit_group();
+            }
+          } else {
+            const uint32_t stg = stg0 + (nstore & 1u) * STG_BYTES;
+            if (lane == 0) bulk_wait_group_read<1>();  // the store that used this buffer is done reading
+            __syncwarp();
+            const uint32_t buf = stg + lane * 128;
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+              const int i = c * 8;
+              st_shared_v4(buf + ((c ^ (lane & 7)) << 4),
+                           pack_bf16x2(__uint_as_float(r[i]) * ab, __uint_as_float(r[i + 1]) * ab),
+                           pack_bf16x2(__uint_as_float(r[i + 2]) * ab, __uint_as_float(r[i + 3]) * ab),
+                           pack_bf16x2(__uint_as_float(r[i + 4]) * ab, __uint_as_float(r[i + 5]) * ab),
+                           pack_bf16x2(__uint_as_float(r[i + 6]) * ab, __uint_as_float(r[i + 7]) * ab));
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              tma_store_2d(&tmY, stg, col0, row0);
+              bulk_commit_group();
+            }
+            ++nstore;
+          }
+          continue;
+        }
+        // direct stores (Y not 16-byte aligned or pitched): one row per lane
+        if (row >= p.M) continue;
+        const bool full = p.vec_store && col0 + static_cast<int>(EPI_N) <= p.N;
         if (p.out_fp32) {
           float* dst = static_cast<float*>(p.y) + static_cast<int64_t>(row) * p.ldy + col0;
           if (full) {
 #pragma unroll
-            for (int i = 0; i < 128; i += 4)
+            for (int i = 0; i < 64; i += 4)
               *reinterpret_cast<float4*>(dst + i) =
-                  make_float4(__uint_as_float(r[i]) * (i < 64 ? ab0 : ab1), __uint_as_float(r[i + 1]) * (i < 64 ? ab0 : ab1),
-                              __uint_as_float(r[i + 2]) * (i < 64 ? ab0 : ab1), __uint_as_float(r[i + 3]) * (i < 64 ? ab0 : ab1));
+                  make_float4(__uint_as_float(r[i]) * ab, __uint_as_float(r[i + 1]) * ab,
+                              __uint_as_float(r[i + 2]) * ab, __uint_as_float(r[i + 3]) * ab);
           } else {
 #pragma unroll
-            for (int i = 0; i < 128; ++i)
-              if (col0 + i < p.N) dst[i] = __uint_as_float(r[i]) * (i < 64 ? ab0 : ab1);
+            for (int i = 0; i < 64; ++i)
+              if (col0 + i < p.N) dst[i] = __uint_as_float(r[i]) * ab;
           }
         } else {
           __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(p.y) + static_cast<int64_t>(row) * p.ldy + col0;
           if (full) {
 #pragma unroll
-            for (int i = 0; i < 128; i += 8) {
+            for (int i = 0; i < 64; i += 8) {
               uint4 v;
-              v.x = pack_bf16x2(__uint_as_float(r[i]) * (i < 64 ? ab0 : ab1), __uint_as_float(r[i + 1]) * (i < 64 ? ab0 : ab1));
-              v.y = pack_bf16x2(__uint_as_float(r[i + 2]) * (i < 64 ? ab0 : ab1), __uint_as_float(r[i + 3]) * (i < 64 ? ab0 : ab1));
-              v.z = pack_bf16x2(__uint_as_float(r[i + 4]) * (i < 64 ? ab0 : ab1), __uint_as_float(r[i + 5]) * (i < 64 ? ab0 : ab1));
-              v.w = pack_bf16x2(__uint_as_float(r[i + 6]) * (i < 64 ? ab0 : ab1), __uint_as_float(r[i + 7]) * (i < 64 ? ab0 : ab1));
+              v.x = pack_bf16x2(__uint_as_float(r[i]) * ab, __uint_as_float(r[i + 1]) * ab);
+              v.y = pack_bf16x2(__uint_as_float(r[i + 2]) * ab, __uint_as_float(r[i + 3]) * ab);
+              v.z = pack_bf16x2(__uint_as_float(r[i + 4]) * ab, __uint_as_float(r[i + 5]) * ab);
+              v.w = pack_bf16x2(__uint_as_float(r[i + 6]) * ab, __uint_as_float(r[i + 7]) * ab);
               *reinterpret_cast<uint4*>(dst + i) = v;
             }
           } else {
 #pragma unroll
-            for (int i = 0; i < 128; ++i)
-              if (col0 + i < p.N) dst[i] = __float2bfloat16_rn(__uint_as_float(r[i]) * (i < 64 ? ab0 : ab1));
+            for (int i = 0; i < 64; ++i)
+              if (col0 + i < p.N) dst[i] = __float2bfloat16_rn(__uint_as_float(r[i]) * ab);
           }
         }
       }
     }
+    // the staging buffers must not be released (CTA exit) while a TMA store
+    // still reads them
+    if (lane == 0) bulk_wait_group_all();
+    __syncwarp();
   }
 
   tc_fence_before();
@@ -461,6 +537,23 @@ nvfp4_status make_code_map(CUtensorMap* map, const void* base, int64_t rows, int
 // 3D uint32 tensor map over a swizzled scale buffer seen as
 // [row blocks][K groups][128 words]: one 512-byte atom per (row block, K
 // group); boxes of 4 K groups x `blocks` row blocks, zero-filled past the end.
+// 2D tensor map over Y [M, N] (row pitch ldy elements) for the epilogue's TMA
+// stores: boxes of 128 bytes x 32 rows with the 128-byte swizzle.
+nvfp4_status make_output_map(CUtensorMap* map, void* y, int64_t M, int64_t N, int64_t ldy, bool fp32) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc) return set_error(NVFP4_ERR_CUDA, "cuTensorMapEncodeTiled entry point not available");
+  const cuuint64_t esize = fp32 ? 4 : 2;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(M)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(ldy) * esize};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(128 / esize), 32};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(map, fp32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, y, dims,
+                   strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return set_error(NVFP4_ERR_CUDA, "cuTensorMapEncodeTiled(Y) failed (%d)", (int)r);
+  return NVFP4_OK;
+}
+
 nvfp4_status make_scale_map(CUtensorMap* map, const void* base, int64_t rows, int64_t K,
                             uint32_t blocks) {
   EncodeTiledFn enc = get_encode_fn();
@@ -570,11 +663,15 @@ nvfp4_status gemm_impl(const char* fn, const void* a_codes, const void* a_scales
   p.num_tiles = static_cast<uint32_t>(num_tiles);
   p.out_fp32 = out_dtype == NVFP4_OUT_FP32;
   p.vec_store = aligned16(y) && ((ldy * (p.out_fp32 ? 4 : 2)) % 16 == 0);
+  p.tma_store = p.vec_store;
+  CUtensorMap ty;
+  std::memset(&ty, 0, sizeof(ty));
+  if (p.tma_store && (st = make_output_map(&ty, y, M, N, ldy, p.out_fp32 != 0)) != NVFP4_OK) return st;
   p.timeout_ns = g_timeout_ns;
   p.debug_flags = g_debug_flags;
   // one CTA pair per two SMs, never more pairs than tiles
   const int64_t pairs = std::max<int64_t>(1, std::min<int64_t>(num_tiles, sms / 2));
-  gemm_kernel<<<static_cast<unsigned>(2 * pairs), kThreads, SMEM_BYTES, s>>>(ta, tb, tsa, tsb, p);
+  gemm_kernel<<<static_cast<unsigned>(2 * pairs), kThreads, SMEM_BYTES, s>>>(ta, tb, tsa, tsb, ty, p);
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_status(e, "gemm_kernel launch");
   return NVFP4_OK;

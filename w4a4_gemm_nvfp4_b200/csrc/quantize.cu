@@ -154,33 +154,31 @@ __device__ __forceinline__ uint32_t e2m1x2_round(float hi, float lo, float& qlo,
   return byte;
 }
 
-// Packed binary32 pairs (one IEEE RNE operation per lane, like the scalar
-// instruction on each lane).
+// Packed binary32 pairs held in one 64-bit register pair (one IEEE RNE
+// operation per lane, like the scalar instruction on each lane).
 struct f2 {
-  float a, b;
+  uint64_t v;
+  __device__ __forceinline__ float a() const { return __uint_as_float(static_cast<uint32_t>(v)); }
+  __device__ __forceinline__ float b() const { return __uint_as_float(static_cast<uint32_t>(v >> 32)); }
 };
+__device__ __forceinline__ f2 make_f2(float a, float b) {
+  f2 r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r.v) : "f"(a), "f"(b));
+  return r;
+}
 __device__ __forceinline__ f2 mul2(f2 x, f2 y) {
   f2 r;
-  asm("{\n\t.reg .b64 p, q, o;\n\tmov.b64 p, {%2, %3};\n\tmov.b64 q, {%4, %5};\n\t"
-      "mul.rn.f32x2 o, p, q;\n\tmov.b64 {%0, %1}, o;\n\t}"
-      : "=f"(r.a), "=f"(r.b)
-      : "f"(x.a), "f"(x.b), "f"(y.a), "f"(y.b));
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r.v) : "l"(x.v), "l"(y.v));
   return r;
 }
 __device__ __forceinline__ f2 fma2(f2 x, f2 y, f2 z) {
   f2 r;
-  asm("{\n\t.reg .b64 p, q, s, o;\n\tmov.b64 p, {%2, %3};\n\tmov.b64 q, {%4, %5};\n\t"
-      "mov.b64 s, {%6, %7};\n\tfma.rn.f32x2 o, p, q, s;\n\tmov.b64 {%0, %1}, o;\n\t}"
-      : "=f"(r.a), "=f"(r.b)
-      : "f"(x.a), "f"(x.b), "f"(y.a), "f"(y.b), "f"(z.a), "f"(z.b));
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r.v) : "l"(x.v), "l"(y.v), "l"(z.v));
   return r;
 }
 __device__ __forceinline__ f2 add2(f2 x, f2 y) {
   f2 r;
-  asm("{\n\t.reg .b64 p, q, o;\n\tmov.b64 p, {%2, %3};\n\tmov.b64 q, {%4, %5};\n\t"
-      "add.rn.f32x2 o, p, q;\n\tmov.b64 {%0, %1}, o;\n\t}"
-      : "=f"(r.a), "=f"(r.b)
-      : "f"(x.a), "f"(x.b), "f"(y.a), "f"(y.b));
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r.v) : "l"(x.v), "l"(y.v));
   return r;
 }
 
@@ -195,13 +193,13 @@ enum { kRuleMax = 0, kRuleMae = 1, kRuleMse = 2 };
 // 16 values are held as pairs p[j] = (x_j, x_{j+8}), j < 8; codes byte j holds
 // elements 2j, 2j+1 (low nibble first).
 __device__ __forceinline__ uint2 candidate_codes(const f2 p[8], float r) {
-  const f2 rr = {r, r};
+  const f2 rr = make_f2(r, r);
   uint32_t bytes[8];
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
     const f2 v0 = mul2(p[2 * j], rr), v1 = mul2(p[2 * j + 1], rr);
-    bytes[j] = e2m1x2_encode(v1.a, v0.a);
-    bytes[j + 4] = e2m1x2_encode(v1.b, v0.b);
+    bytes[j] = e2m1x2_encode(v1.a(), v0.a());
+    bytes[j + 4] = e2m1x2_encode(v1.b(), v0.b());
   }
   return make_uint2(bytes[0] | (bytes[1] << 8) | (bytes[2] << 16) | (bytes[3] << 24),
                     bytes[4] | (bytes[5] << 8) | (bytes[6] << 16) | (bytes[7] << 24));
@@ -215,8 +213,8 @@ __device__ __forceinline__ uint2 candidate_codes(const f2 p[8], float r) {
 //   (w_0 + w_1, w_2 + w_3)                = (z_0, z_1),    then z_0 + z_1.
 template <int RULE>
 __device__ __forceinline__ float candidate(const f2 p[8], float d, float r, uint2& codes) {
-  const f2 rr = {r, r};
-  const f2 nd = {-d, -d};
+  const f2 rr = make_f2(r, r);
+  const f2 nd = make_f2(-d, -d);
   f2 v[8];
 #pragma unroll
   for (int j = 0; j < 8; ++j) v[j] = mul2(p[j], rr);
@@ -226,21 +224,21 @@ __device__ __forceinline__ float candidate(const f2 p[8], float d, float r, uint
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
     // byte j: elements 2j, 2j+1 (first half); byte j+4: elements 2j+8, 2j+9
-    bytes[j] = e2m1x2_round(v[2 * j + 1].a, v[2 * j].a, q[2 * j], q[2 * j + 1]);
-    bytes[j + 4] = e2m1x2_round(v[2 * j + 1].b, v[2 * j].b, q[2 * j + 8], q[2 * j + 9]);
+    bytes[j] = e2m1x2_round(v[2 * j + 1].a(), v[2 * j].a(), q[2 * j], q[2 * j + 1]);
+    bytes[j + 4] = e2m1x2_round(v[2 * j + 1].b(), v[2 * j].b(), q[2 * j + 8], q[2 * j + 9]);
   }
   codes.x = bytes[0] | (bytes[1] << 8) | (bytes[2] << 16) | (bytes[3] << 24);
   codes.y = bytes[4] | (bytes[5] << 8) | (bytes[6] << 16) | (bytes[7] << 24);
   // e = fma(-q, d, x), paired like p
   f2 e[8];
 #pragma unroll
-  for (int j = 0; j < 8; ++j) e[j] = fma2(f2{q[j], q[j + 8]}, nd, p[j]);
+  for (int j = 0; j < 8; ++j) e[j] = fma2(make_f2(q[j], q[j + 8]), nd, p[j]);
   if (RULE == kRuleMax) {
     float m0 = 0.0f, m1 = 0.0f;
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
-      m0 = fmaxf(m0, fabsf(e[j].a));
-      m1 = fmaxf(m1, fabsf(e[j].b));
+      m0 = fmaxf(m0, fabsf(e[j].a()));
+      m1 = fmaxf(m1, fabsf(e[j].b()));
     }
     return fmaxf(m0, m1);
   }
@@ -250,12 +248,12 @@ __device__ __forceinline__ float candidate(const f2 p[8], float d, float r, uint
     for (int j = 0; j < 8; ++j) t[j] = mul2(e[j], e[j]);
   } else {
 #pragma unroll
-    for (int j = 0; j < 8; ++j) t[j] = f2{fabsf(e[j].a), fabsf(e[j].b)};
+    for (int j = 0; j < 8; ++j) t[j] = make_f2(fabsf(e[j].a()), fabsf(e[j].b()));
   }
   const f2 u0 = add2(t[0], t[1]), u1 = add2(t[2], t[3]), u2 = add2(t[4], t[5]), u3 = add2(t[6], t[7]);
   const f2 w0 = add2(u0, u1), w1 = add2(u2, u3);
   const f2 z = add2(w0, w1);
-  return __fadd_rn(z.a, z.b);
+  return __fadd_rn(z.a(), z.b());
 }
 
 // Per-call constants of the block step.  The scale quotient b / (alpha*Q) must
@@ -278,19 +276,21 @@ __device__ __forceinline__ bool needs_exact_quotient(float q) {
 // Quantize one block held as 8 words of bf16 pairs (element 2j in the low
 // half of word j).  dr[c] = (d, r) of E4M3 scale code c: d = val(c) * alpha,
 // r = 1/d (0 if infinite).
+// Returns the block's max |x| bit pattern (0x7F80 and above: Inf or NaN).
 template <bool FOUR_OVER_SIX, int RULE>
-__device__ __forceinline__ void quantize_block(const uint4& lo, const uint4& hi, const BlockConsts& k,
-                                               const float2* dr, uint2& codes, uint32_t& scale) {
+__device__ __forceinline__ uint32_t quantize_block(const uint4& lo, const uint4& hi, const BlockConsts& k,
+                                                   const float2* dr, uint2& codes, uint32_t& scale) {
   const uint32_t w[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
   uint32_t m = absmax4(lo, 0u);
   m = absmax4(hi, m);
-  const float b = __uint_as_float(max(m & 0xFFFFu, m >> 16) << 16);
+  const uint32_t bbits = max(m & 0xFFFFu, m >> 16);
+  const float b = __uint_as_float(bbits << 16);
   // p[j] = (x_j, x_{j+8}): x_2i is the low half of word i, x_2i+1 the high half
   f2 p[8];
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    p[2 * i] = f2{__uint_as_float(w[i] << 16), __uint_as_float(w[i + 4] << 16)};
-    p[2 * i + 1] = f2{__uint_as_float(w[i] & 0xFFFF0000u), __uint_as_float(w[i + 4] & 0xFFFF0000u)};
+    p[2 * i] = make_f2(__uint_as_float(w[i] << 16), __uint_as_float(w[i + 4] << 16));
+    p[2 * i + 1] = make_f2(__uint_as_float(w[i] & 0xFFFF0000u), __uint_as_float(w[i + 4] & 0xFFFF0000u));
   }
   float s6raw = __fmul_rn(b, k.inv6);
   float s4raw = FOUR_OVER_SIX ? __fmul_rn(b, k.inv4) : 0.0f;
@@ -303,7 +303,7 @@ __device__ __forceinline__ void quantize_block(const uint4& lo, const uint4& hi,
   if (!FOUR_OVER_SIX) {
     codes = candidate_codes(p, dr6.y);
     scale = sc & 0xFFu;
-    return;
+    return bbits;
   }
   const float2 dr4 = dr[sc >> 8];
   uint2 c6, c4;
@@ -312,6 +312,7 @@ __device__ __forceinline__ void quantize_block(const uint4& lo, const uint4& hi,
   const bool pick4 = E4 < E6;  // ties keep scale 6
   codes = pick4 ? c4 : c6;
   scale = pick4 ? (sc >> 8) : (sc & 0xFFu);
+  return bbits;
 }
 
 struct QuantParams {
@@ -384,68 +385,87 @@ __global__ void __launch_bounds__(kQuantThreads)
   // ---- lane -> (row, 16-element block) inside a warp task ----
   // task = (row_block * 16 + piece) * kgroups + kgroup; a piece is 32 bytes of
   // a 512-byte scale atom: atom byte o = 32*piece + lane holds the scale of
-  // row (o/16) + 32*((o/4)%4) and K-block o%4 of the atom.  Each warp walks
-  // its tasks with a fixed stride, loading the next task's block while it
-  // quantizes the current one.
+  // row (o/16) + 32*((o/4)%4) and K-block o%4 of the atom.  Each CTA takes
+  // one contiguous run of tasks and its warps interleave over it (warp w:
+  // tasks start + w, start + w + 8, ...), so the CTA streams 8 neighbouring
+  // K groups (1 KB of each of 8 rows) at a time and a warp's next task is
+  // 8 K groups on: the source, code and scale pointers step by 1 KB, 256 B
+  // and 4 KB, except where a run crosses into the next piece.  Each warp
+  // loads its next task's block while it quantizes the current one.
   const int row_in_atom = ((lane >> 2) & 3) * 32 + (lane >> 4);
   const int kb_in_group = lane & 3;
-  const uint32_t stride = gridDim.x * kQuantWarps;
-  const uint32_t stride_hi = stride / p.kgroups, stride_lo = stride % p.kgroups;
+  const uint32_t per_cta = (p.ntasks + gridDim.x - 1) / gridDim.x;
+  const uint32_t cta_begin = blockIdx.x * per_cta;  // < 2^31 + 2^14: no wrap-around
+  const uint32_t task_end = min(cta_begin + per_cta, p.ntasks);
+  uint32_t task = cta_begin + warp;
+  if (task >= task_end) return;
   const int64_t half_k = p.K / 2;
-  uint32_t task = blockIdx.x * kQuantWarps + warp;
+  const bool step_in_row = p.kgroups >= kQuantWarps;  // a step of 8 crosses at most one piece
   uint32_t kg = task % p.kgroups, t2 = task / p.kgroups;
-  int64_t row = static_cast<int64_t>(t2 >> 4) * 128 + row_in_atom + 2 * (t2 & 15u);
+
+  // pointers of the lane's block in task (t2, kg)
+  const uint4* src;
+  uint2* dst;
+  uint8_t* sdst;
+  bool row_ok;
+  auto locate = [&](uint32_t t2_, uint32_t kg_) {
+    const int64_t row = static_cast<int64_t>(t2_ >> 4) * 128 + row_in_atom + 2 * (t2_ & 15u);
+    row_ok = row < p.rows;
+    const int64_t kb = static_cast<int64_t>(kg_) * 4 + kb_in_group;
+    src = reinterpret_cast<const uint4*>(p.x + row * p.ldx + kb * 16);
+    dst = reinterpret_cast<uint2*>(p.codes + row * half_k + kb * 8);
+    sdst = p.scales + (static_cast<int64_t>(t2_ >> 4) * p.kgroups + kg_) * 512 + (t2_ & 15u) * 32 + lane;
+  };
+  locate(t2, kg);
   uint4 lo = make_uint4(0, 0, 0, 0), hi = lo;
-  if (task < p.ntasks && row < p.rows) {
-    const uint4* src = reinterpret_cast<const uint4*>(p.x + row * p.ldx + (kg * 4 + kb_in_group) * 16);
+  if (row_ok) {
     lo = ld_stream(src);
     hi = ld_stream(src + 1);
   }
-  while (task < p.ntasks) {
-    // next task (ntasks < 2^31 and stride < 2^16: no wrap-around)
-    const uint32_t ntask = task + stride;
-    uint32_t nkg = kg + stride_lo, nt2 = t2 + stride_hi;
-    if (nkg >= p.kgroups) {
-      nkg -= p.kgroups;
-      ++nt2;
+  for (; task < task_end; task += kQuantWarps) {
+    // next task's pointers and block
+    uint2* cur_dst = dst;
+    uint8_t* cur_sdst = sdst;
+    const bool cur_ok = row_ok;
+    if (!step_in_row) {
+      const uint32_t nt = task + kQuantWarps;
+      kg = nt % p.kgroups;
+      t2 = nt / p.kgroups;
+      locate(t2, kg);
+    } else if ((kg += kQuantWarps) >= p.kgroups) {
+      kg -= p.kgroups;
+      ++t2;
+      locate(t2, kg);
+    } else {
+      src += 8 * kQuantWarps;
+      dst += 4 * kQuantWarps;
+      sdst += 512 * kQuantWarps;
     }
-    const int64_t nrow = static_cast<int64_t>(nt2 >> 4) * 128 + row_in_atom + 2 * (nt2 & 15u);
     uint4 nlo = make_uint4(0, 0, 0, 0), nhi = nlo;
-    if (ntask < p.ntasks && nrow < p.rows) {
-      const uint4* src = reinterpret_cast<const uint4*>(p.x + nrow * p.ldx + (nkg * 4 + kb_in_group) * 16);
+    if (task + kQuantWarps < task_end && row_ok) {
       nlo = ld_stream(src);
       nhi = ld_stream(src + 1);
     }
 
     uint32_t scale = 0;
-    if (row < p.rows) {
+    if (cur_ok) {
       uint2 codes;
-      quantize_block<FOUR_OVER_SIX, RULE>(lo, hi, k, s_dr, codes, scale);
-      const uint32_t bmax = p.alpha_in ? absmax4(hi, absmax4(lo, 0u)) : 0u;
-      if (max(bmax & 0xFFFFu, bmax >> 16) >= 0x7F80u) {
+      const uint32_t bmax = quantize_block<FOUR_OVER_SIX, RULE>(lo, hi, k, s_dr, codes, scale);
+      if (p.alpha_in && bmax >= 0x7F80u) {
         // Inf/NaN in this block (a static alpha skips the tensor check):
         // the block is written as zeros and the call reports it
         codes = make_uint2(0u, 0u);
         scale = 0u;
         p.ws->status = NVFP4_ERR_NONFINITE;
       }
-      *reinterpret_cast<uint2*>(p.codes + row * half_k + (kg * 4 + kb_in_group) * 8) = codes;
+      *cur_dst = codes;
     }
-    p.scales[(static_cast<int64_t>(t2 >> 4) * p.kgroups + kg) * 512 + (t2 & 15u) * 32 + lane] =
-        static_cast<uint8_t>(scale);
-
-    task = ntask;
-    kg = nkg;
-    t2 = nt2;
-    row = nrow;
+    *cur_sdst = static_cast<uint8_t>(scale);
     lo = nlo;
     hi = nhi;
   }
 }
 
-// Grid: one wave of resident CTAs (SMs x CTAs per SM at this kernel's
-// register use), fewer when there are fewer tasks; every warp then walks its
-// tasks with a grid-wide stride.
 template <bool F, int R>
 cudaError_t launch_quantize(int sms, const QuantParams& p, cudaStream_t s) {
   static std::atomic<int> per_sm{0};
