@@ -37,11 +37,13 @@ def test_pr1_operands(recipe):
         assert_quant_equal(q, x, *recipe)
 
 
-def test_strided_rows():
+@pytest.mark.parametrize("ldx_pad", [64, 8])  # 8: rows not 32-byte aligned (two 16-byte loads per block)
+def test_strided_rows(ldx_pad):
     x = workloads.small_operand(200, 256, seed=9).make()
-    q, status = gpu_quantize(x, "four_over_six", "mse", 256.0, ldx_pad=64)
-    assert status == nv.OK
-    assert_quant_equal(q, x, "four_over_six", "mse", 256.0)
+    for recipe in (("four_over_six", "mse", 256.0), ("six", "max", 448.0)):
+        q, status = gpu_quantize(x, *recipe, ldx_pad=ldx_pad)
+        assert status == nv.OK
+        assert_quant_equal(q, x, *recipe)
 
 
 def test_zero_tensor():
