@@ -25,10 +25,11 @@
 //                    every CTA, then makes one HBM pass over x: each lane owns
 //                    one whole 16-element block (two 16-byte loads), so the
 //                    block max and both candidates' errors stay in registers
-//                    with no shuffles; a warp's 32 lanes cover 8 rows x 4
-//                    blocks chosen so that their 32 scale bytes form one
-//                    contiguous 32-byte piece of a 512-byte scale atom, and
-//                    their codes form eight 32-byte row segments.
+//                    with no shuffles.  Blocks are taken in row-major order,
+//                    32 consecutive blocks (1 KB of x) per warp task, so the
+//                    grid sweeps x front to back; every lane writes its 8
+//                    code bytes and its scale byte at that block's place in
+//                    the swizzled scale layout.
 #include <cuda_fp16.h>
 
 #include <algorithm>
@@ -58,6 +59,12 @@ __device__ __forceinline__ uint4 ld_stream(const uint4* p) {
                : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
                : "l"(p));
   return v;
+}
+
+__device__ __forceinline__ void ld_block2(const uint16_t* p, uint4& lo, uint4& hi) {
+  const uint4* q = reinterpret_cast<const uint4*>(p);
+  lo = ld_stream(q);
+  hi = ld_stream(q + 1);
 }
 
 __device__ __forceinline__ uint32_t absmax4(const uint4& v, uint32_t m) {
@@ -382,85 +389,59 @@ __global__ void __launch_bounds__(kQuantThreads)
   }
   __syncthreads();
 
-  // ---- lane -> (row, 16-element block) inside a warp task ----
-  // task = (row_block * 16 + piece) * kgroups + kgroup; a piece is 32 bytes of
-  // a 512-byte scale atom: atom byte o = 32*piece + lane holds the scale of
-  // row (o/16) + 32*((o/4)%4) and K-block o%4 of the atom.  Each CTA takes
-  // one contiguous run of tasks and its warps interleave over it (warp w:
-  // tasks start + w, start + w + 8, ...), so the CTA streams 8 neighbouring
-  // K groups (1 KB of each of 8 rows) at a time and a warp's next task is
-  // 8 K groups on: the source, code and scale pointers step by 1 KB, 256 B
-  // and 4 KB, except where a run crosses into the next piece.  Each warp
-  // loads its next task's block while it quantizes the current one.
-  const int row_in_atom = ((lane >> 2) & 3) * 32 + (lane >> 4);
-  const int kb_in_group = lane & 3;
+  // ---- lane -> (row, 16-element block) ----
+  // Blocks are numbered row-major over the padded rows (a multiple of 128):
+  // g = row * (K/16) + kb.  Warp task t takes blocks 32t .. 32t+31, one per
+  // lane, so a task reads 1 KB of consecutive memory when x is dense; each
+  // CTA takes one contiguous run of tasks and its warps interleave over it
+  // (warp w: tasks start + w, start + w + 8, ...), so the GPU sweeps x front
+  // to back.  Rows past `rows` only write their (zero) scale bytes.  Each
+  // warp loads its next task's block while it quantizes the current one.
+  const uint32_t kbs = static_cast<uint32_t>(p.K / 16);
   const uint32_t per_cta = (p.ntasks + gridDim.x - 1) / gridDim.x;
   const uint32_t cta_begin = blockIdx.x * per_cta;  // < 2^31 + 2^14: no wrap-around
   const uint32_t task_end = min(cta_begin + per_cta, p.ntasks);
   uint32_t task = cta_begin + warp;
   if (task >= task_end) return;
   const int64_t half_k = p.K / 2;
-  const bool step_in_row = p.kgroups >= kQuantWarps;  // a step of 8 crosses at most one piece
-  uint32_t kg = task % p.kgroups, t2 = task / p.kgroups;
+  const uint64_t g0 = static_cast<uint64_t>(task) * 32 + lane;
+  int64_t row = static_cast<int64_t>(g0 / kbs);
+  uint32_t kb = static_cast<uint32_t>(g0 % kbs);
+  const uint32_t step_rows = (32 * kQuantWarps) / kbs, step_kb = (32 * kQuantWarps) % kbs;
+  const int64_t rows_padded = (p.rows + 127) / 128 * 128;
 
-  // pointers of the lane's block in task (t2, kg)
-  const uint4* src;
-  uint2* dst;
-  uint8_t* sdst;
-  bool row_ok;
-  auto locate = [&](uint32_t t2_, uint32_t kg_) {
-    const int64_t row = static_cast<int64_t>(t2_ >> 4) * 128 + row_in_atom + 2 * (t2_ & 15u);
-    row_ok = row < p.rows;
-    const int64_t kb = static_cast<int64_t>(kg_) * 4 + kb_in_group;
-    src = reinterpret_cast<const uint4*>(p.x + row * p.ldx + kb * 16);
-    dst = reinterpret_cast<uint2*>(p.codes + row * half_k + kb * 8);
-    sdst = p.scales + (static_cast<int64_t>(t2_ >> 4) * p.kgroups + kg_) * 512 + (t2_ & 15u) * 32 + lane;
-  };
-  locate(t2, kg);
   uint4 lo = make_uint4(0, 0, 0, 0), hi = lo;
-  if (row_ok) {
-    lo = ld_stream(src);
-    hi = ld_stream(src + 1);
-  }
+  if (row < p.rows) ld_block2(p.x + row * p.ldx + kb * 16, lo, hi);
   for (; task < task_end; task += kQuantWarps) {
-    // next task's pointers and block
-    uint2* cur_dst = dst;
-    uint8_t* cur_sdst = sdst;
-    const bool cur_ok = row_ok;
-    if (!step_in_row) {
-      const uint32_t nt = task + kQuantWarps;
-      kg = nt % p.kgroups;
-      t2 = nt / p.kgroups;
-      locate(t2, kg);
-    } else if ((kg += kQuantWarps) >= p.kgroups) {
-      kg -= p.kgroups;
-      ++t2;
-      locate(t2, kg);
-    } else {
-      src += 8 * kQuantWarps;
-      dst += 4 * kQuantWarps;
-      sdst += 512 * kQuantWarps;
+    const int64_t cur_row = row;
+    const uint32_t cur_kb = kb;
+    row += step_rows;
+    kb += step_kb;
+    if (kb >= kbs) {
+      kb -= kbs;
+      ++row;
     }
     uint4 nlo = make_uint4(0, 0, 0, 0), nhi = nlo;
-    if (task + kQuantWarps < task_end && row_ok) {
-      nlo = ld_stream(src);
-      nhi = ld_stream(src + 1);
-    }
+    if (task + kQuantWarps < task_end && row < p.rows) ld_block2(p.x + row * p.ldx + kb * 16, nlo, nhi);
 
-    uint32_t scale = 0;
-    if (cur_ok) {
-      uint2 codes;
-      const uint32_t bmax = quantize_block<FOUR_OVER_SIX, RULE>(lo, hi, k, s_dr, codes, scale);
-      if (p.alpha_in && bmax >= 0x7F80u) {
-        // Inf/NaN in this block (a static alpha skips the tensor check):
-        // the block is written as zeros and the call reports it
-        codes = make_uint2(0u, 0u);
-        scale = 0u;
-        p.ws->status = NVFP4_ERR_NONFINITE;
+    if (cur_row < rows_padded) {
+      uint32_t scale = 0;
+      if (cur_row < p.rows) {
+        uint2 codes;
+        const uint32_t bmax = quantize_block<FOUR_OVER_SIX, RULE>(lo, hi, k, s_dr, codes, scale);
+        if (p.alpha_in && bmax >= 0x7F80u) {
+          // Inf/NaN in this block (a static alpha skips the tensor check):
+          // the block is written as zeros and the call reports it
+          codes = make_uint2(0u, 0u);
+          scale = 0u;
+          p.ws->status = NVFP4_ERR_NONFINITE;
+        }
+        *reinterpret_cast<uint2*>(p.codes + cur_row * half_k + cur_kb * 8) = codes;
       }
-      *cur_dst = codes;
+      const int64_t atom = (cur_row >> 7) * p.kgroups + (cur_kb >> 2);
+      p.scales[atom * 512 + (cur_row & 31) * 16 + ((cur_row >> 5) & 3) * 4 + (cur_kb & 3)] =
+          static_cast<uint8_t>(scale);
     }
-    *cur_sdst = static_cast<uint8_t>(scale);
     lo = nlo;
     hi = nhi;
   }
@@ -527,7 +508,7 @@ nvfp4_status nvfp4_quantize(const void* x, int64_t rows, int64_t K, int64_t ldx,
   if (workspace_bytes < nvfp4_quantize_workspace_bytes(rows, K))
     return set_error(NVFP4_ERR_INVALID_ARG, "nvfp4_quantize: workspace too small");
   const int64_t row_blocks = (rows + 127) / 128;
-  const int64_t ntasks = row_blocks * 16 * (K / 64);
+  const int64_t ntasks = (row_blocks * 128 * (K / 16) + 31) / 32;
   if (ntasks >= 0x80000000ll || rows * ldx > (1ll << 40))
     return set_error(NVFP4_ERR_INVALID_ARG, "nvfp4_quantize: tensor too large");
   int dev = 0, sms = 0;
@@ -647,7 +628,7 @@ extern "C" nvfp4_status nvfp4_quantize_noalloc(const void* x, int64_t rows, int6
       (reinterpret_cast<uintptr_t>(global_scale) & 3u))
     return set_error(NVFP4_ERR_INVALID_ARG, "nvfp4_quantize_noalloc: misaligned buffer");
   const int64_t row_blocks = (rows + 127) / 128;
-  const int64_t ntasks = row_blocks * 16 * (K / 64);
+  const int64_t ntasks = (row_blocks * 128 * (K / 16) + 31) / 32;
   if (ntasks >= 0x80000000ll || rows * ldx > (1ll << 40))
     return set_error(NVFP4_ERR_INVALID_ARG, "nvfp4_quantize_noalloc: tensor too large");
   int dev = 0, sms = 0;
@@ -724,7 +705,7 @@ extern "C" nvfp4_status nvfp4_quantize_with_scale(const void* x, int64_t rows, i
   if (workspace_bytes < sizeof(WorkspaceHeader))
     return set_error(NVFP4_ERR_INVALID_ARG, "nvfp4_quantize_with_scale: workspace too small");
   const int64_t row_blocks = (rows + 127) / 128;
-  const int64_t ntasks = row_blocks * 16 * (K / 64);
+  const int64_t ntasks = (row_blocks * 128 * (K / 16) + 31) / 32;
   if (ntasks >= 0x80000000ll || rows * ldx > (1ll << 40))
     return set_error(NVFP4_ERR_INVALID_ARG, "nvfp4_quantize_with_scale: tensor too large");
   int dev = 0, sms = 0;
