@@ -238,6 +238,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     // -------------------------------------------------- TMA producer ----
     // The whole warp walks the loop; one elected lane issues.
     uint32_t it = 0;  // k-step counter across this pair's tiles
+    // B (the weight) is re-read by every row of output tiles: keep it in L2
+    const uint64_t pol_keep = l2_policy_evict_last();
     bool stop = false;
     for (uint32_t tile = pair; tile < p.num_tiles && !stop; tile += npairs) {
       const int m0 = static_cast<int>(tile / p.n_tiles) * BM;
@@ -258,11 +260,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           if (!((p.debug_flags & 1) && it == 0)) {  // test hook: the first stage never fills
             const int32_t kx = static_cast<int32_t>(kt * BK_BYTES);
             tma_load_2d_pair(sbase + OFF_A + s * A_STAGE, &tmA, fb, kx, a_row);
-            tma_load_2d_pair(sbase + OFF_B + s * B_STAGE, &tmB, fb, kx, b_row);
+            tma_load_2d_pair_hint(sbase + OFF_B + s * B_STAGE, &tmB, fb, kx, b_row, pol_keep);
             tma_load_3d_pair(sbase + OFF_SFA + s * SFA_STAGE, &tmSFA, fb, 0,
                              static_cast<int32_t>(kt * 4), a_row / 128);
-            tma_load_3d_pair(sbase + OFF_SFB + s * SFB_STAGE, &tmSFB, fb, 0,
-                             static_cast<int32_t>(kt * 4), n0 / 128);
+            tma_load_3d_pair_hint(sbase + OFF_SFB + s * SFB_STAGE, &tmSFB, fb, 0,
+                                  static_cast<int32_t>(kt * 4), n0 / 128, pol_keep);
           }
         }
         __syncwarp();
@@ -367,6 +369,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     // this warp's two staging buffers; lane 0 issues (and waits for) every
     // TMA store of the warp, so the bulk groups it waits on are its own
     const uint32_t stg0 = sbase + OFF_STG + static_cast<uint32_t>(quad) * 2 * STG_BYTES;
+    const uint64_t pol_stream = l2_policy_evict_first();  // Y is written once: do not let it evict B
     uint32_t nstore = 0;
     uint32_t local = 0;
     for (uint32_t tile = pair; tile < p.num_tiles; tile += npairs, ++local) {
@@ -421,8 +424,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) {
-              tma_store_2d(&tmY, stg0, col0, row0);
-              tma_store_2d(&tmY, stg0 + STG_BYTES, col0 + 32, row0);
+              tma_store_2d_hint(&tmY, stg0, col0, row0, pol_stream);
+              tma_store_2d_hint(&tmY, stg0 + STG_BYTES, col0 + 32, row0, pol_stream);
               bulk_commit_group();
             }
           } else {
@@ -442,7 +445,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) {
-              tma_store_2d(&tmY, stg, col0, row0);
+              tma_store_2d_hint(&tmY, stg, col0, row0, pol_stream);
               bulk_commit_group();
             }
             ++nstore;
