@@ -129,6 +129,24 @@ NVFP4_API nvfp4_status nvfp4_quantize(const void* x, int64_t rows, int64_t K, in
                             float* global_scale, void* workspace, size_t workspace_bytes,
                             void* stream);
 
+/* The NVFP4 operand of x^T: x is the same bf16 [rows, K] matrix as for
+ * nvfp4_quantize, but the 16-element blocks run along rows (down a column of
+ * x), so codes/scales describe the [K, rows] matrix x^T -- the layout the
+ * weight-gradient and input-gradient GEMMs of training need (the "Four Over
+ * Six (4/6)" summary, "주요 기여 및 결과": 4/6 applied to weights, activations
+ * and gradients in NVFP4 pretraining).  Same alpha (the tensor amax is the
+ * same), same modes, rules and arithmetic per block as nvfp4_quantize.
+ *   codes   [K, rows/2] bytes, nvfp4_codes_bytes(K, rows)
+ *   scales  nvfp4_scales_bytes(K, rows) bytes, swizzled for a [K, rows] operand
+ * Requirements: rows a positive multiple of 64, K a positive multiple of 8,
+ * ldx >= K and ldx % 8 == 0, buffers as nvfp4_quantize, workspace of
+ * nvfp4_quantize_workspace_bytes(rows, K).  Two kernel launches (amax pass,
+ * tiled transpose-quantize). */
+NVFP4_API nvfp4_status nvfp4_quantize_t(const void* x, int64_t rows, int64_t K, int64_t ldx, int mode,
+                                        int rule, float fp8_max, void* codes, void* scales,
+                                        float* global_scale, void* workspace, size_t workspace_bytes,
+                                        void* stream);
+
 /* nvfp4_quantize with a caller-supplied tensor scale: alpha is read from
  * *global_scale (device memory; e.g. calibrated offline, or a previous call's
  * output), the tensor-amax pass and its read of x are skipped, and every

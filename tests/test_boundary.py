@@ -73,6 +73,22 @@ def test_quantize_rejects_bad_arguments(bad):
     assert nv.last_error_message()
 
 
+def _qt(**kw):
+    args = dict(x=FAKE, rows=128, K=72, ldx=72, mode=1, rule=2, fp8_max=256.0, codes=FAKE,
+                scales=FAKE, global_scale=FAKE, workspace=FAKE, workspace_bytes=1 << 20, stream=None)
+    args.update(kw)
+    return nv.nvfp4_quantize_t(*args.values())
+
+
+@pytest.mark.parametrize("bad", [
+    dict(x=None), dict(codes=None), dict(rows=0), dict(rows=32), dict(rows=100), dict(K=0), dict(K=12),
+    dict(ldx=64), dict(ldx=76), dict(mode=5), dict(rule=7), dict(fp8_max=100.0), dict(x=FAKE + 8),
+    dict(workspace_bytes=16),
+])
+def test_quantize_t_rejects_bad_arguments(bad):
+    assert _qt(**bad) == nv.ERR_INVALID_ARG
+
+
 def _qs(**kw):
     args = dict(x=FAKE, rows=64, K=512, ldx=512, mode=1, rule=2, global_scale=FAKE, codes=FAKE,
                 scales=FAKE, workspace=FAKE, workspace_bytes=64, stream=None)
@@ -137,5 +153,6 @@ def test_no_gpu_fails_loudly():
         pytest.skip("a GPU is present")
     assert _q() in (nv.ERR_CUDA, nv.ERR_UNSUPPORTED_DEVICE)
     assert _qs() in (nv.ERR_CUDA, nv.ERR_UNSUPPORTED_DEVICE)
+    assert _qt() in (nv.ERR_CUDA, nv.ERR_UNSUPPORTED_DEVICE)
     assert _gs((64, 128, 256)) in (nv.ERR_CUDA, nv.ERR_UNSUPPORTED_DEVICE)
     assert _g() in (nv.ERR_CUDA, nv.ERR_UNSUPPORTED_DEVICE)

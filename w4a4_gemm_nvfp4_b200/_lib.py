@@ -37,6 +37,8 @@ _SIGNATURES = {
                                       ctypes.c_float, _P, _P, _P, _P, ctypes.c_size_t, _P]),
     "nvfp4_quantize_noalloc": (ctypes.c_int, [_P, _I64, _I64, _I64, ctypes.c_int, ctypes.c_int,
                                               ctypes.c_float, _P, _P, _P, _P]),
+    "nvfp4_quantize_t": (ctypes.c_int, [_P, _I64, _I64, _I64, ctypes.c_int, ctypes.c_int,
+                                        ctypes.c_float, _P, _P, _P, _P, ctypes.c_size_t, _P]),
     "nvfp4_quantize_with_scale": (ctypes.c_int, [_P, _I64, _I64, _I64, ctypes.c_int, ctypes.c_int,
                                                  _P, _P, _P, _P, ctypes.c_size_t, _P]),
     "nvfp4_gemm": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _I64,
@@ -106,6 +108,13 @@ def nvfp4_quantize_noalloc(x, rows, K, ldx, mode, rule, fp8_max, codes, scales, 
     library: no workspace argument, nothing allocated (see include/nvfp4.h)."""
     return load().nvfp4_quantize_noalloc(x, rows, K, ldx, mode, rule, fp8_max, codes, scales,
                                          global_scale, stream)
+
+
+def nvfp4_quantize_t(x, rows, K, ldx, mode, rule, fp8_max, codes, scales, global_scale, workspace,
+                     workspace_bytes, stream) -> int:
+    """The NVFP4 operand of x^T (blocks along the rows of x)."""
+    return load().nvfp4_quantize_t(x, rows, K, ldx, mode, rule, fp8_max, codes, scales, global_scale,
+                                   workspace, workspace_bytes, stream)
 
 
 def nvfp4_quantize_with_scale(x, rows, K, ldx, mode, rule, global_scale, codes, scales, workspace,
@@ -215,6 +224,33 @@ def quantize(x, mode: str = "six", rule: str = "max", fp8_max: float | None = No
                         out.codes.data_ptr(), out.scales.data_ptr(), out.global_scale.data_ptr(),
                         out.workspace.data_ptr(), out.workspace.numel(), _stream_handle(stream))
     _check(st, "nvfp4_quantize")
+    return out
+
+
+def quantize_t(x, mode: str = "six", rule: str = "max", fp8_max: float | None = None,
+               out: NVFP4Tensor | None = None, stream=None) -> NVFP4Tensor:
+    """NVFP4-quantize x^T for a CUDA bf16 matrix x [rows, K] (rows % 64 == 0,
+    K % 8 == 0): the result is the [K, rows] operand, blocks along rows of x."""
+    import torch
+
+    if x.dtype != torch.bfloat16 or x.dim() != 2 or not x.is_cuda:
+        raise ValueError("x must be a 2-D bfloat16 CUDA tensor")
+    if x.stride(1) != 1:
+        raise ValueError("x must have unit stride along K")
+    rows, K = x.shape
+    F = DEFAULT_FP8_MAX[mode] if fp8_max is None else float(fp8_max)
+    if out is None:
+        dev = x.device
+        out = NVFP4Tensor(
+            codes=torch.empty(K, rows // 2, dtype=torch.uint8, device=dev),
+            scales=torch.empty(max(1, nvfp4_scales_bytes(K, rows)), dtype=torch.uint8, device=dev),
+            global_scale=torch.empty(1, dtype=torch.float32, device=dev),
+            workspace=torch.empty(nvfp4_quantize_workspace_bytes(rows, K), dtype=torch.uint8, device=dev),
+            rows=K, K=rows)
+    st = nvfp4_quantize_t(x.data_ptr(), rows, K, x.stride(0), MODES[mode], RULES[rule], F,
+                          out.codes.data_ptr(), out.scales.data_ptr(), out.global_scale.data_ptr(),
+                          out.workspace.data_ptr(), out.workspace.numel(), _stream_handle(stream))
+    _check(st, "nvfp4_quantize_t")
     return out
 
 

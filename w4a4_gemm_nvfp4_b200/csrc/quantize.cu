@@ -337,18 +337,20 @@ struct QuantParams {
   uint32_t kgroups;    // K / 64
 };
 
-template <bool FOUR_OVER_SIX, int RULE>
-__global__ void __launch_bounds__(kQuantThreads)
-    quantize_kernel(const QuantParams p) {
-  // ---- alpha: a caller-supplied static scale, or the tensor amax reduced
-  // from the partials of the amax pass (every CTA reduces the same partials)
+// Start of every quantize kernel: alpha (a caller-supplied static scale, or
+// the tensor amax reduced from the partials of the amax pass -- every CTA
+// reduces the same partials), the per-call constants of the block step and
+// the (d, r) table of every E4M3 scale code.  Returns false when the kernel
+// must stop (non-finite tensor, invalid static alpha); that is uniform over
+// the grid.
+__device__ __forceinline__ bool quant_prologue(const QuantParams& p, BlockConsts& k, float2* s_dr) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   float alpha;
   if (p.alpha_in) {
     alpha = __ldg(p.alpha_in);
     if (!(alpha > 0.0f) || isinf(alpha)) {  // not a positive finite number
       if (blockIdx.x == 0 && threadIdx.x == 0) p.ws->status = NVFP4_ERR_INVALID_ARG;
-      return;
+      return false;
     }
     // the status word was cleared to NVFP4_OK before the launch; CTAs only
     // ever raise it (to NVFP4_ERR_NONFINITE), so their order does not matter
@@ -370,17 +372,14 @@ __global__ void __launch_bounds__(kQuantThreads)
       p.ws->detail = amax_bits;
       *p.global_scale = nonfinite ? __uint_as_float(0x7FC00000u) : alpha;
     }
-    if (nonfinite) return;
+    if (nonfinite) return false;
   }
-  BlockConsts k;
   k.a6 = __fmul_rn(alpha, 6.0f);
   k.a4 = __fmul_rn(alpha, 4.0f);
   k.inv6 = __frcp_rn(k.a6);
   k.inv4 = __frcp_rn(k.a4);
   k.fast_div = k.inv6 >= 1.17549435e-38f && !isinf(k.inv4);
-
   // (d, r) of every E4M3 scale code (0x7F is NaN and never produced)
-  __shared__ float2 s_dr[128];
   if (threadIdx.x < 128) {
     float s, unused;
     e4m3x2_to_f32(threadIdx.x, s, unused);
@@ -388,6 +387,16 @@ __global__ void __launch_bounds__(kQuantThreads)
     s_dr[threadIdx.x] = make_float2(d, safe_recip(d));
   }
   __syncthreads();
+  return true;
+}
+
+template <bool FOUR_OVER_SIX, int RULE>
+__global__ void __launch_bounds__(kQuantThreads)
+    quantize_kernel(const QuantParams p) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  BlockConsts k;
+  __shared__ float2 s_dr[128];
+  if (!quant_prologue(p, k, s_dr)) return;
 
   // ---- lane -> (row, 16-element block) ----
   // Blocks are numbered row-major over the padded rows (a multiple of 128):
@@ -447,6 +456,108 @@ __global__ void __launch_bounds__(kQuantThreads)
   }
 }
 
+// Quantization of x^T: the NVFP4 operand of the [K, rows] matrix x^T, i.e.
+// 16-element blocks along rows (a column of x), as the weight-gradient and
+// input-gradient GEMMs of training need it.  A CTA loads a 128-row x 64-column
+// tile of x into shared memory (16-byte chunks, chunk index XOR-swizzled by
+// the 16-row group so the column reads below hit 32 distinct banks), then
+// thread t quantizes the two columns 2(t>>3), 2(t>>3)+1 over rows
+// 16(t&7) .. 16(t&7)+15 with the same block step as the row-wise kernel.
+// Output row kk of x^T, block mb: codes at kk*(rows/2) + 8*mb, scale in the
+// swizzled layout of a [K, rows] operand; rows kk in [K, ceil(K/128)*128)
+// get zero scales.
+template <bool FOUR_OVER_SIX, int RULE>
+__global__ void __launch_bounds__(kQuantThreads)
+    quantize_t_kernel(const QuantParams p) {
+  BlockConsts k;
+  __shared__ float2 s_dr[128];
+  __shared__ __align__(16) uint32_t tile[128 * 32];  // 128 rows x 128 bytes
+  if (!quant_prologue(p, k, s_dr)) return;
+
+  const int64_t M = p.rows, K = p.K;
+  const int64_t k_pad = (K + 127) / 128 * 128;
+  const uint32_t tiles_m = static_cast<uint32_t>((M + 127) / 128);
+  const uint32_t tiles_k = static_cast<uint32_t>(k_pad / 64);
+  const uint32_t ntiles = tiles_m * tiles_k;
+  const int cp = threadIdx.x >> 3, mb = threadIdx.x & 7;
+  const int64_t half_m = M / 2;
+  const int64_t kgroups_t = M / 64;  // K groups of the transposed operand
+  for (uint32_t t = blockIdx.x; t < ntiles; t += gridDim.x) {
+    const int64_t m0 = static_cast<int64_t>(t % tiles_m) * 128;
+    const int64_t k0 = static_cast<int64_t>(t / tiles_m) * 64;
+    // ---- load: 128 rows x 8 chunks of 16 bytes, 4 per thread ----
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int q = threadIdx.x + i * kQuantThreads;
+      const int r = q >> 3, ch = q & 7;
+      uint4 v = make_uint4(0, 0, 0, 0);
+      if (m0 + r < M && k0 + ch * 8 < K)
+        v = ld_stream(reinterpret_cast<const uint4*>(p.x + (m0 + r) * p.ldx + k0 + ch * 8));
+      *reinterpret_cast<uint4*>(&tile[r * 32 + ((ch ^ ((r >> 4) & 7)) << 2)]) = v;
+    }
+    __syncthreads();
+    // ---- two column blocks per thread ----
+    const int64_t mb_g = m0 / 16 + mb;
+    if (mb_g * 16 < M) {
+      uint32_t wl[8], wh[8];  // column 2cp / 2cp+1 as bf16 pairs (element 2i in the low half)
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int r0 = mb * 16 + 2 * i;
+        const uint32_t a = tile[r0 * 32 + (((cp >> 2) ^ mb) << 2) + (cp & 3)];
+        const uint32_t b = tile[(r0 + 1) * 32 + (((cp >> 2) ^ mb) << 2) + (cp & 3)];
+        wl[i] = __byte_perm(a, b, 0x5410);
+        wh[i] = __byte_perm(a, b, 0x7632);
+      }
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int64_t kk = k0 + 2 * cp + h;
+        if (kk >= k_pad) continue;
+        uint32_t scale = 0;
+        if (kk < K) {
+          const uint32_t* w = h ? wh : wl;
+          const uint4 lo = make_uint4(w[0], w[1], w[2], w[3]), hi = make_uint4(w[4], w[5], w[6], w[7]);
+          uint2 codes;
+          const uint32_t bmax = quantize_block<FOUR_OVER_SIX, RULE>(lo, hi, k, s_dr, codes, scale);
+          if (p.alpha_in && bmax >= 0x7F80u) {
+            codes = make_uint2(0u, 0u);
+            scale = 0u;
+            p.ws->status = NVFP4_ERR_NONFINITE;
+          }
+          *reinterpret_cast<uint2*>(p.codes + kk * half_m + mb_g * 8) = codes;
+        }
+        const int64_t atom = (kk >> 7) * kgroups_t + (mb_g >> 2);
+        p.scales[atom * 512 + (kk & 31) * 16 + ((kk >> 5) & 3) * 4 + (mb_g & 3)] =
+            static_cast<uint8_t>(scale);
+      }
+    }
+    __syncthreads();
+  }
+}
+
+template <bool F, int R>
+cudaError_t launch_quantize_t(int sms, const QuantParams& p, cudaStream_t s) {
+  static std::atomic<int> per_sm{0};
+  int occ = per_sm.load(std::memory_order_relaxed);
+  if (occ == 0) {
+    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, quantize_t_kernel<F, R>,
+                                                                  kQuantThreads, 0);
+    if (e != cudaSuccess) return e;
+    occ = std::max(1, occ);
+    per_sm.store(occ, std::memory_order_relaxed);
+  }
+  const int64_t tiles = ((p.rows + 127) / 128) * (((p.K + 127) / 128 * 128) / 64);
+  const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(tiles, static_cast<int64_t>(sms) * occ)));
+  quantize_t_kernel<F, R><<<grid, kQuantThreads, 0, s>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quantize_t_kernel(int mode, int rule, int sms, const QuantParams& p, cudaStream_t s) {
+  if (mode == NVFP4_MODE_SIX) return launch_quantize_t<false, kRuleMax>(sms, p, s);
+  if (rule == NVFP4_RULE_MAX) return launch_quantize_t<true, kRuleMax>(sms, p, s);
+  if (rule == NVFP4_RULE_MAE) return launch_quantize_t<true, kRuleMae>(sms, p, s);
+  return launch_quantize_t<true, kRuleMse>(sms, p, s);
+}
+
 template <bool F, int R>
 cudaError_t launch_quantize(int sms, const QuantParams& p, cudaStream_t s) {
   static std::atomic<int> per_sm{0};
@@ -484,33 +595,42 @@ size_t nvfp4_quantize_workspace_bytes(int64_t rows, int64_t K) {
   return sizeof(WorkspaceHeader) + sizeof(uint32_t) * kMaxPartials;
 }
 
-nvfp4_status nvfp4_quantize(const void* x, int64_t rows, int64_t K, int64_t ldx, int mode,
-                            int rule, float fp8_max, void* codes, void* scales,
-                            float* global_scale, void* workspace, size_t workspace_bytes,
-                            void* stream) {
+}  // extern "C"
+
+namespace {
+
+// nvfp4_quantize (row-wise blocks of x) and nvfp4_quantize_t (blocks along
+// the rows of x, i.e. the operand of x^T): amax pass, then the quantize kernel.
+nvfp4_status quantize_impl(const char* fn, bool transposed, const void* x, int64_t rows, int64_t K,
+                           int64_t ldx, int mode, int rule, float fp8_max, void* codes, void* scales,
+                           float* global_scale, void* workspace, size_t workspace_bytes, void* stream) {
   if (!x || !codes || !scales || !global_scale || !workspace)
-    return set_error(NVFP4_ERR_INVALID_ARG, "nvfp4_quantize: null pointer argument");
-  if (rows < 1 || K < 64 || K % 64 != 0)
+    return set_error(NVFP4_ERR_INVALID_ARG, "%s: null pointer argument", fn);
+  if (!transposed && (rows < 1 || K < 64 || K % 64 != 0))
     return set_error(NVFP4_ERR_INVALID_ARG,
-                     "nvfp4_quantize: need rows >= 1 and K a positive multiple of 64 (rows=%lld K=%lld)",
+                     "%s: need rows >= 1 and K a positive multiple of 64 (rows=%lld K=%lld)", fn,
                      (long long)rows, (long long)K);
+  if (transposed && (rows < 64 || rows % 64 != 0 || K < 8 || K % 8 != 0))
+    return set_error(NVFP4_ERR_INVALID_ARG,
+                     "%s: need rows a positive multiple of 64 and K a positive multiple of 8 (rows=%lld K=%lld)",
+                     fn, (long long)rows, (long long)K);
   if (ldx < K || ldx % 8 != 0)
-    return set_error(NVFP4_ERR_INVALID_ARG, "nvfp4_quantize: need ldx >= K and ldx %% 8 == 0");
+    return set_error(NVFP4_ERR_INVALID_ARG, "%s: need ldx >= K and ldx %% 8 == 0", fn);
   if (mode != NVFP4_MODE_SIX && mode != NVFP4_MODE_FOUR_OVER_SIX)
-    return set_error(NVFP4_ERR_INVALID_ARG, "nvfp4_quantize: unknown mode %d", mode);
+    return set_error(NVFP4_ERR_INVALID_ARG, "%s: unknown mode %d", fn, mode);
   if (rule != NVFP4_RULE_MAX && rule != NVFP4_RULE_MAE && rule != NVFP4_RULE_MSE)
-    return set_error(NVFP4_ERR_INVALID_ARG, "nvfp4_quantize: unknown rule %d", rule);
+    return set_error(NVFP4_ERR_INVALID_ARG, "%s: unknown rule %d", fn, rule);
   if (!(fp8_max == 448.0f || fp8_max == 256.0f))
-    return set_error(NVFP4_ERR_INVALID_ARG, "nvfp4_quantize: fp8_max must be 448 or 256");
+    return set_error(NVFP4_ERR_INVALID_ARG, "%s: fp8_max must be 448 or 256", fn);
   if (!aligned16(x) || !aligned16(codes) || !aligned16(scales) || !aligned16(workspace) ||
       (reinterpret_cast<uintptr_t>(global_scale) & 3u))
-    return set_error(NVFP4_ERR_INVALID_ARG, "nvfp4_quantize: misaligned buffer");
+    return set_error(NVFP4_ERR_INVALID_ARG, "%s: misaligned buffer", fn);
   if (workspace_bytes < nvfp4_quantize_workspace_bytes(rows, K))
-    return set_error(NVFP4_ERR_INVALID_ARG, "nvfp4_quantize: workspace too small");
+    return set_error(NVFP4_ERR_INVALID_ARG, "%s: workspace too small", fn);
   const int64_t row_blocks = (rows + 127) / 128;
-  const int64_t ntasks = (row_blocks * 128 * (K / 16) + 31) / 32;
+  const int64_t ntasks = transposed ? 0 : (row_blocks * 128 * (K / 16) + 31) / 32;
   if (ntasks >= 0x80000000ll || rows * ldx > (1ll << 40))
-    return set_error(NVFP4_ERR_INVALID_ARG, "nvfp4_quantize: tensor too large");
+    return set_error(NVFP4_ERR_INVALID_ARG, "%s: tensor too large", fn);
   int dev = 0, sms = 0;
   nvfp4_status st = check_device(&dev, &sms);
   if (st != NVFP4_OK) return st;
@@ -548,9 +668,29 @@ nvfp4_status nvfp4_quantize(const void* x, int64_t rows, int64_t K, int64_t ldx,
   p.f6 = fp8_max * 6.0f;
   p.ntasks = static_cast<uint32_t>(ntasks);
   p.kgroups = static_cast<uint32_t>(K / 64);
-  e = launch_quantize_kernel(mode, rule, sms, p, s);
-  if (e != cudaSuccess) return cuda_status(e, "quantize_kernel launch");
+  e = transposed ? launch_quantize_t_kernel(mode, rule, sms, p, s) : launch_quantize_kernel(mode, rule, sms, p, s);
+  if (e != cudaSuccess) return cuda_status(e, "quantize kernel launch");
   return NVFP4_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+nvfp4_status nvfp4_quantize(const void* x, int64_t rows, int64_t K, int64_t ldx, int mode,
+                            int rule, float fp8_max, void* codes, void* scales,
+                            float* global_scale, void* workspace, size_t workspace_bytes,
+                            void* stream) {
+  return quantize_impl("nvfp4_quantize", false, x, rows, K, ldx, mode, rule, fp8_max, codes, scales,
+                       global_scale, workspace, workspace_bytes, stream);
+}
+
+nvfp4_status nvfp4_quantize_t(const void* x, int64_t rows, int64_t K, int64_t ldx, int mode,
+                              int rule, float fp8_max, void* codes, void* scales,
+                              float* global_scale, void* workspace, size_t workspace_bytes,
+                              void* stream) {
+  return quantize_impl("nvfp4_quantize_t", true, x, rows, K, ldx, mode, rule, fp8_max, codes, scales,
+                       global_scale, workspace, workspace_bytes, stream);
 }
 
 }  // extern "C"
