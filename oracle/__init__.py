@@ -82,6 +82,9 @@ def _load():
                                             ctypes.c_int, u8p, u8p]),
                 "or_quantize": (ctypes.c_int, [u16p, i64, i64, i64, ctypes.c_int, ctypes.c_int,
                                                ctypes.c_float, u8p, u8p, f32p]),
+                "or_quantize_arc": (ctypes.c_int, [u16p, i64, i64, i64, ctypes.POINTER(ctypes.c_int32), i64,
+                                                   ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_float,
+                                                   u8p, u8p, f32p]),
                 "or_scales_swizzled_bytes": (i64, [i64, i64]),
                 "or_swizzle_scales": (None, [u8p, i64, i64, u8p]),
                 "or_unswizzle_scales": (None, [u8p, i64, i64, u8p]),
@@ -201,6 +204,34 @@ def quantize(x, mode: int, rule: int, fp8_max: float):
     rc = _load().or_quantize(_ptr(xb, ctypes.c_uint16), rows, K, K, int(mode), int(rule),
                              float(fp8_max), _ptr(codes, ctypes.c_uint8),
                              _ptr(scales, ctypes.c_uint8), ctypes.byref(alpha))
+    if rc != 0:
+        raise NonFiniteInput("tensor holds Inf or NaN")
+    return codes, scales, float(np.float32(alpha.value))
+
+
+AUG_RESIDUAL = 0
+AUG_DUPLICATE = 1
+
+
+def quantize_arc(x, perm, S: int, augment: int, mode: int, rule: int, fp8_max: float):
+    """ARCQuant augmented quantization (ARCQuant page, 기술 요약 / 방법론):
+    channels reordered by `perm`, primary NVFP4 stage, then S augmented
+    channels -- the residual of the first S reordered channels against the
+    primary stage (augment=AUG_RESIDUAL) or a copy of them (AUG_DUPLICATE, for
+    weights) -- quantized with the same alpha.  Returns (codes [rows,
+    (K+S)/2], canonical scales [rows, (K+S)/16], alpha)."""
+    xb = as_bf16_bits(x)
+    rows, K = xb.shape
+    p = np.ascontiguousarray(np.asarray(perm, dtype=np.int32))
+    assert p.shape == (K,) and sorted(p.tolist()) == list(range(K))
+    assert K % 16 == 0 and S % 16 == 0 and 0 <= S <= K
+    codes = np.zeros((rows, (K + S) // 2), np.uint8)
+    scales = np.zeros((rows, (K + S) // 16), np.uint8)
+    alpha = ctypes.c_float(0)
+    rc = _load().or_quantize_arc(_ptr(xb, ctypes.c_uint16), rows, K, K, _ptr(p, ctypes.c_int32), S,
+                                 int(augment), int(mode), int(rule), float(fp8_max),
+                                 _ptr(codes, ctypes.c_uint8), _ptr(scales, ctypes.c_uint8),
+                                 ctypes.byref(alpha))
     if rc != 0:
         raise NonFiniteInput("tensor holds Inf or NaN")
     return codes, scales, float(np.float32(alpha.value))

@@ -220,6 +220,58 @@ void or_quantize_block(const float x[16], float alpha, int mode, int rule,
   if (err4) *err4 = e4;
 }
 
+/* -------------------------------------------- augmented residual channels --- */
+
+/* ARCQuant (ARCQuant page, 기술 요약 / 방법론): the activation's K channels are
+ * reordered by a calibration permutation (outliers first); the primary stage is
+ * the usual NVFP4 quantization of the reordered row; the residual stage takes
+ * the first S reordered channels, forms their residual against the primary
+ * stage, e_j = fmaf(-val(q_j), d, x_j) with d = val(s)*alpha of the block, and
+ * quantizes it as S more NVFP4 channels (same alpha, mode and rule) appended
+ * along K, so one GEMM over K + S adds the correction.  augment == 1 instead
+ * appends a plain copy of the first S reordered channels (the matching weight
+ * columns are duplicated).  Output per row: K + S channels; codes packed
+ * [rows, (K+S)/2], canonical scales [rows, (K+S)/16].  Returns 0, or 1 when x
+ * holds a non-finite value (outputs untouched). */
+int or_quantize_arc(const uint16_t* x, int64_t rows, int64_t K, int64_t ldx, const int32_t* perm,
+                    int64_t S, int augment, int mode, int rule, float fp8_max, uint8_t* codes,
+                    uint8_t* scales, float* alpha_out) {
+  int bad = 0;
+  float amax = or_amax_bf16(x, rows, K, ldx, &bad);
+  if (bad) return 1;
+  float alpha = or_global_scale(amax, fp8_max);
+  const int64_t KA = K + S;
+  for (int64_t r = 0; r < rows; ++r) {
+    for (int64_t j = 0; j < K / 16; ++j) {
+      float xb[16];
+      uint8_t q[16], s;
+      for (int i = 0; i < 16; ++i) xb[i] = bf16_to_f32(x[r * ldx + perm[j * 16 + i]]);
+      or_quantize_block(xb, alpha, mode, rule, q, &s, 0, 0, 0);
+      scales[r * (KA / 16) + j] = s;
+      for (int i = 0; i < 8; ++i)
+        codes[r * (KA / 2) + j * 8 + i] = (uint8_t)((q[2 * i] & 15u) | ((q[2 * i + 1] & 15u) << 4));
+      if (j * 16 >= S) continue;
+      /* the block's augmented channels K + 16j .. K + 16j + 15 */
+      const int64_t ja = K / 16 + j;
+      uint8_t qa[16], sa;
+      if (augment == 1) {
+        memcpy(qa, q, 16);
+        sa = s;
+      } else {
+        float e[16];
+        const float d = or_e4m3_value(s) * alpha;
+        for (int i = 0; i < 16; ++i) e[i] = fmaf(-or_e2m1_value(q[i]), d, xb[i]);
+        or_quantize_block(e, alpha, mode, rule, qa, &sa, 0, 0, 0);
+      }
+      scales[r * (KA / 16) + ja] = sa;
+      for (int i = 0; i < 8; ++i)
+        codes[r * (KA / 2) + ja * 8 + i] = (uint8_t)((qa[2 * i] & 15u) | ((qa[2 * i + 1] & 15u) << 4));
+    }
+  }
+  if (alpha_out) *alpha_out = alpha;
+  return 0;
+}
+
 /* ------------------------------------------------------------ a tensor --- */
 
 /* Quantize rows of a bf16 tensor with a given alpha.  codes: [nrows, K/2]
