@@ -129,6 +129,27 @@ NVFP4_API nvfp4_status nvfp4_quantize(const void* x, int64_t rows, int64_t K, in
                             float* global_scale, void* workspace, size_t workspace_bytes,
                             void* stream);
 
+/* Augmented residual channels (ARCQuant page, "기술 요약" / "방법론"): the
+ * NVFP4 operand of the [rows, K + S] matrix whose first K channels are the
+ * channels of x in the order perm (outlier channels first, as calibration
+ * ranks them) and whose last S channels are
+ *   augment = 0: the residual e = x - q*d of the first S reordered channels
+ *                against their own quantization (activations), or
+ *   augment = 1: a copy of the first S reordered channels (the weight, whose
+ *                matching columns are duplicated),
+ * all quantized with the same alpha (the amax of x), mode and rule, so that
+ * one nvfp4_gemm over K + S adds the residual correction in its accumulator.
+ *   perm    device int32[K], a permutation of 0..K-1 (entries outside 0..K-1
+ *           are read as channel 0)
+ *   S       0 <= S <= K, S % 64 == 0
+ *   codes   [rows, (K+S)/2];  scales  nvfp4_scales_bytes(rows, K + S)
+ * Requirements otherwise as nvfp4_quantize, and K <= 16384 (rows and the
+ * permutation are staged in shared memory).  Two kernel launches. */
+NVFP4_API nvfp4_status nvfp4_quantize_arc(const void* x, int64_t rows, int64_t K, int64_t ldx,
+                                          const int32_t* perm, int64_t S, int augment, int mode, int rule,
+                                          float fp8_max, void* codes, void* scales, float* global_scale,
+                                          void* workspace, size_t workspace_bytes, void* stream);
+
 /* The NVFP4 operand of x^T: x is the same bf16 [rows, K] matrix as for
  * nvfp4_quantize, but the 16-element blocks run along rows (down a column of
  * x), so codes/scales describe the [K, rows] matrix x^T -- the layout the

@@ -89,6 +89,22 @@ def test_quantize_t_rejects_bad_arguments(bad):
     assert _qt(**bad) == nv.ERR_INVALID_ARG
 
 
+def _qa(**kw):
+    args = dict(x=FAKE, rows=64, K=512, ldx=512, perm=FAKE, S=64, augment=0, mode=1, rule=2, fp8_max=256.0,
+                codes=FAKE, scales=FAKE, global_scale=FAKE, workspace=FAKE, workspace_bytes=1 << 20,
+                stream=None)
+    args.update(kw)
+    return nv.nvfp4_quantize_arc(*args.values())
+
+
+@pytest.mark.parametrize("bad", [
+    dict(perm=None), dict(perm=FAKE + 2), dict(S=-64), dict(S=32), dict(S=576), dict(K=16448, ldx=16448),
+    dict(augment=2), dict(x=None), dict(K=48), dict(mode=3), dict(fp8_max=1.0),
+])
+def test_quantize_arc_rejects_bad_arguments(bad):
+    assert _qa(**bad) == nv.ERR_INVALID_ARG
+
+
 def _qs(**kw):
     args = dict(x=FAKE, rows=64, K=512, ldx=512, mode=1, rule=2, global_scale=FAKE, codes=FAKE,
                 scales=FAKE, workspace=FAKE, workspace_bytes=64, stream=None)
@@ -154,5 +170,6 @@ def test_no_gpu_fails_loudly():
     assert _q() in (nv.ERR_CUDA, nv.ERR_UNSUPPORTED_DEVICE)
     assert _qs() in (nv.ERR_CUDA, nv.ERR_UNSUPPORTED_DEVICE)
     assert _qt() in (nv.ERR_CUDA, nv.ERR_UNSUPPORTED_DEVICE)
+    assert _qa() in (nv.ERR_CUDA, nv.ERR_UNSUPPORTED_DEVICE)
     assert _gs((64, 128, 256)) in (nv.ERR_CUDA, nv.ERR_UNSUPPORTED_DEVICE)
     assert _g() in (nv.ERR_CUDA, nv.ERR_UNSUPPORTED_DEVICE)

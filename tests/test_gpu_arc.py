@@ -1,0 +1,97 @@
+"""Parity of nvfp4_quantize_arc (ARCQuant augmented residual channels) with
+the oracle, bit-exact, and of the augmented GEMM over K + S with the fp64
+oracle; the augmented product must also be closer to the exact bf16 product
+than the plain W4A4 one on outlier-heavy activations."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+import w4a4_gemm_nvfp4_b200 as nv
+from gpu_util import MODE, RULE, assert_gemm_close, to_np
+
+pytestmark = pytest.mark.gpu
+
+RECIPES = [("six", "max", 448.0), ("four_over_six", "mse", 256.0), ("four_over_six", "mae", 256.0),
+           ("four_over_six", "max", 256.0)]
+
+
+def outlier_perm(x: torch.Tensor) -> np.ndarray:
+    """Channels by descending column absmax (the calibration ranking)."""
+    amax = x.float().abs().amax(dim=0).numpy()
+    return np.argsort(-amax, kind="stable").astype(np.int32)
+
+
+def gpu_arc(x_cpu, perm, S, augment, mode, rule, F, canary=0xA5):
+    rows, K = x_cpu.shape
+    KA = K + S
+    out = nv.NVFP4Tensor(
+        codes=torch.full((rows, KA // 2), canary, dtype=torch.uint8, device="cuda"),
+        scales=torch.full((nv.nvfp4_scales_bytes(rows, KA),), canary, dtype=torch.uint8, device="cuda"),
+        global_scale=torch.full((1,), -1.0, dtype=torch.float32, device="cuda"),
+        workspace=torch.full((nv.nvfp4_quantize_workspace_bytes(rows, K),), 0xFF, dtype=torch.uint8,
+                             device="cuda"),
+        rows=rows, K=KA)
+    nv.quantize_arc(x_cpu.cuda(), torch.from_numpy(perm).cuda(), S, augment, mode, rule, F, out=out)
+    return out, nv.device_status(out.workspace)
+
+
+def assert_arc_equal(q, x, perm, S, augment, mode, rule, F):
+    rows, K = x.shape
+    oc, os_, oa = oracle.quantize_arc(x, perm, S, augment, MODE[mode], RULE[rule], F)
+    assert float(q.global_scale.cpu()[0]) == np.float32(oa)
+    gc = to_np(q.codes)
+    bad = np.argwhere(gc != oc)
+    assert bad.size == 0, f"{len(bad)} code bytes differ, first {bad[:5].tolist()}"
+    swz = oracle.swizzle_scales(os_, rows, K + S)
+    gs = to_np(q.scales)
+    bad = np.nonzero(gs != swz)[0]
+    assert bad.size == 0, f"{bad.size} scale bytes differ, first {bad[:5].tolist()}"
+
+
+@pytest.mark.parametrize("recipe", RECIPES, ids=lambda r: "-".join(map(str, r)))
+@pytest.mark.parametrize("shape,S", [((1, 64), 64), ((129, 256), 64), ((300, 512), 128), ((64, 1024), 0),
+                                     ((200, 5120), 256)], ids=lambda v: str(v))
+@pytest.mark.parametrize("augment", [nv.AUG_RESIDUAL, nv.AUG_DUPLICATE])
+def test_quantize_arc_matches_oracle(shape, S, recipe, augment):
+    x = workloads.small_operand(*shape, seed=shape[0] + shape[1] + S, kind="t").make()
+    perm = outlier_perm(x)
+    q, st = gpu_arc(x, perm, S, augment, *recipe)
+    assert st == nv.OK
+    assert_arc_equal(q, x, perm, S, augment, *recipe)
+
+
+def test_random_permutation_and_full_augment():
+    x = workloads.small_operand(70, 192, seed=9, kind="normal").make()
+    perm = torch.randperm(192, generator=torch.Generator().manual_seed(4)).numpy().astype(np.int32)
+    q, st = gpu_arc(x, perm, 192, nv.AUG_RESIDUAL, "four_over_six", "mse", 256.0)
+    assert st == nv.OK
+    assert_arc_equal(q, x, perm, 192, nv.AUG_RESIDUAL, "four_over_six", "mse", 256.0)
+
+
+def test_augmented_gemm_matches_oracle_and_beats_plain():
+    """Y = [X_p | R] . [W_p | W_S]^T over K + S: parity with the fp64 oracle
+    on the same operands, and a smaller error against the bf16 product than
+    plain W4A4 on outlier-heavy activations."""
+    M, N, K, S = 256, 384, 1024, 128
+    x = workloads.Operand(M, K, "normal", 1.0, outliers="channels", out_frac=0.02, out_mult=60.0,
+                          seed=21).make()
+    w = workloads.Operand(N, K, "normal", 0.02, seed=22).make()
+    perm = outlier_perm(x)
+    qx, st = gpu_arc(x, perm, S, nv.AUG_RESIDUAL, "six", "max", 448.0)
+    assert st == nv.OK
+    qw, st = gpu_arc(w, perm, S, nv.AUG_DUPLICATE, "six", "max", 448.0)
+    assert st == nv.OK
+    y = to_np(nv.gemm(qx, qw, out_dtype=torch.float32))
+    xc, xs, xa = oracle.quantize_arc(x, perm, S, oracle.AUG_RESIDUAL, oracle.MODE_SIX, oracle.RULE_MAX, 448.0)
+    wc, ws, wa = oracle.quantize_arc(w, perm, S, oracle.AUG_DUPLICATE, oracle.MODE_SIX, oracle.RULE_MAX, 448.0)
+    ref, guard = oracle.gemm_reference(xc, xs, xa, wc, ws, wa)
+    assert_gemm_close(y, ref, guard)
+    exact = x.double().numpy() @ w.double().numpy().T
+    pc, ps, pa = oracle.quantize(x, oracle.MODE_SIX, oracle.RULE_MAX, 448.0)
+    qc, qs, qa = oracle.quantize(w, oracle.MODE_SIX, oracle.RULE_MAX, 448.0)
+    plain, _ = oracle.gemm_reference(pc, ps, pa, qc, qs, qa)
+    err_aug = np.abs(y - exact).mean()
+    err_plain = np.abs(plain - exact).mean()
+    assert err_aug < err_plain, (err_aug, err_plain)

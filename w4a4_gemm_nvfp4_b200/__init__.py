@@ -16,4 +16,4 @@ from ._lib import (  # noqa: F401
     last_error_message, load, nvfp4_codes_bytes, nvfp4_gemm, nvfp4_gemm_workspace_bytes,
     nvfp4_get_device_status, nvfp4_quantize, nvfp4_quantize_noalloc, nvfp4_quantize_with_scale,
     nvfp4_quantize_workspace_bytes, nvfp4_scales_bytes,
-    quantize, quantize_t, nvfp4_quantize_t, status_string, testing_set_gemm_wait)
+    quantize, quantize_t, nvfp4_quantize_t, quantize_arc, nvfp4_quantize_arc, AUG_RESIDUAL, AUG_DUPLICATE, status_string, testing_set_gemm_wait)

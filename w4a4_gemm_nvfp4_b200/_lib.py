@@ -37,6 +37,8 @@ _SIGNATURES = {
                                       ctypes.c_float, _P, _P, _P, _P, ctypes.c_size_t, _P]),
     "nvfp4_quantize_noalloc": (ctypes.c_int, [_P, _I64, _I64, _I64, ctypes.c_int, ctypes.c_int,
                                               ctypes.c_float, _P, _P, _P, _P]),
+    "nvfp4_quantize_arc": (ctypes.c_int, [_P, _I64, _I64, _I64, _P, _I64, ctypes.c_int, ctypes.c_int,
+                                          ctypes.c_int, ctypes.c_float, _P, _P, _P, _P, ctypes.c_size_t, _P]),
     "nvfp4_quantize_t": (ctypes.c_int, [_P, _I64, _I64, _I64, ctypes.c_int, ctypes.c_int,
                                         ctypes.c_float, _P, _P, _P, _P, ctypes.c_size_t, _P]),
     "nvfp4_quantize_with_scale": (ctypes.c_int, [_P, _I64, _I64, _I64, ctypes.c_int, ctypes.c_int,
@@ -108,6 +110,13 @@ def nvfp4_quantize_noalloc(x, rows, K, ldx, mode, rule, fp8_max, codes, scales, 
     library: no workspace argument, nothing allocated (see include/nvfp4.h)."""
     return load().nvfp4_quantize_noalloc(x, rows, K, ldx, mode, rule, fp8_max, codes, scales,
                                          global_scale, stream)
+
+
+def nvfp4_quantize_arc(x, rows, K, ldx, perm, S, augment, mode, rule, fp8_max, codes, scales,
+                       global_scale, workspace, workspace_bytes, stream) -> int:
+    """Augmented residual-channel quantization (perm: device int32[K])."""
+    return load().nvfp4_quantize_arc(x, rows, K, ldx, perm, S, augment, mode, rule, fp8_max, codes,
+                                     scales, global_scale, workspace, workspace_bytes, stream)
 
 
 def nvfp4_quantize_t(x, rows, K, ldx, mode, rule, fp8_max, codes, scales, global_scale, workspace,
@@ -224,6 +233,44 @@ def quantize(x, mode: str = "six", rule: str = "max", fp8_max: float | None = No
                         out.codes.data_ptr(), out.scales.data_ptr(), out.global_scale.data_ptr(),
                         out.workspace.data_ptr(), out.workspace.numel(), _stream_handle(stream))
     _check(st, "nvfp4_quantize")
+    return out
+
+
+AUG_RESIDUAL = 0
+AUG_DUPLICATE = 1
+
+
+def quantize_arc(x, perm, S: int, augment: int = AUG_RESIDUAL, mode: str = "six", rule: str = "max",
+                 fp8_max: float | None = None, out: NVFP4Tensor | None = None, stream=None) -> NVFP4Tensor:
+    """ARCQuant augmented quantization of a CUDA bf16 matrix x [rows, K]:
+    channels in the order ``perm`` (an int32 CUDA tensor, a permutation of
+    0..K-1), then S appended channels -- the residual of the first S
+    reordered channels (AUG_RESIDUAL, activations) or their copy
+    (AUG_DUPLICATE, weights).  The result is the [rows, K + S] operand."""
+    import torch
+
+    if x.dtype != torch.bfloat16 or x.dim() != 2 or not x.is_cuda:
+        raise ValueError("x must be a 2-D bfloat16 CUDA tensor")
+    if x.stride(1) != 1:
+        raise ValueError("x must have unit stride along K")
+    rows, K = x.shape
+    if perm.dtype != torch.int32 or perm.numel() != K or not perm.is_cuda:
+        raise ValueError("perm must be an int32 CUDA tensor with K entries")
+    F = DEFAULT_FP8_MAX[mode] if fp8_max is None else float(fp8_max)
+    KA = K + S
+    if out is None:
+        dev = x.device
+        out = NVFP4Tensor(
+            codes=torch.empty(rows, KA // 2, dtype=torch.uint8, device=dev),
+            scales=torch.empty(max(1, nvfp4_scales_bytes(rows, KA)), dtype=torch.uint8, device=dev),
+            global_scale=torch.empty(1, dtype=torch.float32, device=dev),
+            workspace=torch.empty(nvfp4_quantize_workspace_bytes(rows, K), dtype=torch.uint8, device=dev),
+            rows=rows, K=KA)
+    st = nvfp4_quantize_arc(x.data_ptr(), rows, K, x.stride(0), perm.data_ptr(), S, augment, MODES[mode],
+                            RULES[rule], F, out.codes.data_ptr(), out.scales.data_ptr(),
+                            out.global_scale.data_ptr(), out.workspace.data_ptr(), out.workspace.numel(),
+                            _stream_handle(stream))
+    _check(st, "nvfp4_quantize_arc")
     return out
 
 

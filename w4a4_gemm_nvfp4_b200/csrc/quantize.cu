@@ -43,6 +43,8 @@ namespace {
 
 constexpr int kAmaxThreads = 512;
 constexpr int kMaxPartials = 4096;
+constexpr int kArcRows = 4;          // rows per step of the augmented quantizer
+constexpr int64_t kArcMaxK = 16384;  // its shared memory: 2 bytes x K x (1 + kArcRows)
 constexpr int kQuantThreads = 256;
 constexpr int kQuantWarps = kQuantThreads / 32;
 constexpr uint32_t kAbsMask2 = 0x7FFF7FFFu;  // clears both bf16 sign bits
@@ -283,22 +285,11 @@ __device__ __forceinline__ bool needs_exact_quotient(float q) {
 // Quantize one block held as 8 words of bf16 pairs (element 2j in the low
 // half of word j).  dr[c] = (d, r) of E4M3 scale code c: d = val(c) * alpha,
 // r = 1/d (0 if infinite).
-// Returns the block's max |x| bit pattern (0x7F80 and above: Inf or NaN).
+// The block step on 16 binary32 values held as pairs p[j] = (x_j, x_{j+8})
+// with block max b: scale(s) and codes of the chosen candidate.
 template <bool FOUR_OVER_SIX, int RULE>
-__device__ __forceinline__ uint32_t quantize_block(const uint4& lo, const uint4& hi, const BlockConsts& k,
-                                                   const float2* dr, uint2& codes, uint32_t& scale) {
-  const uint32_t w[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
-  uint32_t m = absmax4(lo, 0u);
-  m = absmax4(hi, m);
-  const uint32_t bbits = max(m & 0xFFFFu, m >> 16);
-  const float b = __uint_as_float(bbits << 16);
-  // p[j] = (x_j, x_{j+8}): x_2i is the low half of word i, x_2i+1 the high half
-  f2 p[8];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    p[2 * i] = make_f2(__uint_as_float(w[i] << 16), __uint_as_float(w[i + 4] << 16));
-    p[2 * i + 1] = make_f2(__uint_as_float(w[i] & 0xFFFF0000u), __uint_as_float(w[i + 4] & 0xFFFF0000u));
-  }
+__device__ __forceinline__ void quantize_pairs(const f2 p[8], float b, const BlockConsts& k,
+                                               const float2* dr, uint2& codes, uint32_t& scale) {
   float s6raw = __fmul_rn(b, k.inv6);
   float s4raw = FOUR_OVER_SIX ? __fmul_rn(b, k.inv4) : 0.0f;
   if (!k.fast_div || needs_exact_quotient(s6raw) || (FOUR_OVER_SIX && needs_exact_quotient(s4raw))) {
@@ -310,7 +301,7 @@ __device__ __forceinline__ uint32_t quantize_block(const uint4& lo, const uint4&
   if (!FOUR_OVER_SIX) {
     codes = candidate_codes(p, dr6.y);
     scale = sc & 0xFFu;
-    return bbits;
+    return;
   }
   const float2 dr4 = dr[sc >> 8];
   uint2 c6, c4;
@@ -319,6 +310,30 @@ __device__ __forceinline__ uint32_t quantize_block(const uint4& lo, const uint4&
   const bool pick4 = E4 < E6;  // ties keep scale 6
   codes = pick4 ? c4 : c6;
   scale = pick4 ? (sc >> 8) : (sc & 0xFFu);
+}
+
+// bf16 block (8 words of bf16 pairs, element 2j in the low half of word j) ->
+// binary32 pairs p[j] = (x_j, x_{j+8}); returns the block's max |x| bit
+// pattern (0x7F80 and above: Inf or NaN).
+__device__ __forceinline__ uint32_t unpack_block(const uint4& lo, const uint4& hi, f2 p[8]) {
+  const uint32_t w[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+  uint32_t m = absmax4(lo, 0u);
+  m = absmax4(hi, m);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    p[2 * i] = make_f2(__uint_as_float(w[i] << 16), __uint_as_float(w[i + 4] << 16));
+    p[2 * i + 1] = make_f2(__uint_as_float(w[i] & 0xFFFF0000u), __uint_as_float(w[i + 4] & 0xFFFF0000u));
+  }
+  return max(m & 0xFFFFu, m >> 16);
+}
+
+// Quantize one bf16 block; returns its max |x| bit pattern.
+template <bool FOUR_OVER_SIX, int RULE>
+__device__ __forceinline__ uint32_t quantize_block(const uint4& lo, const uint4& hi, const BlockConsts& k,
+                                                   const float2* dr, uint2& codes, uint32_t& scale) {
+  f2 p[8];
+  const uint32_t bbits = unpack_block(lo, hi, p);
+  quantize_pairs<FOUR_OVER_SIX, RULE>(p, __uint_as_float(bbits << 16), k, dr, codes, scale);
   return bbits;
 }
 
@@ -335,6 +350,10 @@ struct QuantParams {
   float f6;            // fp8_max * 6
   uint32_t ntasks;     // ceil(rows/128) * 16 * (K/64)
   uint32_t kgroups;    // K / 64
+  // augmented (ARCQuant) quantization only
+  const int32_t* perm = nullptr;  // channel order, K entries
+  int64_t S = 0;                  // augmented channels
+  int augment = 0;                // 0: residual of the first S reordered channels, 1: their copy
 };
 
 // Start of every quantize kernel: alpha (a caller-supplied static scale, or
@@ -534,6 +553,149 @@ __global__ void __launch_bounds__(kQuantThreads)
   }
 }
 
+// E2M1 codes (element i in nibble i of c.x for i < 8, of c.y for i >= 8) back
+// to binary32 pairs q[j] = (val(code j), val(code j+8)), exact via f16.
+__device__ __forceinline__ void decode_pairs(const uint2 c, f2 q[8]) {
+  float v[16];
+#pragma unroll
+  for (int b = 0; b < 4; ++b) {
+    asm("{\n\t.reg .b8 c;\n\t.reg .b32 h2;\n\t.reg .f16 h0, h1;\n\t"
+        "cvt.u8.u32 c, %2;\n\t"
+        "cvt.rn.f16x2.e2m1x2 h2, c;\n\t"
+        "mov.b32 {h0, h1}, h2;\n\t"
+        "cvt.f32.f16 %0, h0;\n\t"
+        "cvt.f32.f16 %1, h1;\n\t}"
+        : "=f"(v[2 * b]), "=f"(v[2 * b + 1])
+        : "r"((c.x >> (8 * b)) & 0xFFu));
+    asm("{\n\t.reg .b8 c;\n\t.reg .b32 h2;\n\t.reg .f16 h0, h1;\n\t"
+        "cvt.u8.u32 c, %2;\n\t"
+        "cvt.rn.f16x2.e2m1x2 h2, c;\n\t"
+        "mov.b32 {h0, h1}, h2;\n\t"
+        "cvt.f32.f16 %0, h0;\n\t"
+        "cvt.f32.f16 %1, h1;\n\t}"
+        : "=f"(v[8 + 2 * b]), "=f"(v[8 + 2 * b + 1])
+        : "r"((c.y >> (8 * b)) & 0xFFu));
+  }
+#pragma unroll
+  for (int j = 0; j < 8; ++j) q[j] = make_f2(v[j], v[j + 8]);
+}
+
+// Augmented quantization (ARCQuant page, 기술 요약 / 방법론): channels of x
+// taken in the order perm, the usual block step on them (primary stage), and
+// S appended channels -- the residual e = fma(-q, d, x) of the first S
+// reordered channels against the primary stage, quantized with the same block
+// step (augment 0), or a copy of them (augment 1, for the weight).  Each CTA
+// takes kArcRows rows at a time: the rows and the permutation sit in shared
+// memory (2 bytes per channel each), so the channel gather reads shared
+// memory only.
+// Output: the [rows, K + S] operand (codes and swizzled scales).
+template <bool FOUR_OVER_SIX, int RULE>
+__global__ void __launch_bounds__(kQuantThreads)
+    quantize_arc_kernel(const QuantParams p) {
+  BlockConsts k;
+  __shared__ float2 s_dr[128];
+  extern __shared__ __align__(16) uint16_t s_dyn[];  // [K] permutation, then [K] row
+  if (!quant_prologue(p, k, s_dr)) return;
+
+  const int64_t K = p.K, KA = p.K + p.S;
+  uint16_t* s_perm = s_dyn;
+  uint16_t* s_rows = s_dyn + K;  // kArcRows rows
+  for (int64_t i = threadIdx.x; i < K; i += kQuantThreads) {
+    const int32_t c = p.perm[i];
+    s_perm[i] = static_cast<uint16_t>(c >= 0 && c < K ? c : 0);  // out-of-range entries read channel 0
+  }
+  const int64_t rows_padded = (p.rows + 127) / 128 * 128;
+  const int64_t half_ka = KA / 2, kgroups_a = KA / 64;
+  const int nprim = static_cast<int>(K / 16), nres = static_cast<int>(p.S / 16);
+  // kArcRows consecutive rows per step (rows_padded is a multiple of 128)
+  for (int64_t row0 = static_cast<int64_t>(blockIdx.x) * kArcRows; row0 < rows_padded;
+       row0 += static_cast<int64_t>(gridDim.x) * kArcRows) {
+    __syncthreads();  // the permutation is staged / the previous rows are consumed
+    for (int rr = 0; rr < kArcRows; ++rr) {
+      if (row0 + rr >= p.rows) break;
+      const uint4* src = reinterpret_cast<const uint4*>(p.x + (row0 + rr) * p.ldx);
+      uint4* dst = reinterpret_cast<uint4*>(s_rows + rr * K);
+      for (int64_t c = threadIdx.x; c < K / 8; c += kQuantThreads) dst[c] = ld_stream(src + c);
+    }
+    __syncthreads();
+    for (int jr = threadIdx.x; jr < kArcRows * nprim; jr += kQuantThreads) {
+      const int rr = jr / nprim, j = jr - rr * nprim;
+      const int64_t row = row0 + rr;
+      const bool live = row < p.rows;
+      const uint16_t* s_row = s_rows + rr * K;
+      const int64_t atom_row = (row >> 7) * kgroups_a;
+      const int64_t in_atom = (row & 31) * 16 + ((row >> 5) & 3) * 4;
+      uint32_t scale = 0, scale_a = 0;
+      uint2 codes = make_uint2(0u, 0u), codes_a = codes;
+      if (live) {
+        // gather the block's 16 channels as bf16 pairs (element 2i low)
+        uint32_t w[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          w[i] = static_cast<uint32_t>(s_row[s_perm[16 * j + 2 * i]]) |
+                 (static_cast<uint32_t>(s_row[s_perm[16 * j + 2 * i + 1]]) << 16);
+        f2 px[8];
+        const uint32_t bbits = unpack_block(make_uint4(w[0], w[1], w[2], w[3]),
+                                            make_uint4(w[4], w[5], w[6], w[7]), px);
+        quantize_pairs<FOUR_OVER_SIX, RULE>(px, __uint_as_float(bbits << 16), k, s_dr, codes, scale);
+        if (j < nres) {
+          if (p.augment) {
+            codes_a = codes;
+            scale_a = scale;
+          } else {
+            const float d = s_dr[scale].x;
+            const f2 nd = make_f2(-d, -d);
+            f2 q[8], e[8];
+            decode_pairs(codes, q);
+            float b = 0.0f;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              e[i] = fma2(q[i], nd, px[i]);
+              b = fmaxf(b, fmaxf(fabsf(e[i].a()), fabsf(e[i].b())));
+            }
+            quantize_pairs<FOUR_OVER_SIX, RULE>(e, b, k, s_dr, codes_a, scale_a);
+          }
+        }
+        *reinterpret_cast<uint2*>(p.codes + row * half_ka + j * 8) = codes;
+        if (j < nres) *reinterpret_cast<uint2*>(p.codes + row * half_ka + (nprim + j) * 8) = codes_a;
+      }
+      p.scales[(atom_row + (j >> 2)) * 512 + in_atom + (j & 3)] = static_cast<uint8_t>(scale);
+      if (j < nres) {
+        const int ja = nprim + j;
+        p.scales[(atom_row + (ja >> 2)) * 512 + in_atom + (ja & 3)] = static_cast<uint8_t>(scale_a);
+      }
+    }
+  }
+}
+
+template <bool F, int R>
+cudaError_t launch_quantize_arc(int sms, const QuantParams& p, cudaStream_t s) {
+  const size_t smem = static_cast<size_t>(p.K) * 2 * (1 + kArcRows);
+  static std::atomic<int> attr_done{0};
+  if (!attr_done.load(std::memory_order_relaxed)) {
+    cudaError_t e = cudaFuncSetAttribute(quantize_arc_kernel<F, R>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(kArcMaxK * 2 * (1 + kArcRows)));
+    if (e != cudaSuccess) return e;
+    attr_done.store(1, std::memory_order_relaxed);
+  }
+  int occ = 0;
+  cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, quantize_arc_kernel<F, R>,
+                                                                kQuantThreads, smem);
+  if (e != cudaSuccess) return e;
+  const int64_t steps = (p.rows + 127) / 128 * 128 / kArcRows;
+  const int grid = static_cast<int>(std::max<int64_t>(
+      1, std::min<int64_t>(steps, static_cast<int64_t>(sms) * std::max(1, occ))));
+  quantize_arc_kernel<F, R><<<grid, kQuantThreads, smem, s>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quantize_arc_kernel(int mode, int rule, int sms, const QuantParams& p, cudaStream_t s) {
+  if (mode == NVFP4_MODE_SIX) return launch_quantize_arc<false, kRuleMax>(sms, p, s);
+  if (rule == NVFP4_RULE_MAX) return launch_quantize_arc<true, kRuleMax>(sms, p, s);
+  if (rule == NVFP4_RULE_MAE) return launch_quantize_arc<true, kRuleMae>(sms, p, s);
+  return launch_quantize_arc<true, kRuleMse>(sms, p, s);
+}
+
 template <bool F, int R>
 cudaError_t launch_quantize_t(int sms, const QuantParams& p, cudaStream_t s) {
   static std::atomic<int> per_sm{0};
@@ -601,11 +763,23 @@ namespace {
 
 // nvfp4_quantize (row-wise blocks of x) and nvfp4_quantize_t (blocks along
 // the rows of x, i.e. the operand of x^T): amax pass, then the quantize kernel.
-nvfp4_status quantize_impl(const char* fn, bool transposed, const void* x, int64_t rows, int64_t K,
+enum class QuantKind { kRows, kTransposed, kAugmented };
+
+nvfp4_status quantize_impl(const char* fn, QuantKind kind, const void* x, int64_t rows, int64_t K,
                            int64_t ldx, int mode, int rule, float fp8_max, void* codes, void* scales,
-                           float* global_scale, void* workspace, size_t workspace_bytes, void* stream) {
+                           float* global_scale, void* workspace, size_t workspace_bytes, void* stream,
+                           const int32_t* perm = nullptr, int64_t S = 0, int augment = 0) {
+  const bool transposed = kind == QuantKind::kTransposed;
   if (!x || !codes || !scales || !global_scale || !workspace)
     return set_error(NVFP4_ERR_INVALID_ARG, "%s: null pointer argument", fn);
+  if (kind == QuantKind::kAugmented) {
+    if (!perm || (reinterpret_cast<uintptr_t>(perm) & 3u))
+      return set_error(NVFP4_ERR_INVALID_ARG, "%s: perm must be a non-null 4-byte aligned device pointer", fn);
+    if (S < 0 || S % 64 != 0 || S > K)
+      return set_error(NVFP4_ERR_INVALID_ARG, "%s: need 0 <= S <= K and S %% 64 == 0 (S=%lld)", fn, (long long)S);
+    if (K > kArcMaxK) return set_error(NVFP4_ERR_INVALID_ARG, "%s: K above %lld", fn, (long long)kArcMaxK);
+    if (augment != 0 && augment != 1) return set_error(NVFP4_ERR_INVALID_ARG, "%s: augment must be 0 or 1", fn);
+  }
   if (!transposed && (rows < 1 || K < 64 || K % 64 != 0))
     return set_error(NVFP4_ERR_INVALID_ARG,
                      "%s: need rows >= 1 and K a positive multiple of 64 (rows=%lld K=%lld)", fn,
@@ -628,7 +802,7 @@ nvfp4_status quantize_impl(const char* fn, bool transposed, const void* x, int64
   if (workspace_bytes < nvfp4_quantize_workspace_bytes(rows, K))
     return set_error(NVFP4_ERR_INVALID_ARG, "%s: workspace too small", fn);
   const int64_t row_blocks = (rows + 127) / 128;
-  const int64_t ntasks = transposed ? 0 : (row_blocks * 128 * (K / 16) + 31) / 32;
+  const int64_t ntasks = kind == QuantKind::kRows ? (row_blocks * 128 * (K / 16) + 31) / 32 : 0;
   if (ntasks >= 0x80000000ll || rows * ldx > (1ll << 40))
     return set_error(NVFP4_ERR_INVALID_ARG, "%s: tensor too large", fn);
   int dev = 0, sms = 0;
@@ -668,7 +842,12 @@ nvfp4_status quantize_impl(const char* fn, bool transposed, const void* x, int64
   p.f6 = fp8_max * 6.0f;
   p.ntasks = static_cast<uint32_t>(ntasks);
   p.kgroups = static_cast<uint32_t>(K / 64);
-  e = transposed ? launch_quantize_t_kernel(mode, rule, sms, p, s) : launch_quantize_kernel(mode, rule, sms, p, s);
+  p.perm = perm;
+  p.S = S;
+  p.augment = augment;
+  e = kind == QuantKind::kTransposed ? launch_quantize_t_kernel(mode, rule, sms, p, s)
+      : kind == QuantKind::kAugmented ? launch_quantize_arc_kernel(mode, rule, sms, p, s)
+                                       : launch_quantize_kernel(mode, rule, sms, p, s);
   if (e != cudaSuccess) return cuda_status(e, "quantize kernel launch");
   return NVFP4_OK;
 }
@@ -681,15 +860,23 @@ nvfp4_status nvfp4_quantize(const void* x, int64_t rows, int64_t K, int64_t ldx,
                             int rule, float fp8_max, void* codes, void* scales,
                             float* global_scale, void* workspace, size_t workspace_bytes,
                             void* stream) {
-  return quantize_impl("nvfp4_quantize", false, x, rows, K, ldx, mode, rule, fp8_max, codes, scales,
+  return quantize_impl("nvfp4_quantize", QuantKind::kRows, x, rows, K, ldx, mode, rule, fp8_max, codes, scales,
                        global_scale, workspace, workspace_bytes, stream);
+}
+
+nvfp4_status nvfp4_quantize_arc(const void* x, int64_t rows, int64_t K, int64_t ldx,
+                                const int32_t* perm, int64_t S, int augment, int mode, int rule,
+                                float fp8_max, void* codes, void* scales, float* global_scale,
+                                void* workspace, size_t workspace_bytes, void* stream) {
+  return quantize_impl("nvfp4_quantize_arc", QuantKind::kAugmented, x, rows, K, ldx, mode, rule, fp8_max,
+                       codes, scales, global_scale, workspace, workspace_bytes, stream, perm, S, augment);
 }
 
 nvfp4_status nvfp4_quantize_t(const void* x, int64_t rows, int64_t K, int64_t ldx, int mode,
                               int rule, float fp8_max, void* codes, void* scales,
                               float* global_scale, void* workspace, size_t workspace_bytes,
                               void* stream) {
-  return quantize_impl("nvfp4_quantize_t", true, x, rows, K, ldx, mode, rule, fp8_max, codes, scales,
+  return quantize_impl("nvfp4_quantize_t", QuantKind::kTransposed, x, rows, K, ldx, mode, rule, fp8_max, codes, scales,
                        global_scale, workspace, workspace_bytes, stream);
 }
 
