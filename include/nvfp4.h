@@ -223,6 +223,25 @@ NVFP4_API nvfp4_status nvfp4_gemm(const void* a_codes, const void* a_scales, con
                         int64_t M, int64_t N, int64_t K, void* y, int64_t ldy, int out_dtype,
                         void* workspace, size_t workspace_bytes, void* stream);
 
+/* nvfp4_gemm whose epilogue writes Y as an NVFP4 operand instead of bf16: Y is
+ * rounded to bf16 exactly as nvfp4_gemm's bf16 output would be, then each
+ * 16-column block goes through the block step of nvfp4_quantize (mode, rule)
+ * against the caller-supplied tensor scale *y_alpha (device), so the result
+ * equals nvfp4_gemm (bf16) followed by nvfp4_quantize_with_scale, bit for bit,
+ * without Y ever being written in bf16.  This is the quantization fused into
+ * the producing op's epilogue that a calibrated (static) alpha makes possible
+ * (Minima page, "심층 분석": calibrated module-level scales).
+ *   y_codes   [M, N/2], 16-byte aligned;  y_scales  nvfp4_scales_bytes(M, N)
+ * Requirements as nvfp4_gemm plus N % 64 == 0.  Device status as
+ * nvfp4_quantize_with_scale: NVFP4_ERR_INVALID_ARG when *y_alpha is not a
+ * positive finite number (nothing is written), NVFP4_ERR_NONFINITE when a
+ * block of Y holds Inf/NaN (written as zeros).  One memset, one kernel. */
+NVFP4_API nvfp4_status nvfp4_gemm_quantized(const void* a_codes, const void* a_scales, const float* a_global,
+                                            const void* b_codes, const void* b_scales, const float* b_global,
+                                            int64_t M, int64_t N, int64_t K, int mode, int rule,
+                                            const float* y_alpha, void* y_codes, void* y_scales,
+                                            void* workspace, size_t workspace_bytes, void* stream);
+
 /* nvfp4_gemm with one B global scale per output-column segment, for one GEMM
  * over several weights fused along N (e.g. the Q, K and V projections, or
  * gate and up), each quantized with its own tensor scale -- for instance

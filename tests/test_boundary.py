@@ -139,6 +139,22 @@ def test_gemm_rejects_bad_arguments(bad):
     assert _g(**bad) == nv.ERR_INVALID_ARG
 
 
+def _gq(**kw):
+    args = dict(a_codes=FAKE, a_scales=FAKE, a_global=FAKE, b_codes=FAKE, b_scales=FAKE, b_global=FAKE,
+                M=64, N=256, K=512, mode=1, rule=2, y_alpha=FAKE, y_codes=FAKE, y_scales=FAKE, workspace=FAKE,
+                workspace_bytes=64, stream=None)
+    args.update(kw)
+    return nv.nvfp4_gemm_quantized(*args.values())
+
+
+@pytest.mark.parametrize("bad", [
+    dict(y_alpha=None), dict(y_codes=None), dict(y_scales=None), dict(N=96), dict(mode=4), dict(rule=9),
+    dict(y_codes=FAKE + 8), dict(y_alpha=FAKE + 1), dict(K=100), dict(M=0),
+])
+def test_gemm_quantized_rejects_bad_arguments(bad):
+    assert _gq(**bad) == nv.ERR_INVALID_ARG
+
+
 def _gs(ends=(256,), nseg=None, **kw):
     import ctypes as C
     arr = (C.c_int64 * max(1, len(ends)))(*ends)
@@ -171,5 +187,6 @@ def test_no_gpu_fails_loudly():
     assert _qs() in (nv.ERR_CUDA, nv.ERR_UNSUPPORTED_DEVICE)
     assert _qt() in (nv.ERR_CUDA, nv.ERR_UNSUPPORTED_DEVICE)
     assert _qa() in (nv.ERR_CUDA, nv.ERR_UNSUPPORTED_DEVICE)
+    assert _gq() in (nv.ERR_CUDA, nv.ERR_UNSUPPORTED_DEVICE)
     assert _gs((64, 128, 256)) in (nv.ERR_CUDA, nv.ERR_UNSUPPORTED_DEVICE)
     assert _g() in (nv.ERR_CUDA, nv.ERR_UNSUPPORTED_DEVICE)

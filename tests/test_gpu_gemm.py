@@ -187,3 +187,27 @@ def test_gemm_segmented_one_segment_is_gemm():
     y2 = nv.gemm_segmented(A, B, B.global_scale.clone(), [520], out_dtype=torch.float32)
     torch.cuda.synchronize()
     assert torch.equal(y1, y2)
+
+
+# ----------------------------------------------- NVFP4 output (static alpha) --
+
+@pytest.mark.parametrize("M,N,K", [(64, 128, 512), (200, 320, 256), (300, 1024, 1024)])
+@pytest.mark.parametrize("recipe", [("six", "max"), ("four_over_six", "mse"), ("four_over_six", "mae"),
+                                    ("four_over_six", "max")], ids=lambda r: "-".join(r))
+def test_gemm_quantized_output_equals_gemm_then_quantize(M, N, K, recipe):
+    """The fused epilogue equals nvfp4_gemm (bf16 Y) followed by
+    nvfp4_quantize_with_scale, bit for bit, and the oracle's row quantizer on
+    that bf16 Y at the same alpha."""
+    mode, rule = recipe
+    ac, as_, aa = _quantized(M, K, 31, ("four_over_six", "mse", 256.0))
+    bc, bs, ba = _quantized(N, K, 32, ("six", "max", 448.0), kind="normal")
+    A, B = upload_operand(ac, as_, aa), upload_operand(bc, bs, ba)
+    y = nv.gemm(A, B, out_dtype=torch.bfloat16)
+    alpha = torch.tensor([float(y.float().abs().max()) / (6 * 448.0) * 1.3], dtype=torch.float32, device="cuda")
+    ref = nv.quantize(y, mode, rule, out=None, global_scale=alpha)
+    q = nv.gemm_quantized(A, B, alpha, mode, rule)
+    assert nv.device_status(q.workspace) == nv.OK
+    assert torch.equal(q.codes, ref.codes) and torch.equal(q.scales, ref.scales)
+    oc, os_ = oracle.quantize_rows(y.cpu(), float(alpha.cpu()[0]), MODE[mode], RULE[rule])
+    assert np.array_equal(to_np(q.codes), oc)
+    assert np.array_equal(to_np(q.scales), oracle.swizzle_scales(os_, M, N))

@@ -12,7 +12,7 @@ a ctypes binding around its C ABI (``include/nvfp4.h``).
 from ._lib import (  # noqa: F401
     DEFAULT_FP8_MAX, ERR_CUDA, ERR_INVALID_ARG, ERR_NONFINITE, ERR_TIMEOUT, ERR_UNSUPPORTED_DEVICE,
     LIB_PATH, MODES, OK, OUT_BF16, OUT_FP32, RULES, NVFP4Error, NVFP4Tensor, device_status, gemm,
-    gemm_segmented, nvfp4_gemm_segmented,
+    gemm_segmented, nvfp4_gemm_segmented, gemm_quantized, nvfp4_gemm_quantized,
     last_error_message, load, nvfp4_codes_bytes, nvfp4_gemm, nvfp4_gemm_workspace_bytes,
     nvfp4_get_device_status, nvfp4_quantize, nvfp4_quantize_noalloc, nvfp4_quantize_with_scale,
     nvfp4_quantize_workspace_bytes, nvfp4_scales_bytes,

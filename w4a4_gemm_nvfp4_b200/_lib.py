@@ -45,6 +45,8 @@ _SIGNATURES = {
                                                  _P, _P, _P, _P, ctypes.c_size_t, _P]),
     "nvfp4_gemm": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _I64,
                                   ctypes.c_int, _P, ctypes.c_size_t, _P]),
+    "nvfp4_gemm_quantized": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, ctypes.c_int, ctypes.c_int,
+                                            _P, _P, _P, _P, ctypes.c_size_t, _P]),
     "nvfp4_gemm_segmented": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, ctypes.c_int, _I64, _I64,
                                             _I64, _P, _I64, ctypes.c_int, _P, ctypes.c_size_t, _P]),
     "nvfp4_get_device_status": (ctypes.c_int, [_P, _P]),
@@ -138,6 +140,14 @@ def nvfp4_gemm(a_codes, a_scales, a_global, b_codes, b_scales, b_global, M, N, K
                out_dtype, workspace, workspace_bytes, stream) -> int:
     return load().nvfp4_gemm(a_codes, a_scales, a_global, b_codes, b_scales, b_global, M, N, K, y,
                              ldy, out_dtype, workspace, workspace_bytes, stream)
+
+
+def nvfp4_gemm_quantized(a_codes, a_scales, a_global, b_codes, b_scales, b_global, M, N, K, mode, rule,
+                         y_alpha, y_codes, y_scales, workspace, workspace_bytes, stream) -> int:
+    """nvfp4_gemm with Y written as an NVFP4 operand (static alpha)."""
+    return load().nvfp4_gemm_quantized(a_codes, a_scales, a_global, b_codes, b_scales, b_global, M, N, K,
+                                       mode, rule, y_alpha, y_codes, y_scales, workspace, workspace_bytes,
+                                       stream)
 
 
 def nvfp4_gemm_segmented(a_codes, a_scales, a_global, b_codes, b_scales, b_globals, seg_ends, nseg,
@@ -320,6 +330,32 @@ def gemm(a: NVFP4Tensor, b: NVFP4Tensor, out_dtype=None, out=None, workspace=Non
                     out.data_ptr(), out.stride(0), code, workspace.data_ptr(), workspace.numel(),
                     _stream_handle(stream))
     _check(st, "nvfp4_gemm")
+    return out
+
+
+def gemm_quantized(a: NVFP4Tensor, b: NVFP4Tensor, y_alpha, mode: str = "six", rule: str = "max",
+                   out: NVFP4Tensor | None = None, stream=None) -> NVFP4Tensor:
+    """Y = A_hat @ B_hat^T written directly as an NVFP4 [M, N] operand,
+    quantized against the float32 CUDA tensor ``y_alpha`` (one element)."""
+    import torch
+
+    if a.K != b.K:
+        raise ValueError("operands disagree on K")
+    M, N = a.rows, b.rows
+    dev = a.codes.device
+    if out is None:
+        out = NVFP4Tensor(
+            codes=torch.empty(M, N // 2, dtype=torch.uint8, device=dev),
+            scales=torch.empty(max(1, nvfp4_scales_bytes(M, N)), dtype=torch.uint8, device=dev),
+            global_scale=y_alpha.reshape(1),
+            workspace=torch.empty(nvfp4_gemm_workspace_bytes(), dtype=torch.uint8, device=dev),
+            rows=M, K=N)
+    st = nvfp4_gemm_quantized(a.codes.data_ptr(), a.scales.data_ptr(), a.global_scale.data_ptr(),
+                              b.codes.data_ptr(), b.scales.data_ptr(), b.global_scale.data_ptr(), M, N, a.K,
+                              MODES[mode], RULES[rule], y_alpha.data_ptr(), out.codes.data_ptr(),
+                              out.scales.data_ptr(), out.workspace.data_ptr(), out.workspace.numel(),
+                              _stream_handle(stream))
+    _check(st, "nvfp4_gemm_quantized")
     return out
 
 

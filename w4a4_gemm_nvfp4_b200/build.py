@@ -22,9 +22,10 @@ LIB = os.path.join(PKG, "libnvfp4.so")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 COMMON = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC,-fvisibility=hidden", "-I", INCLUDE, "-I", CSRC]
-# Per-file extra flags: the quantizer's arithmetic must not be contracted
-# into FMAs behind the explicit intrinsics' back.
-EXTRA = {"quantize.cu": ["-fmad=false"]}
+# Per-file extra flags: the block step's arithmetic (quantizer kernels, and
+# the GEMM epilogue that writes an NVFP4 output) must not be contracted into
+# FMAs behind the explicit intrinsics' back.
+EXTRA = {"quantize.cu": ["-fmad=false"], "gemm.cu": ["-fmad=false"]}
 SOURCES = ["api.cu", "quantize.cu", "gemm.cu"]
 
 

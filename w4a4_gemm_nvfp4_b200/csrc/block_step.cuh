@@ -1,0 +1,300 @@
+// block_step.cuh -- the NVFP4 block step shared by the quantizer kernels and
+// the GEMM epilogue that writes a quantized output.
+//
+// Definition ("Four Over Six (4/6)" technical summary,
+// gist.science/ko/paper/2512.02010; sections "문제 제기", "적응형 블록 스케일링
+// 알고리즘", "구현 세부 사항"):
+//   per 16-element block, b = max|x|; for Q in {6} or {6, 4}:
+//     s = E4M3_RNE_satfinite(b / (alpha*Q)), d = s*alpha, r = 1/d (0 if inf)
+//     q_i = E2M1_RNE_satfinite(x_i * r), e_i = fma(-q_i, d, x_i)
+//     E_Q = max|e| | sum|e| | sum e^2 (contiguous pairwise tree)
+//   keep Q = 4 iff E_4 < E_6.
+// Every step is one binary32 operation (explicit __f*_rn intrinsics and
+// packed f32x2 PTX), so the result does not depend on FMA contraction.
+#pragma once
+
+#include <cstdint>
+
+namespace nvfp4 {
+namespace {
+
+constexpr uint32_t kAbsMask2 = 0x7FFF7FFFu;  // clears both bf16 sign bits
+
+__device__ __forceinline__ uint32_t max_u16x2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("max.u16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
+__device__ __forceinline__ uint32_t absmax4(const uint4& v, uint32_t m) {
+  m = max_u16x2(m, v.x & kAbsMask2);
+  m = max_u16x2(m, v.y & kAbsMask2);
+  m = max_u16x2(m, v.z & kAbsMask2);
+  return max_u16x2(m, v.w & kAbsMask2);
+}
+
+// ------------------------------------------------------- conversions ----
+
+// Two binary32 -> two E4M3 (RNE, saturating to 448): lo byte from `lo`.
+__device__ __forceinline__ uint32_t cvt_e4m3x2(float hi, float lo) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+// Two E4M3 (byte pair) -> two binary32 (exact, via f16).
+__device__ __forceinline__ void e4m3x2_to_f32(uint32_t pair, float& lo, float& hi) {
+  asm("{\n\t.reg .b32 h2;\n\t.reg .f16 h0, h1;\n\t"
+      "cvt.rn.f16x2.e4m3x2 h2, %2;\n\t"
+      "mov.b32 {h0, h1}, h2;\n\t"
+      "cvt.f32.f16 %0, h0;\n\t"
+      "cvt.f32.f16 %1, h1;\n\t}"
+      : "=f"(lo), "=f"(hi)
+      : "h"(static_cast<uint16_t>(pair)));
+}
+// Two binary32 -> E2M1 codes (RNE, saturating to 6, sign kept); the code byte
+// holds `lo` in its low nibble.
+__device__ __forceinline__ uint32_t e2m1x2_encode(float hi, float lo) {
+  uint32_t byte;
+  asm("{\n\t.reg .b8 c;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 c, %1, %2;\n\t"
+      "cvt.u32.u8 %0, c;\n\t}"
+      : "=r"(byte)
+      : "f"(hi), "f"(lo));
+  return byte;
+}
+// e2m1x2_encode, plus the two code values back as binary32 (exact, via f16).
+__device__ __forceinline__ uint32_t e2m1x2_round(float hi, float lo, float& qlo, float& qhi) {
+  uint32_t byte;
+  asm("{\n\t.reg .b8 c;\n\t.reg .b32 h2;\n\t.reg .f16 h0, h1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 c, %3, %4;\n\t"
+      "cvt.rn.f16x2.e2m1x2 h2, c;\n\t"
+      "mov.b32 {h0, h1}, h2;\n\t"
+      "cvt.f32.f16 %1, h0;\n\t"
+      "cvt.f32.f16 %2, h1;\n\t"
+      "cvt.u32.u8 %0, c;\n\t}"
+      : "=r"(byte), "=f"(qlo), "=f"(qhi)
+      : "f"(hi), "f"(lo));
+  return byte;
+}
+
+// Packed binary32 pairs held in one 64-bit register pair (one IEEE RNE
+// operation per lane, like the scalar instruction on each lane).
+struct f2 {
+  uint64_t v;
+  __device__ __forceinline__ float a() const { return __uint_as_float(static_cast<uint32_t>(v)); }
+  __device__ __forceinline__ float b() const { return __uint_as_float(static_cast<uint32_t>(v >> 32)); }
+};
+__device__ __forceinline__ f2 make_f2(float a, float b) {
+  f2 r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r.v) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ f2 mul2(f2 x, f2 y) {
+  f2 r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r.v) : "l"(x.v), "l"(y.v));
+  return r;
+}
+__device__ __forceinline__ f2 fma2(f2 x, f2 y, f2 z) {
+  f2 r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r.v) : "l"(x.v), "l"(y.v), "l"(z.v));
+  return r;
+}
+__device__ __forceinline__ f2 add2(f2 x, f2 y) {
+  f2 r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r.v) : "l"(x.v), "l"(y.v));
+  return r;
+}
+
+__device__ __forceinline__ float safe_recip(float d) {
+  float r = __frcp_rn(d);
+  return isinf(r) ? 0.0f : r;  // d == 0 or 1/d overflowed
+}
+
+enum { kRuleMax = 0, kRuleMae = 1, kRuleMse = 2 };
+
+// Codes of one candidate: v = x * r per element, E2M1-rounded.  The block's
+// 16 values are held as pairs p[j] = (x_j, x_{j+8}), j < 8; codes byte j holds
+// elements 2j, 2j+1 (low nibble first).
+__device__ __forceinline__ uint2 candidate_codes(const f2 p[8], float r) {
+  const f2 rr = make_f2(r, r);
+  uint32_t bytes[8];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const f2 v0 = mul2(p[2 * j], rr), v1 = mul2(p[2 * j + 1], rr);
+    bytes[j] = e2m1x2_encode(v1.a(), v0.a());
+    bytes[j + 4] = e2m1x2_encode(v1.b(), v0.b());
+  }
+  return make_uint2(bytes[0] | (bytes[1] << 8) | (bytes[2] << 16) | (bytes[3] << 24),
+                    bytes[4] | (bytes[5] << 8) | (bytes[6] << 16) | (bytes[7] << 24));
+}
+
+// One candidate with its block error under RULE.  With the (x_j, x_{j+8})
+// pairing the contiguous pairwise tree of the error terms
+// ((t0+t1)+(t2+t3))+... is exactly three packed additions and one scalar one:
+//   (t_2i + t_2i+1, t_2i+8 + t_2i+9)      = (u_i, u_i+4)   i < 4
+//   (u_2i + u_2i+1, u_2i+4 + u_2i+5)      = (w_i, w_i+2)   i < 2
+//   (w_0 + w_1, w_2 + w_3)                = (z_0, z_1),    then z_0 + z_1.
+template <int RULE>
+__device__ __forceinline__ float candidate(const f2 p[8], float d, float r, uint2& codes) {
+  const f2 rr = make_f2(r, r);
+  const f2 nd = make_f2(-d, -d);
+  f2 v[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) v[j] = mul2(p[j], rr);
+  // element k is v[k % 8].a (k < 8) or v[k % 8].b (k >= 8)
+  float q[16];
+  uint32_t bytes[8];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    // byte j: elements 2j, 2j+1 (first half); byte j+4: elements 2j+8, 2j+9
+    bytes[j] = e2m1x2_round(v[2 * j + 1].a(), v[2 * j].a(), q[2 * j], q[2 * j + 1]);
+    bytes[j + 4] = e2m1x2_round(v[2 * j + 1].b(), v[2 * j].b(), q[2 * j + 8], q[2 * j + 9]);
+  }
+  codes.x = bytes[0] | (bytes[1] << 8) | (bytes[2] << 16) | (bytes[3] << 24);
+  codes.y = bytes[4] | (bytes[5] << 8) | (bytes[6] << 16) | (bytes[7] << 24);
+  // e = fma(-q, d, x), paired like p
+  f2 e[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) e[j] = fma2(make_f2(q[j], q[j + 8]), nd, p[j]);
+  if (RULE == kRuleMax) {
+    float m0 = 0.0f, m1 = 0.0f;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      m0 = fmaxf(m0, fabsf(e[j].a()));
+      m1 = fmaxf(m1, fabsf(e[j].b()));
+    }
+    return fmaxf(m0, m1);
+  }
+  f2 t[8];
+  if (RULE == kRuleMse) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) t[j] = mul2(e[j], e[j]);
+  } else {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) t[j] = make_f2(fabsf(e[j].a()), fabsf(e[j].b()));
+  }
+  const f2 u0 = add2(t[0], t[1]), u1 = add2(t[2], t[3]), u2 = add2(t[4], t[5]), u3 = add2(t[6], t[7]);
+  const f2 w0 = add2(u0, u1), w1 = add2(u2, u3);
+  const f2 z = add2(w0, w1);
+  return __fadd_rn(z.a(), z.b());
+}
+
+// Per-call constants of the block step.  The scale quotient b / (alpha*Q) must
+// be the correctly rounded binary32 quotient before its E4M3 rounding; it is
+// taken as b * fl(1/(alpha*Q)), which is within 3 units in the last place of
+// the quotient, and recomputed by a true division whenever that distance
+// could change the E4M3 result: below the E4M3 normal range (2^-6), or with
+// the 20 bits under E4M3's 3-bit mantissa within 5 units of the rounding
+// midpoint 0x80000.  Above 448 both saturate to 448.
+struct BlockConsts {
+  float a6, a4;      // alpha * 6, alpha * 4
+  float inv6, inv4;  // fl(1 / a6), fl(1 / a4)
+  bool fast_div;     // both reciprocals finite and normal
+};
+__device__ __forceinline__ bool needs_exact_quotient(float q) {
+  const uint32_t b = __float_as_uint(q);
+  return b < 0x3C800008u || ((b & 0xFFFFFu) - 0x7FFFBu) < 11u;
+}
+
+// Quantize one block held as 8 words of bf16 pairs (element 2j in the low
+// half of word j).  dr[c] = (d, r) of E4M3 scale code c: d = val(c) * alpha,
+// r = 1/d (0 if infinite).
+// The block step on 16 binary32 values held as pairs p[j] = (x_j, x_{j+8})
+// with block max b: scale(s) and codes of the chosen candidate.
+template <bool FOUR_OVER_SIX, int RULE>
+__device__ __forceinline__ void quantize_pairs(const f2 p[8], float b, const BlockConsts& k,
+                                               const float2* dr, uint2& codes, uint32_t& scale) {
+  float s6raw = __fmul_rn(b, k.inv6);
+  float s4raw = FOUR_OVER_SIX ? __fmul_rn(b, k.inv4) : 0.0f;
+  if (!k.fast_div || needs_exact_quotient(s6raw) || (FOUR_OVER_SIX && needs_exact_quotient(s4raw))) {
+    s6raw = __fdiv_rn(b, k.a6);
+    if (FOUR_OVER_SIX) s4raw = __fdiv_rn(b, k.a4);
+  }
+  const uint32_t sc = cvt_e4m3x2(s4raw, s6raw);  // low byte: scale-6, high byte: scale-4
+  const float2 dr6 = dr[sc & 0xFFu];
+  if (!FOUR_OVER_SIX) {
+    codes = candidate_codes(p, dr6.y);
+    scale = sc & 0xFFu;
+    return;
+  }
+  const float2 dr4 = dr[sc >> 8];
+  uint2 c6, c4;
+  const float E6 = candidate<RULE>(p, dr6.x, dr6.y, c6);
+  const float E4 = candidate<RULE>(p, dr4.x, dr4.y, c4);
+  const bool pick4 = E4 < E6;  // ties keep scale 6
+  codes = pick4 ? c4 : c6;
+  scale = pick4 ? (sc >> 8) : (sc & 0xFFu);
+}
+
+// bf16 block (8 words of bf16 pairs, element 2j in the low half of word j) ->
+// binary32 pairs p[j] = (x_j, x_{j+8}); returns the block's max |x| bit
+// pattern (0x7F80 and above: Inf or NaN).
+__device__ __forceinline__ uint32_t unpack_block(const uint4& lo, const uint4& hi, f2 p[8]) {
+  const uint32_t w[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+  uint32_t m = absmax4(lo, 0u);
+  m = absmax4(hi, m);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    p[2 * i] = make_f2(__uint_as_float(w[i] << 16), __uint_as_float(w[i + 4] << 16));
+    p[2 * i + 1] = make_f2(__uint_as_float(w[i] & 0xFFFF0000u), __uint_as_float(w[i + 4] & 0xFFFF0000u));
+  }
+  return max(m & 0xFFFFu, m >> 16);
+}
+
+// Quantize one bf16 block; returns its max |x| bit pattern.
+template <bool FOUR_OVER_SIX, int RULE>
+__device__ __forceinline__ uint32_t quantize_block(const uint4& lo, const uint4& hi, const BlockConsts& k,
+                                                   const float2* dr, uint2& codes, uint32_t& scale) {
+  f2 p[8];
+  const uint32_t bbits = unpack_block(lo, hi, p);
+  quantize_pairs<FOUR_OVER_SIX, RULE>(p, __uint_as_float(bbits << 16), k, dr, codes, scale);
+  return bbits;
+}
+
+// E2M1 codes (element i in nibble i of c.x for i < 8, of c.y for i >= 8) back
+// to binary32 pairs q[j] = (val(code j), val(code j+8)), exact via f16.
+__device__ __forceinline__ void decode_pairs(const uint2 c, f2 q[8]) {
+  float v[16];
+#pragma unroll
+  for (int b = 0; b < 4; ++b) {
+    asm("{\n\t.reg .b8 c;\n\t.reg .b32 h2;\n\t.reg .f16 h0, h1;\n\t"
+        "cvt.u8.u32 c, %2;\n\t"
+        "cvt.rn.f16x2.e2m1x2 h2, c;\n\t"
+        "mov.b32 {h0, h1}, h2;\n\t"
+        "cvt.f32.f16 %0, h0;\n\t"
+        "cvt.f32.f16 %1, h1;\n\t}"
+        : "=f"(v[2 * b]), "=f"(v[2 * b + 1])
+        : "r"((c.x >> (8 * b)) & 0xFFu));
+    asm("{\n\t.reg .b8 c;\n\t.reg .b32 h2;\n\t.reg .f16 h0, h1;\n\t"
+        "cvt.u8.u32 c, %2;\n\t"
+        "cvt.rn.f16x2.e2m1x2 h2, c;\n\t"
+        "mov.b32 {h0, h1}, h2;\n\t"
+        "cvt.f32.f16 %0, h0;\n\t"
+        "cvt.f32.f16 %1, h1;\n\t}"
+        : "=f"(v[8 + 2 * b]), "=f"(v[8 + 2 * b + 1])
+        : "r"((c.y >> (8 * b)) & 0xFFu));
+  }
+#pragma unroll
+  for (int j = 0; j < 8; ++j) q[j] = make_f2(v[j], v[j + 8]);
+}
+
+// Per-call constants and the (d, r) table of every E4M3 scale code for a
+// given alpha; the table needs 128 threads (thread t fills entry t).
+__device__ __forceinline__ void make_block_consts(float alpha, BlockConsts& k) {
+  k.a6 = __fmul_rn(alpha, 6.0f);
+  k.a4 = __fmul_rn(alpha, 4.0f);
+  k.inv6 = __frcp_rn(k.a6);
+  k.inv4 = __frcp_rn(k.a4);
+  k.fast_div = k.inv6 >= 1.17549435e-38f && !isinf(k.inv4);
+}
+__device__ __forceinline__ void fill_scale_table(float alpha, float2* dr, uint32_t t) {
+  if (t < 128) {
+    float s, unused;
+    e4m3x2_to_f32(t, s, unused);
+    const float d = t == 0x7F ? 0.0f : __fmul_rn(s, alpha);  // 0x7F is NaN and never produced
+    dr[t] = make_float2(d, safe_recip(d));
+  }
+}
+
+}  // namespace
+}  // namespace nvfp4

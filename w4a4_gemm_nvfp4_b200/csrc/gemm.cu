@@ -52,6 +52,7 @@
 #include <cstring>
 #include <mutex>
 
+#include "block_step.cuh"
 #include "common.cuh"
 #include "nvfp4_testing.h"
 
@@ -175,6 +176,10 @@ struct GemmParams {
   int out_fp32;
   int vec_store;          // rows of Y start 16-byte aligned: vector stores
   int tma_store;          // Y base and row pitch 16-byte aligned: TMA stores through shared memory
+  // NVFP4 output (epilogue kinds 1..4): Y quantized with a caller-supplied alpha
+  const float* q_alpha;
+  uint8_t* q_codes;       // [M, N/2]
+  uint8_t* q_scales;      // swizzled, nvfp4_scales_bytes(M, N)
   uint64_t timeout_ns;
   int debug_flags;        // bit 0: never issue the first stage's copies (timeout test)
 };
@@ -186,6 +191,9 @@ __device__ __forceinline__ void record_timeout(const GemmParams& p, volatile int
   p.ws->status = NVFP4_ERR_TIMEOUT;
 }
 
+// EPI: 0 = bf16 / fp32 output; 1 = NVFP4 output, scale-6; 2, 3, 4 = NVFP4
+// output, Four-Over-Six with the max / MAE / MSE rule.
+template <int EPI>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const __grid_constant__ CUtensorMap tmSFA, const __grid_constant__ CUtensorMap tmSFB,
@@ -366,6 +374,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       while (sg + 1 < p.nseg && col >= p.seg_end[sg]) ++sg;
       return __fmul_rn(alpha_a, __ldg(p.b_global + sg));
     };
+    // NVFP4 output: the block step's constants and (d, r) table for the
+    // output alpha, in the staging area (which the NVFP4 output does not use)
+    BlockConsts qk;
+    float2* q_dr = reinterpret_cast<float2*>(smem + OFF_STG);
+    bool q_ok = true;
+    if (EPI > 0) {
+      const float qa = __ldg(p.q_alpha);
+      q_ok = qa > 0.0f && !isinf(qa);  // a positive finite number, else nothing is written
+      make_block_consts(q_ok ? qa : 1.0f, qk);
+      fill_scale_table(q_ok ? qa : 1.0f, q_dr, threadIdx.x - 64);  // 128 epilogue threads, 128 entries
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      if (!q_ok && threadIdx.x == 64 && rank == 0 && pair == 0) p.ws->status = NVFP4_ERR_INVALID_ARG;
+    }
+    const int64_t q_rows_padded = (static_cast<int64_t>(p.M) + 127) / 128 * 128;
     // this warp's two staging buffers; lane 0 issues (and waits for) every
     // TMA store of the warp, so the bulk groups it waits on are its own
     const uint32_t stg0 = sbase + OFF_STG + static_cast<uint32_t>(quad) * 2 * STG_BYTES;
@@ -401,6 +423,46 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           if (lane == 0) mbar_arrive_cluster(acc_free_leader);
         }
         const int col0 = n0 + sub * static_cast<int>(EPI_N);
+        if (EPI > 0) {
+          // Y rounded to bf16 as the plain output would be, then the block
+          // step over its four 16-column blocks (N % 64 == 0)
+          if (col0 >= p.N || row >= q_rows_padded || !q_ok) continue;
+          const float ab = segment_scale(col0);
+          uint32_t scales4 = 0;
+          uint32_t cw[8];
+          if (row < p.M) {
+#pragma unroll
+            for (int blk = 0; blk < 4; ++blk) {
+              uint32_t w[8];
+#pragma unroll
+              for (int i = 0; i < 8; ++i)
+                w[i] = pack_bf16x2(__uint_as_float(r[16 * blk + 2 * i]) * ab,
+                                   __uint_as_float(r[16 * blk + 2 * i + 1]) * ab);
+              uint2 codes;
+              uint32_t scale;
+              const uint4 lo = make_uint4(w[0], w[1], w[2], w[3]), hi = make_uint4(w[4], w[5], w[6], w[7]);
+              uint32_t bmax;
+              if (EPI == 1) bmax = quantize_block<false, kRuleMax>(lo, hi, qk, q_dr, codes, scale);
+              else if (EPI == 2) bmax = quantize_block<true, kRuleMax>(lo, hi, qk, q_dr, codes, scale);
+              else if (EPI == 3) bmax = quantize_block<true, kRuleMae>(lo, hi, qk, q_dr, codes, scale);
+              else bmax = quantize_block<true, kRuleMse>(lo, hi, qk, q_dr, codes, scale);
+              if (bmax >= 0x7F80u) {  // Inf/NaN in the block: written as zeros, reported
+                codes = make_uint2(0u, 0u);
+                scale = 0u;
+                p.ws->status = NVFP4_ERR_NONFINITE;
+              }
+              cw[2 * blk] = codes.x;
+              cw[2 * blk + 1] = codes.y;
+              scales4 |= scale << (8 * blk);
+            }
+            uint4* dst = reinterpret_cast<uint4*>(p.q_codes + static_cast<int64_t>(row) * (p.N / 2) + col0 / 2);
+            dst[0] = make_uint4(cw[0], cw[1], cw[2], cw[3]);
+            dst[1] = make_uint4(cw[4], cw[5], cw[6], cw[7]);
+          }
+          const int64_t atom = (static_cast<int64_t>(row) >> 7) * (p.N / 64) + col0 / 64;
+          *reinterpret_cast<uint32_t*>(p.q_scales + atom * 512 + (row & 31) * 16 + ((row >> 5) & 3) * 4) = scales4;
+          continue;
+        }
         if (row0 >= p.M || col0 >= p.N) continue;  // warp-uniform
         const float ab = segment_scale(col0);
         if (p.tma_store) {
@@ -595,13 +657,36 @@ void nvfp4_testing_set_gemm_wait(uint64_t timeout_ns, int debug_flags) {
 
 namespace {
 
+template <int EPI>
+cudaError_t launch_gemm(unsigned grid, cudaStream_t s, const CUtensorMap& ta, const CUtensorMap& tb,
+                        const CUtensorMap& tsa, const CUtensorMap& tsb, const CUtensorMap& ty,
+                        const GemmParams& p) {
+  static std::once_flag attr_once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(attr_once, [] {
+    attr_err = cudaFuncSetAttribute(gemm_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    static_cast<int>(SMEM_BYTES));
+  });
+  if (attr_err != cudaSuccess) return attr_err;
+  gemm_kernel<EPI><<<grid, kThreads, SMEM_BYTES, s>>>(ta, tb, tsa, tsb, ty, p);
+  return cudaGetLastError();
+}
+
+// epi: 0 = bf16 / fp32 Y; 1..4 = NVFP4 Y (q_* arguments), see gemm_kernel.
 nvfp4_status gemm_impl(const char* fn, const void* a_codes, const void* a_scales, const float* a_global,
                        const void* b_codes, const void* b_scales, const float* b_global,
                        const int64_t* seg_ends, int nseg, int64_t M, int64_t N, int64_t K, void* y,
                        int64_t ldy, int out_dtype, void* workspace, size_t workspace_bytes,
-                       void* stream) {
+                       void* stream, int epi = 0, const float* q_alpha = nullptr,
+                       void* q_codes = nullptr, void* q_scales = nullptr) {
   if (!a_codes || !a_scales || !a_global || !b_codes || !b_scales || !b_global || !y || !workspace)
     return set_error(NVFP4_ERR_INVALID_ARG, "%s: null pointer argument", fn);
+  if (epi > 0) {
+    if (!q_alpha || !q_codes || !q_scales) return set_error(NVFP4_ERR_INVALID_ARG, "%s: null pointer argument", fn);
+    if (N % 64 != 0) return set_error(NVFP4_ERR_INVALID_ARG, "%s: need N %% 64 == 0 for an NVFP4 output", fn);
+    if (!aligned16(q_codes) || !aligned16(q_scales) || (reinterpret_cast<uintptr_t>(q_alpha) & 3u))
+      return set_error(NVFP4_ERR_INVALID_ARG, "%s: misaligned buffer", fn);
+  }
   if (M < 1 || N < 1 || K < 64 || K % 64 != 0)
     return set_error(NVFP4_ERR_INVALID_ARG, "%s: need M, N >= 1 and K a positive multiple of 64 (M=%lld N=%lld K=%lld)", fn,
                      (long long)M, (long long)N, (long long)K);
@@ -636,14 +721,6 @@ nvfp4_status gemm_impl(const char* fn, const void* a_codes, const void* a_scales
   if ((st = make_scale_map(&tsa, a_scales, M, K, 1)) != NVFP4_OK) return st;
   if ((st = make_scale_map(&tsb, b_scales, N, K, 2)) != NVFP4_OK) return st;
 
-  static std::once_flag attr_once;
-  static cudaError_t attr_err = cudaSuccess;
-  std::call_once(attr_once, [] {
-    attr_err = cudaFuncSetAttribute(gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    static_cast<int>(SMEM_BYTES));
-  });
-  if (attr_err != cudaSuccess) return cuda_status(attr_err, "cudaFuncSetAttribute(gemm_kernel)");
-
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t e = cudaMemsetAsync(workspace, 0, sizeof(WorkspaceHeader), s);
   if (e != cudaSuccess) return cuda_status(e, "cudaMemsetAsync(status)");
@@ -666,7 +743,10 @@ nvfp4_status gemm_impl(const char* fn, const void* a_codes, const void* a_scales
   p.num_tiles = static_cast<uint32_t>(num_tiles);
   p.out_fp32 = out_dtype == NVFP4_OUT_FP32;
   p.vec_store = aligned16(y) && ((ldy * (p.out_fp32 ? 4 : 2)) % 16 == 0);
-  p.tma_store = p.vec_store;
+  p.tma_store = p.vec_store && epi == 0;
+  p.q_alpha = q_alpha;
+  p.q_codes = static_cast<uint8_t*>(q_codes);
+  p.q_scales = static_cast<uint8_t*>(q_scales);
   CUtensorMap ty;
   std::memset(&ty, 0, sizeof(ty));
   if (p.tma_store && (st = make_output_map(&ty, y, M, N, ldy, p.out_fp32 != 0)) != NVFP4_OK) return st;
@@ -674,8 +754,14 @@ nvfp4_status gemm_impl(const char* fn, const void* a_codes, const void* a_scales
   p.debug_flags = g_debug_flags;
   // one CTA pair per two SMs, never more pairs than tiles
   const int64_t pairs = std::max<int64_t>(1, std::min<int64_t>(num_tiles, sms / 2));
-  gemm_kernel<<<static_cast<unsigned>(2 * pairs), kThreads, SMEM_BYTES, s>>>(ta, tb, tsa, tsb, ty, p);
-  e = cudaGetLastError();
+  const unsigned grid = static_cast<unsigned>(2 * pairs);
+  switch (epi) {
+    case 0: e = launch_gemm<0>(grid, s, ta, tb, tsa, tsb, ty, p); break;
+    case 1: e = launch_gemm<1>(grid, s, ta, tb, tsa, tsb, ty, p); break;
+    case 2: e = launch_gemm<2>(grid, s, ta, tb, tsa, tsb, ty, p); break;
+    case 3: e = launch_gemm<3>(grid, s, ta, tb, tsa, tsb, ty, p); break;
+    default: e = launch_gemm<4>(grid, s, ta, tb, tsa, tsb, ty, p); break;
+  }
   if (e != cudaSuccess) return cuda_status(e, "gemm_kernel launch");
   return NVFP4_OK;
 }
@@ -691,6 +777,23 @@ nvfp4_status nvfp4_gemm(const void* a_codes, const void* a_scales, const float* 
   const int64_t end = N;
   return gemm_impl("nvfp4_gemm", a_codes, a_scales, a_global, b_codes, b_scales, b_global, &end, 1,
                    M, N, K, y, ldy, out_dtype, workspace, workspace_bytes, stream);
+}
+
+nvfp4_status nvfp4_gemm_quantized(const void* a_codes, const void* a_scales, const float* a_global,
+                                  const void* b_codes, const void* b_scales, const float* b_global,
+                                  int64_t M, int64_t N, int64_t K, int mode, int rule, const float* y_alpha,
+                                  void* y_codes, void* y_scales, void* workspace, size_t workspace_bytes,
+                                  void* stream) {
+  if (mode != NVFP4_MODE_SIX && mode != NVFP4_MODE_FOUR_OVER_SIX)
+    return set_error(NVFP4_ERR_INVALID_ARG, "nvfp4_gemm_quantized: unknown mode %d", mode);
+  if (rule != NVFP4_RULE_MAX && rule != NVFP4_RULE_MAE && rule != NVFP4_RULE_MSE)
+    return set_error(NVFP4_ERR_INVALID_ARG, "nvfp4_gemm_quantized: unknown rule %d", rule);
+  const int epi = mode == NVFP4_MODE_SIX ? 1 : (rule == NVFP4_RULE_MAX ? 2 : rule == NVFP4_RULE_MAE ? 3 : 4);
+  const int64_t end = N;
+  // y / ldy are not written with an NVFP4 output; y_codes stands in for the pointer checks
+  return gemm_impl("nvfp4_gemm_quantized", a_codes, a_scales, a_global, b_codes, b_scales, b_global, &end,
+                   1, M, N, K, y_codes, N, NVFP4_OUT_BF16, workspace, workspace_bytes, stream, epi, y_alpha,
+                   y_codes, y_scales);
 }
 
 nvfp4_status nvfp4_gemm_segmented(const void* a_codes, const void* a_scales, const float* a_global,
