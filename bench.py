@@ -397,6 +397,80 @@ def run_reference(args, world, rank):
     }
 
 
+def run_sweep(args):
+    """The quantizer sweep over the C2 shapes and recipes, and the GEMM of each
+    configured workload: one JSON line per item (1 GPU; not the headline)."""
+    import w4a4_gemm_nvfp4_b200 as nv
+
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    peaks = _peaks()
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+    flush_rd = torch.zeros(L2_FLUSH_BYTES // 8, dtype=torch.int64, device=device)
+    flush_sum = torch.zeros((), dtype=torch.int64, device=device)
+    stream = torch.cuda.current_stream(device)
+
+    def timed(fn, n):
+        for _ in range(3):
+            fn()
+        ts = []
+        for i in range(n):
+            flush.fill_(i & 0xFF)
+            torch.sum(flush_rd, dim=0, out=flush_sum)
+            torch.cuda._sleep(HOST_LEAD_CYCLES)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            ts.append(e0.elapsed_time(e1))
+        return statistics.median(ts)
+
+    for rows, K in workloads.SWEEP_SHAPES:
+        x = workloads.sweep_operand(rows, K, seed=0).make().to(device)
+        six_kernel = None
+        for m, r, F in workloads.SWEEP_RECIPES:
+            q = nv.quantize(x, m, r, F)
+            qs = nv.quantize(x, m, r, global_scale=q.global_scale)
+            t_e2e = timed(lambda: nv.quantize(x, m, r, F, out=q), args.steps)
+            t_k = timed(lambda: nv.quantize(x, m, r, out=qs, global_scale=q.global_scale), args.steps)
+            assert nv.device_status(q.workspace) == nv.OK and nv.device_status(qs.workspace) == nv.OK
+            if m == "six":
+                six_kernel = t_k
+            n = rows * K
+            print(json.dumps({
+                "sweep": "quantize", "rows": rows, "K": K, "recipe": f"{m}-{r}-{F:g}",
+                "ms_kernel": round(t_k, 4), "GBps_kernel": round(QUANT_BYTES_PER_ELEM * n / t_k / 1e6, 1),
+                "frac_hbm_kernel": round(QUANT_BYTES_PER_ELEM * n / t_k / 1e6 / peaks["hbm"], 4),
+                "ms_end_to_end": round(t_e2e, 4),
+                "GBps_end_to_end": round((QUANT_BYTES_PER_ELEM + AMAX_BYTES_PER_ELEM) * n / t_e2e / 1e6, 1),
+                "overhead_vs_six_kernel": None if m == "six" else round(t_k / six_kernel - 1.0, 4),
+                "l2": "flushed between iterations", "median_of": args.steps}), flush=True)
+        del x
+        torch.cuda.empty_cache()
+    fp4_peak = 4.0 * peaks["bf16"]
+    for name in ("mlp8b", "attn27b", "prefill"):
+        wl = workloads.WORKLOADS[name]
+        xm, xr, xF = wl.x_recipes[-1]
+        wm, wr, wF = wl.w_recipe
+        x = wl.x.make().to(device)
+        w = wl.w.make().to(device)
+        qx = nv.quantize(x, xm, xr, xF)
+        qw = nv.quantize(w, wm, wr, wF)
+        y = torch.empty(wl.M, wl.N, dtype=torch.bfloat16, device=device)
+        ws = torch.zeros(nv.nvfp4_gemm_workspace_bytes(), dtype=torch.uint8, device=device)
+        t = timed(lambda: nv.gemm(qx, qw, out=y, workspace=ws), args.steps)
+        assert nv.device_status(ws) == nv.OK
+        tf = 2.0 * wl.M * wl.N * wl.K / t / 1e9
+        print(json.dumps({
+            "sweep": "gemm", "workload": name, "M": wl.M, "N": wl.N, "K": wl.K,
+            "x_recipe": f"{xm}-{xr}-{xF:g}", "w_recipe": f"{wm}-{wr}-{wF:g}",
+            "ms": round(t, 4), "TFLOPs": round(tf, 1), "frac_fp4_peak": round(tf / fp4_peak, 4),
+            "l2": "flushed between iterations", "median_of": args.steps}), flush=True)
+        del x, w, qx, qw, y
+        torch.cuda.empty_cache()
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -408,6 +482,9 @@ def main():
                     help="mode,rule,fp8_max for X (default four_over_six,mse,256)")
     ap.add_argument("--cpu-rows", type=int, default=256, help="X rows per oracle step (reference arm)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--sweep", action="store_true",
+                    help="instead of the headline step: the quantizer sweep and every GEMM workload, "
+                         "one JSON line each (1 GPU)")
     args = ap.parse_args()
     m, r, f = args.x_recipe.split(",")
     args.x_recipe = (m, r, float(f))
@@ -415,6 +492,10 @@ def main():
         ap.error("--warmup must be >= 3")
 
     world, rank, local = _dist()
+    if args.sweep:
+        if world == 1 and args.impl == "ours":
+            run_sweep(args)
+        return
     if args.impl == "reference":
         if rank == 0:
             print(json.dumps(run_reference(args, world, rank)), flush=True)
