@@ -24,7 +24,7 @@
  *          section "문제 정의" (problem definition): NVFP4 blocks are 16
  *          elements along the reduction dimension.
  *
- * Readings where the pages are silent (each one is listed in the design doc):
+ * Readings where the pages are silent:
  *   - alpha = amax / (F * 6) with F = fp8_max in {448, 256}; alpha = 1 when
  *     amax == 0; a non-finite amax is an error.
  *   - every step is one IEEE-754 binary32 operation, round-to-nearest-even,

@@ -117,7 +117,7 @@ struct QuantParams {
   WorkspaceHeader* ws;
   int nparts;
   float f6;            // fp8_max * 6
-  uint32_t ntasks;     // ceil(rows/128) * 16 * (K/64)
+  uint32_t ntasks;     // row-wise kernel: warp tasks of 32 blocks over the rows padded to 128
   uint32_t kgroups;    // K / 64
   // augmented (ARCQuant) quantization only
   const int32_t* perm = nullptr;  // channel order, K entries
