@@ -62,19 +62,31 @@ __device__ __forceinline__ uint32_t e2m1x2_encode(float hi, float lo) {
       : "f"(hi), "f"(lo));
   return byte;
 }
-// e2m1x2_encode, plus the two code values back as binary32 (exact, via f16).
-__device__ __forceinline__ uint32_t e2m1x2_round(float hi, float lo, float& qlo, float& qhi) {
-  uint32_t byte;
-  asm("{\n\t.reg .b8 c;\n\t.reg .b32 h2;\n\t.reg .f16 h0, h1;\n\t"
-      "cvt.rn.satfinite.e2m1x2.f32 c, %3, %4;\n\t"
-      "cvt.rn.f16x2.e2m1x2 h2, c;\n\t"
-      "mov.b32 {h0, h1}, h2;\n\t"
-      "cvt.f32.f16 %1, h0;\n\t"
-      "cvt.f32.f16 %2, h1;\n\t"
-      "cvt.u32.u8 %0, c;\n\t}"
-      : "=r"(byte), "=f"(qlo), "=f"(qhi)
-      : "f"(hi), "f"(lo));
-  return byte;
+// Eight binary32 (elements 0..7) -> one word of eight E2M1 codes (element i
+// in nibble i; RNE, saturating to 6, sign kept), and the eight code values
+// back as binary32 (exact, via f16).
+__device__ __forceinline__ uint32_t e2m1x8_round(const float x[8], float q[8]) {
+  uint32_t w;
+  asm("{\n\t.reg .b8 c0, c1, c2, c3;\n\t.reg .b32 h<4>;\n\t.reg .f16 f<8>;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 c0, %10, %9;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 c1, %12, %11;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 c2, %14, %13;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 c3, %16, %15;\n\t"
+      "mov.b32 %0, {c0, c1, c2, c3};\n\t"
+      "cvt.rn.f16x2.e2m1x2 h0, c0;\n\t"
+      "cvt.rn.f16x2.e2m1x2 h1, c1;\n\t"
+      "cvt.rn.f16x2.e2m1x2 h2, c2;\n\t"
+      "cvt.rn.f16x2.e2m1x2 h3, c3;\n\t"
+      "mov.b32 {f0, f1}, h0;\n\tmov.b32 {f2, f3}, h1;\n\t"
+      "mov.b32 {f4, f5}, h2;\n\tmov.b32 {f6, f7}, h3;\n\t"
+      "cvt.f32.f16 %1, f0;\n\tcvt.f32.f16 %2, f1;\n\t"
+      "cvt.f32.f16 %3, f2;\n\tcvt.f32.f16 %4, f3;\n\t"
+      "cvt.f32.f16 %5, f4;\n\tcvt.f32.f16 %6, f5;\n\t"
+      "cvt.f32.f16 %7, f6;\n\tcvt.f32.f16 %8, f7;\n\t}"
+      : "=r"(w), "=f"(q[0]), "=f"(q[1]), "=f"(q[2]), "=f"(q[3]), "=f"(q[4]), "=f"(q[5]),
+        "=f"(q[6]), "=f"(q[7])
+      : "f"(x[0]), "f"(x[1]), "f"(x[2]), "f"(x[3]), "f"(x[4]), "f"(x[5]), "f"(x[6]), "f"(x[7]));
+  return w;
 }
 
 // Packed binary32 pairs held in one 64-bit register pair (one IEEE RNE
@@ -142,16 +154,14 @@ __device__ __forceinline__ float candidate(const f2 p[8], float d, float r, uint
 #pragma unroll
   for (int j = 0; j < 8; ++j) v[j] = mul2(p[j], rr);
   // element k is v[k % 8].a (k < 8) or v[k % 8].b (k >= 8)
-  float q[16];
-  uint32_t bytes[8];
+  float xa[8], xb[8], q[16];
 #pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    // byte j: elements 2j, 2j+1 (first half); byte j+4: elements 2j+8, 2j+9
-    bytes[j] = e2m1x2_round(v[2 * j + 1].a(), v[2 * j].a(), q[2 * j], q[2 * j + 1]);
-    bytes[j + 4] = e2m1x2_round(v[2 * j + 1].b(), v[2 * j].b(), q[2 * j + 8], q[2 * j + 9]);
+  for (int j = 0; j < 8; ++j) {
+    xa[j] = v[j].a();
+    xb[j] = v[j].b();
   }
-  codes.x = bytes[0] | (bytes[1] << 8) | (bytes[2] << 16) | (bytes[3] << 24);
-  codes.y = bytes[4] | (bytes[5] << 8) | (bytes[6] << 16) | (bytes[7] << 24);
+  codes.x = e2m1x8_round(xa, q);
+  codes.y = e2m1x8_round(xb, q + 8);
   // e = fma(-q, d, x), paired like p
   f2 e[8];
 #pragma unroll
