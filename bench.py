@@ -128,6 +128,17 @@ def _barrier(world):
         torch.distributed.barrier()
 
 
+def rank_x_operand(wl, rank: int):
+    """Rank r's activations: the workload's X recipe with its own seed (weak
+    scaling: every rank quantizes and multiplies a different X, same W)."""
+    return workloads.Operand(**{**wl.x.__dict__, "seed": wl.x.seed + 101 * rank})
+
+
+def job_tflops(world: int, flops_per_rank: float, ms_max: float) -> float:
+    """Whole-job throughput: all ranks' flops over the slowest rank's time."""
+    return world * flops_per_rank / (ms_max * 1e-3) / 1e12
+
+
 def _max_over_ranks(world, value: float, device) -> float:
     if world == 1:
         return value
@@ -148,7 +159,7 @@ def run_ours(args, world, rank, local):
     wm, wr, wF = wl.w_recipe
     M, N, K = wl.M, wl.N, wl.K
     # each rank gets its own activations (weak scaling), same weights
-    xop = workloads.Operand(**{**wl.x.__dict__, "seed": wl.x.seed + 101 * rank})
+    xop = rank_x_operand(wl, rank)
     x_host = xop.make().pin_memory()
     x = x_host.to(device)
     w = wl.w.make().to(device)
@@ -258,7 +269,7 @@ def run_ours(args, world, rank, local):
     fp4_peak = 4.0 * peaks["bf16"]
     gemm_tflops = flops / (ms_gemm * 1e-3) / 1e12
     quant_gbs = (QUANT_BYTES_PER_ELEM + AMAX_BYTES_PER_ELEM) * M * K / (ms_quant * 1e-3) / 1e9
-    value = world * flops / (ms_step * 1e-3) / 1e12
+    value = job_tflops(world, flops, ms_step)
     result = {
         "metric": METRIC,
         "value": round(value, 2),
@@ -310,7 +321,7 @@ def run_ours(args, world, rank, local):
             "ms_gemm_after_six": round(_max_over_ranks(world, statistics.mean(tg6), device), 4),
         },
         "e2e": {
-            "value": round(world * flops / (ms_e2e * 1e-3) / 1e12, 2),
+            "value": round(job_tflops(world, flops, ms_e2e), 2),
             "unit": "TFLOP/s",
             "h2d_bytes_per_step": M * K * 2,
             "d2h_bytes_per_step": M * N * 2,
