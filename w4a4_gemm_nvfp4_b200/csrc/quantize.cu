@@ -362,11 +362,13 @@ __global__ void __launch_bounds__(kQuantThreads)
       uint2 codes = make_uint2(0u, 0u), codes_a = codes;
       if (live) {
         // gather the block's 16 channels as bf16 pairs (element 2i low)
+        const uint4 pi0 = reinterpret_cast<const uint4*>(s_perm + 16 * j)[0];
+        const uint4 pi1 = reinterpret_cast<const uint4*>(s_perm + 16 * j)[1];
+        const uint32_t pw[8] = {pi0.x, pi0.y, pi0.z, pi0.w, pi1.x, pi1.y, pi1.z, pi1.w};
         uint32_t w[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i)
-          w[i] = static_cast<uint32_t>(s_row[s_perm[16 * j + 2 * i]]) |
-                 (static_cast<uint32_t>(s_row[s_perm[16 * j + 2 * i + 1]]) << 16);
+          w[i] = static_cast<uint32_t>(s_row[pw[i] & 0xFFFFu]) | (static_cast<uint32_t>(s_row[pw[i] >> 16]) << 16);
         f2 px[8];
         const uint32_t bbits = unpack_block(make_uint4(w[0], w[1], w[2], w[3]),
                                             make_uint4(w[4], w[5], w[6], w[7]), px);
