@@ -2,7 +2,10 @@
  * nvfp4.h -- C ABI of libnvfp4.so: NVFP4 W4A4 linear-layer kernels for
  * NVIDIA B200 (sm_100a).
  *
- * Two operations, both asynchronous on a caller-supplied CUDA stream:
+ * Two core operations, both asynchronous on a caller-supplied CUDA stream
+ * (variants declared further down: a static tensor scale, quantization of
+ * x^T, ARCQuant augmented residual channels, an allocation-free quantizer,
+ * per-segment B scales, and a GEMM that writes an NVFP4 output):
  *
  *  nvfp4_quantize  16-element block-scaled NVFP4 quantization of a bf16
  *                  matrix: E2M1 codes, one FP8 E4M3 scale per 16 elements
@@ -52,14 +55,16 @@
  *           (nvfp4_scales_bytes).  16-byte aligned.
  *   global_scale  one fp32 in device memory (alpha).
  *   Y       bf16 or fp32 [M, N], row-major, row stride ldy >= N elements,
- *           aligned to its element size (rows that start 16-byte aligned get
- *           vector stores).
+ *           aligned to its element size.  When its base and row pitch are
+ *           16-byte aligned the epilogue stores through TMA, otherwise with
+ *           direct stores.
  *
  * Errors: every call validates its arguments on the host and returns a status
  * without launching anything when they are invalid.  Conditions only the GPU
  * can see (non-finite input to nvfp4_quantize, a static alpha that is not a
- * positive finite number, a bounded wait that ran out in nvfp4_gemm) are written to a status word in the call's workspace and read
- * by nvfp4_get_device_status.  Launch failures return NVFP4_ERR_CUDA with
+ * positive finite number, a bounded wait that ran out in nvfp4_gemm) are
+ * written to a status word in the call's workspace and read by
+ * nvfp4_get_device_status.  Launch failures return NVFP4_ERR_CUDA with
  * the CUDA message available from nvfp4_last_error_message.
  *
  * Streams are passed as void* and must be a cudaStream_t of the current
