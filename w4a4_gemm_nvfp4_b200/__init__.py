@@ -2,12 +2,22 @@
 
 ``quantize`` -- 16-element block-scaled NVFP4 quantization (scale-to-6 or
 Four-Over-Six with a max / MAE / MSE selection rule) of a bf16 CUDA matrix,
-writing codes and scales in the layout the block-scaled tensor-core MMA reads.
-``gemm`` -- Y = A_hat @ B_hat^T on two such operands (tcgen05 block-scaled FP4
-MMA, fp32 accumulation, bf16 or fp32 output).
+writing codes and scales in the layout the block-scaled tensor-core MMA reads;
+with ``global_scale=`` a caller-supplied (e.g. calibrated) tensor scale
+replaces the amax pass.
+``quantize_t`` -- the same for x^T (blocks down the columns of x), the layout
+of the gradient GEMMs in training.
+``quantize_arc`` -- ARCQuant augmented residual channels: channels in a
+calibration order plus S appended channels holding the residual of the first
+S (activations) or a copy of them (weights), for one GEMM over K + S.
+``gemm`` -- Y = A_hat @ B_hat^T on two NVFP4 operands (tcgen05 block-scaled FP4
+MMA, fp32 accumulation, bf16 or fp32 output); ``gemm_segmented`` applies one
+B global scale per output-column segment (fused projections);
+``gemm_quantized`` writes Y directly as an NVFP4 operand against a static
+output scale.
 
-Both run in libnvfp4.so (CUDA, built in-tree by ``build.py``); this package is
-a ctypes binding around its C ABI (``include/nvfp4.h``).
+All of it runs in libnvfp4.so (CUDA, built in-tree by ``build.py``); this
+package is a ctypes binding around its C ABI (``include/nvfp4.h``).
 """
 from ._lib import (  # noqa: F401
     DEFAULT_FP8_MAX, ERR_CUDA, ERR_INVALID_ARG, ERR_NONFINITE, ERR_TIMEOUT, ERR_UNSUPPORTED_DEVICE,
