@@ -105,6 +105,20 @@ def test_one_hot_k_block_pins_scale_layout(kb):
     assert np.array_equal(y.astype(np.float64), ref)
 
 
+def test_tile_order_with_partial_last_group():
+    """The output tiles are walked in groups of 32 rows of 256-row tiles.
+    M = 8488 gives 34 rows of tiles: one full group and a ragged group of two.
+    Every output element is checked, so a tile that is skipped or computed
+    twice in the last group fails."""
+    M, N, K = 33 * 256 + 40, 3 * 256 + 64, 256
+    rng = np.random.default_rng(8488)
+    ac, as_ = _random_operand(M, K, rng)
+    bc, bs = _random_operand(N, K, rng)
+    ref, guard = oracle.gemm_reference(ac, as_, 0.5, bc, bs, 2.0)
+    y = _run(upload_operand(ac, as_, 0.5), upload_operand(bc, bs, 2.0), torch.float32)
+    assert_gemm_close(y, ref, guard)
+
+
 # ------------------------------------------------ full sizes, sampled rows --
 
 @pytest.mark.slow
