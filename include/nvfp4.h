@@ -203,7 +203,7 @@ NVFP4_API nvfp4_status nvfp4_quantize_with_scale(const void* x, int64_t rows, in
  * device array of 16448 bytes inside this library, held on every GPU that
  * loads it until the process exits; a launch whose amax pass would need more
  * than its 4096 partial slots is rejected with NVFP4_ERR_INVALID_ARG (a B200
- * uses at most 592).  Nothing in the scratch has to start at zero: every call
+ * uses at most 296, two per SM).  Nothing in the scratch has to start at zero: every call
  * writes what it later reads.  All calls on a device share the array, so calls
  * that may overlap on the GPU race and must be ordered by the caller (same
  * stream, or events).  The first call on each device looks up the array's

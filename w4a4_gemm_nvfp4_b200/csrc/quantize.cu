@@ -496,25 +496,21 @@ size_t nvfp4_quantize_workspace_bytes(int64_t rows, int64_t K) {
 
 namespace {
 
-// nvfp4_quantize (row-wise blocks of x) and nvfp4_quantize_t (blocks along
-// the rows of x, i.e. the operand of x^T): amax pass, then the quantize kernel.
-enum class QuantKind { kRows, kTransposed, kAugmented };
+// ------------------------------------------------------------ host side --
+// Warp tasks of the row-wise kernel: 32 blocks of 16 elements each, over the
+// rows padded to a multiple of 128.
+int64_t row_tasks(int64_t rows, int64_t K) { return ((rows + 127) / 128 * 128 * (K / 16) + 31) / 32; }
 
-nvfp4_status quantize_impl(const char* fn, QuantKind kind, const void* x, int64_t rows, int64_t K,
-                           int64_t ldx, int mode, int rule, float fp8_max, void* codes, void* scales,
-                           float* global_scale, void* workspace, size_t workspace_bytes, void* stream,
-                           const int32_t* perm = nullptr, int64_t S = 0, int augment = 0) {
-  const bool transposed = kind == QuantKind::kTransposed;
-  if (!x || !codes || !scales || !global_scale || !workspace)
+// Checks shared by every quantize entry point: pointers, shape, row pitch,
+// mode, rule, alignment and the size limits of the kernels' index arithmetic.
+// `scale_ptr` is the global-scale output (dynamic alpha) or input (static
+// alpha).  Row-wise blocks need K a multiple of 64; the transposed form
+// (blocks down the columns) needs rows a multiple of 64 and K of 8.
+nvfp4_status check_quant_args(const char* fn, bool transposed, const void* x, int64_t rows, int64_t K,
+                              int64_t ldx, int mode, int rule, const void* codes, const void* scales,
+                              const void* scale_ptr) {
+  if (!x || !codes || !scales || !scale_ptr)
     return set_error(NVFP4_ERR_INVALID_ARG, "%s: null pointer argument", fn);
-  if (kind == QuantKind::kAugmented) {
-    if (!perm || (reinterpret_cast<uintptr_t>(perm) & 3u))
-      return set_error(NVFP4_ERR_INVALID_ARG, "%s: perm must be a non-null 4-byte aligned device pointer", fn);
-    if (S < 0 || S % 64 != 0 || S > K)
-      return set_error(NVFP4_ERR_INVALID_ARG, "%s: need 0 <= S <= K and S %% 64 == 0 (S=%lld)", fn, (long long)S);
-    if (K > kArcMaxK) return set_error(NVFP4_ERR_INVALID_ARG, "%s: K above %lld", fn, (long long)kArcMaxK);
-    if (augment != 0 && augment != 1) return set_error(NVFP4_ERR_INVALID_ARG, "%s: augment must be 0 or 1", fn);
-  }
   if (!transposed && (rows < 1 || K < 64 || K % 64 != 0))
     return set_error(NVFP4_ERR_INVALID_ARG,
                      "%s: need rows >= 1 and K a positive multiple of 64 (rows=%lld K=%lld)", fn,
@@ -529,39 +525,37 @@ nvfp4_status quantize_impl(const char* fn, QuantKind kind, const void* x, int64_
     return set_error(NVFP4_ERR_INVALID_ARG, "%s: unknown mode %d", fn, mode);
   if (rule != NVFP4_RULE_MAX && rule != NVFP4_RULE_MAE && rule != NVFP4_RULE_MSE)
     return set_error(NVFP4_ERR_INVALID_ARG, "%s: unknown rule %d", fn, rule);
+  if (!aligned16(x) || !aligned16(codes) || !aligned16(scales) ||
+      (reinterpret_cast<uintptr_t>(scale_ptr) & 3u))
+    return set_error(NVFP4_ERR_INVALID_ARG, "%s: misaligned buffer", fn);
+  // at most 2^40 elements of x (rows * ldx), and a 32-bit warp-task counter
+  // in the row-wise kernel
+  if (rows > (int64_t{1} << 40) / ldx || row_tasks(rows, K) >= 0x80000000ll)
+    return set_error(NVFP4_ERR_INVALID_ARG, "%s: tensor too large", fn);
+  return NVFP4_OK;
+}
+
+nvfp4_status check_fp8_max(const char* fn, float fp8_max) {
   if (!(fp8_max == 448.0f || fp8_max == 256.0f))
     return set_error(NVFP4_ERR_INVALID_ARG, "%s: fp8_max must be 448 or 256", fn);
-  if (!aligned16(x) || !aligned16(codes) || !aligned16(scales) || !aligned16(workspace) ||
-      (reinterpret_cast<uintptr_t>(global_scale) & 3u))
-    return set_error(NVFP4_ERR_INVALID_ARG, "%s: misaligned buffer", fn);
-  if (workspace_bytes < nvfp4_quantize_workspace_bytes(rows, K))
-    return set_error(NVFP4_ERR_INVALID_ARG, "%s: workspace too small", fn);
-  const int64_t row_blocks = (rows + 127) / 128;
-  const int64_t ntasks = kind == QuantKind::kRows ? (row_blocks * 128 * (K / 16) + 31) / 32 : 0;
-  if (ntasks >= 0x80000000ll || rows * ldx > (1ll << 40))
-    return set_error(NVFP4_ERR_INVALID_ARG, "%s: tensor too large", fn);
-  int dev = 0, sms = 0;
-  nvfp4_status st = check_device(&dev, &sms);
-  if (st != NVFP4_OK) return st;
+  return NVFP4_OK;
+}
 
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  auto* ws = static_cast<WorkspaceHeader*>(workspace);
-  auto* partials = reinterpret_cast<uint32_t*>(static_cast<char*>(workspace) + sizeof(WorkspaceHeader));
+// CTAs of the amax pass: enough for eight 16-byte loads per thread, at most
+// two per SM (dense x), or one per row up to two per SM (pitched x).
+int amax_grid_size(int64_t rows, int64_t K, int64_t ldx, int sms) {
+  int64_t g;
+  if (ldx == K)
+    g = std::min<int64_t>((rows * K / 8 + kAmaxThreads * 8 - 1) / (kAmaxThreads * 8), int64_t{sms} * 2);
+  else
+    g = std::min<int64_t>(rows, int64_t{sms} * 2);
+  return static_cast<int>(std::max<int64_t>(1, g));
+}
 
-  int amax_grid;
-  if (ldx == K) {
-    const int64_t nvec = rows * K / 8;
-    amax_grid = static_cast<int>(std::min<int64_t>((nvec + kAmaxThreads * 8 - 1) / (kAmaxThreads * 8),
-                                                   static_cast<int64_t>(sms) * 2));
-  } else {
-    amax_grid = static_cast<int>(std::min<int64_t>(rows, static_cast<int64_t>(sms) * 2));
-  }
-  amax_grid = std::max(1, std::min(amax_grid, kMaxPartials));
-  amax_kernel<<<amax_grid, kAmaxThreads, 0, s>>>(static_cast<const uint16_t*>(x), rows, K, ldx,
-                                                  partials);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return cuda_status(e, "amax_kernel launch");
-
+// Kernel parameters common to every entry point; the caller sets the alpha
+// source (partials + nparts + f6 and global_scale, or alpha_in).
+QuantParams base_params(const void* x, int64_t rows, int64_t K, int64_t ldx, void* codes, void* scales,
+                        WorkspaceHeader* ws) {
   QuantParams p;
   p.x = static_cast<const uint16_t*>(x);
   p.rows = rows;
@@ -569,22 +563,73 @@ nvfp4_status quantize_impl(const char* fn, QuantKind kind, const void* x, int64_
   p.ldx = ldx;
   p.codes = static_cast<uint8_t*>(codes);
   p.scales = static_cast<uint8_t*>(scales);
-  p.global_scale = global_scale;
-  p.partials = partials;
+  p.global_scale = nullptr;
+  p.partials = nullptr;
   p.alpha_in = nullptr;
   p.ws = ws;
+  p.nparts = 0;
+  p.f6 = 0.0f;
+  p.ntasks = static_cast<uint32_t>(row_tasks(rows, K));
+  p.kgroups = static_cast<uint32_t>(K / 64);
+  return p;
+}
+
+// The amax pass into `partials` (amax_grid CTAs), then the quantize kernel
+// of `kind` with alpha reduced from those partials.
+enum class QuantKind { kRows, kTransposed, kAugmented };
+
+nvfp4_status launch_dynamic(QuantKind kind, QuantParams p, int mode, int rule, float fp8_max,
+                            float* global_scale, uint32_t* partials, int amax_grid, int sms,
+                            cudaStream_t s) {
+  amax_kernel<<<amax_grid, kAmaxThreads, 0, s>>>(p.x, p.rows, p.K, p.ldx, partials);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_status(e, "amax_kernel launch");
+  p.global_scale = global_scale;
+  p.partials = partials;
   p.nparts = amax_grid;
   p.f6 = fp8_max * 6.0f;
-  p.ntasks = static_cast<uint32_t>(ntasks);
-  p.kgroups = static_cast<uint32_t>(K / 64);
-  p.perm = perm;
-  p.S = S;
-  p.augment = augment;
   e = kind == QuantKind::kTransposed ? launch_quantize_t_kernel(mode, rule, sms, p, s)
       : kind == QuantKind::kAugmented ? launch_quantize_arc_kernel(mode, rule, sms, p, s)
                                        : launch_quantize_kernel(mode, rule, sms, p, s);
   if (e != cudaSuccess) return cuda_status(e, "quantize kernel launch");
   return NVFP4_OK;
+}
+
+// nvfp4_quantize (row-wise blocks of x), nvfp4_quantize_t (blocks along the
+// rows of x, i.e. the operand of x^T) and nvfp4_quantize_arc (row-wise with
+// reordered and augmented channels), with the caller's workspace.
+nvfp4_status quantize_impl(const char* fn, QuantKind kind, const void* x, int64_t rows, int64_t K,
+                           int64_t ldx, int mode, int rule, float fp8_max, void* codes, void* scales,
+                           float* global_scale, void* workspace, size_t workspace_bytes, void* stream,
+                           const int32_t* perm = nullptr, int64_t S = 0, int augment = 0) {
+  nvfp4_status st = check_quant_args(fn, kind == QuantKind::kTransposed, x, rows, K, ldx, mode, rule, codes,
+                                     scales, global_scale);
+  if (st != NVFP4_OK) return st;
+  if ((st = check_fp8_max(fn, fp8_max)) != NVFP4_OK) return st;
+  if (kind == QuantKind::kAugmented) {
+    if (!perm || (reinterpret_cast<uintptr_t>(perm) & 3u))
+      return set_error(NVFP4_ERR_INVALID_ARG, "%s: perm must be a non-null 4-byte aligned device pointer", fn);
+    if (S < 0 || S % 64 != 0 || S > K)
+      return set_error(NVFP4_ERR_INVALID_ARG, "%s: need 0 <= S <= K and S %% 64 == 0 (S=%lld)", fn, (long long)S);
+    if (K > kArcMaxK) return set_error(NVFP4_ERR_INVALID_ARG, "%s: K above %lld", fn, (long long)kArcMaxK);
+    if (augment != 0 && augment != 1) return set_error(NVFP4_ERR_INVALID_ARG, "%s: augment must be 0 or 1", fn);
+  }
+  if (!workspace || !aligned16(workspace))
+    return set_error(NVFP4_ERR_INVALID_ARG, "%s: workspace must be a non-null 16-byte aligned pointer", fn);
+  if (workspace_bytes < nvfp4_quantize_workspace_bytes(rows, K))
+    return set_error(NVFP4_ERR_INVALID_ARG, "%s: workspace too small", fn);
+  int dev = 0, sms = 0;
+  if ((st = check_device(&dev, &sms)) != NVFP4_OK) return st;
+
+  auto* ws = static_cast<WorkspaceHeader*>(workspace);
+  auto* partials = reinterpret_cast<uint32_t*>(static_cast<char*>(workspace) + sizeof(WorkspaceHeader));
+  QuantParams p = base_params(x, rows, K, ldx, codes, scales, ws);
+  p.perm = perm;
+  p.S = S;
+  p.augment = augment;
+  const int amax_grid = std::min(amax_grid_size(rows, K, ldx, sms), kMaxPartials);
+  return launch_dynamic(kind, p, mode, rule, fp8_max, global_scale, partials, amax_grid, sms,
+                        static_cast<cudaStream_t>(stream));
 }
 
 }  // namespace
@@ -631,7 +676,7 @@ nvfp4_status nvfp4_quantize_t(const void* x, int64_t rows, int64_t K, int64_t ld
 //
 // The array below is held by every GPU that loads this library, from module
 // load until process exit.  Its size bounds the amax pass at kMaxPartials
-// CTAs (the launch uses at most 4 per SM, 592 on a B200); a launch that would
+// CTAs (the launch uses at most 2 per SM, 296 on a B200); a launch that would
 // need more is rejected.  Nothing in it has to start at zero: each call's amax
 // kernel writes every partial slot the following quantize kernel reads, and
 // the quantize kernel writes the status word.  All calls on a device share it,
@@ -672,74 +717,23 @@ nvfp4_status noalloc_scratch(int dev, void** out) {
 extern "C" nvfp4_status nvfp4_quantize_noalloc(const void* x, int64_t rows, int64_t K, int64_t ldx,
                                                int mode, int rule, float fp8_max, void* codes,
                                                void* scales, float* global_scale, void* stream) {
-  if (!x || !codes || !scales || !global_scale)
-    return set_error(NVFP4_ERR_INVALID_ARG, "nvfp4_quantize_noalloc: null pointer argument");
-  if (rows < 1 || K < 64 || K % 64 != 0)
-    return set_error(NVFP4_ERR_INVALID_ARG,
-                     "nvfp4_quantize_noalloc: need rows >= 1 and K a positive multiple of 64 (rows=%lld K=%lld)",
-                     (long long)rows, (long long)K);
-  if (ldx < K || ldx % 8 != 0)
-    return set_error(NVFP4_ERR_INVALID_ARG, "nvfp4_quantize_noalloc: need ldx >= K and ldx %% 8 == 0");
-  if (mode != NVFP4_MODE_SIX && mode != NVFP4_MODE_FOUR_OVER_SIX)
-    return set_error(NVFP4_ERR_INVALID_ARG, "nvfp4_quantize_noalloc: unknown mode %d", mode);
-  if (rule != NVFP4_RULE_MAX && rule != NVFP4_RULE_MAE && rule != NVFP4_RULE_MSE)
-    return set_error(NVFP4_ERR_INVALID_ARG, "nvfp4_quantize_noalloc: unknown rule %d", rule);
-  if (!(fp8_max == 448.0f || fp8_max == 256.0f))
-    return set_error(NVFP4_ERR_INVALID_ARG, "nvfp4_quantize_noalloc: fp8_max must be 448 or 256");
-  if (!aligned16(x) || !aligned16(codes) || !aligned16(scales) ||
-      (reinterpret_cast<uintptr_t>(global_scale) & 3u))
-    return set_error(NVFP4_ERR_INVALID_ARG, "nvfp4_quantize_noalloc: misaligned buffer");
-  const int64_t row_blocks = (rows + 127) / 128;
-  const int64_t ntasks = (row_blocks * 128 * (K / 16) + 31) / 32;
-  if (ntasks >= 0x80000000ll || rows * ldx > (1ll << 40))
-    return set_error(NVFP4_ERR_INVALID_ARG, "nvfp4_quantize_noalloc: tensor too large");
-  int dev = 0, sms = 0;
-  nvfp4_status st = check_device(&dev, &sms);
+  const char* fn = "nvfp4_quantize_noalloc";
+  nvfp4_status st = check_quant_args(fn, false, x, rows, K, ldx, mode, rule, codes, scales, global_scale);
   if (st != NVFP4_OK) return st;
-
-  int amax_grid;
-  if (ldx == K) {
-    const int64_t nvec = rows * K / 8;
-    amax_grid = static_cast<int>(std::min<int64_t>((nvec + kAmaxThreads * 8 - 1) / (kAmaxThreads * 8),
-                                                   static_cast<int64_t>(sms) * 2));
-  } else {
-    amax_grid = static_cast<int>(std::min<int64_t>(rows, static_cast<int64_t>(sms) * 2));
-  }
-  amax_grid = std::max(1, amax_grid);
+  if ((st = check_fp8_max(fn, fp8_max)) != NVFP4_OK) return st;
+  int dev = 0, sms = 0;
+  if ((st = check_device(&dev, &sms)) != NVFP4_OK) return st;
+  const int amax_grid = amax_grid_size(rows, K, ldx, sms);
   if (amax_grid > kMaxPartials)
     return set_error(NVFP4_ERR_INVALID_ARG,
-                     "nvfp4_quantize_noalloc: the amax pass needs %d partial slots but the static "
-                     "scratch holds %d (%zu bytes)", amax_grid, kMaxPartials, kNoAllocScratchBytes);
-
+                     "%s: the amax pass needs %d partial slots but the static scratch holds %d (%zu bytes)", fn,
+                     amax_grid, kMaxPartials, kNoAllocScratchBytes);
   void* scratch = nullptr;
   if ((st = noalloc_scratch(dev, &scratch)) != NVFP4_OK) return st;
   auto* ws = static_cast<WorkspaceHeader*>(scratch);
   auto* partials = reinterpret_cast<uint32_t*>(static_cast<char*>(scratch) + sizeof(WorkspaceHeader));
-
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  amax_kernel<<<amax_grid, kAmaxThreads, 0, s>>>(static_cast<const uint16_t*>(x), rows, K, ldx,
-                                                  partials);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return cuda_status(e, "amax_kernel launch");
-
-  QuantParams p;
-  p.x = static_cast<const uint16_t*>(x);
-  p.rows = rows;
-  p.K = K;
-  p.ldx = ldx;
-  p.codes = static_cast<uint8_t*>(codes);
-  p.scales = static_cast<uint8_t*>(scales);
-  p.global_scale = global_scale;
-  p.partials = partials;
-  p.alpha_in = nullptr;
-  p.ws = ws;
-  p.nparts = amax_grid;
-  p.f6 = fp8_max * 6.0f;
-  p.ntasks = static_cast<uint32_t>(ntasks);
-  p.kgroups = static_cast<uint32_t>(K / 64);
-  e = launch_quantize_kernel(mode, rule, sms, p, s);
-  if (e != cudaSuccess) return cuda_status(e, "quantize_kernel launch");
-  return NVFP4_OK;
+  return launch_dynamic(QuantKind::kRows, base_params(x, rows, K, ldx, codes, scales, ws), mode, rule, fp8_max,
+                        global_scale, partials, amax_grid, sms, static_cast<cudaStream_t>(stream));
 }
 
 // ------------------------------------------------------ static tensor scale --
@@ -750,44 +744,17 @@ extern "C" nvfp4_status nvfp4_quantize_with_scale(const void* x, int64_t rows, i
                                                   int mode, int rule, const float* global_scale,
                                                   void* codes, void* scales, void* workspace,
                                                   size_t workspace_bytes, void* stream) {
-  if (!x || !codes || !scales || !global_scale || !workspace)
-    return set_error(NVFP4_ERR_INVALID_ARG, "nvfp4_quantize_with_scale: null pointer argument");
-  if (rows < 1 || K < 64 || K % 64 != 0)
-    return set_error(NVFP4_ERR_INVALID_ARG,
-                     "nvfp4_quantize_with_scale: need rows >= 1 and K a positive multiple of 64");
-  if (ldx < K || ldx % 8 != 0)
-    return set_error(NVFP4_ERR_INVALID_ARG, "nvfp4_quantize_with_scale: need ldx >= K and ldx %% 8 == 0");
-  if (mode != NVFP4_MODE_SIX && mode != NVFP4_MODE_FOUR_OVER_SIX)
-    return set_error(NVFP4_ERR_INVALID_ARG, "nvfp4_quantize_with_scale: unknown mode %d", mode);
-  if (rule != NVFP4_RULE_MAX && rule != NVFP4_RULE_MAE && rule != NVFP4_RULE_MSE)
-    return set_error(NVFP4_ERR_INVALID_ARG, "nvfp4_quantize_with_scale: unknown rule %d", rule);
-  if (!aligned16(x) || !aligned16(codes) || !aligned16(scales) || !aligned16(workspace) ||
-      (reinterpret_cast<uintptr_t>(global_scale) & 3u))
-    return set_error(NVFP4_ERR_INVALID_ARG, "nvfp4_quantize_with_scale: misaligned buffer");
-  if (workspace_bytes < sizeof(WorkspaceHeader))
-    return set_error(NVFP4_ERR_INVALID_ARG, "nvfp4_quantize_with_scale: workspace too small");
-  const int64_t row_blocks = (rows + 127) / 128;
-  const int64_t ntasks = (row_blocks * 128 * (K / 16) + 31) / 32;
-  if (ntasks >= 0x80000000ll || rows * ldx > (1ll << 40))
-    return set_error(NVFP4_ERR_INVALID_ARG, "nvfp4_quantize_with_scale: tensor too large");
-  int dev = 0, sms = 0;
-  nvfp4_status st = check_device(&dev, &sms);
+  const char* fn = "nvfp4_quantize_with_scale";
+  nvfp4_status st = check_quant_args(fn, false, x, rows, K, ldx, mode, rule, codes, scales, global_scale);
   if (st != NVFP4_OK) return st;
-  QuantParams p;
-  p.x = static_cast<const uint16_t*>(x);
-  p.rows = rows;
-  p.K = K;
-  p.ldx = ldx;
-  p.codes = static_cast<uint8_t*>(codes);
-  p.scales = static_cast<uint8_t*>(scales);
-  p.global_scale = nullptr;
-  p.partials = nullptr;
+  if (!workspace || !aligned16(workspace))
+    return set_error(NVFP4_ERR_INVALID_ARG, "%s: workspace must be a non-null 16-byte aligned pointer", fn);
+  if (workspace_bytes < sizeof(WorkspaceHeader))
+    return set_error(NVFP4_ERR_INVALID_ARG, "%s: workspace too small", fn);
+  int dev = 0, sms = 0;
+  if ((st = check_device(&dev, &sms)) != NVFP4_OK) return st;
+  QuantParams p = base_params(x, rows, K, ldx, codes, scales, static_cast<WorkspaceHeader*>(workspace));
   p.alpha_in = global_scale;
-  p.ws = static_cast<WorkspaceHeader*>(workspace);
-  p.nparts = 0;
-  p.f6 = 0.0f;
-  p.ntasks = static_cast<uint32_t>(ntasks);
-  p.kgroups = static_cast<uint32_t>(K / 64);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t e = cudaMemsetAsync(workspace, 0, 2 * sizeof(uint32_t), s);  // status, detail
   if (e != cudaSuccess) return cuda_status(e, "nvfp4_quantize_with_scale: status reset");
