@@ -365,6 +365,17 @@ def _w_dequant(wl):
 
 
 def _cores():
+    """Threads the oracle sample runs on: the fp64 GEMM's BLAS pool (the C
+    quantizer is single-threaded and the smaller part), else the CPU affinity."""
+    try:
+        import numpy  # noqa: F401  (loads the BLAS library threadpoolctl inspects)
+        from threadpoolctl import threadpool_info
+
+        blas = [i["num_threads"] for i in threadpool_info() if i.get("user_api") == "blas"]
+        if blas:
+            return max(blas)
+    except Exception:
+        pass
     try:
         return len(os.sched_getaffinity(0))
     except AttributeError:
@@ -381,7 +392,7 @@ def cpu_baseline(args, sample_rows=64):
             "kind": "oracle",
             "sample": f"{sample_rows} rows of X ({wl.K} wide) quantized by the C oracle (1 thread) + "
                       f"fp64 numpy GEMM against the oracle-dequantized W {wl.N}x{wl.K} "
-                      f"(BLAS threads); W quantization untimed; {dt:.1f} s"}
+                      f"({_cores()} BLAS threads); W quantization untimed; {dt:.1f} s"}
 
 
 def run_reference(args, world, rank):
@@ -397,7 +408,7 @@ def run_reference(args, world, rank):
     dt = time.perf_counter() - t0
     value = flops / dt / 1e12
     sample = (f"each step: {rows} rows of X quantized by the C oracle (1 thread) + fp64 numpy "
-              f"GEMM against the oracle-dequantized W {wl.N}x{wl.K}")
+              f"GEMM against the oracle-dequantized W {wl.N}x{wl.K} ({_cores()} BLAS threads)")
     return {
         "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
