@@ -3,8 +3,9 @@
 The functions named like the C ABI (``nvfp4_quantize``, ``nvfp4_gemm``, ...)
 take raw integers (device pointers, sizes, a cudaStream_t handle) and return
 the C status.  ``quantize`` / ``gemm`` wrap them for torch CUDA tensors:
-they allocate outputs with torch, pass pointers and the current stream, and
-raise ``NVFP4Error`` on a non-OK status.  Every step of the computation runs
+they allocate outputs with torch, check every buffer they are given against
+the shape, dtype and device the call reads or writes, pass pointers and the
+current stream, and raise ``NVFP4Error`` on a non-OK status.  Every step of the computation runs
 in the library's kernels; there is no CPU or PyTorch fallback, and importing
 this module on a machine without the built library raises at first use.
 """
@@ -200,6 +201,70 @@ def _check(status: int, what: str) -> None:
         raise NVFP4Error(status, what)
 
 
+# The C ABI takes raw pointers and cannot see buffer sizes, so the wrappers
+# check every torch buffer they pass against the shape the call will read or
+# write: a buffer that is too small, of another dtype or on another device is
+# rejected here instead of being overrun on the GPU.
+
+def _require(t, name: str, dtype, min_numel: int, device, contiguous: bool = True) -> None:
+    import torch
+
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, not {t.dtype}")
+    if t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+    if contiguous and not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if t.numel() < min_numel:
+        raise ValueError(f"{name} holds {t.numel()} elements, the call needs {min_numel}")
+
+
+def _check_operand(q: "NVFP4Tensor", name: str, rows: int, K: int, device, global_scale: bool = True,
+                   workspace: bool = False) -> None:
+    """q's buffers hold (or will hold) a [rows, K] NVFP4 operand on `device`."""
+    import torch
+
+    if (q.rows, q.K) != (rows, K):
+        raise ValueError(f"{name} describes a [{q.rows}, {q.K}] operand, the call needs [{rows}, {K}]")
+    _require(q.codes, f"{name}.codes", torch.uint8, rows * (K // 2), device)
+    _require(q.scales, f"{name}.scales", torch.uint8, nvfp4_scales_bytes(rows, K), device)
+    if global_scale:
+        _require(q.global_scale, f"{name}.global_scale", torch.float32, 1, device, contiguous=False)
+    if workspace:
+        _require(q.workspace, f"{name}.workspace", torch.uint8, 0, device)
+
+
+def _check_output(y, M: int, N: int, dtype, device) -> None:
+    """y is an [M, N] matrix of `dtype` on `device` with unit column stride
+    (rows may be padded: the row pitch is passed as ldy)."""
+    import torch
+
+    if not isinstance(y, torch.Tensor):
+        raise TypeError("out must be a torch.Tensor")
+    if y.dtype != dtype:
+        raise ValueError(f"out must be {dtype}, not {y.dtype}")
+    if y.device != device:
+        raise ValueError(f"out is on {y.device}, expected {device}")
+    if y.dim() != 2 or tuple(y.shape) != (M, N):
+        raise ValueError(f"out must have shape ({M}, {N}), not {tuple(y.shape)}")
+    if y.stride(1) != 1 or y.stride(0) < N:
+        raise ValueError("out must have unit stride along N and a row pitch of at least N")
+
+
+def _out_code(out_dtype, out):
+    """The C output code for out_dtype (default: out's dtype, else bf16)."""
+    import torch
+
+    if out_dtype is None:
+        out_dtype = out.dtype if out is not None else torch.bfloat16
+    codes = {torch.bfloat16: OUT_BF16, torch.float32: OUT_FP32}
+    if out_dtype not in codes:
+        raise ValueError(f"out_dtype must be torch.bfloat16 or torch.float32, not {out_dtype}")
+    return out_dtype, codes[out_dtype]
+
+
 def quantize(x, mode: str = "six", rule: str = "max", fp8_max: float | None = None,
              out: NVFP4Tensor | None = None, stream=None, global_scale=None) -> NVFP4Tensor:
     """NVFP4-quantize a CUDA bf16 matrix [rows, K] (K % 64 == 0).
@@ -230,6 +295,7 @@ def quantize(x, mode: str = "six", rule: str = "max", fp8_max: float | None = No
                           else global_scale.reshape(1)),
             workspace=torch.empty(nvfp4_quantize_workspace_bytes(rows, K), dtype=torch.uint8, device=dev),
             rows=rows, K=K)
+    _check_operand(out, "out", rows, K, x.device, workspace=True)
     if global_scale is not None:
         if out.global_scale.data_ptr() != global_scale.data_ptr():
             out.global_scale.copy_(global_scale.reshape(1))
@@ -276,6 +342,9 @@ def quantize_arc(x, perm, S: int, augment: int = AUG_RESIDUAL, mode: str = "six"
             global_scale=torch.empty(1, dtype=torch.float32, device=dev),
             workspace=torch.empty(nvfp4_quantize_workspace_bytes(rows, K), dtype=torch.uint8, device=dev),
             rows=rows, K=KA)
+    if perm.device != x.device:
+        raise ValueError("perm must be on x's device")
+    _check_operand(out, "out", rows, KA, x.device, workspace=True)
     st = nvfp4_quantize_arc(x.data_ptr(), rows, K, x.stride(0), perm.data_ptr(), S, augment, MODES[mode],
                             RULES[rule], F, out.codes.data_ptr(), out.scales.data_ptr(),
                             out.global_scale.data_ptr(), out.workspace.data_ptr(), out.workspace.numel(),
@@ -304,6 +373,7 @@ def quantize_t(x, mode: str = "six", rule: str = "max", fp8_max: float | None = 
             global_scale=torch.empty(1, dtype=torch.float32, device=dev),
             workspace=torch.empty(nvfp4_quantize_workspace_bytes(rows, K), dtype=torch.uint8, device=dev),
             rows=K, K=rows)
+    _check_operand(out, "out", K, rows, x.device, workspace=True)
     st = nvfp4_quantize_t(x.data_ptr(), rows, K, x.stride(0), MODES[mode], RULES[rule], F,
                           out.codes.data_ptr(), out.scales.data_ptr(), out.global_scale.data_ptr(),
                           out.workspace.data_ptr(), out.workspace.numel(), _stream_handle(stream))
@@ -318,13 +388,17 @@ def gemm(a: NVFP4Tensor, b: NVFP4Tensor, out_dtype=None, out=None, workspace=Non
 
     if a.K != b.K:
         raise ValueError("operands disagree on K")
-    out_dtype = torch.bfloat16 if out_dtype is None else out_dtype
-    code = {torch.bfloat16: OUT_BF16, torch.float32: OUT_FP32}[out_dtype]
+    out_dtype, code = _out_code(out_dtype, out)
     M, N, K = a.rows, b.rows, a.K
+    dev = a.codes.device
+    _check_operand(a, "a", M, K, dev)
+    _check_operand(b, "b", N, K, dev)
     if out is None:
-        out = torch.empty(M, N, dtype=out_dtype, device=a.codes.device)
+        out = torch.empty(M, N, dtype=out_dtype, device=dev)
     if workspace is None:
-        workspace = torch.empty(nvfp4_gemm_workspace_bytes(), dtype=torch.uint8, device=a.codes.device)
+        workspace = torch.empty(nvfp4_gemm_workspace_bytes(), dtype=torch.uint8, device=dev)
+    _check_output(out, M, N, out_dtype, dev)
+    _require(workspace, "workspace", torch.uint8, 0, dev)
     st = nvfp4_gemm(a.codes.data_ptr(), a.scales.data_ptr(), a.global_scale.data_ptr(),
                     b.codes.data_ptr(), b.scales.data_ptr(), b.global_scale.data_ptr(), M, N, K,
                     out.data_ptr(), out.stride(0), code, workspace.data_ptr(), workspace.numel(),
@@ -343,6 +417,9 @@ def gemm_quantized(a: NVFP4Tensor, b: NVFP4Tensor, y_alpha, mode: str = "six", r
         raise ValueError("operands disagree on K")
     M, N = a.rows, b.rows
     dev = a.codes.device
+    _check_operand(a, "a", M, a.K, dev)
+    _check_operand(b, "b", N, b.K, dev)
+    _require(y_alpha, "y_alpha", torch.float32, 1, dev, contiguous=False)
     if out is None:
         out = NVFP4Tensor(
             codes=torch.empty(M, N // 2, dtype=torch.uint8, device=dev),
@@ -350,6 +427,7 @@ def gemm_quantized(a: NVFP4Tensor, b: NVFP4Tensor, y_alpha, mode: str = "six", r
             global_scale=y_alpha.reshape(1),
             workspace=torch.empty(nvfp4_gemm_workspace_bytes(), dtype=torch.uint8, device=dev),
             rows=M, K=N)
+    _check_operand(out, "out", M, N, dev, global_scale=False, workspace=True)
     st = nvfp4_gemm_quantized(a.codes.data_ptr(), a.scales.data_ptr(), a.global_scale.data_ptr(),
                               b.codes.data_ptr(), b.scales.data_ptr(), b.global_scale.data_ptr(), M, N, a.K,
                               MODES[mode], RULES[rule], y_alpha.data_ptr(), out.codes.data_ptr(),
@@ -371,13 +449,19 @@ def gemm_segmented(a: NVFP4Tensor, b: NVFP4Tensor, b_globals, seg_ends, out_dtyp
     ends = (ctypes.c_int64 * len(seg_ends))(*[int(e) for e in seg_ends])
     if b_globals.dtype != torch.float32 or b_globals.numel() != len(seg_ends) or not b_globals.is_cuda:
         raise ValueError("b_globals must be a float32 CUDA tensor with one entry per segment")
-    out_dtype = torch.bfloat16 if out_dtype is None else out_dtype
-    code = {torch.bfloat16: OUT_BF16, torch.float32: OUT_FP32}[out_dtype]
+    out_dtype, code = _out_code(out_dtype, out)
     M, N, K = a.rows, b.rows, a.K
+    dev = a.codes.device
+    _check_operand(a, "a", M, K, dev)
+    _check_operand(b, "b", N, K, dev, global_scale=False)
+    if b_globals.device != dev:
+        raise ValueError("b_globals must be on the operands' device")
     if out is None:
-        out = torch.empty(M, N, dtype=out_dtype, device=a.codes.device)
+        out = torch.empty(M, N, dtype=out_dtype, device=dev)
     if workspace is None:
-        workspace = torch.empty(nvfp4_gemm_workspace_bytes(), dtype=torch.uint8, device=a.codes.device)
+        workspace = torch.empty(nvfp4_gemm_workspace_bytes(), dtype=torch.uint8, device=dev)
+    _check_output(out, M, N, out_dtype, dev)
+    _require(workspace, "workspace", torch.uint8, 0, dev)
     st = nvfp4_gemm_segmented(a.codes.data_ptr(), a.scales.data_ptr(), a.global_scale.data_ptr(),
                               b.codes.data_ptr(), b.scales.data_ptr(), b_globals.data_ptr(),
                               ctypes.addressof(ends), len(seg_ends), M, N, K, out.data_ptr(),
