@@ -530,7 +530,7 @@ def main():
     if world > 1:
         import datetime
 
-        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                              device_id=torch.device("cuda", local))
     try:
         res = run_ours(args, world, rank, local)
