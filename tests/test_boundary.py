@@ -73,6 +73,33 @@ def test_quantize_rejects_bad_arguments(bad):
     assert nv.last_error_message()
 
 
+def _qn(**kw):
+    args = dict(x=FAKE, rows=64, K=512, ldx=512, mode=1, rule=2, fp8_max=256.0, codes=FAKE,
+                scales=FAKE, global_scale=FAKE, stream=None)
+    args.update(kw)
+    return nv.nvfp4_quantize_noalloc(*args.values())
+
+
+@pytest.mark.parametrize("bad", [
+    dict(x=None), dict(codes=None), dict(scales=None), dict(global_scale=None), dict(rows=0),
+    dict(K=48), dict(ldx=256), dict(ldx=516), dict(mode=2), dict(rule=3), dict(fp8_max=300.0),
+    dict(x=FAKE + 8), dict(scales=FAKE + 4), dict(global_scale=FAKE + 2),
+    dict(rows=1 << 31, K=1024, ldx=1024),
+])
+def test_quantize_noalloc_rejects_bad_arguments(bad):
+    assert _qn(**bad) == nv.ERR_INVALID_ARG
+    assert nv.last_error_message()
+
+
+@pytest.mark.parametrize("rows,K,ldx", [(1 << 31, 1024, 1024), (1 << 30, 64, 1 << 11), ((1 << 62), 64, 64)])
+def test_oversized_tensors_are_rejected(rows, K, ldx):
+    """More than 2^40 elements of x (rows * ldx), including products that
+    would overflow 64 bits, are an argument error, not a launch."""
+    assert _q(rows=rows, K=K, ldx=ldx) == nv.ERR_INVALID_ARG
+    assert "too large" in nv.last_error_message()
+    assert _qs(rows=rows, K=K, ldx=ldx) == nv.ERR_INVALID_ARG
+
+
 def _qt(**kw):
     args = dict(x=FAKE, rows=128, K=72, ldx=72, mode=1, rule=2, fp8_max=256.0, codes=FAKE,
                 scales=FAKE, global_scale=FAKE, workspace=FAKE, workspace_bytes=1 << 20, stream=None)
@@ -134,6 +161,7 @@ def _g(**kw):
     dict(a_codes=None), dict(b_scales=None), dict(y=None), dict(workspace=None), dict(M=0),
     dict(N=-1), dict(K=32), dict(K=100), dict(ldy=128), dict(ldy=255), dict(out_dtype=2),
     dict(y=FAKE + 1), dict(a_global=FAKE + 1), dict(workspace_bytes=4),
+    dict(M=1 << 31), dict(N=1 << 31, ldy=1 << 31), dict(K=1 << 31),
 ])
 def test_gemm_rejects_bad_arguments(bad):
     assert _g(**bad) == nv.ERR_INVALID_ARG
