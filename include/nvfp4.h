@@ -219,8 +219,8 @@ NVFP4_API nvfp4_status nvfp4_quantize_noalloc(const void* x, int64_t rows, int64
  *   a_codes/a_scales/a_global  operand A (M rows), as nvfp4_quantize wrote it
  *   b_codes/b_scales/b_global  operand B (N rows, e.g. a weight [N, K])
  *   out_dtype  NVFP4_OUT_BF16 (round-to-nearest-even) or NVFP4_OUT_FP32.
- * Requirements: M, N >= 1, K >= 64, K % 64 == 0, ldy >= N, code and scale
- * buffers 16-byte aligned, Y aligned to its element size, workspace
+ * Requirements: 1 <= M, N, K <= 2^30, K % 64 == 0, N <= ldy <= 2^40, code
+ * and scale buffers 16-byte aligned, Y aligned to its element size, workspace
  * (>= nvfp4_gemm_workspace_bytes(), 16-byte aligned) for the status word.
  * Enqueues a 64-byte memset of the status word and one kernel launch. */
 NVFP4_API nvfp4_status nvfp4_gemm(const void* a_codes, const void* a_scales, const float* a_global,

@@ -161,7 +161,7 @@ def _g(**kw):
     dict(a_codes=None), dict(b_scales=None), dict(y=None), dict(workspace=None), dict(M=0),
     dict(N=-1), dict(K=32), dict(K=100), dict(ldy=128), dict(ldy=255), dict(out_dtype=2),
     dict(y=FAKE + 1), dict(a_global=FAKE + 1), dict(workspace_bytes=4),
-    dict(M=1 << 31), dict(N=1 << 31, ldy=1 << 31), dict(K=1 << 31),
+    dict(M=1 << 31), dict(N=1 << 31, ldy=1 << 31), dict(K=1 << 31), dict(ldy=(1 << 40) + 1), dict(ldy=1 << 62),
 ])
 def test_gemm_rejects_bad_arguments(bad):
     assert _g(**bad) == nv.ERR_INVALID_ARG
@@ -218,3 +218,5 @@ def test_no_gpu_fails_loudly():
     assert _gq() in (nv.ERR_CUDA, nv.ERR_UNSUPPORTED_DEVICE)
     assert _gs((64, 128, 256)) in (nv.ERR_CUDA, nv.ERR_UNSUPPORTED_DEVICE)
     assert _g() in (nv.ERR_CUDA, nv.ERR_UNSUPPORTED_DEVICE)
+    assert _g(ldy=1 << 40) in (nv.ERR_CUDA, nv.ERR_UNSUPPORTED_DEVICE)  # the largest legal row pitch
+    assert _qn() in (nv.ERR_CUDA, nv.ERR_UNSUPPORTED_DEVICE)

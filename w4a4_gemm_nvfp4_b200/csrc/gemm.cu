@@ -706,7 +706,7 @@ nvfp4_status gemm_impl(const char* fn, const void* a_codes, const void* a_scales
                      (long long)M, (long long)N, (long long)K);
   if (M > (1ll << 30) || N > (1ll << 30) || K > (1ll << 30))
     return set_error(NVFP4_ERR_INVALID_ARG, "%s: dimension too large", fn);
-  if (ldy < N) return set_error(NVFP4_ERR_INVALID_ARG, "%s: need ldy >= N", fn);
+  if (ldy < N || ldy > (int64_t{1} << 40)) return set_error(NVFP4_ERR_INVALID_ARG, "%s: need N <= ldy <= 2^40", fn);
   if (out_dtype != NVFP4_OUT_BF16 && out_dtype != NVFP4_OUT_FP32)
     return set_error(NVFP4_ERR_INVALID_ARG, "%s: unknown out_dtype %d", fn, out_dtype);
   if (!aligned16(a_codes) || !aligned16(b_codes) || !aligned16(a_scales) || !aligned16(b_scales) ||
