@@ -123,6 +123,7 @@ NVFP4_API size_t nvfp4_gemm_workspace_bytes(void);
  *            The pages use 448 for scale-6 and 256 for 4/6; any pairing is
  *            accepted.
  * Requirements: rows >= 1, K >= 64, K % 64 == 0, ldx >= K, ldx % 8 == 0,
+ * rows * ldx <= 2^40 and (rows rounded up to 128) * K < 2^40 elements,
  * x / codes / scales / workspace 16-byte aligned, global_scale 4-byte
  * aligned, workspace_bytes >= nvfp4_quantize_workspace_bytes(rows, K).
  * Writes codes, every byte of scales (padding = 0), *global_scale and the
