@@ -2,8 +2,10 @@
 
 Pinned against: the E2M1 grid the Four-Over-Six summary prints (section
 "문제 제기"), a hand-worked rounding table, an independent per-binade rint
-formulation over a dense sweep, and torch's float8_e4m3fn cast (a library
-routine) over every code, midpoint and a log-uniform sweep.
+formulation over a dense sweep, torch's float8_e4m3fn cast (a library
+routine) over every code, midpoint and a log-uniform sweep, and brute-force
+nearest-value enumeration over both grids (E4M3's built from the format's
+definition).
 """
 import numpy as np
 import pytest
@@ -109,3 +111,63 @@ def test_e4m3_subnormal_ties():
     # 3 * 2^-10 is the midpoint of codes 1 and 2: even code 2.
     assert oracle.e4m3_encode(3 * 2.0 ** -10) == 2
     assert oracle.e4m3_encode(0.0) == 0
+
+
+# ------------------------------------------- brute-force nearest value --
+# Round-to-nearest-even by enumeration: the nearest grid value wins; of two
+# equally near ones, the code with an even mantissa (bit 0 clear) wins; with
+# saturation nothing is above the largest finite value.  The grids come from
+# the format definitions, not from the oracle or torch.
+
+def _e4m3_grid() -> np.ndarray:
+    """All 127 non-negative finite E4M3 values (bias 7, 3 mantissa bits,
+    subnormals at exponent field 0, code 0x7F is NaN), by code."""
+    vals = []
+    for code in range(0x7F):
+        e, m = code >> 3, code & 7
+        vals.append(m / 8 * 2.0 ** -6 if e == 0 else (1 + m / 8) * 2.0 ** (e - 7))
+    return np.array(vals)
+
+
+def _nearest_even(v: np.ndarray, grid: np.ndarray) -> np.ndarray:
+    """Code of the grid value nearest to |v|; ties to the even code.  Above
+    the largest value the nearest is that value; clamping first keeps the
+    binary64 distances exact (|v| - g for a huge v would round to a tie)."""
+    a = np.minimum(np.abs(v.astype(np.float64)), grid[-1])
+    d = np.abs(a[:, None] - grid[None, :])
+    best = d.min(axis=1, keepdims=True)
+    tied = d == best
+    even = tied & (np.arange(grid.size)[None, :] % 2 == 0)
+    pick_even = even.any(axis=1)
+    return np.where(pick_even, even.argmax(axis=1), tied.argmax(axis=1))
+
+
+def test_e2m1_encode_is_nearest_grid_value_by_enumeration():
+    grid = np.array([_grid()[c] for c in range(8)])          # the pages' grid
+    rng = np.random.default_rng(1)
+    mids = (grid[:-1] + grid[1:]) / 2
+    vals = np.concatenate([
+        rng.uniform(-7, 7, 20000), np.exp2(rng.uniform(-30, 3, 5000)),
+        mids, np.nextafter(mids.astype(np.float32), np.float32(0)),
+        np.nextafter(mids.astype(np.float32), np.float32(10)), grid, [6.5, 7.0, 1e20, 0.0]]).astype(np.float32)
+    vals = np.concatenate([vals, -vals])
+    ref = _nearest_even(vals, grid) + 8 * np.signbit(vals)
+    got = np.array([oracle.e2m1_encode(float(v)) for v in vals])
+    bad = np.nonzero(got != ref)[0]
+    assert bad.size == 0, [(float(vals[i]), int(got[i]), int(ref[i])) for i in bad[:10]]
+
+
+def test_e4m3_encode_is_nearest_grid_value_by_enumeration():
+    grid = _e4m3_grid()
+    assert grid[1] == 2.0 ** -9 and grid[8] == 2.0 ** -6 and grid[0x7E] == 448.0
+    rng = np.random.default_rng(2)
+    mids = (grid[:-1] + grid[1:]) / 2
+    m32 = mids.astype(np.float32)
+    assert np.array_equal(m32.astype(np.float64), mids)          # midpoints are exact in binary32
+    vals = np.concatenate([
+        np.exp2(rng.uniform(-14, 10, 30000)), grid, m32, np.nextafter(m32, np.float32(0)),
+        np.nextafter(m32, np.float32(1000)), [449.0, 464.0, 480.0, 1e6, 0.0]]).astype(np.float32)
+    ref = _nearest_even(vals, grid)                               # saturates at 448 by construction
+    got = np.array([oracle.e4m3_encode(float(v)) for v in vals])
+    bad = np.nonzero(got != ref)[0]
+    assert bad.size == 0, [(float(vals[i]), int(got[i]), int(ref[i])) for i in bad[:10]]
