@@ -210,7 +210,8 @@ def test_tiny_alpha_gives_zero_codes_not_nan():
     blk[1] = np.float32(-(2.0 ** -131))
     alpha = oracle.global_scale(float(blk[0]), 448.0)
     d = _e4m3_val(oracle.quantize_candidate(blk, alpha, 6.0, oracle.RULE_MAX)[1]) * alpha
-    assert np.isinf(np.float32(1.0) / np.float32(d))
+    with np.errstate(over="ignore"):  # the overflow is the point of this case
+        assert np.isinf(np.float32(1.0) / np.float32(d))
     codes, s, chose4, e6, e4 = oracle.quantize_block(blk, alpha, oracle.MODE_FOUR_OVER_SIX, oracle.RULE_MAX)
     assert list(codes[:2]) == [0, 8] and not codes[2:].any()
     assert e6 == np.float32(2.0 ** -130) and e4 == e6 and not chose4
