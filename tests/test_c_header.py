@@ -12,6 +12,18 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 INCLUDE = os.path.join(ROOT, "include")
 LIBDIR = os.path.join(ROOT, "w4a4_gemm_nvfp4_b200")
 
+
+@pytest.fixture
+def scratch():
+    """A scratch folder inside the repository's (git-ignored) build folder."""
+    import pathlib
+
+    d = pathlib.Path(ROOT, "_build", "c_abi_test", str(os.getpid()))
+    d.mkdir(parents=True, exist_ok=True)
+    yield d
+    shutil.rmtree(d, ignore_errors=True)
+
+
 PROGRAM = r"""
 #include <stdio.h>
 #include <string.h>
@@ -53,22 +65,22 @@ def _compiler(name):
 
 
 @pytest.mark.parametrize("lang", ["c99", "c++17"])
-def test_headers_compile_strictly(lang, tmp_path):
+def test_headers_compile_strictly(lang, scratch):
     cc = _compiler("gcc" if lang == "c99" else "g++")
-    src = tmp_path / ("t.c" if lang == "c99" else "t.cc")
+    src = scratch / ("t.c" if lang == "c99" else "t.cc")
     src.write_text('#include "nvfp4.h"\n#include "nvfp4_testing.h"\nint main(void) { return 0; }\n')
     subprocess.run([cc, f"-std={lang}", "-Wall", "-Wextra", "-pedantic", "-Werror", "-I", INCLUDE,
                     "-fsyntax-only", str(src)], check=True, capture_output=True)
 
 
-def test_c_program_links_and_validates_on_the_host(tmp_path):
+def test_c_program_links_and_validates_on_the_host(scratch):
     lib = os.path.join(LIBDIR, "libnvfp4.so")
     if not os.path.exists(lib):
         pytest.skip("libnvfp4.so is not built")
     cc = _compiler("gcc")
-    src = tmp_path / "abi.c"
+    src = scratch / "abi.c"
     src.write_text(PROGRAM)
-    exe = tmp_path / "abi"
+    exe = scratch / "abi"
     subprocess.run([cc, "-std=c99", "-Wall", "-Werror", "-I", INCLUDE, str(src), "-L", LIBDIR, "-lnvfp4",
                     f"-Wl,-rpath,{LIBDIR}", "-o", str(exe)], check=True, capture_output=True)
     r = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
