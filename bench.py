@@ -473,6 +473,25 @@ def run_sweep(args):
                 "GBps_end_to_end": round((QUANT_BYTES_PER_ELEM + AMAX_BYTES_PER_ELEM) * n / t_e2e / 1e6, 1),
                 "overhead_vs_six_kernel": None if m == "six" else round(t_k / six_kernel - 1.0, 4),
                 "l2": "flushed between iterations", "median_of": args.steps}), flush=True)
+            # the other quantizer entry points, amax pass included: blocks down
+            # the columns (x^T), and 128 augmented residual channels
+            n_bytes = (QUANT_BYTES_PER_ELEM + AMAX_BYTES_PER_ELEM) * n
+            qt = nv.quantize_t(x, m, r, F)
+            t_t = timed(lambda: nv.quantize_t(x, m, r, F, out=qt), args.steps)
+            assert nv.device_status(qt.workspace) == nv.OK
+            S = 128
+            perm = torch.randperm(K, generator=torch.Generator().manual_seed(5)).to(torch.int32).to(device)
+            qa = nv.quantize_arc(x, perm, S, nv.AUG_RESIDUAL, m, r, F)
+            t_a = timed(lambda: nv.quantize_arc(x, perm, S, nv.AUG_RESIDUAL, m, r, F, out=qa), args.steps)
+            assert nv.device_status(qa.workspace) == nv.OK
+            arc_bytes = (2.0 + AMAX_BYTES_PER_ELEM + (QUANT_BYTES_PER_ELEM - 2.0) * (K + S) / K) * n
+            print(json.dumps({
+                "sweep": "quantize_variants", "rows": rows, "K": K, "recipe": f"{m}-{r}-{F:g}",
+                "ms_transposed": round(t_t, 4), "GBps_transposed": round(n_bytes / t_t / 1e6, 1),
+                "ms_arc_S128": round(t_a, 4), "GBps_arc_S128": round(arc_bytes / t_a / 1e6, 1),
+                "arc_overhead_vs_rows": round(t_a / t_e2e - 1.0, 4),
+                "l2": "flushed between iterations", "median_of": args.steps}), flush=True)
+            del qt, qa
         del x
         torch.cuda.empty_cache()
     fp4_peak = 4.0 * peaks["bf16"]
@@ -494,7 +513,26 @@ def run_sweep(args):
             "x_recipe": f"{xm}-{xr}-{xF:g}", "w_recipe": f"{wm}-{wr}-{wF:g}",
             "ms": round(t, 4), "TFLOPs": round(tf, 1), "frac_fp4_peak": round(tf / fp4_peak, 4),
             "l2": "flushed between iterations", "median_of": args.steps}), flush=True)
-        del x, w, qx, qw, y
+        # the GEMM variants on the same operands: two output-column segments
+        # with their own B scales, and Y written as an NVFP4 operand (4/6-MSE)
+        half = wl.N // 2 // 64 * 64
+        b_globals = torch.stack([qw.global_scale[0]] * 2)
+        t_seg = timed(lambda: nv.gemm_segmented(qx, qw, b_globals, [half, wl.N], out=y, workspace=ws),
+                      args.steps)
+        assert nv.device_status(ws) == nv.OK
+        y_alpha = torch.tensor([max(float(y.abs().max()), 1e-30) / (6 * 256.0)], dtype=torch.float32,
+                               device=device)
+        qy = nv.gemm_quantized(qx, qw, y_alpha, "four_over_six", "mse")
+        t_q = timed(lambda: nv.gemm_quantized(qx, qw, y_alpha, "four_over_six", "mse", out=qy), args.steps)
+        assert nv.device_status(qy.workspace) == nv.OK
+        flops = 2.0 * wl.M * wl.N * wl.K
+        print(json.dumps({
+            "sweep": "gemm_variants", "workload": name, "M": wl.M, "N": wl.N, "K": wl.K,
+            "ms_segmented_2": round(t_seg, 4), "TFLOPs_segmented_2": round(flops / t_seg / 1e9, 1),
+            "ms_nvfp4_out_46mse": round(t_q, 4), "TFLOPs_nvfp4_out_46mse": round(flops / t_q / 1e9, 1),
+            "frac_fp4_peak_nvfp4_out": round(flops / t_q / 1e9 / fp4_peak, 4),
+            "l2": "flushed between iterations", "median_of": args.steps}), flush=True)
+        del x, w, qx, qw, y, qy
         torch.cuda.empty_cache()
 
 
