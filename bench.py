@@ -331,7 +331,7 @@ def run_ours(args, world, rank, local):
         "clocks": clocks.summary(),
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        result["cpu_baseline"] = cpu_baseline(args, sample_rows=1024)
+        result["cpu_baseline"] = cpu_baseline(args, sample_rows=8192)  # about 10 s of CPU work
     return result
 
 
