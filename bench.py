@@ -71,11 +71,24 @@ class ClockSampler:
         self._stop = None
         self._thread = None
         self.error = None
+        self.match = None
+
+    def _handle(self, pynvml):
+        """NVML handle of the CUDA device being timed.  NVML numbers every GPU
+        of the machine, CUDA only the visible ones, so the two indexes can
+        differ; the UUID names the same GPU in both."""
+        try:
+            u = str(torch.cuda.get_device_properties(self.gpu).uuid)
+            self.match = "uuid"
+            return pynvml.nvmlDeviceGetHandleByUUID(u if u.startswith("GPU-") else "GPU-" + u)
+        except Exception:
+            self.match = "index"
+            return pynvml.nvmlDeviceGetHandleByIndex(self.gpu)
 
     def _run(self):
         import pynvml
 
-        h = pynvml.nvmlDeviceGetHandleByIndex(self.gpu)
+        h = self._handle(pynvml)
         self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
         while not self._stop.is_set():
             self.samples.append(pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM))
@@ -113,7 +126,7 @@ class ClockSampler:
                     "reasons": [self.error or "no samples"]}
         return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
                 "sm_mhz_min": min(self.samples), "reasons": sorted(self.reasons),
-                "samples": len(self.samples)}
+                "samples": len(self.samples), "nvml_device_by": self.match}
 
 
 def _dist():
