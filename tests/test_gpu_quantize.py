@@ -147,3 +147,44 @@ def test_config_operands_full_size_sampled(name):
         _check_sampled(x, recipe)
     w = _full_tensor((name, "w"), wl.w.make)
     _check_sampled(w, wl.w_recipe)
+
+
+def _reading_pin_cases():
+    import test_oracle_readings as tr
+    return tr.CASES
+
+
+@pytest.mark.parametrize("case", _reading_pin_cases(), ids=lambda c: c["name"])
+def test_reading_pins(case):
+    """The blocks that pin the quotient order, the reciprocal-multiply scaling
+    and the pairwise error sum (tests/golden/reading_pins.txt, derived in
+    exact arithmetic): every quantizer kernel gives the stored bits."""
+    import test_oracle_readings as tr
+
+    x = tr._tensor(case)
+    recipe = (case["mode"], case["rule"], case["F"])
+
+    def block1(codes_row, scales_swz):
+        unpacked = [int(v) for b in codes_row[8:16] for v in (b & 15, b >> 4)]
+        return unpacked, int(scales_swz[1])  # row 0, K block 1 of the first atom
+
+    # row-wise kernel (amax pass included)
+    q, status = gpu_quantize(x, *recipe)
+    assert status == nv.OK
+    assert block1(to_np(q.codes)[0], to_np(q.scales)) == (case["codes"], case["scale"])
+    assert_quant_equal(q, x, *recipe)
+    # static alpha: the quantize kernel alone, at the golden tensor's alpha
+    qs = nv.quantize(x.cuda(), case["mode"], case["rule"], global_scale=q.global_scale.clone())
+    assert nv.device_status(qs.workspace) == nv.OK
+    assert block1(to_np(qs.codes)[0], to_np(qs.scales)) == (case["codes"], case["scale"])
+    # column-wise kernel: the golden row as column 0 of a 64 x 8 matrix
+    xt = torch.zeros(64, 8, dtype=torch.bfloat16)
+    xt[:, 0] = x[0]
+    qt = nv.quantize_t(xt.cuda(), *recipe)
+    assert nv.device_status(qt.workspace) == nv.OK
+    assert block1(to_np(qt.codes)[0], to_np(qt.scales)) == (case["codes"], case["scale"])
+    # augmented-channel kernel with the identity order and no extra channels
+    perm = torch.arange(64, dtype=torch.int32, device="cuda")
+    qa = nv.quantize_arc(x.cuda(), perm, 0, nv.AUG_RESIDUAL, *recipe)
+    assert nv.device_status(qa.workspace) == nv.OK
+    assert block1(to_np(qa.codes)[0], to_np(qa.scales)) == (case["codes"], case["scale"])
