@@ -209,7 +209,11 @@ NVFP4_API nvfp4_status nvfp4_quantize_with_scale(const void* x, int64_t rows, in
  * that may overlap on the GPU race and must be ordered by the caller (same
  * stream, or events).  The first call on each device looks up the array's
  * device address with cudaGetSymbolAddress (with that device current); make
- * that first call before any stream capture.  Non-finite input shows as a NaN
+ * that first call before any stream capture.  The array belongs to the CUDA
+ * context that loaded this library's module: the lookup is repeated on the
+ * first call in every other context of the device (a driver-API context, or
+ * the primary context after cudaDeviceReset re-created it), and that call
+ * too should come before any stream capture.  Non-finite input shows as a NaN
  * *global_scale (there is no workspace status word to read).  Allocates
  * nothing: no cudaMalloc, cudaFree or allocating library routine. */
 NVFP4_API nvfp4_status nvfp4_quantize_noalloc(const void* x, int64_t rows, int64_t K, int64_t ldx,

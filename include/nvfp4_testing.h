@@ -14,9 +14,10 @@
 extern "C" {
 #endif
 
-/* Sets, for the following nvfp4_gemm calls in this process, the deadline of
- * every bounded wait inside the GEMM kernel (timeout_ns; 0 restores the
- * default of 4 s) and debug flags (bit 0: the producer never issues the
+/* Sets, for the following nvfp4_gemm calls in this process, the timeout of
+ * every bounded wait inside the GEMM kernel (timeout_ns, counted from the
+ * start of each wait, so it bounds a lack of progress, not the kernel's run
+ * time; 0 restores the default of 4 s) and debug flags (bit 0: the producer never issues the
  * copies of the first pipeline stage, so the consumer's wait for it runs out
  * and the kernel reports NVFP4_ERR_TIMEOUT through the workspace status word
  * after draining its in-flight work).  Not thread-safe; tests only. */

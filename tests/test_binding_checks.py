@@ -84,3 +84,14 @@ def test_scalar_buffers():
         L._require(torch.empty(0, dtype=torch.float32), "alpha", torch.float32, 1, CPU, contiguous=False)
     with pytest.raises(TypeError):
         L._require(0.5, "alpha", torch.float32, 1, CPU)
+
+
+def test_row_pitch_of_a_single_row_is_its_length():
+    """torch may give a size-1 dimension any stride (0 after some views); the
+    binding passes the row length as the pitch of a one-row tensor."""
+    from w4a4_gemm_nvfp4_b200._lib import _row_pitch
+
+    one = torch.zeros(64, dtype=torch.bfloat16).as_strided((1, 64), (0, 1))
+    assert one.stride(0) == 0 and _row_pitch(one) == 64
+    many = torch.zeros(3, 80, dtype=torch.bfloat16)[:, :64]
+    assert _row_pitch(many) == 80

@@ -225,3 +225,26 @@ def test_gemm_quantized_output_equals_gemm_then_quantize(M, N, K, recipe):
     oc, os_ = oracle.quantize_rows(y.cpu(), float(alpha.cpu()[0]), MODE[mode], RULE[rule])
     assert np.array_equal(to_np(q.codes), oc)
     assert np.array_equal(to_np(q.scales), oracle.swizzle_scales(os_, M, N))
+
+
+@pytest.mark.skipif(torch.cuda.device_count() < 2, reason="needs two visible GPUs")
+def test_second_device_after_the_first():
+    """Kernel attributes (the GEMM's and the augmented quantizer's shared-memory
+    opt-in) belong to each device's context: a call on device 1 after calls on
+    device 0 must launch and be right."""
+    ac, as_, aa = _quantized(256, 512, 51, ("four_over_six", "mse", 256.0))
+    bc, bs, ba = _quantized(384, 512, 52, ("six", "max", 448.0), kind="normal")
+    ref, guard = oracle.gemm_reference(ac, as_, aa, bc, bs, ba)
+    x = workloads.small_operand(128, 512, seed=53).make()
+    perm = torch.arange(512, dtype=torch.int32)
+    for dev in (0, 1):
+        with torch.cuda.device(dev):
+            A, B = upload_operand(ac, as_, aa), upload_operand(bc, bs, ba)
+            assert A.codes.device.index == dev
+            y = nv.gemm(A, B, out_dtype=torch.float32)
+            ws = torch.zeros(nv.nvfp4_gemm_workspace_bytes(), dtype=torch.uint8, device="cuda")
+            nv.gemm(A, B, out_dtype=torch.float32, out=y, workspace=ws)
+            assert nv.device_status(ws) == nv.OK
+            assert_gemm_close(to_np(y), ref, guard)
+            qa = nv.quantize_arc(x.cuda(), perm.cuda(), 64, nv.AUG_RESIDUAL, "four_over_six", "mse", 256.0)
+            assert nv.device_status(qa.workspace) == nv.OK

@@ -56,7 +56,7 @@ def _tensor(case) -> torch.Tensor:
     row = np.zeros(64, np.float32)
     row[0] = case["amax"]
     row[16:32] = case["block"]
-    t = torch.from_numpy(row[None, :]).to(torch.bfloat16)
+    t = torch.from_numpy(row.reshape(1, 64).copy()).to(torch.bfloat16)
     assert np.array_equal(t.float().numpy(), row[None, :]), "golden values must be bf16-exact"
     return t
 

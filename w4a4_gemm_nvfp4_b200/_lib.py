@@ -249,8 +249,15 @@ def _check_output(y, M: int, N: int, dtype, device) -> None:
         raise ValueError(f"out is on {y.device}, expected {device}")
     if y.dim() != 2 or tuple(y.shape) != (M, N):
         raise ValueError(f"out must have shape ({M}, {N}), not {tuple(y.shape)}")
-    if y.stride(1) != 1 or y.stride(0) < N:
+    if y.stride(1) != 1 or _row_pitch(y) < N:
         raise ValueError("out must have unit stride along N and a row pitch of at least N")
+
+
+def _row_pitch(x) -> int:
+    """Row pitch of a 2-D tensor in elements.  A single row has no pitch to
+    speak of (torch may report any stride for a size-1 dimension), so its
+    row length stands in."""
+    return x.shape[1] if x.shape[0] == 1 else x.stride(0)
 
 
 def _out_code(out_dtype, out):
@@ -299,13 +306,13 @@ def quantize(x, mode: str = "six", rule: str = "max", fp8_max: float | None = No
     if global_scale is not None:
         if out.global_scale.data_ptr() != global_scale.data_ptr():
             out.global_scale.copy_(global_scale.reshape(1))
-        st = nvfp4_quantize_with_scale(x.data_ptr(), rows, K, x.stride(0), MODES[mode], RULES[rule],
+        st = nvfp4_quantize_with_scale(x.data_ptr(), rows, K, _row_pitch(x), MODES[mode], RULES[rule],
                                        out.global_scale.data_ptr(), out.codes.data_ptr(),
                                        out.scales.data_ptr(), out.workspace.data_ptr(),
                                        out.workspace.numel(), _stream_handle(stream))
         _check(st, "nvfp4_quantize_with_scale")
         return out
-    st = nvfp4_quantize(x.data_ptr(), rows, K, x.stride(0), MODES[mode], RULES[rule], F,
+    st = nvfp4_quantize(x.data_ptr(), rows, K, _row_pitch(x), MODES[mode], RULES[rule], F,
                         out.codes.data_ptr(), out.scales.data_ptr(), out.global_scale.data_ptr(),
                         out.workspace.data_ptr(), out.workspace.numel(), _stream_handle(stream))
     _check(st, "nvfp4_quantize")
@@ -345,7 +352,7 @@ def quantize_arc(x, perm, S: int, augment: int = AUG_RESIDUAL, mode: str = "six"
     if perm.device != x.device:
         raise ValueError("perm must be on x's device")
     _check_operand(out, "out", rows, KA, x.device, workspace=True)
-    st = nvfp4_quantize_arc(x.data_ptr(), rows, K, x.stride(0), perm.data_ptr(), S, augment, MODES[mode],
+    st = nvfp4_quantize_arc(x.data_ptr(), rows, K, _row_pitch(x), perm.data_ptr(), S, augment, MODES[mode],
                             RULES[rule], F, out.codes.data_ptr(), out.scales.data_ptr(),
                             out.global_scale.data_ptr(), out.workspace.data_ptr(), out.workspace.numel(),
                             _stream_handle(stream))
@@ -374,7 +381,7 @@ def quantize_t(x, mode: str = "six", rule: str = "max", fp8_max: float | None = 
             workspace=torch.empty(nvfp4_quantize_workspace_bytes(rows, K), dtype=torch.uint8, device=dev),
             rows=K, K=rows)
     _check_operand(out, "out", K, rows, x.device, workspace=True)
-    st = nvfp4_quantize_t(x.data_ptr(), rows, K, x.stride(0), MODES[mode], RULES[rule], F,
+    st = nvfp4_quantize_t(x.data_ptr(), rows, K, _row_pitch(x), MODES[mode], RULES[rule], F,
                           out.codes.data_ptr(), out.scales.data_ptr(), out.global_scale.data_ptr(),
                           out.workspace.data_ptr(), out.workspace.numel(), _stream_handle(stream))
     _check(st, "nvfp4_quantize_t")
@@ -401,7 +408,7 @@ def gemm(a: NVFP4Tensor, b: NVFP4Tensor, out_dtype=None, out=None, workspace=Non
     _require(workspace, "workspace", torch.uint8, 0, dev)
     st = nvfp4_gemm(a.codes.data_ptr(), a.scales.data_ptr(), a.global_scale.data_ptr(),
                     b.codes.data_ptr(), b.scales.data_ptr(), b.global_scale.data_ptr(), M, N, K,
-                    out.data_ptr(), out.stride(0), code, workspace.data_ptr(), workspace.numel(),
+                    out.data_ptr(), _row_pitch(out), code, workspace.data_ptr(), workspace.numel(),
                     _stream_handle(stream))
     _check(st, "nvfp4_gemm")
     return out
@@ -465,7 +472,7 @@ def gemm_segmented(a: NVFP4Tensor, b: NVFP4Tensor, b_globals, seg_ends, out_dtyp
     st = nvfp4_gemm_segmented(a.codes.data_ptr(), a.scales.data_ptr(), a.global_scale.data_ptr(),
                               b.codes.data_ptr(), b.scales.data_ptr(), b_globals.data_ptr(),
                               ctypes.addressof(ends), len(seg_ends), M, N, K, out.data_ptr(),
-                              out.stride(0), code, workspace.data_ptr(), workspace.numel(),
+                              _row_pitch(out), code, workspace.data_ptr(), workspace.numel(),
                               _stream_handle(stream))
     _check(st, "nvfp4_gemm_segmented")
     return out

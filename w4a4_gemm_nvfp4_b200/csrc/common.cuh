@@ -6,6 +6,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <mutex>
+
 #include "nvfp4.h"
 
 namespace nvfp4 {
@@ -20,6 +22,42 @@ nvfp4_status check_device(int* device, int* num_sms);
 nvfp4_status cuda_status(cudaError_t err, const char* what);
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// The driver's unique id of the CUDA context current on this thread (ids are
+// never reused within a process, unlike context handles), or 0 when no
+// context is current or the driver cannot be asked.
+uint64_t current_context_id();
+
+// A value computed once per CUDA context of each device: kernel attributes,
+// occupancy and symbol addresses belong to the context that loaded the
+// module, so a device whose primary context was reset (cudaDeviceReset) or
+// replaced gets them computed again.
+constexpr int kMaxDevices = 64;
+template <typename T>
+struct PerContextCache {
+  std::mutex mu;
+  uint64_t ctx[kMaxDevices] = {};
+  T value[kMaxDevices] = {};
+};
+// The cached value for device `dev` (the current device) in the current
+// context; `make(T*)` computes it (returning a cudaError_t) when the context
+// changed or nothing is cached yet.  When no context id can be read the value
+// is recomputed on every call.
+template <typename T, typename Make>
+cudaError_t per_context(PerContextCache<T>& c, int dev, Make make, T* out) {
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lk(c.mu);
+  const uint64_t id = current_context_id();
+  if (id == 0 || c.ctx[dev] != id) {
+    T v{};
+    const cudaError_t e = make(&v);
+    if (e != cudaSuccess) return e;
+    c.value[dev] = v;
+    c.ctx[dev] = current_context_id();  // the computation may have created the context
+  }
+  *out = c.value[dev];
+  return cudaSuccess;
+}
 
 // Status words live at the start of every workspace.
 struct WorkspaceHeader {
@@ -49,9 +87,6 @@ __device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
                : "memory");
 }
-__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
-}
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
@@ -65,16 +100,21 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 }
 
 // Bounded wait: spins on try_wait until the phase with `parity` completed,
-// `*abort` became non-zero, or `deadline_ns` (globaltimer) passed.  Returns
-// true when the phase completed.
+// `*abort` became non-zero, or `timeout_ns` passed (on %globaltimer) since
+// this wait first checked the clock.  The limit is on a lack of progress:
+// every wait gets the whole timeout, however long the kernel has run.
+// Returns true when the phase completed.
 __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
                                                   const volatile int* abort,
-                                                  uint64_t deadline_ns) {
+                                                  uint64_t timeout_ns) {
+  uint64_t start = 0;
   for (uint32_t it = 0;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 63u) == 63u) {
       if (*abort) return false;
-      if (global_timer_ns() > deadline_ns) return false;
+      const uint64_t now = global_timer_ns();
+      if (start == 0) start = now;
+      else if (now - start > timeout_ns) return false;
     }
   }
 }
@@ -94,26 +134,6 @@ __device__ __forceinline__ bool elect_one() {
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(pred));
   return pred != 0;
-}
-
-// TMA: 2D tiled tensor load into shared memory, completing on `bar`.
-__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
-                                            int32_t c0, int32_t c1) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1)
-      : "memory");
-}
-
-// 3D tiled tensor load into this CTA's shared memory, completing on its own `bar`.
-__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
-                                            int32_t c0, int32_t c1, int32_t c2) {
-  asm volatile(
-      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "r"(c2)
-      : "memory");
 }
 
 // TMA for one CTA of a CTA pair (cta_group::2): the destination is this CTA's
@@ -177,16 +197,6 @@ __device__ __forceinline__ void tma_store_2d_hint(const CUtensorMap* map, uint32
       : "memory");
 }
 
-// TMA: 2D tiled tensor store from this CTA's shared memory (bulk-group
-// completion; out-of-range parts of the box are not written).
-__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, uint32_t src, int32_t c0,
-                                             int32_t c1) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.global.shared::cta.tile.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
-          reinterpret_cast<uint64_t>(map)),
-      "r"(src), "r"(c0), "r"(c1)
-      : "memory");
-}
 __device__ __forceinline__ void bulk_commit_group() {
   asm volatile("cp.async.bulk.commit_group;" ::: "memory");
 }
@@ -223,35 +233,12 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar_cluster) {
                : "memory");
 }
 
-// Plain (non-tensor) bulk copy global -> shared, completing on `bar`.
-// Both addresses 16-byte aligned, bytes a multiple of 16.
-__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes,
-                                          uint32_t bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-          dst),
-      "l"(src), "r"(bytes), "r"(bar)
-      : "memory");
-}
-
 __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
 
 // ----------------------------------------------------------- tcgen05 ----
 
-__device__ __forceinline__ void tmem_alloc(uint32_t dst_smem, uint32_t ncols) {
-  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem),
-               "r"(ncols)
-               : "memory");
-}
-__device__ __forceinline__ void tmem_relinquish() {
-  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
-  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
-               : "memory");
-}
 __device__ __forceinline__ void tc_fence_before() {
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
 }
@@ -277,13 +264,6 @@ __device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols
 __device__ __forceinline__ void tc_commit_pair(uint32_t bar_cluster) {
   asm volatile(
       "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar_cluster)
-      : "memory");
-}
-
-// Arrive on `bar` once every previously issued tcgen05 op of this thread completed.
-__device__ __forceinline__ void tc_commit(uint32_t bar) {
-  asm volatile(
-      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
       : "memory");
 }
 

@@ -43,9 +43,11 @@
 // buffer suffices.  The epilogue loads the shared columns 192..255 first,
 // releases them to the next tile's MMAs at once, and stores the rest of tile
 // i while the mainloop of tile i+1 runs.
-// Every wait is bounded by a deadline on %globaltimer; a wait that runs out
-// records NVFP4_ERR_TIMEOUT in the workspace, raises a CTA-wide abort flag,
-// and every role drains what it has in flight before TMEM is freed.
+// Every wait is bounded: a wait that makes no progress for the timeout (4 s
+// by default, on %globaltimer) records NVFP4_ERR_TIMEOUT in the workspace,
+// raises a CTA-wide abort flag, and every role drains what it has in flight
+// before TMEM is freed.  The bound is per wait, so a long GEMM whose waits
+// keep completing never times out.
 #include <cuda_bf16.h>
 
 #include <algorithm>
@@ -254,7 +256,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   cluster_sync_all();  // both CTAs' barriers exist before anyone signals them
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint64_t deadline = global_timer_ns() + p.timeout_ns;
 
   if (warp == 0) {
     // -------------------------------------------------- TMA producer ----
@@ -271,7 +272,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       for (uint32_t kt = 0; kt < p.ktiles; ++kt, ++it) {
         const uint32_t s = it % STAGES, ph = (it / STAGES) & 1u;
         if (it >= STAGES &&
-            !__all_sync(0xffffffffu, mbar_wait_bounded(bar_empty + 8 * s, ph ^ 1u, abort, deadline))) {
+            !__all_sync(0xffffffffu, mbar_wait_bounded(bar_empty + 8 * s, ph ^ 1u, abort, p.timeout_ns))) {
           if (lane == 0 && !*abort) record_timeout(p, abort, 1);
           stop = true;
           break;
@@ -298,14 +299,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       // (they complete once both CTAs' bytes arrived); the other CTA, whose
       // copies complete on the leader's barriers, waits out a 2 ms grace
       // period instead -- a bulk copy of a few KB lands in microseconds.
-      const uint64_t now = global_timer_ns();
       if (rank == 0) {
         const volatile int no_abort = 0;
         const uint32_t first = it > STAGES ? it - STAGES : 0;
         for (uint32_t k = first; k < it; ++k)
-          mbar_wait_bounded(bar_full + 8 * (k % STAGES), (k / STAGES) & 1u, &no_abort,
-                            now + 100000000ull);
+          mbar_wait_bounded(bar_full + 8 * (k % STAGES), (k / STAGES) & 1u, &no_abort, 100000000ull);
       } else {
+        const uint64_t now = global_timer_ns();
         while (global_timer_ns() < now + 2000000ull) {
         }
       }
@@ -324,7 +324,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         // The accumulator this tile writes overlaps the previous tile's
         // first-drained subtiles: wait until both CTAs' epilogues released them.
         if (local > 0 &&
-            !__all_sync(0xffffffffu, mbar_wait_bounded(bar_acc_free, (local - 1) & 1u, abort, deadline))) {
+            !__all_sync(0xffffffffu, mbar_wait_bounded(bar_acc_free, (local - 1) & 1u, abort, p.timeout_ns))) {
           if (lane == 0 && !*abort) record_timeout(p, abort, 4);
           break;
         }
@@ -332,7 +332,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const uint32_t acc = tmem + ((local & 1u) ? TM_ACC1 : 0u);
         for (uint32_t kt = 0; kt < p.ktiles; ++kt, ++it) {
           const uint32_t s = it % STAGES, ph = (it / STAGES) & 1u;
-          if (!__all_sync(0xffffffffu, mbar_wait_bounded(bar_full + 8 * s, ph, abort, deadline))) {
+          if (!__all_sync(0xffffffffu, mbar_wait_bounded(bar_full + 8 * s, ph, abort, p.timeout_ns))) {
             if (lane == 0 && !*abort) record_timeout(p, abort, 2);
             stop = true;
             break;
@@ -371,7 +371,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         // Drain the MMAs already issued before TMEM is released.
         const volatile int no_abort = 0;
         tc_commit_pair(map_to_rank(bar_drain, 0));
-        mbar_wait_bounded(bar_drain, 0, &no_abort, global_timer_ns() + 100000000ull);
+        mbar_wait_bounded(bar_drain, 0, &no_abort, 100000000ull);
       }
       __syncwarp();
     }
@@ -409,7 +409,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     uint32_t nstore = 0;
     uint32_t local = 0;
     for (uint32_t tile = pair; tile < p.num_tiles; tile += npairs, ++local) {
-      bool ok = mbar_wait_bounded(bar_acc_full, local & 1u, abort, deadline);
+      bool ok = mbar_wait_bounded(bar_acc_full, local & 1u, abort, p.timeout_ns);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) {
         if (lane == 0 && !*abort) record_timeout(p, abort, 3);
@@ -651,7 +651,7 @@ nvfp4_status make_scale_map(CUtensorMap* map, const void* base, int64_t rows, in
 
 }  // namespace
 
-// Test hooks (not part of the public header): bounded-wait deadline and
+// Test hooks (not part of the public header): bounded-wait timeout and
 // debug flags for the next nvfp4_gemm calls on this process.
 static uint64_t g_timeout_ns = 4000000000ull;  // 4 s
 static int g_debug_flags = 0;
@@ -672,15 +672,17 @@ void nvfp4_testing_set_gemm_wait(uint64_t timeout_ns, int debug_flags) {
 namespace {
 
 template <int EPI>
-cudaError_t launch_gemm(unsigned grid, cudaStream_t s, const CUtensorMap& ta, const CUtensorMap& tb,
+cudaError_t launch_gemm(int dev, unsigned grid, cudaStream_t s, const CUtensorMap& ta, const CUtensorMap& tb,
                         const CUtensorMap& tsa, const CUtensorMap& tsb, const CUtensorMap& ty,
                         const GemmParams& p) {
-  static std::once_flag attr_once;
-  static cudaError_t attr_err = cudaSuccess;
-  std::call_once(attr_once, [] {
-    attr_err = cudaFuncSetAttribute(gemm_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    static_cast<int>(SMEM_BYTES));
-  });
+  // the shared-memory opt-in is an attribute of the kernel in this context
+  static PerContextCache<int> attr;
+  int done = 0;
+  const cudaError_t attr_err = per_context(attr, dev, [](int* v) {
+    *v = 1;
+    return cudaFuncSetAttribute(gemm_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                static_cast<int>(SMEM_BYTES));
+  }, &done);
   if (attr_err != cudaSuccess) return attr_err;
   gemm_kernel<EPI><<<grid, kThreads, SMEM_BYTES, s>>>(ta, tb, tsa, tsb, ty, p);
   return cudaGetLastError();
@@ -771,11 +773,11 @@ nvfp4_status gemm_impl(const char* fn, const void* a_codes, const void* a_scales
   const int64_t pairs = std::max<int64_t>(1, std::min<int64_t>(num_tiles, sms / 2));
   const unsigned grid = static_cast<unsigned>(2 * pairs);
   switch (epi) {
-    case 0: e = launch_gemm<0>(grid, s, ta, tb, tsa, tsb, ty, p); break;
-    case 1: e = launch_gemm<1>(grid, s, ta, tb, tsa, tsb, ty, p); break;
-    case 2: e = launch_gemm<2>(grid, s, ta, tb, tsa, tsb, ty, p); break;
-    case 3: e = launch_gemm<3>(grid, s, ta, tb, tsa, tsb, ty, p); break;
-    default: e = launch_gemm<4>(grid, s, ta, tb, tsa, tsb, ty, p); break;
+    case 0: e = launch_gemm<0>(dev, grid, s, ta, tb, tsa, tsb, ty, p); break;
+    case 1: e = launch_gemm<1>(dev, grid, s, ta, tb, tsa, tsb, ty, p); break;
+    case 2: e = launch_gemm<2>(dev, grid, s, ta, tb, tsa, tsb, ty, p); break;
+    case 3: e = launch_gemm<3>(dev, grid, s, ta, tb, tsa, tsb, ty, p); break;
+    default: e = launch_gemm<4>(dev, grid, s, ta, tb, tsa, tsb, ty, p); break;
   }
   if (e != cudaSuccess) return cuda_status(e, "gemm_kernel launch");
   return NVFP4_OK;

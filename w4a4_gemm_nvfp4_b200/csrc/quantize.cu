@@ -33,8 +33,6 @@
 #include <cuda_fp16.h>
 
 #include <algorithm>
-#include <atomic>
-#include <mutex>
 
 #include "block_step.cuh"
 #include "common.cuh"
@@ -404,18 +402,19 @@ __global__ void __launch_bounds__(kQuantThreads)
 }
 
 template <bool F, int R>
-cudaError_t launch_quantize_arc(int sms, const QuantParams& p, cudaStream_t s) {
+cudaError_t launch_quantize_arc(int dev, int sms, const QuantParams& p, cudaStream_t s) {
   const size_t smem = static_cast<size_t>(p.K) * 2 * (1 + kArcRows);
-  static std::atomic<int> attr_done{0};
-  if (!attr_done.load(std::memory_order_relaxed)) {
-    cudaError_t e = cudaFuncSetAttribute(quantize_arc_kernel<F, R>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(kArcMaxK * 2 * (1 + kArcRows)));
-    if (e != cudaSuccess) return e;
-    attr_done.store(1, std::memory_order_relaxed);
-  }
+  // the shared-memory opt-in is an attribute of the kernel in this context
+  static PerContextCache<int> attr;
+  int done = 0;
+  cudaError_t e = per_context(attr, dev, [](int* v) {
+    *v = 1;
+    return cudaFuncSetAttribute(quantize_arc_kernel<F, R>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                static_cast<int>(kArcMaxK * 2 * (1 + kArcRows)));
+  }, &done);
+  if (e != cudaSuccess) return e;
   int occ = 0;
-  cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, quantize_arc_kernel<F, R>,
-                                                                kQuantThreads, smem);
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, quantize_arc_kernel<F, R>, kQuantThreads, smem);
   if (e != cudaSuccess) return e;
   const int64_t steps = (p.rows + 127) / 128 * 128 / kArcRows;
   const int grid = static_cast<int>(std::max<int64_t>(
@@ -424,59 +423,59 @@ cudaError_t launch_quantize_arc(int sms, const QuantParams& p, cudaStream_t s) {
   return cudaGetLastError();
 }
 
-cudaError_t launch_quantize_arc_kernel(int mode, int rule, int sms, const QuantParams& p, cudaStream_t s) {
-  if (mode == NVFP4_MODE_SIX) return launch_quantize_arc<false, kRuleMax>(sms, p, s);
-  if (rule == NVFP4_RULE_MAX) return launch_quantize_arc<true, kRuleMax>(sms, p, s);
-  if (rule == NVFP4_RULE_MAE) return launch_quantize_arc<true, kRuleMae>(sms, p, s);
-  return launch_quantize_arc<true, kRuleMse>(sms, p, s);
+cudaError_t launch_quantize_arc_kernel(int mode, int rule, int dev, int sms, const QuantParams& p,
+                                       cudaStream_t s) {
+  if (mode == NVFP4_MODE_SIX) return launch_quantize_arc<false, kRuleMax>(dev, sms, p, s);
+  if (rule == NVFP4_RULE_MAX) return launch_quantize_arc<true, kRuleMax>(dev, sms, p, s);
+  if (rule == NVFP4_RULE_MAE) return launch_quantize_arc<true, kRuleMae>(dev, sms, p, s);
+  return launch_quantize_arc<true, kRuleMse>(dev, sms, p, s);
 }
 
 template <bool F, int R>
-cudaError_t launch_quantize_t(int sms, const QuantParams& p, cudaStream_t s) {
-  static std::atomic<int> per_sm{0};
-  int occ = per_sm.load(std::memory_order_relaxed);
-  if (occ == 0) {
-    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, quantize_t_kernel<F, R>,
-                                                                  kQuantThreads, 0);
-    if (e != cudaSuccess) return e;
-    occ = std::max(1, occ);
-    per_sm.store(occ, std::memory_order_relaxed);
-  }
+cudaError_t launch_quantize_t(int dev, int sms, const QuantParams& p, cudaStream_t s) {
+  static PerContextCache<int> per_sm;
+  int occ = 0;
+  cudaError_t e = per_context(per_sm, dev, [](int* v) {
+    const cudaError_t r = cudaOccupancyMaxActiveBlocksPerMultiprocessor(v, quantize_t_kernel<F, R>, kQuantThreads, 0);
+    *v = std::max(1, *v);
+    return r;
+  }, &occ);
+  if (e != cudaSuccess) return e;
   const int64_t tiles = ((p.rows + 127) / 128) * (((p.K + 127) / 128 * 128) / 64);
   const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(tiles, static_cast<int64_t>(sms) * occ)));
   quantize_t_kernel<F, R><<<grid, kQuantThreads, 0, s>>>(p);
   return cudaGetLastError();
 }
 
-cudaError_t launch_quantize_t_kernel(int mode, int rule, int sms, const QuantParams& p, cudaStream_t s) {
-  if (mode == NVFP4_MODE_SIX) return launch_quantize_t<false, kRuleMax>(sms, p, s);
-  if (rule == NVFP4_RULE_MAX) return launch_quantize_t<true, kRuleMax>(sms, p, s);
-  if (rule == NVFP4_RULE_MAE) return launch_quantize_t<true, kRuleMae>(sms, p, s);
-  return launch_quantize_t<true, kRuleMse>(sms, p, s);
+cudaError_t launch_quantize_t_kernel(int mode, int rule, int dev, int sms, const QuantParams& p,
+                                     cudaStream_t s) {
+  if (mode == NVFP4_MODE_SIX) return launch_quantize_t<false, kRuleMax>(dev, sms, p, s);
+  if (rule == NVFP4_RULE_MAX) return launch_quantize_t<true, kRuleMax>(dev, sms, p, s);
+  if (rule == NVFP4_RULE_MAE) return launch_quantize_t<true, kRuleMae>(dev, sms, p, s);
+  return launch_quantize_t<true, kRuleMse>(dev, sms, p, s);
 }
 
 template <bool F, int R>
-cudaError_t launch_quantize(int sms, const QuantParams& p, cudaStream_t s) {
-  static std::atomic<int> per_sm{0};
-  int occ = per_sm.load(std::memory_order_relaxed);
-  if (occ == 0) {
-    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, quantize_kernel<F, R>,
-                                                                  kQuantThreads, 0);
-    if (e != cudaSuccess) return e;
-    occ = std::max(1, occ);
-    per_sm.store(occ, std::memory_order_relaxed);
-  }
+cudaError_t launch_quantize(int dev, int sms, const QuantParams& p, cudaStream_t s) {
+  static PerContextCache<int> per_sm;
+  int occ = 0;
+  cudaError_t e = per_context(per_sm, dev, [](int* v) {
+    const cudaError_t r = cudaOccupancyMaxActiveBlocksPerMultiprocessor(v, quantize_kernel<F, R>, kQuantThreads, 0);
+    *v = std::max(1, *v);
+    return r;
+  }, &occ);
+  if (e != cudaSuccess) return e;
   const int64_t want = (static_cast<int64_t>(p.ntasks) + kQuantWarps - 1) / kQuantWarps;
   const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(want, static_cast<int64_t>(sms) * occ)));
   quantize_kernel<F, R><<<grid, kQuantThreads, 0, s>>>(p);
   return cudaGetLastError();
 }
 
-cudaError_t launch_quantize_kernel(int mode, int rule, int sms, const QuantParams& p, cudaStream_t s) {
-  if (mode == NVFP4_MODE_SIX) return launch_quantize<false, kRuleMax>(sms, p, s);
-  if (rule == NVFP4_RULE_MAX) return launch_quantize<true, kRuleMax>(sms, p, s);
-  if (rule == NVFP4_RULE_MAE) return launch_quantize<true, kRuleMae>(sms, p, s);
-  return launch_quantize<true, kRuleMse>(sms, p, s);
+cudaError_t launch_quantize_kernel(int mode, int rule, int dev, int sms, const QuantParams& p, cudaStream_t s) {
+  if (mode == NVFP4_MODE_SIX) return launch_quantize<false, kRuleMax>(dev, sms, p, s);
+  if (rule == NVFP4_RULE_MAX) return launch_quantize<true, kRuleMax>(dev, sms, p, s);
+  if (rule == NVFP4_RULE_MAE) return launch_quantize<true, kRuleMae>(dev, sms, p, s);
+  return launch_quantize<true, kRuleMse>(dev, sms, p, s);
 }
 
 }  // namespace
@@ -579,7 +578,7 @@ QuantParams base_params(const void* x, int64_t rows, int64_t K, int64_t ldx, voi
 enum class QuantKind { kRows, kTransposed, kAugmented };
 
 nvfp4_status launch_dynamic(QuantKind kind, QuantParams p, int mode, int rule, float fp8_max,
-                            float* global_scale, uint32_t* partials, int amax_grid, int sms,
+                            float* global_scale, uint32_t* partials, int amax_grid, int dev, int sms,
                             cudaStream_t s) {
   amax_kernel<<<amax_grid, kAmaxThreads, 0, s>>>(p.x, p.rows, p.K, p.ldx, partials);
   cudaError_t e = cudaGetLastError();
@@ -588,9 +587,9 @@ nvfp4_status launch_dynamic(QuantKind kind, QuantParams p, int mode, int rule, f
   p.partials = partials;
   p.nparts = amax_grid;
   p.f6 = fp8_max * 6.0f;
-  e = kind == QuantKind::kTransposed ? launch_quantize_t_kernel(mode, rule, sms, p, s)
-      : kind == QuantKind::kAugmented ? launch_quantize_arc_kernel(mode, rule, sms, p, s)
-                                       : launch_quantize_kernel(mode, rule, sms, p, s);
+  e = kind == QuantKind::kTransposed ? launch_quantize_t_kernel(mode, rule, dev, sms, p, s)
+      : kind == QuantKind::kAugmented ? launch_quantize_arc_kernel(mode, rule, dev, sms, p, s)
+                                       : launch_quantize_kernel(mode, rule, dev, sms, p, s);
   if (e != cudaSuccess) return cuda_status(e, "quantize kernel launch");
   return NVFP4_OK;
 }
@@ -628,7 +627,7 @@ nvfp4_status quantize_impl(const char* fn, QuantKind kind, const void* x, int64_
   p.S = S;
   p.augment = augment;
   const int amax_grid = std::min(amax_grid_size(rows, K, ldx, sms), kMaxPartials);
-  return launch_dynamic(kind, p, mode, rule, fp8_max, global_scale, partials, amax_grid, sms,
+  return launch_dynamic(kind, p, mode, rule, fp8_max, global_scale, partials, amax_grid, dev, sms,
                         static_cast<cudaStream_t>(stream));
 }
 
@@ -689,25 +688,19 @@ namespace {
 constexpr size_t kNoAllocScratchBytes = sizeof(WorkspaceHeader) + sizeof(uint32_t) * kMaxPartials;
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
-constexpr int kNoAllocMaxDevices = 64;
-static std::mutex g_noalloc_mu;
-static void* g_noalloc_addr[kNoAllocMaxDevices];
+static PerContextCache<void*> g_noalloc_addr;
 
 // Device address of g_noalloc_scratch on the current device `dev`, looked up
-// once per device (the first call on a device does this set-up).  In host
-// code the array's name is only a host-side stand-in for the symbol, never a
-// device address, so kernels must get this pointer instead.
+// with that device current once per CUDA context: the first call on a device
+// does this set-up, and so does the first call after the device's context
+// was reset or replaced (the module, and with it the array, is loaded anew).
+// In host code the array's name is only a host-side stand-in for the symbol,
+// never a device address, so kernels must get this pointer instead.
 nvfp4_status noalloc_scratch(int dev, void** out) {
-  if (dev < 0 || dev >= kNoAllocMaxDevices)
-    return set_error(NVFP4_ERR_UNSUPPORTED_DEVICE, "nvfp4_quantize_noalloc: device %d", dev);
-  std::lock_guard<std::mutex> lk(g_noalloc_mu);
-  if (!g_noalloc_addr[dev]) {
-    void* p = nullptr;
-    cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-    if (e != cudaSuccess) return cuda_status(e, "cudaGetSymbolAddress(noalloc scratch)");
-    g_noalloc_addr[dev] = p;
-  }
-  *out = g_noalloc_addr[dev];
+  cudaError_t e = per_context(g_noalloc_addr, dev, [](void** p) {
+    return cudaGetSymbolAddress(p, g_noalloc_scratch);
+  }, out);
+  if (e != cudaSuccess) return cuda_status(e, "cudaGetSymbolAddress(noalloc scratch)");
   return NVFP4_OK;
 }
 
@@ -733,7 +726,7 @@ extern "C" nvfp4_status nvfp4_quantize_noalloc(const void* x, int64_t rows, int6
   auto* ws = static_cast<WorkspaceHeader*>(scratch);
   auto* partials = reinterpret_cast<uint32_t*>(static_cast<char*>(scratch) + sizeof(WorkspaceHeader));
   return launch_dynamic(QuantKind::kRows, base_params(x, rows, K, ldx, codes, scales, ws), mode, rule, fp8_max,
-                        global_scale, partials, amax_grid, sms, static_cast<cudaStream_t>(stream));
+                        global_scale, partials, amax_grid, dev, sms, static_cast<cudaStream_t>(stream));
 }
 
 // ------------------------------------------------------ static tensor scale --
@@ -758,7 +751,7 @@ extern "C" nvfp4_status nvfp4_quantize_with_scale(const void* x, int64_t rows, i
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t e = cudaMemsetAsync(workspace, 0, 2 * sizeof(uint32_t), s);  // status, detail
   if (e != cudaSuccess) return cuda_status(e, "nvfp4_quantize_with_scale: status reset");
-  e = launch_quantize_kernel(mode, rule, sms, p, s);
+  e = launch_quantize_kernel(mode, rule, dev, sms, p, s);
   if (e != cudaSuccess) return cuda_status(e, "quantize_kernel launch");
   return NVFP4_OK;
 }
