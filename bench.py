@@ -3,7 +3,9 @@
 One step = the whole path on one batch: tensor amax -> Four-Over-Six (MSE,
 fp8_max 256) quantization of X -> NVFP4 GEMM against a pre-quantized weight
 (scale-6, fp8_max 448) -> bf16 Y, on the long-prefill MLP shape
-(X 32768 x 5120, W 17408 x 5120).  `value` is whole-job GEMM-equivalent
+(X 32768 x 5120, W 17408 x 5120), as one nvfp4_quantize_gemm call (each
+kernel a programmatic dependent of the one before it).  The breakdown times
+the same step as two calls with an event between quantize and GEMM.  `value` is whole-job GEMM-equivalent
 throughput, 2*M*N*K per step per GPU summed over ranks / step time (TFLOP/s);
 the JSON line also carries the quantizer's GB/s and the GEMM's TFLOP/s with
 their roofline fractions.
@@ -147,6 +149,14 @@ def rank_x_operand(wl, rank: int):
     return workloads.Operand(**{**wl.x.__dict__, "seed": wl.x.seed + 101 * rank})
 
 
+def spread(ts) -> dict:
+    """Median, 10th and 90th percentile (nearest rank) of per-step times, ms."""
+    xs = sorted(ts)
+    pick = lambda q: xs[min(len(xs) - 1, max(0, int(round(q * (len(xs) - 1)))))]
+    return {"median": round(statistics.median(xs), 4), "p10": round(pick(0.1), 4), "p90": round(pick(0.9), 4),
+            "n": len(xs)}
+
+
 def job_tflops(world: int, flops_per_rank: float, ms_max: float) -> float:
     """Whole-job throughput: all ranks' flops over the slowest rank's time."""
     return world * flops_per_rank / (ms_max * 1e-3) / 1e12
@@ -204,11 +214,28 @@ def run_ours(args, world, rank, local):
         if ev:
             ev[2].record(stream)
 
+    def fused_step():
+        # the whole path in one call: amax -> quantize X -> GEMM, each kernel
+        # a programmatic dependent of the one before it
+        nv.quantize_gemm(x, qw, xm, xr, xF, out_dtype=torch.bfloat16, x_out=qx, out=y, workspace=gws)
+
     for _ in range(args.warmup):
+        fused_step()
         step(qx, xm, xr, xF)
         step(q6, "six", "max", 448.0)
     torch.cuda.synchronize()
     assert nv.device_status(qx.workspace) == nv.OK and nv.device_status(gws) == nv.OK
+
+    def timed_fused(steps):
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+        for i in range(steps):
+            flush_l2(i)                             # L2 flush between steps (untimed)
+            torch.cuda._sleep(HOST_LEAD_CYCLES)     # GPU busy while the host enqueues the step
+            evs[i][0].record(stream)
+            fused_step()
+            evs[i][1].record(stream)
+        torch.cuda.synchronize()
+        return [a.elapsed_time(b) for a, b in evs]
 
     def timed(qbuf, mode, rule, F, steps):
         evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
@@ -224,7 +251,12 @@ def run_ours(args, world, rank, local):
     _barrier(world)
     torch.cuda.synchronize()
     with ClockSampler(local) as clocks:
-        tq, tg = timed(qx, xm, xr, xF, args.steps)
+        steps_ms = timed_fused(args.steps)          # the headline: K whole steps
+    assert nv.device_status(qx.workspace) == nv.OK and nv.device_status(gws) == nv.OK
+    # the breakdown: the same step as two calls with an event between them
+    _barrier(world)
+    torch.cuda.synchronize()
+    tq, tg = timed(qx, xm, xr, xF, args.steps)
     _barrier(world)
     torch.cuda.synchronize()
     tq6, tg6 = timed(q6, "six", "max", 448.0, args.steps)
@@ -256,7 +288,37 @@ def run_ours(args, world, rank, local):
     ms_qstatic = _max_over_ranks(world, ms_qstatic, device)
     ms_qstatic6 = _max_over_ranks(world, ms_qstatic6, device)
 
-    ms_step = _max_over_ranks(world, statistics.mean(a + b for a, b in zip(tq, tg)), device)
+    # the "next" entry points on the same operands: the GEMM writing Y as an
+    # NVFP4 operand (4/6-MSE at a static output alpha), and the augmented-
+    # channel step (ARCQuant: 128 residual channels of the most outlying
+    # columns, then the GEMM over K + 128 against the weight with those
+    # columns duplicated)
+    S_ARC = 128
+    y_alpha = (y.float().abs().amax() / (6 * 256.0)).reshape(1).to(torch.float32)
+    qy = nv.gemm_quantized(qx, qw, y_alpha, "four_over_six", "mse")
+    perm = x.float().abs().amax(dim=0).argsort(descending=True).to(torch.int32)
+    qw_arc = nv.quantize_arc(wl.w.make().to(device), perm, S_ARC, nv.AUG_DUPLICATE, wm, wr, wF)
+    qa = nv.quantize_arc(x, perm, S_ARC, nv.AUG_RESIDUAL, xm, xr, xF)
+    y_arc = torch.empty_like(y)
+    _barrier(world)
+    torch.cuda.synchronize()
+    ms_qout = time_op(lambda: nv.gemm_quantized(qx, qw, y_alpha, "four_over_six", "mse", out=qy), args.steps)
+    ms_arc_q = time_op(lambda: nv.quantize_arc(x, perm, S_ARC, nv.AUG_RESIDUAL, xm, xr, xF, out=qa), args.steps)
+
+    def arc_step():
+        nv.quantize_arc(x, perm, S_ARC, nv.AUG_RESIDUAL, xm, xr, xF, out=qa)
+        nv.gemm(qa, qw_arc, out_dtype=torch.bfloat16, out=y_arc, workspace=gws)
+
+    ms_arc_step = time_op(arc_step, args.steps)
+    assert (nv.device_status(qy.workspace) == nv.OK and nv.device_status(qa.workspace) == nv.OK
+            and nv.device_status(gws) == nv.OK)
+    ms_qout = _max_over_ranks(world, ms_qout, device)
+    ms_arc_q = _max_over_ranks(world, ms_arc_q, device)
+    ms_arc_step = _max_over_ranks(world, ms_arc_step, device)
+    del qy, qa, qw_arc, y_arc
+
+    ms_step = _max_over_ranks(world, statistics.mean(steps_ms), device)
+    ms_two_calls = _max_over_ranks(world, statistics.mean(a + b for a, b in zip(tq, tg)), device)
     ms_quant = _max_over_ranks(world, statistics.mean(tq), device)
     ms_gemm = _max_over_ranks(world, statistics.mean(tg), device)
     ms_quant6 = _max_over_ranks(world, statistics.mean(tq6), device)
@@ -270,8 +332,7 @@ def run_ours(args, world, rank, local):
     e0.record(stream)
     for _ in range(e2e_steps):
         x.copy_(x_host, non_blocking=True)
-        nv.quantize(x, xm, xr, xF, out=qx)
-        nv.gemm(qx, qw, out_dtype=torch.bfloat16, out=y, workspace=gws)
+        fused_step()
         y_host.copy_(y, non_blocking=True)
     e1.record(stream)
     torch.cuda.synchronize()
@@ -317,6 +378,7 @@ def run_ours(args, world, rank, local):
             "traffic_detail": GEMM_PREFILL_TRAFFIC if args.workload == "prefill" else None,
         },
         "breakdown": {
+            "ms_step_two_calls": round(ms_two_calls, 4),
             "ms_quantize_46": round(ms_quant, 4),
             "ms_quantize_six": round(ms_quant6, 4),
             "overhead_46_vs_six": round(ms_quant / ms_quant6 - 1.0, 4),
@@ -332,6 +394,18 @@ def run_ours(args, world, rank, local):
             "ms_gemm": round(ms_gemm, 4),
             "gemm_TFLOPs": round(gemm_tflops, 1),
             "ms_gemm_after_six": round(_max_over_ranks(world, statistics.mean(tg6), device), 4),
+            "ms_gemm_nvfp4_out_46mse": round(ms_qout, 4),
+            "gemm_nvfp4_out_TFLOPs": round(flops / (ms_qout * 1e-3) / 1e12, 1),
+            "gemm_nvfp4_out_frac_fp4_peak": round(flops / (ms_qout * 1e-3) / 1e12 / fp4_peak, 4),
+            "ms_quantize_arc_S128": round(ms_arc_q, 4),
+            "ms_step_arc_S128": round(ms_arc_step, 4),
+            "arc_step_overhead_vs_step": round(ms_arc_step / ms_step - 1.0, 4),
+        },
+        "stats": {
+            "what": "per-step CUDA-event times of this rank (rank 0), ms",
+            "ms_per_step": spread(steps_ms),
+            "ms_quantize_46": spread(tq),
+            "ms_gemm": spread(tg),
         },
         "e2e": {
             "value": round(job_tflops(world, flops, ms_e2e), 2),
@@ -344,7 +418,7 @@ def run_ours(args, world, rank, local):
         "clocks": clocks.summary(),
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        result["cpu_baseline"] = cpu_baseline(args, sample_rows=8192)  # about 10 s of CPU work
+        result["cpu_baseline"] = cpu_baseline(args, sample_rows=1024)  # about 40 s of CPU work in all
     return result
 
 
@@ -395,17 +469,95 @@ def _cores():
         return os.cpu_count()
 
 
+def _host_threads() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def cpu_quantizer_baseline(wl, x_recipe):
+    """The oracle quantizer on the workload's whole X: amax, then every block,
+    single-threaded and on all host threads (row slices, one oracle call per
+    slice; ctypes releases the GIL during each), results checked identical.
+    GB/s over the same 4.5625 B/element as the GPU's end-to-end figure."""
+    from concurrent.futures import ThreadPoolExecutor
+
+    import numpy as np
+
+    import oracle
+
+    mode = {"six": oracle.MODE_SIX, "four_over_six": oracle.MODE_FOUR_OVER_SIX}
+    rule = {"max": oracle.RULE_MAX, "mae": oracle.RULE_MAE, "mse": oracle.RULE_MSE}
+    xm, xr, xF = x_recipe
+    x = wl.x.make()
+    rows, K = x.shape
+    bits = oracle.as_bf16_bits(x)
+    t0 = time.perf_counter()
+    amax, _ = oracle.amax(bits)
+    alpha = oracle.global_scale(amax, xF)
+    t_amax = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    c1, s1 = oracle.quantize_rows(bits, alpha, mode[xm], rule[xr])
+    t1 = time.perf_counter() - t0 + t_amax
+    threads = _host_threads()
+    edges = np.linspace(0, rows, threads + 1).astype(int)
+    t0 = time.perf_counter()
+    amax_n, _ = oracle.amax(bits)   # the amax pass again, inside the multi-threaded time
+    with ThreadPoolExecutor(threads) as pool:
+        parts = list(pool.map(lambda i: oracle.quantize_rows(bits[edges[i]:edges[i + 1]], alpha, mode[xm], rule[xr]),
+                              range(threads)))
+    tn = time.perf_counter() - t0
+    identical = (amax_n == amax and np.array_equal(np.concatenate([p[0] for p in parts]), c1)
+                 and np.array_equal(np.concatenate([p[1] for p in parts]), s1))
+    nbytes = (QUANT_BYTES_PER_ELEM + AMAX_BYTES_PER_ELEM) * rows * K
+    return {"GBps_1_thread": round(nbytes / t1 / 1e9, 4), "GBps_all_threads": round(nbytes / tn / 1e9, 4),
+            "threads": threads, "s_1_thread": round(t1, 2), "s_all_threads": round(tn, 2),
+            "identical": bool(identical),
+            "sample": f"the whole X ({rows}x{K}, {xm}-{xr}, fp8_max {xF:g}): amax + every block; the "
+                      f"multi-threaded run splits the rows over {threads} threads"}
+
+
+def cpu_gemm_baseline(wl, x_recipe, rows=256):
+    """The oracle GEMM (fp64 matmul of the exactly dequantized operands) on a
+    slice of `rows` rows of X; the full-size time is extrapolated."""
+    import oracle
+
+    mode = {"six": oracle.MODE_SIX, "four_over_six": oracle.MODE_FOUR_OVER_SIX}
+    rule = {"max": oracle.RULE_MAX, "mae": oracle.RULE_MAE, "mse": oracle.RULE_MSE}
+    xm, xr, xF = x_recipe
+    w_deq = _w_dequant(wl)
+    x = workloads.Operand(**{**wl.x.__dict__, "rows": rows}).make()
+    xc, xs, xa = oracle.quantize(x, mode[xm], rule[xr], xF)
+    t0 = time.perf_counter()
+    xd = oracle.dequantize(xc, xs, xa)
+    _ = xd @ w_deq.T
+    dt = time.perf_counter() - t0
+    flops = 2.0 * rows * wl.N * wl.K
+    return {"GFLOPs": round(flops / dt / 1e9, 2), "rows": rows, "threads": _cores(), "s": round(dt, 3),
+            "full_size_s_extrapolated": round(dt * wl.M / rows, 1),
+            "sample": f"{rows} rows of X dequantized and multiplied in fp64 by the dequantized W {wl.N}x{wl.K} "
+                      f"(BLAS threads {_cores()}); the full-size time is that x {wl.M}/{rows}, extrapolated"}
+
+
 def cpu_baseline(args, sample_rows=64):
+    """The oracle timed on this host: a bounded sample of the whole step
+    (quantize `sample_rows` rows of X, then their fp64 GEMM against the
+    dequantized W) as the headline figure, plus the quantizer on the whole X
+    and the GEMM on a 256-row slice as separate records."""
     wl = workloads.WORKLOADS[args.workload]
     w_deq = _w_dequant(wl)
     t0 = time.perf_counter()
     flops = _oracle_sample(wl, args.x_recipe, sample_rows, w_deq)
     dt = time.perf_counter() - t0
+    del w_deq
     return {"value": round(flops / dt / 1e12, 6), "unit": "TFLOP/s", "cores": _cores(),
             "kind": "oracle",
             "sample": f"{sample_rows} rows of X ({wl.K} wide) quantized by the C oracle (1 thread) + "
                       f"fp64 numpy GEMM against the oracle-dequantized W {wl.N}x{wl.K} "
-                      f"({_cores()} BLAS threads); W quantization untimed; {dt:.1f} s"}
+                      f"({_cores()} BLAS threads); W quantization untimed; {dt:.1f} s",
+            "quantizer": cpu_quantizer_baseline(wl, args.x_recipe),
+            "gemm": cpu_gemm_baseline(wl, args.x_recipe)}
 
 
 def run_reference(args, world, rank):

@@ -5,7 +5,8 @@
  * Two core operations, both asynchronous on a caller-supplied CUDA stream
  * (variants declared further down: a static tensor scale, quantization of
  * x^T, ARCQuant augmented residual channels, an allocation-free quantizer,
- * per-segment B scales, and a GEMM that writes an NVFP4 output):
+ * per-segment B scales, a GEMM that writes an NVFP4 output, and one call that
+ * quantizes the activations and runs the GEMM):
  *
  *  nvfp4_quantize  16-element block-scaled NVFP4 quantization of a bf16
  *                  matrix: E2M1 codes, one FP8 E4M3 scale per 16 elements
@@ -62,7 +63,7 @@
  * Errors: every call validates its arguments on the host and returns a status
  * without launching anything when they are invalid.  Conditions only the GPU
  * can see (non-finite input to nvfp4_quantize, a static alpha that is not a
- * positive finite number, a bounded wait that ran out in nvfp4_gemm) are
+ * positive finite number, a bounded device wait that ran out) are
  * written to a status word in the call's workspace and read by
  * nvfp4_get_device_status.  Launch failures return NVFP4_ERR_CUDA with
  * the CUDA message available from nvfp4_last_error_message.
@@ -123,13 +124,16 @@ NVFP4_API size_t nvfp4_gemm_workspace_bytes(void);
  *            The pages use 448 for scale-6 and 256 for 4/6; any pairing is
  *            accepted.
  * Requirements: rows >= 1, K >= 64, K % 64 == 0, ldx >= K, ldx % 8 == 0,
- * rows * ldx <= 2^40 and (rows rounded up to 128) * K < 2^40 elements,
+ * rows * ldx <= 2^40 and (rows rounded up to 128) * (K rounded up to 512)
+ * < 2^40 elements,
  * x / codes / scales / workspace 16-byte aligned, global_scale 4-byte
  * aligned, workspace_bytes >= nvfp4_quantize_workspace_bytes(rows, K).
  * Writes codes, every byte of scales (padding = 0), *global_scale and the
  * workspace status word.  When x holds Inf or NaN the status word becomes
  * NVFP4_ERR_NONFINITE, *global_scale becomes NaN, and codes/scales are left
- * unwritten.  Returns once both kernels are enqueued (two launches). */
+ * unwritten.  Returns once both kernels are enqueued: the amax pass, then the
+ * quantize kernel as its programmatic dependent (scheduled while the amax pass
+ * drains; it waits for the pass before reading anything). */
 NVFP4_API nvfp4_status nvfp4_quantize(const void* x, int64_t rows, int64_t K, int64_t ldx, int mode,
                             int rule, float fp8_max, void* codes, void* scales,
                             float* global_scale, void* workspace, size_t workspace_bytes,
@@ -274,6 +278,27 @@ NVFP4_API nvfp4_status nvfp4_gemm_segmented(const void* a_codes, const void* a_s
                                             const int64_t* seg_ends, int nseg, int64_t M, int64_t N,
                                             int64_t K, void* y, int64_t ldy, int out_dtype,
                                             void* workspace, size_t workspace_bytes, void* stream);
+
+/* The W4A4 linear layer in one call: quantize the activations x [M, K] as
+ * nvfp4_quantize does (into x_codes / x_scales / *x_global_scale, with
+ * x_workspace), then Y [M, N] = X_hat . W_hat^T as nvfp4_gemm does, against
+ * a weight already quantized (w_codes / w_scales / w_global, N rows).  The
+ * long-prefill path of the Minima page ("산업 영향"): quantize -> GEMM on one
+ * stream.  Enqueues the GEMM's 64-byte status reset, the amax pass, the
+ * quantize kernel and the GEMM kernel, each kernel a programmatic dependent
+ * of the one before it (it is scheduled while that one drains and waits for
+ * it before touching memory), so the quantizer's and the GEMM's prologues
+ * overlap the preceding kernel's tail.  Results are those of the two calls
+ * made one after the other, bit for bit.  Arguments and requirements are
+ * those of nvfp4_quantize and nvfp4_gemm; every one is checked before
+ * anything is enqueued.  Device status: x_workspace as nvfp4_quantize,
+ * workspace as nvfp4_gemm. */
+NVFP4_API nvfp4_status nvfp4_quantize_gemm(const void* x, int64_t M, int64_t K, int64_t ldx, int mode, int rule,
+                                           float fp8_max, void* x_codes, void* x_scales, float* x_global_scale,
+                                           void* x_workspace, size_t x_workspace_bytes, const void* w_codes,
+                                           const void* w_scales, const float* w_global, int64_t N, void* y,
+                                           int64_t ldy, int out_dtype, void* workspace, size_t workspace_bytes,
+                                           void* stream);
 
 /* Synchronizes `stream`, then returns the status word the last call that used
  * `workspace` wrote (NVFP4_OK, NVFP4_ERR_INVALID_ARG, NVFP4_ERR_NONFINITE or

@@ -220,3 +220,33 @@ def test_no_gpu_fails_loudly():
     assert _g() in (nv.ERR_CUDA, nv.ERR_UNSUPPORTED_DEVICE)
     assert _g(ldy=1 << 40) in (nv.ERR_CUDA, nv.ERR_UNSUPPORTED_DEVICE)  # the largest legal row pitch
     assert _qn() in (nv.ERR_CUDA, nv.ERR_UNSUPPORTED_DEVICE)
+
+
+def _qg(**kw):
+    args = dict(x=FAKE, M=64, K=512, ldx=512, mode=1, rule=2, fp8_max=256.0, x_codes=FAKE, x_scales=FAKE,
+                x_global_scale=FAKE, x_workspace=FAKE, x_workspace_bytes=1 << 20, w_codes=FAKE, w_scales=FAKE,
+                w_global=FAKE, N=256, y=FAKE, ldy=256, out_dtype=0, workspace=FAKE, workspace_bytes=64,
+                stream=None)
+    args.update(kw)
+    return nv.nvfp4_quantize_gemm(*args.values())
+
+
+@pytest.mark.parametrize("bad", [
+    # the quantize half
+    dict(x=None), dict(x_codes=None), dict(x_global_scale=None), dict(x_workspace=None), dict(M=0), dict(K=96),
+    dict(ldx=256), dict(mode=2), dict(rule=5), dict(fp8_max=100.0), dict(x_workspace_bytes=16),
+    # the GEMM half
+    dict(w_codes=None), dict(w_scales=None), dict(w_global=None), dict(y=None), dict(workspace=None), dict(N=0),
+    dict(ldy=128), dict(out_dtype=3), dict(y=FAKE + 1), dict(workspace_bytes=4), dict(w_global=FAKE + 2),
+])
+def test_quantize_gemm_rejects_bad_arguments(bad):
+    assert _qg(**bad) == nv.ERR_INVALID_ARG
+    assert nv.last_error_message().startswith("nvfp4_quantize_gemm")
+
+
+def test_quantize_gemm_without_gpu_fails_loudly():
+    import torch
+
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    assert _qg() in (nv.ERR_CUDA, nv.ERR_UNSUPPORTED_DEVICE)

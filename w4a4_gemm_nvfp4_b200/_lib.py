@@ -50,6 +50,9 @@ _SIGNATURES = {
                                             _P, _P, _P, _P, ctypes.c_size_t, _P]),
     "nvfp4_gemm_segmented": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, ctypes.c_int, _I64, _I64,
                                             _I64, _P, _I64, ctypes.c_int, _P, ctypes.c_size_t, _P]),
+    "nvfp4_quantize_gemm": (ctypes.c_int, [_P, _I64, _I64, _I64, ctypes.c_int, ctypes.c_int, ctypes.c_float,
+                                           _P, _P, _P, _P, ctypes.c_size_t, _P, _P, _P, _I64, _P, _I64,
+                                           ctypes.c_int, _P, ctypes.c_size_t, _P]),
     "nvfp4_get_device_status": (ctypes.c_int, [_P, _P]),
     "nvfp4_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "nvfp4_last_error_message": (ctypes.c_char_p, []),
@@ -158,6 +161,14 @@ def nvfp4_gemm_segmented(a_codes, a_scales, a_global, b_codes, b_scales, b_globa
     return load().nvfp4_gemm_segmented(a_codes, a_scales, a_global, b_codes, b_scales, b_globals,
                                        seg_ends, nseg, M, N, K, y, ldy, out_dtype, workspace,
                                        workspace_bytes, stream)
+
+
+def nvfp4_quantize_gemm(x, M, K, ldx, mode, rule, fp8_max, x_codes, x_scales, x_global_scale, x_workspace,
+                        x_workspace_bytes, w_codes, w_scales, w_global, N, y, ldy, out_dtype, workspace,
+                        workspace_bytes, stream) -> int:
+    return load().nvfp4_quantize_gemm(x, M, K, ldx, mode, rule, fp8_max, x_codes, x_scales, x_global_scale,
+                                      x_workspace, x_workspace_bytes, w_codes, w_scales, w_global, N, y, ldy,
+                                      out_dtype, workspace, workspace_bytes, stream)
 
 
 def nvfp4_get_device_status(workspace, stream) -> int:
@@ -412,6 +423,50 @@ def gemm(a: NVFP4Tensor, b: NVFP4Tensor, out_dtype=None, out=None, workspace=Non
                     _stream_handle(stream))
     _check(st, "nvfp4_gemm")
     return out
+
+
+def quantize_gemm(x, w: NVFP4Tensor, mode: str = "six", rule: str = "max", fp8_max: float | None = None,
+                  out_dtype=None, x_out: NVFP4Tensor | None = None, out=None, workspace=None, stream=None):
+    """The W4A4 linear layer in one call: quantize the bf16 CUDA activations
+    x [M, K] (into ``x_out``, which then holds the NVFP4 operand of x), then
+    Y = X_hat @ W_hat^T against the pre-quantized weight ``w`` [N, K].  The
+    quantize and GEMM kernels run as programmatic dependents of the kernel
+    before them.  Returns (x_out, Y)."""
+    import torch
+
+    if x.dtype != torch.bfloat16 or x.dim() != 2 or not x.is_cuda:
+        raise ValueError("x must be a 2-D bfloat16 CUDA tensor")
+    if x.stride(1) != 1:
+        raise ValueError("x must have unit stride along K")
+    M, K = x.shape
+    if w.K != K:
+        raise ValueError("x and w disagree on K")
+    N = w.rows
+    dev = x.device
+    F = DEFAULT_FP8_MAX[mode] if fp8_max is None else float(fp8_max)
+    out_dtype, code = _out_code(out_dtype, out)
+    if x_out is None:
+        x_out = NVFP4Tensor(
+            codes=torch.empty(M, K // 2, dtype=torch.uint8, device=dev),
+            scales=torch.empty(max(1, nvfp4_scales_bytes(M, K)), dtype=torch.uint8, device=dev),
+            global_scale=torch.empty(1, dtype=torch.float32, device=dev),
+            workspace=torch.empty(nvfp4_quantize_workspace_bytes(M, K), dtype=torch.uint8, device=dev),
+            rows=M, K=K)
+    _check_operand(x_out, "x_out", M, K, dev, workspace=True)
+    _check_operand(w, "w", N, K, dev)
+    if out is None:
+        out = torch.empty(M, N, dtype=out_dtype, device=dev)
+    if workspace is None:
+        workspace = torch.empty(nvfp4_gemm_workspace_bytes(), dtype=torch.uint8, device=dev)
+    _check_output(out, M, N, out_dtype, dev)
+    _require(workspace, "workspace", torch.uint8, 0, dev)
+    st = nvfp4_quantize_gemm(x.data_ptr(), M, K, _row_pitch(x), MODES[mode], RULES[rule], F,
+                             x_out.codes.data_ptr(), x_out.scales.data_ptr(), x_out.global_scale.data_ptr(),
+                             x_out.workspace.data_ptr(), x_out.workspace.numel(), w.codes.data_ptr(),
+                             w.scales.data_ptr(), w.global_scale.data_ptr(), N, out.data_ptr(), _row_pitch(out),
+                             code, workspace.data_ptr(), workspace.numel(), _stream_handle(stream))
+    _check(st, "nvfp4_quantize_gemm")
+    return x_out, out
 
 
 def gemm_quantized(a: NVFP4Tensor, b: NVFP4Tensor, y_alpha, mode: str = "six", rule: str = "max",

@@ -236,19 +236,45 @@ __device__ __forceinline__ void quantize_pairs(const f2 p[8], float b, const Blo
   scale = pick4 ? (sc >> 8) : (sc & 0xFFu);
 }
 
+// Three-input maximum that propagates NaN (one instruction on sm_100; the
+// compiler folds fabsf of an operand into it).
+__device__ __forceinline__ float max3_nan(float a, float b, float c) {
+  float d;
+  asm("max.NaN.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
 // bf16 block (8 words of bf16 pairs, element 2j in the low half of word j) ->
 // binary32 pairs p[j] = (x_j, x_{j+8}); returns the block's max |x| bit
 // pattern (0x7F80 and above: Inf or NaN).
 __device__ __forceinline__ uint32_t unpack_block(const uint4& lo, const uint4& hi, f2 p[8]) {
   const uint32_t w[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
-  uint32_t m = absmax4(lo, 0u);
-  m = absmax4(hi, m);
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    p[2 * i] = make_f2(__uint_as_float(w[i] << 16), __uint_as_float(w[i + 4] << 16));
-    p[2 * i + 1] = make_f2(__uint_as_float(w[i] & 0xFFFF0000u), __uint_as_float(w[i + 4] & 0xFFFF0000u));
+    // bf16 -> binary32 as a mixed-precision add of -0 (exact for every bf16
+    // value, signed zeros included), which runs on the FMA pipe instead of
+    // taking integer shifts and masks
+    float a0, a1, b0, b1;
+    asm("{\n\t.reg .b16 l0, h0, l1, h1;\n\t"
+        "mov.b32 {l0, h0}, %4;\n\t"
+        "mov.b32 {l1, h1}, %5;\n\t"
+        "add.rn.f32.bf16 %0, l0, 0f80000000;\n\t"
+        "add.rn.f32.bf16 %1, l1, 0f80000000;\n\t"
+        "add.rn.f32.bf16 %2, h0, 0f80000000;\n\t"
+        "add.rn.f32.bf16 %3, h1, 0f80000000;\n\t}"
+        : "=f"(a0), "=f"(a1), "=f"(b0), "=f"(b1)
+        : "r"(w[i]), "r"(w[i + 4]));
+    p[2 * i] = make_f2(a0, a1);
+    p[2 * i + 1] = make_f2(b0, b1);
   }
-  return max(m & 0xFFFFu, m >> 16);
+  // max |x| of the 16 values (exact: a maximum of bf16 values), NaN kept
+  const float m0 = max3_nan(fabsf(p[0].a()), fabsf(p[1].a()), fabsf(p[2].a()));
+  const float m1 = max3_nan(fabsf(p[3].a()), fabsf(p[4].a()), fabsf(p[5].a()));
+  const float m2 = max3_nan(fabsf(p[6].a()), fabsf(p[7].a()), fabsf(p[0].b()));
+  const float m3 = max3_nan(fabsf(p[1].b()), fabsf(p[2].b()), fabsf(p[3].b()));
+  const float m4 = max3_nan(fabsf(p[4].b()), fabsf(p[5].b()), fabsf(p[6].b()));
+  const float m = max3_nan(max3_nan(m0, m1, m2), max3_nan(m3, m4, fabsf(p[7].b())), 0.0f);
+  return __float_as_uint(m) >> 16;  // its bf16 bit pattern
 }
 
 // Quantize one bf16 block; returns its max |x| bit pattern.

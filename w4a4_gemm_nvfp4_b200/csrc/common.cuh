@@ -7,6 +7,7 @@
 #include <stdint.h>
 
 #include <mutex>
+#include <utility>
 
 #include "nvfp4.h"
 
@@ -22,6 +23,35 @@ nvfp4_status check_device(int* device, int* num_sms);
 nvfp4_status cuda_status(cudaError_t err, const char* what);
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// nvfp4_quantize's argument checks alone (no device check; enqueues nothing), and its whole work
+// (checks, amax pass, quantize kernel), with `fn` naming the entry point in
+// error messages: for entry points that quantize and then go on.
+nvfp4_status quantize_rows_check(const char* fn, const void* x, int64_t rows, int64_t K, int64_t ldx, int mode,
+                                 int rule, float fp8_max, const void* codes, const void* scales,
+                                 const float* global_scale, const void* workspace, size_t workspace_bytes);
+nvfp4_status quantize_rows_enqueue(const char* fn, const void* x, int64_t rows, int64_t K, int64_t ldx, int mode,
+                                   int rule, float fp8_max, void* codes, void* scales, float* global_scale,
+                                   void* workspace, size_t workspace_bytes, void* stream);
+
+// Launches `kernel` on `stream`, as a programmatic dependent of the previous
+// kernel on the stream when `pdl` is set (the kernel must then call
+// pdl_wait() before touching memory that kernel uses).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_kernel(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                          bool pdl, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = pdl ? 1 : 0;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 // The driver's unique id of the CUDA context current on this thread (ids are
 // never reused within a process, unlike context handles), or 0 when no
@@ -231,6 +261,19 @@ __device__ __forceinline__ void cluster_sync_all() {
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar_cluster) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster)
                : "memory");
+}
+
+// Programmatic dependent launch.  A kernel launched as a programmatic
+// dependent of the previous kernel on its stream may start while that kernel
+// still runs; pdl_wait() blocks until the previous kernel has completed and
+// its memory writes are visible, so it must come before the first access to
+// anything the previous kernel touches.  For a kernel launched normally it
+// returns at once.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+// Lets a programmatic dependent of this grid start once every CTA of this
+// grid has called it (or exited); the dependent still waits in pdl_wait().
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
 __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {

@@ -256,6 +256,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   cluster_sync_all();  // both CTAs' barriers exist before anyone signals them
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // launched as a programmatic dependent of the quantize kernel that writes
+  // A: everything above overlapped that kernel's tail; no global memory is
+  // touched before it has finished
+  pdl_wait();
 
   if (warp == 0) {
     // -------------------------------------------------- TMA producer ----
@@ -672,9 +676,9 @@ void nvfp4_testing_set_gemm_wait(uint64_t timeout_ns, int debug_flags) {
 namespace {
 
 template <int EPI>
-cudaError_t launch_gemm(int dev, unsigned grid, cudaStream_t s, const CUtensorMap& ta, const CUtensorMap& tb,
-                        const CUtensorMap& tsa, const CUtensorMap& tsb, const CUtensorMap& ty,
-                        const GemmParams& p) {
+cudaError_t launch_gemm(int dev, unsigned grid, cudaStream_t s, bool pdl, const CUtensorMap& ta,
+                        const CUtensorMap& tb, const CUtensorMap& tsa, const CUtensorMap& tsb,
+                        const CUtensorMap& ty, const GemmParams& p) {
   // the shared-memory opt-in is an attribute of the kernel in this context
   static PerContextCache<int> attr;
   int done = 0;
@@ -684,17 +688,27 @@ cudaError_t launch_gemm(int dev, unsigned grid, cudaStream_t s, const CUtensorMa
                                 static_cast<int>(SMEM_BYTES));
   }, &done);
   if (attr_err != cudaSuccess) return attr_err;
-  gemm_kernel<EPI><<<grid, kThreads, SMEM_BYTES, s>>>(ta, tb, tsa, tsb, ty, p);
-  return cudaGetLastError();
+  return launch_kernel(gemm_kernel<EPI>, dim3(grid), dim3(kThreads), SMEM_BYTES, s, pdl, ta, tb, tsa, tsb, ty, p);
 }
 
+// A GEMM checked and ready to launch: tensor maps and kernel parameters.
+struct GemmLaunch {
+  CUtensorMap ta, tb, tsa, tsb, ty;
+  GemmParams p;
+  unsigned grid;
+  int epi;
+  int dev;
+  void* workspace;
+};
+
+// Checks the arguments and prepares the launch; enqueues nothing.
 // epi: 0 = bf16 / fp32 Y; 1..4 = NVFP4 Y (q_* arguments), see gemm_kernel.
-nvfp4_status gemm_impl(const char* fn, const void* a_codes, const void* a_scales, const float* a_global,
-                       const void* b_codes, const void* b_scales, const float* b_global,
-                       const int64_t* seg_ends, int nseg, int64_t M, int64_t N, int64_t K, void* y,
-                       int64_t ldy, int out_dtype, void* workspace, size_t workspace_bytes,
-                       void* stream, int epi = 0, const float* q_alpha = nullptr,
-                       void* q_codes = nullptr, void* q_scales = nullptr) {
+nvfp4_status gemm_prepare(GemmLaunch* L, const char* fn, const void* a_codes, const void* a_scales,
+                          const float* a_global, const void* b_codes, const void* b_scales,
+                          const float* b_global, const int64_t* seg_ends, int nseg, int64_t M, int64_t N,
+                          int64_t K, void* y, int64_t ldy, int out_dtype, void* workspace,
+                          size_t workspace_bytes, int epi, const float* q_alpha, void* q_codes,
+                          void* q_scales) {
   if (!a_codes || !a_scales || !a_global || !b_codes || !b_scales || !b_global || !y || !workspace)
     return set_error(NVFP4_ERR_INVALID_ARG, "%s: null pointer argument", fn);
   if (epi > 0) {
@@ -731,17 +745,12 @@ nvfp4_status gemm_impl(const char* fn, const void* a_codes, const void* a_scales
   nvfp4_status st = check_device(&dev, &sms);
   if (st != NVFP4_OK) return st;
 
-  CUtensorMap ta, tb, tsa, tsb;
-  if ((st = make_code_map(&ta, a_codes, M, K)) != NVFP4_OK) return st;
-  if ((st = make_code_map(&tb, b_codes, N, K)) != NVFP4_OK) return st;
-  if ((st = make_scale_map(&tsa, a_scales, M, K, 1)) != NVFP4_OK) return st;
-  if ((st = make_scale_map(&tsb, b_scales, N, K, 2)) != NVFP4_OK) return st;
+  if ((st = make_code_map(&L->ta, a_codes, M, K)) != NVFP4_OK) return st;
+  if ((st = make_code_map(&L->tb, b_codes, N, K)) != NVFP4_OK) return st;
+  if ((st = make_scale_map(&L->tsa, a_scales, M, K, 1)) != NVFP4_OK) return st;
+  if ((st = make_scale_map(&L->tsb, b_scales, N, K, 2)) != NVFP4_OK) return st;
 
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  cudaError_t e = cudaMemsetAsync(workspace, 0, sizeof(WorkspaceHeader), s);
-  if (e != cudaSuccess) return cuda_status(e, "cudaMemsetAsync(status)");
-
-  GemmParams p;
+  GemmParams& p = L->p;
   p.a_global = a_global;
   p.b_global = b_global;
   p.nseg = nseg;
@@ -764,23 +773,49 @@ nvfp4_status gemm_impl(const char* fn, const void* a_codes, const void* a_scales
   p.q_alpha = q_alpha;
   p.q_codes = static_cast<uint8_t*>(q_codes);
   p.q_scales = static_cast<uint8_t*>(q_scales);
-  CUtensorMap ty;
-  std::memset(&ty, 0, sizeof(ty));
-  if (p.tma_store && (st = make_output_map(&ty, y, M, N, ldy, p.out_fp32 != 0)) != NVFP4_OK) return st;
+  std::memset(&L->ty, 0, sizeof(L->ty));
+  if (p.tma_store && (st = make_output_map(&L->ty, y, M, N, ldy, p.out_fp32 != 0)) != NVFP4_OK) return st;
   p.timeout_ns = g_timeout_ns;
   p.debug_flags = g_debug_flags;
   // one CTA pair per two SMs, never more pairs than tiles
   const int64_t pairs = std::max<int64_t>(1, std::min<int64_t>(num_tiles, sms / 2));
-  const unsigned grid = static_cast<unsigned>(2 * pairs);
-  switch (epi) {
-    case 0: e = launch_gemm<0>(dev, grid, s, ta, tb, tsa, tsb, ty, p); break;
-    case 1: e = launch_gemm<1>(dev, grid, s, ta, tb, tsa, tsb, ty, p); break;
-    case 2: e = launch_gemm<2>(dev, grid, s, ta, tb, tsa, tsb, ty, p); break;
-    case 3: e = launch_gemm<3>(dev, grid, s, ta, tb, tsa, tsb, ty, p); break;
-    default: e = launch_gemm<4>(dev, grid, s, ta, tb, tsa, tsb, ty, p); break;
+  L->grid = static_cast<unsigned>(2 * pairs);
+  L->epi = epi;
+  L->dev = dev;
+  L->workspace = workspace;
+  return NVFP4_OK;
+}
+
+// Enqueues the status-word reset (unless the caller already did) and the
+// kernel, as a programmatic dependent of the previous kernel when `pdl` is
+// set (only useful when that kernel immediately precedes it on the stream).
+nvfp4_status gemm_enqueue(const GemmLaunch& L, cudaStream_t s, bool clear_status, bool pdl) {
+  cudaError_t e;
+  if (clear_status && (e = cudaMemsetAsync(L.workspace, 0, sizeof(WorkspaceHeader), s)) != cudaSuccess)
+    return cuda_status(e, "cudaMemsetAsync(status)");
+  switch (L.epi) {
+    case 0: e = launch_gemm<0>(L.dev, L.grid, s, pdl, L.ta, L.tb, L.tsa, L.tsb, L.ty, L.p); break;
+    case 1: e = launch_gemm<1>(L.dev, L.grid, s, pdl, L.ta, L.tb, L.tsa, L.tsb, L.ty, L.p); break;
+    case 2: e = launch_gemm<2>(L.dev, L.grid, s, pdl, L.ta, L.tb, L.tsa, L.tsb, L.ty, L.p); break;
+    case 3: e = launch_gemm<3>(L.dev, L.grid, s, pdl, L.ta, L.tb, L.tsa, L.tsb, L.ty, L.p); break;
+    default: e = launch_gemm<4>(L.dev, L.grid, s, pdl, L.ta, L.tb, L.tsa, L.tsb, L.ty, L.p); break;
   }
   if (e != cudaSuccess) return cuda_status(e, "gemm_kernel launch");
   return NVFP4_OK;
+}
+
+nvfp4_status gemm_impl(const char* fn, const void* a_codes, const void* a_scales, const float* a_global,
+                       const void* b_codes, const void* b_scales, const float* b_global,
+                       const int64_t* seg_ends, int nseg, int64_t M, int64_t N, int64_t K, void* y,
+                       int64_t ldy, int out_dtype, void* workspace, size_t workspace_bytes,
+                       void* stream, int epi = 0, const float* q_alpha = nullptr,
+                       void* q_codes = nullptr, void* q_scales = nullptr) {
+  GemmLaunch L;
+  nvfp4_status st = gemm_prepare(&L, fn, a_codes, a_scales, a_global, b_codes, b_scales, b_global, seg_ends,
+                                 nseg, M, N, K, y, ldy, out_dtype, workspace, workspace_bytes, epi, q_alpha,
+                                 q_codes, q_scales);
+  if (st != NVFP4_OK) return st;
+  return gemm_enqueue(L, static_cast<cudaStream_t>(stream), true, false);
 }
 
 }  // namespace
@@ -811,6 +846,33 @@ nvfp4_status nvfp4_gemm_quantized(const void* a_codes, const void* a_scales, con
   return gemm_impl("nvfp4_gemm_quantized", a_codes, a_scales, a_global, b_codes, b_scales, b_global, &end,
                    1, M, N, K, y_codes, N, NVFP4_OUT_BF16, workspace, workspace_bytes, stream, epi, y_alpha,
                    y_codes, y_scales);
+}
+
+nvfp4_status nvfp4_quantize_gemm(const void* x, int64_t M, int64_t K, int64_t ldx, int mode, int rule,
+                                 float fp8_max, void* x_codes, void* x_scales, float* x_global_scale,
+                                 void* x_workspace, size_t x_workspace_bytes, const void* w_codes,
+                                 const void* w_scales, const float* w_global, int64_t N, void* y, int64_t ldy,
+                                 int out_dtype, void* workspace, size_t workspace_bytes, void* stream) {
+  const char* fn = "nvfp4_quantize_gemm";
+  // every check of both halves before anything is enqueued
+  nvfp4_status st = quantize_rows_check(fn, x, M, K, ldx, mode, rule, fp8_max, x_codes, x_scales,
+                                        x_global_scale, x_workspace, x_workspace_bytes);
+  if (st != NVFP4_OK) return st;
+  GemmLaunch L;
+  const int64_t end = N;
+  if ((st = gemm_prepare(&L, fn, x_codes, x_scales, x_global_scale, w_codes, w_scales, w_global, &end, 1, M, N, K,
+                         y, ldy, out_dtype, workspace, workspace_bytes, 0, nullptr, nullptr, nullptr)) != NVFP4_OK)
+    return st;
+  // The GEMM's status word is cleared first, so that on the stream the GEMM
+  // follows the quantize kernel directly and starts as its programmatic
+  // dependent: its prologue overlaps the quantizer's tail.
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemsetAsync(workspace, 0, sizeof(WorkspaceHeader), s);
+  if (e != cudaSuccess) return cuda_status(e, "cudaMemsetAsync(status)");
+  if ((st = quantize_rows_enqueue(fn, x, M, K, ldx, mode, rule, fp8_max, x_codes, x_scales, x_global_scale,
+                                  x_workspace, x_workspace_bytes, stream)) != NVFP4_OK)
+    return st;
+  return gemm_enqueue(L, s, false, true);
 }
 
 nvfp4_status nvfp4_gemm_segmented(const void* a_codes, const void* a_scales, const float* a_global,

@@ -55,12 +55,6 @@ __device__ __forceinline__ uint4 ld_stream(const uint4* p) {
   return v;
 }
 
-__device__ __forceinline__ void ld_block2(const uint16_t* p, uint4& lo, uint4& hi) {
-  const uint4* q = reinterpret_cast<const uint4*>(p);
-  lo = ld_stream(q);
-  hi = ld_stream(q + 1);
-}
-
 // ------------------------------------------------------------- amax pass --
 // Magnitudes compare like their bit patterns once the sign is cleared, and
 // every NaN pattern (> 0x7F80) compares above Inf (0x7F80) above any finite
@@ -69,6 +63,7 @@ __device__ __forceinline__ void ld_block2(const uint16_t* p, uint4& lo, uint4& h
 __global__ void __launch_bounds__(kAmaxThreads, 2)
     amax_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t K, int64_t ldx,
                 uint32_t* __restrict__ partials) {
+  pdl_launch_dependents();  // the quantize kernel may be scheduled now; it waits for this grid's end
   uint32_t m = 0;
   if (ldx == K) {
     const uint4* v = reinterpret_cast<const uint4*>(x);
@@ -115,7 +110,8 @@ struct QuantParams {
   WorkspaceHeader* ws;
   int nparts;
   float f6;            // fp8_max * 6
-  uint32_t ntasks;     // row-wise kernel: warp tasks of 32 blocks over the rows padded to 128
+  uint32_t ntasks;     // row-wise kernel: 512-element chunks over the rows padded to 128
+  uint32_t chunks;     // row-wise kernel: chunks per row, ceil(K / 512)
   uint32_t kgroups;    // K / 64
   // augmented (ARCQuant) quantization only
   const int32_t* perm = nullptr;  // channel order, K entries
@@ -131,6 +127,11 @@ struct QuantParams {
 // the grid.
 __device__ __forceinline__ bool quant_prologue(const QuantParams& p, BlockConsts& k, float2* s_dr) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  // launched as a programmatic dependent of the amax pass (dynamic alpha):
+  // let the next kernel be scheduled, then wait for the amax pass to finish
+  // before reading its partials, and before any other access to memory
+  pdl_launch_dependents();
+  pdl_wait();
   float alpha;
   if (p.alpha_in) {
     alpha = __ldg(p.alpha_in);
@@ -166,6 +167,25 @@ __device__ __forceinline__ bool quant_prologue(const QuantParams& p, BlockConsts
   return true;
 }
 
+// Warp tasks of the row-wise kernel: chunks of 32 consecutive 16-element
+// blocks (512 elements) of one row, lane i taking block i; the last chunk of a
+// row is partial when K % 512 != 0.  Tasks are numbered row-major over the
+// rows padded to a multiple of 128 and each warp takes one contiguous run of
+// them, so inside a row its lanes' pointers into x, the codes and the
+// swizzled scales all advance by constants (512 elements, 256 bytes, 4096
+// bytes: the next K group of atoms) and only a row change recomputes them.
+// Rows past `rows` only write their (zero) scale bytes.  Each warp loads its
+// next task's block while it quantizes the current one.
+__device__ __forceinline__ void ld_block2(const uint16_t* p, uint4& lo, uint4& hi) {
+  const uint4* q = reinterpret_cast<const uint4*>(p);
+  lo = ld_stream(q);
+  hi = ld_stream(q + 1);
+}
+
+__device__ __forceinline__ int64_t scale_row_offset(int64_t row, uint32_t kgroups) {
+  return ((row >> 7) * kgroups) * 512 + (row & 31) * 16 + ((row >> 5) & 3) * 4;
+}
+
 template <bool FOUR_OVER_SIX, int RULE>
 // Four CTAs per SM: measured faster than five or six in both modes.
 __global__ void __launch_bounds__(kQuantThreads, 4)
@@ -175,44 +195,52 @@ __global__ void __launch_bounds__(kQuantThreads, 4)
   __shared__ float2 s_dr[128];
   if (!quant_prologue(p, k, s_dr)) return;
 
-  // ---- lane -> (row, 16-element block) ----
-  // Blocks are numbered row-major over the padded rows (a multiple of 128):
-  // g = row * (K/16) + kb.  Warp task t takes blocks 32t .. 32t+31, one per
-  // lane, so a task reads 1 KB of consecutive memory when x is dense; each
-  // CTA takes one contiguous run of tasks and its warps interleave over it
-  // (warp w: tasks start + w, start + w + 8, ...), so the GPU sweeps x front
-  // to back.  Rows past `rows` only write their (zero) scale bytes.  Each
-  // warp loads its next task's block while it quantizes the current one.
+  // this warp's run of tasks [t, t_end): tasks split evenly over all warps
+  const uint32_t nwarps = gridDim.x * kQuantWarps;
+  const uint32_t gw = blockIdx.x * kQuantWarps + warp;
+  const uint32_t base = p.ntasks / nwarps, extra = p.ntasks % nwarps;
+  uint32_t t = gw * base + min(gw, extra);
+  const uint32_t t_end = t + base + (gw < extra ? 1u : 0u);
+  if (t >= t_end) return;
+  const uint32_t cpr = p.chunks;                       // chunks per row
   const uint32_t kbs = static_cast<uint32_t>(p.K / 16);
-  const uint32_t per_cta = (p.ntasks + gridDim.x - 1) / gridDim.x;
-  const uint32_t cta_begin = blockIdx.x * per_cta;  // < 2^31 + 2^14: no wrap-around
-  const uint32_t task_end = min(cta_begin + per_cta, p.ntasks);
-  uint32_t task = cta_begin + warp;
-  if (task >= task_end) return;
+  // lanes past the last block of a row (only in a partial last chunk)
+  const bool lane_in_last = static_cast<uint32_t>(lane) < kbs - (cpr - 1) * 32;
+  int64_t row = t / cpr;
+  uint32_t chunk = t - static_cast<uint32_t>(row) * cpr;
   const int64_t half_k = p.K / 2;
-  const uint64_t g0 = static_cast<uint64_t>(task) * 32 + lane;
-  int64_t row = static_cast<int64_t>(g0 / kbs);
-  uint32_t kb = static_cast<uint32_t>(g0 % kbs);
-  const uint32_t step_rows = (32 * kQuantWarps) / kbs, step_kb = (32 * kQuantWarps) % kbs;
-  const int64_t rows_padded = (p.rows + 127) / 128 * 128;
+  const uint32_t lane_scale = static_cast<uint32_t>(lane >> 2) * 512 + (lane & 3);
+  // lane pointers of the current task
+  const uint16_t* xp = p.x + row * p.ldx + chunk * 512 + lane * 16;
+  uint8_t* cp = p.codes + row * half_k + chunk * 256 + lane * 8;
+  uint8_t* sp = p.scales + scale_row_offset(row, p.kgroups) + chunk * 4096 + lane_scale;
 
   uint4 lo = make_uint4(0, 0, 0, 0), hi = lo;
-  if (row < p.rows) ld_block2(p.x + row * p.ldx + kb * 16, lo, hi);
-  for (; task < task_end; task += kQuantWarps) {
-    const int64_t cur_row = row;
-    const uint32_t cur_kb = kb;
-    row += step_rows;
-    kb += step_kb;
-    if (kb >= kbs) {
-      kb -= kbs;
+  if (row < p.rows && (chunk + 1 < cpr || lane_in_last)) ld_block2(xp, lo, hi);
+  for (;;) {
+    const bool live = chunk + 1 < cpr || lane_in_last;
+    const bool real_row = row < p.rows;
+    uint8_t* const cur_cp = cp;
+    uint8_t* const cur_sp = sp;
+    // advance to the next task and start its load
+    if (++chunk < cpr) {
+      xp += 512;
+      cp += 256;
+      sp += 4096;
+    } else {
+      chunk = 0;
       ++row;
+      xp = p.x + row * p.ldx + lane * 16;
+      cp = p.codes + row * half_k + lane * 8;
+      sp = p.scales + scale_row_offset(row, p.kgroups) + lane_scale;
     }
+    const bool more = ++t < t_end;
     uint4 nlo = make_uint4(0, 0, 0, 0), nhi = nlo;
-    if (task + kQuantWarps < task_end && row < p.rows) ld_block2(p.x + row * p.ldx + kb * 16, nlo, nhi);
+    if (more && row < p.rows && (chunk + 1 < cpr || lane_in_last)) ld_block2(xp, nlo, nhi);
 
-    if (cur_row < rows_padded) {
+    if (live) {
       uint32_t scale = 0;
-      if (cur_row < p.rows) {
+      if (real_row) {
         uint2 codes;
         const uint32_t bmax = quantize_block<FOUR_OVER_SIX, RULE>(lo, hi, k, s_dr, codes, scale);
         if (p.alpha_in && bmax >= 0x7F80u) {
@@ -222,12 +250,11 @@ __global__ void __launch_bounds__(kQuantThreads, 4)
           scale = 0u;
           p.ws->status = NVFP4_ERR_NONFINITE;
         }
-        *reinterpret_cast<uint2*>(p.codes + cur_row * half_k + cur_kb * 8) = codes;
+        *reinterpret_cast<uint2*>(cur_cp) = codes;
       }
-      const int64_t atom = (cur_row >> 7) * p.kgroups + (cur_kb >> 2);
-      p.scales[atom * 512 + (cur_row & 31) * 16 + ((cur_row >> 5) & 3) * 4 + (cur_kb & 3)] =
-          static_cast<uint8_t>(scale);
+      *cur_sp = static_cast<uint8_t>(scale);
     }
+    if (!more) break;
     lo = nlo;
     hi = nhi;
   }
@@ -402,7 +429,7 @@ __global__ void __launch_bounds__(kQuantThreads)
 }
 
 template <bool F, int R>
-cudaError_t launch_quantize_arc(int dev, int sms, const QuantParams& p, cudaStream_t s) {
+cudaError_t launch_quantize_arc(int dev, int sms, const QuantParams& p, cudaStream_t s, bool pdl) {
   const size_t smem = static_cast<size_t>(p.K) * 2 * (1 + kArcRows);
   // the shared-memory opt-in is an attribute of the kernel in this context
   static PerContextCache<int> attr;
@@ -419,20 +446,19 @@ cudaError_t launch_quantize_arc(int dev, int sms, const QuantParams& p, cudaStre
   const int64_t steps = (p.rows + 127) / 128 * 128 / kArcRows;
   const int grid = static_cast<int>(std::max<int64_t>(
       1, std::min<int64_t>(steps, static_cast<int64_t>(sms) * std::max(1, occ))));
-  quantize_arc_kernel<F, R><<<grid, kQuantThreads, smem, s>>>(p);
-  return cudaGetLastError();
+  return launch_kernel(quantize_arc_kernel<F, R>, dim3(grid), dim3(kQuantThreads), smem, s, pdl, p);
 }
 
 cudaError_t launch_quantize_arc_kernel(int mode, int rule, int dev, int sms, const QuantParams& p,
-                                       cudaStream_t s) {
-  if (mode == NVFP4_MODE_SIX) return launch_quantize_arc<false, kRuleMax>(dev, sms, p, s);
-  if (rule == NVFP4_RULE_MAX) return launch_quantize_arc<true, kRuleMax>(dev, sms, p, s);
-  if (rule == NVFP4_RULE_MAE) return launch_quantize_arc<true, kRuleMae>(dev, sms, p, s);
-  return launch_quantize_arc<true, kRuleMse>(dev, sms, p, s);
+                                       cudaStream_t s, bool pdl) {
+  if (mode == NVFP4_MODE_SIX) return launch_quantize_arc<false, kRuleMax>(dev, sms, p, s, pdl);
+  if (rule == NVFP4_RULE_MAX) return launch_quantize_arc<true, kRuleMax>(dev, sms, p, s, pdl);
+  if (rule == NVFP4_RULE_MAE) return launch_quantize_arc<true, kRuleMae>(dev, sms, p, s, pdl);
+  return launch_quantize_arc<true, kRuleMse>(dev, sms, p, s, pdl);
 }
 
 template <bool F, int R>
-cudaError_t launch_quantize_t(int dev, int sms, const QuantParams& p, cudaStream_t s) {
+cudaError_t launch_quantize_t(int dev, int sms, const QuantParams& p, cudaStream_t s, bool pdl) {
   static PerContextCache<int> per_sm;
   int occ = 0;
   cudaError_t e = per_context(per_sm, dev, [](int* v) {
@@ -443,20 +469,19 @@ cudaError_t launch_quantize_t(int dev, int sms, const QuantParams& p, cudaStream
   if (e != cudaSuccess) return e;
   const int64_t tiles = ((p.rows + 127) / 128) * (((p.K + 127) / 128 * 128) / 64);
   const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(tiles, static_cast<int64_t>(sms) * occ)));
-  quantize_t_kernel<F, R><<<grid, kQuantThreads, 0, s>>>(p);
-  return cudaGetLastError();
+  return launch_kernel(quantize_t_kernel<F, R>, dim3(grid), dim3(kQuantThreads), 0, s, pdl, p);
 }
 
 cudaError_t launch_quantize_t_kernel(int mode, int rule, int dev, int sms, const QuantParams& p,
-                                     cudaStream_t s) {
-  if (mode == NVFP4_MODE_SIX) return launch_quantize_t<false, kRuleMax>(dev, sms, p, s);
-  if (rule == NVFP4_RULE_MAX) return launch_quantize_t<true, kRuleMax>(dev, sms, p, s);
-  if (rule == NVFP4_RULE_MAE) return launch_quantize_t<true, kRuleMae>(dev, sms, p, s);
-  return launch_quantize_t<true, kRuleMse>(dev, sms, p, s);
+                                     cudaStream_t s, bool pdl) {
+  if (mode == NVFP4_MODE_SIX) return launch_quantize_t<false, kRuleMax>(dev, sms, p, s, pdl);
+  if (rule == NVFP4_RULE_MAX) return launch_quantize_t<true, kRuleMax>(dev, sms, p, s, pdl);
+  if (rule == NVFP4_RULE_MAE) return launch_quantize_t<true, kRuleMae>(dev, sms, p, s, pdl);
+  return launch_quantize_t<true, kRuleMse>(dev, sms, p, s, pdl);
 }
 
 template <bool F, int R>
-cudaError_t launch_quantize(int dev, int sms, const QuantParams& p, cudaStream_t s) {
+cudaError_t launch_quantize(int dev, int sms, const QuantParams& p, cudaStream_t s, bool pdl) {
   static PerContextCache<int> per_sm;
   int occ = 0;
   cudaError_t e = per_context(per_sm, dev, [](int* v) {
@@ -467,15 +492,15 @@ cudaError_t launch_quantize(int dev, int sms, const QuantParams& p, cudaStream_t
   if (e != cudaSuccess) return e;
   const int64_t want = (static_cast<int64_t>(p.ntasks) + kQuantWarps - 1) / kQuantWarps;
   const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(want, static_cast<int64_t>(sms) * occ)));
-  quantize_kernel<F, R><<<grid, kQuantThreads, 0, s>>>(p);
-  return cudaGetLastError();
+  return launch_kernel(quantize_kernel<F, R>, dim3(grid), dim3(kQuantThreads), 0, s, pdl, p);
 }
 
-cudaError_t launch_quantize_kernel(int mode, int rule, int dev, int sms, const QuantParams& p, cudaStream_t s) {
-  if (mode == NVFP4_MODE_SIX) return launch_quantize<false, kRuleMax>(dev, sms, p, s);
-  if (rule == NVFP4_RULE_MAX) return launch_quantize<true, kRuleMax>(dev, sms, p, s);
-  if (rule == NVFP4_RULE_MAE) return launch_quantize<true, kRuleMae>(dev, sms, p, s);
-  return launch_quantize<true, kRuleMse>(dev, sms, p, s);
+cudaError_t launch_quantize_kernel(int mode, int rule, int dev, int sms, const QuantParams& p, cudaStream_t s,
+                                   bool pdl) {
+  if (mode == NVFP4_MODE_SIX) return launch_quantize<false, kRuleMax>(dev, sms, p, s, pdl);
+  if (rule == NVFP4_RULE_MAX) return launch_quantize<true, kRuleMax>(dev, sms, p, s, pdl);
+  if (rule == NVFP4_RULE_MAE) return launch_quantize<true, kRuleMae>(dev, sms, p, s, pdl);
+  return launch_quantize<true, kRuleMse>(dev, sms, p, s, pdl);
 }
 
 }  // namespace
@@ -496,9 +521,9 @@ size_t nvfp4_quantize_workspace_bytes(int64_t rows, int64_t K) {
 namespace {
 
 // ------------------------------------------------------------ host side --
-// Warp tasks of the row-wise kernel: 32 blocks of 16 elements each, over the
-// rows padded to a multiple of 128.
-int64_t row_tasks(int64_t rows, int64_t K) { return ((rows + 127) / 128 * 128 * (K / 16) + 31) / 32; }
+// Warp tasks of the row-wise kernel: chunks of 32 blocks of 16 elements (the
+// last chunk of a row may be partial) over the rows padded to a multiple of 128.
+int64_t row_tasks(int64_t rows, int64_t K) { return (rows + 127) / 128 * 128 * ((K + 511) / 512); }
 
 // Checks shared by every quantize entry point: pointers, shape, row pitch,
 // mode, rule, alignment and the size limits of the kernels' index arithmetic.
@@ -569,6 +594,7 @@ QuantParams base_params(const void* x, int64_t rows, int64_t K, int64_t ldx, voi
   p.nparts = 0;
   p.f6 = 0.0f;
   p.ntasks = static_cast<uint32_t>(row_tasks(rows, K));
+  p.chunks = static_cast<uint32_t>((K + 511) / 512);
   p.kgroups = static_cast<uint32_t>(K / 64);
   return p;
 }
@@ -587,9 +613,11 @@ nvfp4_status launch_dynamic(QuantKind kind, QuantParams p, int mode, int rule, f
   p.partials = partials;
   p.nparts = amax_grid;
   p.f6 = fp8_max * 6.0f;
-  e = kind == QuantKind::kTransposed ? launch_quantize_t_kernel(mode, rule, dev, sms, p, s)
-      : kind == QuantKind::kAugmented ? launch_quantize_arc_kernel(mode, rule, dev, sms, p, s)
-                                       : launch_quantize_kernel(mode, rule, dev, sms, p, s);
+  // the quantize kernel is a programmatic dependent of the amax pass: it is
+  // scheduled while the amax pass drains and waits for it in its prologue
+  e = kind == QuantKind::kTransposed ? launch_quantize_t_kernel(mode, rule, dev, sms, p, s, true)
+      : kind == QuantKind::kAugmented ? launch_quantize_arc_kernel(mode, rule, dev, sms, p, s, true)
+                                       : launch_quantize_kernel(mode, rule, dev, sms, p, s, true);
   if (e != cudaSuccess) return cuda_status(e, "quantize kernel launch");
   return NVFP4_OK;
 }
@@ -597,10 +625,12 @@ nvfp4_status launch_dynamic(QuantKind kind, QuantParams p, int mode, int rule, f
 // nvfp4_quantize (row-wise blocks of x), nvfp4_quantize_t (blocks along the
 // rows of x, i.e. the operand of x^T) and nvfp4_quantize_arc (row-wise with
 // reordered and augmented channels), with the caller's workspace.
-nvfp4_status quantize_impl(const char* fn, QuantKind kind, const void* x, int64_t rows, int64_t K,
-                           int64_t ldx, int mode, int rule, float fp8_max, void* codes, void* scales,
-                           float* global_scale, void* workspace, size_t workspace_bytes, void* stream,
-                           const int32_t* perm = nullptr, int64_t S = 0, int augment = 0) {
+// Every host-side argument check of a dynamic-alpha quantize call (not the
+// device check); enqueues nothing.
+nvfp4_status check_quantize_call(const char* fn, QuantKind kind, const void* x, int64_t rows, int64_t K,
+                                 int64_t ldx, int mode, int rule, float fp8_max, const void* codes,
+                                 const void* scales, const float* global_scale, const void* workspace,
+                                 size_t workspace_bytes, const int32_t* perm, int64_t S, int augment) {
   nvfp4_status st = check_quant_args(fn, kind == QuantKind::kTransposed, x, rows, K, ldx, mode, rule, codes,
                                      scales, global_scale);
   if (st != NVFP4_OK) return st;
@@ -617,6 +647,16 @@ nvfp4_status quantize_impl(const char* fn, QuantKind kind, const void* x, int64_
     return set_error(NVFP4_ERR_INVALID_ARG, "%s: workspace must be a non-null 16-byte aligned pointer", fn);
   if (workspace_bytes < nvfp4_quantize_workspace_bytes(rows, K))
     return set_error(NVFP4_ERR_INVALID_ARG, "%s: workspace too small", fn);
+  return NVFP4_OK;
+}
+
+nvfp4_status quantize_impl(const char* fn, QuantKind kind, const void* x, int64_t rows, int64_t K,
+                           int64_t ldx, int mode, int rule, float fp8_max, void* codes, void* scales,
+                           float* global_scale, void* workspace, size_t workspace_bytes, void* stream,
+                           const int32_t* perm = nullptr, int64_t S = 0, int augment = 0) {
+  nvfp4_status st = check_quantize_call(fn, kind, x, rows, K, ldx, mode, rule, fp8_max, codes, scales,
+                                        global_scale, workspace, workspace_bytes, perm, S, augment);
+  if (st != NVFP4_OK) return st;
   int dev = 0, sms = 0;
   if ((st = check_device(&dev, &sms)) != NVFP4_OK) return st;
 
@@ -632,6 +672,24 @@ nvfp4_status quantize_impl(const char* fn, QuantKind kind, const void* x, int64_
 }
 
 }  // namespace
+
+namespace nvfp4 {
+
+nvfp4_status quantize_rows_check(const char* fn, const void* x, int64_t rows, int64_t K, int64_t ldx, int mode,
+                                 int rule, float fp8_max, const void* codes, const void* scales,
+                                 const float* global_scale, const void* workspace, size_t workspace_bytes) {
+  return check_quantize_call(fn, QuantKind::kRows, x, rows, K, ldx, mode, rule, fp8_max, codes, scales,
+                             global_scale, workspace, workspace_bytes, nullptr, 0, 0);
+}
+
+nvfp4_status quantize_rows_enqueue(const char* fn, const void* x, int64_t rows, int64_t K, int64_t ldx, int mode,
+                                   int rule, float fp8_max, void* codes, void* scales, float* global_scale,
+                                   void* workspace, size_t workspace_bytes, void* stream) {
+  return quantize_impl(fn, QuantKind::kRows, x, rows, K, ldx, mode, rule, fp8_max, codes, scales, global_scale,
+                       workspace, workspace_bytes, stream);
+}
+
+}  // namespace nvfp4
 
 extern "C" {
 
@@ -751,7 +809,7 @@ extern "C" nvfp4_status nvfp4_quantize_with_scale(const void* x, int64_t rows, i
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t e = cudaMemsetAsync(workspace, 0, 2 * sizeof(uint32_t), s);  // status, detail
   if (e != cudaSuccess) return cuda_status(e, "nvfp4_quantize_with_scale: status reset");
-  e = launch_quantize_kernel(mode, rule, dev, sms, p, s);
+  e = launch_quantize_kernel(mode, rule, dev, sms, p, s, false);
   if (e != cudaSuccess) return cuda_status(e, "quantize_kernel launch");
   return NVFP4_OK;
 }
