@@ -20,6 +20,8 @@ oracle (the plain, slow definition) on a bounded sample of the same workload.
 from __future__ import annotations
 
 import argparse
+import dataclasses
+import hashlib
 import json
 import os
 import statistics
@@ -41,8 +43,34 @@ AMAX_BYTES_PER_ELEM = 2.0
 # the events: the host's launch overhead then overlaps GPU work instead of
 # showing up as idle time between the start event and the first kernel.
 HOST_LEAD_CYCLES = 400_000
+# dram__bytes_read.sum + dram__bytes_write.sum of one gemm_kernel launch on the
+# full-size prefill workload (one-pass ncu capture), recorded with the SHA-1 of
+# the kernel's sources at capture time; the bench reports it only while those
+# sources are unchanged
 GEMM_PREFILL_TRAFFIC = {"bytes": 1.465e9, "read": 0.365e9, "write": 1.10e9,
-                        "algorithmic": 1.285e9, "source": "ncu one-pass dram__bytes capture of gemm_kernel"}
+                        "algorithmic": 1.285e9, "captured": "unknown", "kernel_sources_sha1": "unknown",
+                        "source": "ncu one-pass dram__bytes capture of gemm_kernel"}
+GEMM_KERNEL_SOURCES = ("w4a4_gemm_nvfp4_b200/csrc/gemm.cu", "w4a4_gemm_nvfp4_b200/csrc/common.cuh",
+                       "w4a4_gemm_nvfp4_b200/csrc/block_step.cuh")
+
+
+def gemm_sources_sha1() -> str:
+    h = hashlib.sha1()
+    for rel in GEMM_KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def recorded_traffic(args):
+    """The recorded per-launch DRAM traffic of the GEMM, or None when the
+    workload is not the full-size prefill one or the kernel's sources changed
+    since the capture."""
+    if args.workload != "prefill" or args.x_rows:
+        return None
+    if GEMM_PREFILL_TRAFFIC["kernel_sources_sha1"] != gemm_sources_sha1():
+        return None
+    return GEMM_PREFILL_TRAFFIC
 
 
 def _peaks():
@@ -143,6 +171,15 @@ def _barrier(world):
         torch.distributed.barrier()
 
 
+def workload_of(args):
+    """The named workload; --x-rows replaces the number of X rows (smaller
+    captures of the same kernels)."""
+    wl = workloads.WORKLOADS[args.workload]
+    if args.x_rows:
+        wl = dataclasses.replace(wl, x=dataclasses.replace(wl.x, rows=args.x_rows))
+    return wl
+
+
 def rank_x_operand(wl, rank: int):
     """Rank r's activations: the workload's X recipe with its own seed (weak
     scaling: every rank quantizes and multiplies a different X, same W)."""
@@ -177,7 +214,8 @@ def run_ours(args, world, rank, local):
 
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
-    wl = workloads.WORKLOADS[args.workload]
+    wl = workload_of(args)
+    traffic = recorded_traffic(args)
     xm, xr, xF = args.x_recipe
     wm, wr, wF = wl.w_recipe
     M, N, K = wl.M, wl.N, wl.K
@@ -276,17 +314,16 @@ def run_ours(args, world, rank, local):
             fn()
             evs[i][1].record(stream)
         torch.cuda.synchronize()
-        return statistics.mean(a.elapsed_time(b) for a, b in evs)
+        return [a.elapsed_time(b) for a, b in evs]
 
     _barrier(world)
     torch.cuda.synchronize()
-    ms_qstatic = time_op(lambda: nv.quantize(x, xm, xr, out=qs, global_scale=qx.global_scale),
+    t_qstatic = time_op(lambda: nv.quantize(x, xm, xr, out=qs, global_scale=qx.global_scale), args.steps)
+    t_qstatic6 = time_op(lambda: nv.quantize(x, "six", "max", out=qs6, global_scale=q6.global_scale),
                          args.steps)
-    ms_qstatic6 = time_op(lambda: nv.quantize(x, "six", "max", out=qs6, global_scale=q6.global_scale),
-                          args.steps)
     assert nv.device_status(qs.workspace) == nv.OK and nv.device_status(qs6.workspace) == nv.OK
-    ms_qstatic = _max_over_ranks(world, ms_qstatic, device)
-    ms_qstatic6 = _max_over_ranks(world, ms_qstatic6, device)
+    ms_qstatic = _max_over_ranks(world, statistics.mean(t_qstatic), device)
+    ms_qstatic6 = _max_over_ranks(world, statistics.mean(t_qstatic6), device)
 
     # the "next" entry points on the same operands: the GEMM writing Y as an
     # NVFP4 operand (4/6-MSE at a static output alpha), and the augmented-
@@ -312,9 +349,9 @@ def run_ours(args, world, rank, local):
     ms_arc_step = time_op(arc_step, args.steps)
     assert (nv.device_status(qy.workspace) == nv.OK and nv.device_status(qa.workspace) == nv.OK
             and nv.device_status(gws) == nv.OK)
-    ms_qout = _max_over_ranks(world, ms_qout, device)
-    ms_arc_q = _max_over_ranks(world, ms_arc_q, device)
-    ms_arc_step = _max_over_ranks(world, ms_arc_step, device)
+    ms_qout = _max_over_ranks(world, statistics.mean(ms_qout), device)
+    ms_arc_q = _max_over_ranks(world, statistics.mean(ms_arc_q), device)
+    ms_arc_step = _max_over_ranks(world, statistics.mean(ms_arc_step), device)
     del qy, qa, qw_arc, y_arc
 
     ms_step = _max_over_ranks(world, statistics.mean(steps_ms), device)
@@ -372,10 +409,11 @@ def run_ours(args, world, rank, local):
             "unit": "TFLOP/s",
             "frac": round(gemm_tflops / fp4_peak, 4),
             "peak_source": f"4 x {peaks['source']} bf16 burst ({peaks['bf16']} TF/s)",
-            # dram__bytes_read.sum + dram__bytes_write.sum of one gemm_kernel launch on this
-            # workload (one-pass ncu capture): 0.365 GB + 1.10 GB; recorded, not measured here
-            "traffic": GEMM_PREFILL_TRAFFIC["bytes"] if args.workload == "prefill" else None,
-            "traffic_detail": GEMM_PREFILL_TRAFFIC if args.workload == "prefill" else None,
+            # recorded from an ncu capture of this kernel version, not measured here
+            "traffic": traffic["bytes"] if traffic else None,
+            "traffic_detail": traffic if traffic else {
+                "why_null": "no capture of the current kernel sources on this workload",
+                "kernel_sources_sha1": gemm_sources_sha1()},
         },
         "breakdown": {
             "ms_step_two_calls": round(ms_two_calls, 4),
@@ -406,6 +444,8 @@ def run_ours(args, world, rank, local):
             "ms_per_step": spread(steps_ms),
             "ms_quantize_46": spread(tq),
             "ms_gemm": spread(tg),
+            "ms_quantize_kernel_46_static_alpha": spread(t_qstatic),
+            "ms_quantize_kernel_six_static_alpha": spread(t_qstatic6),
         },
         "e2e": {
             "value": round(job_tflops(world, flops, ms_e2e), 2),
@@ -545,7 +585,7 @@ def cpu_baseline(args, sample_rows=64):
     (quantize `sample_rows` rows of X, then their fp64 GEMM against the
     dequantized W) as the headline figure, plus the quantizer on the whole X
     and the GEMM on a 256-row slice as separate records."""
-    wl = workloads.WORKLOADS[args.workload]
+    wl = workload_of(args)
     w_deq = _w_dequant(wl)
     t0 = time.perf_counter()
     flops = _oracle_sample(wl, args.x_recipe, sample_rows, w_deq)
@@ -561,7 +601,7 @@ def cpu_baseline(args, sample_rows=64):
 
 
 def run_reference(args, world, rank):
-    wl = workloads.WORKLOADS[args.workload]
+    wl = workload_of(args)
     w_deq = _w_dequant(wl)
     rows = args.cpu_rows
     for _ in range(args.warmup):
@@ -712,6 +752,8 @@ def main():
                     help="mode,rule,fp8_max for X (default four_over_six,mse,256)")
     ap.add_argument("--cpu-rows", type=int, default=256, help="X rows per oracle step (reference arm)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--x-rows", type=int, default=0,
+                    help="replace the workload's X rows (profiling captures of a smaller case)")
     ap.add_argument("--sweep", action="store_true",
                     help="instead of the headline step: the quantizer sweep and every GEMM workload, "
                          "one JSON line each (1 GPU)")

@@ -33,6 +33,14 @@ __device__ __forceinline__ uint32_t absmax4(const uint4& v, uint32_t m) {
   return max_u16x2(m, v.w & kAbsMask2);
 }
 
+// Three-input maximum that propagates NaN (one instruction on sm_100; the
+// compiler folds fabsf of an operand into it).
+__device__ __forceinline__ float max3_nan(float a, float b, float c) {
+  float d;
+  asm("max.NaN.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
 // ------------------------------------------------------- conversions ----
 
 // Two binary32 -> two E4M3 (RNE, saturating to 448): lo byte from `lo`.
@@ -62,33 +70,6 @@ __device__ __forceinline__ uint32_t e2m1x2_encode(float hi, float lo) {
       : "f"(hi), "f"(lo));
   return byte;
 }
-// Eight binary32 (elements 0..7) -> one word of eight E2M1 codes (element i
-// in nibble i; RNE, saturating to 6, sign kept), and the eight code values
-// back as binary32 (exact, via f16).
-__device__ __forceinline__ uint32_t e2m1x8_round(const float x[8], float q[8]) {
-  uint32_t w;
-  asm("{\n\t.reg .b8 c0, c1, c2, c3;\n\t.reg .b32 h<4>;\n\t.reg .f16 f<8>;\n\t"
-      "cvt.rn.satfinite.e2m1x2.f32 c0, %10, %9;\n\t"
-      "cvt.rn.satfinite.e2m1x2.f32 c1, %12, %11;\n\t"
-      "cvt.rn.satfinite.e2m1x2.f32 c2, %14, %13;\n\t"
-      "cvt.rn.satfinite.e2m1x2.f32 c3, %16, %15;\n\t"
-      "mov.b32 %0, {c0, c1, c2, c3};\n\t"
-      "cvt.rn.f16x2.e2m1x2 h0, c0;\n\t"
-      "cvt.rn.f16x2.e2m1x2 h1, c1;\n\t"
-      "cvt.rn.f16x2.e2m1x2 h2, c2;\n\t"
-      "cvt.rn.f16x2.e2m1x2 h3, c3;\n\t"
-      "mov.b32 {f0, f1}, h0;\n\tmov.b32 {f2, f3}, h1;\n\t"
-      "mov.b32 {f4, f5}, h2;\n\tmov.b32 {f6, f7}, h3;\n\t"
-      "cvt.f32.f16 %1, f0;\n\tcvt.f32.f16 %2, f1;\n\t"
-      "cvt.f32.f16 %3, f2;\n\tcvt.f32.f16 %4, f3;\n\t"
-      "cvt.f32.f16 %5, f4;\n\tcvt.f32.f16 %6, f5;\n\t"
-      "cvt.f32.f16 %7, f6;\n\tcvt.f32.f16 %8, f7;\n\t}"
-      : "=r"(w), "=f"(q[0]), "=f"(q[1]), "=f"(q[2]), "=f"(q[3]), "=f"(q[4]), "=f"(q[5]),
-        "=f"(q[6]), "=f"(q[7])
-      : "f"(x[0]), "f"(x[1]), "f"(x[2]), "f"(x[3]), "f"(x[4]), "f"(x[5]), "f"(x[6]), "f"(x[7]));
-  return w;
-}
-
 // Packed binary32 pairs held in one 64-bit register pair (one IEEE RNE
 // operation per lane, like the scalar instruction on each lane).
 struct f2 {
@@ -124,11 +105,28 @@ __device__ __forceinline__ float safe_recip(float d) {
 
 enum { kRuleMax = 0, kRuleMae = 1, kRuleMse = 2 };
 
+// The block step's per-scale-code constants, one 16-byte shared-memory entry
+// per E4M3 code c: (r, r) and (-d, -d) with d = val(c) * alpha and r = 1/d
+// (0 if infinite), already paired for the packed f32x2 arithmetic.
+struct __align__(16) ScaleEntry {
+  f2 rr;  // (r, r)
+  f2 nd;  // (-d, -d)
+};
+__device__ __forceinline__ void load_entry(const ScaleEntry* tab, uint32_t code, f2& rr, f2& nd) {
+  asm("ld.shared.v2.b64 {%0, %1}, [%2];"
+      : "=l"(rr.v), "=l"(nd.v)
+      : "r"(static_cast<uint32_t>(__cvta_generic_to_shared(tab + code))));
+}
+__device__ __forceinline__ f2 load_rr(const ScaleEntry* tab, uint32_t code) {
+  f2 rr;
+  asm("ld.shared.b64 %0, [%1];" : "=l"(rr.v) : "r"(static_cast<uint32_t>(__cvta_generic_to_shared(tab + code))));
+  return rr;
+}
+
 // Codes of one candidate: v = x * r per element, E2M1-rounded.  The block's
 // 16 values are held as pairs p[j] = (x_j, x_{j+8}), j < 8; codes byte j holds
 // elements 2j, 2j+1 (low nibble first).
-__device__ __forceinline__ uint2 candidate_codes(const f2 p[8], float r) {
-  const f2 rr = make_f2(r, r);
+__device__ __forceinline__ uint2 candidate_codes(const f2 p[8], f2 rr) {
   uint32_t bytes[8];
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
@@ -146,34 +144,62 @@ __device__ __forceinline__ uint2 candidate_codes(const f2 p[8], float r) {
 //   (t_2i + t_2i+1, t_2i+8 + t_2i+9)      = (u_i, u_i+4)   i < 4
 //   (u_2i + u_2i+1, u_2i+4 + u_2i+5)      = (w_i, w_i+2)   i < 2
 //   (w_0 + w_1, w_2 + w_3)                = (z_0, z_1),    then z_0 + z_1.
+// E2M1 encode of v (pairs v[j] = (v_j, v_{j+8})) into the two code words
+// (element i in nibble i of codes.x for i < 8, of codes.y for i >= 8; RNE,
+// saturating to 6, sign kept) and the code values back as binary32 (exact,
+// via f16), written directly as the pairs q[j] = (val(code j), val(code
+// j+8)) that the packed error arithmetic takes.
+__device__ __forceinline__ void encode_decode(const f2 v[8], uint2& codes, f2 q[8]) {
+  asm("{\n\t.reg .f32 a<8>, b<8>, qa<8>, qb<8>;\n\t.reg .b8 cx<4>, cy<4>;\n\t"
+      ".reg .b32 hx<4>, hy<4>;\n\t.reg .f16 fa<8>, fb<8>;\n\t"
+      "mov.b64 {a0, b0}, %10;\n\tmov.b64 {a1, b1}, %11;\n\tmov.b64 {a2, b2}, %12;\n\tmov.b64 {a3, b3}, %13;\n\t"
+      "mov.b64 {a4, b4}, %14;\n\tmov.b64 {a5, b5}, %15;\n\tmov.b64 {a6, b6}, %16;\n\tmov.b64 {a7, b7}, %17;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 cx0, a1, a0;\n\tcvt.rn.satfinite.e2m1x2.f32 cx1, a3, a2;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 cx2, a5, a4;\n\tcvt.rn.satfinite.e2m1x2.f32 cx3, a7, a6;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 cy0, b1, b0;\n\tcvt.rn.satfinite.e2m1x2.f32 cy1, b3, b2;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 cy2, b5, b4;\n\tcvt.rn.satfinite.e2m1x2.f32 cy3, b7, b6;\n\t"
+      "mov.b32 %0, {cx0, cx1, cx2, cx3};\n\tmov.b32 %1, {cy0, cy1, cy2, cy3};\n\t"
+      "cvt.rn.f16x2.e2m1x2 hx0, cx0;\n\tcvt.rn.f16x2.e2m1x2 hx1, cx1;\n\t"
+      "cvt.rn.f16x2.e2m1x2 hx2, cx2;\n\tcvt.rn.f16x2.e2m1x2 hx3, cx3;\n\t"
+      "cvt.rn.f16x2.e2m1x2 hy0, cy0;\n\tcvt.rn.f16x2.e2m1x2 hy1, cy1;\n\t"
+      "cvt.rn.f16x2.e2m1x2 hy2, cy2;\n\tcvt.rn.f16x2.e2m1x2 hy3, cy3;\n\t"
+      "mov.b32 {fa0, fa1}, hx0;\n\tmov.b32 {fa2, fa3}, hx1;\n\tmov.b32 {fa4, fa5}, hx2;\n\tmov.b32 {fa6, fa7}, hx3;\n\t"
+      "mov.b32 {fb0, fb1}, hy0;\n\tmov.b32 {fb2, fb3}, hy1;\n\tmov.b32 {fb4, fb5}, hy2;\n\tmov.b32 {fb6, fb7}, hy3;\n\t"
+      "cvt.f32.f16 qa0, fa0;\n\tcvt.f32.f16 qb0, fb0;\n\tmov.b64 %2, {qa0, qb0};\n\t"
+      "cvt.f32.f16 qa1, fa1;\n\tcvt.f32.f16 qb1, fb1;\n\tmov.b64 %3, {qa1, qb1};\n\t"
+      "cvt.f32.f16 qa2, fa2;\n\tcvt.f32.f16 qb2, fb2;\n\tmov.b64 %4, {qa2, qb2};\n\t"
+      "cvt.f32.f16 qa3, fa3;\n\tcvt.f32.f16 qb3, fb3;\n\tmov.b64 %5, {qa3, qb3};\n\t"
+      "cvt.f32.f16 qa4, fa4;\n\tcvt.f32.f16 qb4, fb4;\n\tmov.b64 %6, {qa4, qb4};\n\t"
+      "cvt.f32.f16 qa5, fa5;\n\tcvt.f32.f16 qb5, fb5;\n\tmov.b64 %7, {qa5, qb5};\n\t"
+      "cvt.f32.f16 qa6, fa6;\n\tcvt.f32.f16 qb6, fb6;\n\tmov.b64 %8, {qa6, qb6};\n\t"
+      "cvt.f32.f16 qa7, fa7;\n\tcvt.f32.f16 qb7, fb7;\n\tmov.b64 %9, {qa7, qb7};\n\t}"
+      : "=r"(codes.x), "=r"(codes.y), "=l"(q[0].v), "=l"(q[1].v), "=l"(q[2].v), "=l"(q[3].v), "=l"(q[4].v),
+        "=l"(q[5].v), "=l"(q[6].v), "=l"(q[7].v)
+      : "l"(v[0].v), "l"(v[1].v), "l"(v[2].v), "l"(v[3].v), "l"(v[4].v), "l"(v[5].v), "l"(v[6].v), "l"(v[7].v));
+}
+
+// One candidate with its block error under RULE.  With the (x_j, x_{j+8})
+// pairing the contiguous pairwise tree of the error terms
+// ((t0+t1)+(t2+t3))+... is exactly three packed additions and one scalar one:
+//   (t_2i + t_2i+1, t_2i+8 + t_2i+9)      = (u_i, u_i+4)   i < 4
+//   (u_2i + u_2i+1, u_2i+4 + u_2i+5)      = (w_i, w_i+2)   i < 2
+//   (w_0 + w_1, w_2 + w_3)                = (z_0, z_1),    then z_0 + z_1.
 template <int RULE>
-__device__ __forceinline__ float candidate(const f2 p[8], float d, float r, uint2& codes) {
-  const f2 rr = make_f2(r, r);
-  const f2 nd = make_f2(-d, -d);
-  f2 v[8];
+__device__ __forceinline__ float candidate(const f2 p[8], f2 rr, f2 nd, uint2& codes) {
+  f2 v[8], q[8];
 #pragma unroll
   for (int j = 0; j < 8; ++j) v[j] = mul2(p[j], rr);
-  // element k is v[k % 8].a (k < 8) or v[k % 8].b (k >= 8)
-  float xa[8], xb[8], q[16];
-#pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    xa[j] = v[j].a();
-    xb[j] = v[j].b();
-  }
-  codes.x = e2m1x8_round(xa, q);
-  codes.y = e2m1x8_round(xb, q + 8);
+  encode_decode(v, codes, q);
   // e = fma(-q, d, x), paired like p
   f2 e[8];
 #pragma unroll
-  for (int j = 0; j < 8; ++j) e[j] = fma2(make_f2(q[j], q[j + 8]), nd, p[j]);
+  for (int j = 0; j < 8; ++j) e[j] = fma2(q[j], nd, p[j]);
   if (RULE == kRuleMax) {
-    float m0 = 0.0f, m1 = 0.0f;
+    // max |e| (exact in any order; the errors are finite), one pair at a time
+    float m = 0.0f;
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      m0 = fmaxf(m0, fabsf(e[j].a()));
-      m1 = fmaxf(m1, fabsf(e[j].b()));
-    }
-    return fmaxf(m0, m1);
+    for (int j = 0; j < 8; ++j) m = max3_nan(m, fabsf(e[j].a()), fabsf(e[j].b()));
+    return m;
   }
   f2 t[8];
   if (RULE == kRuleMse) {
@@ -181,7 +207,7 @@ __device__ __forceinline__ float candidate(const f2 p[8], float d, float r, uint
     for (int j = 0; j < 8; ++j) t[j] = mul2(e[j], e[j]);
   } else {
 #pragma unroll
-    for (int j = 0; j < 8; ++j) t[j] = make_f2(fabsf(e[j].a()), fabsf(e[j].b()));
+    for (int j = 0; j < 8; ++j) t[j].v = e[j].v & 0x7FFFFFFF7FFFFFFFull;  // |e| of both lanes
   }
   const f2 u0 = add2(t[0], t[1]), u1 = add2(t[2], t[3]), u2 = add2(t[4], t[5]), u3 = add2(t[6], t[7]);
   const f2 w0 = add2(u0, u1), w1 = add2(u2, u3);
@@ -206,14 +232,12 @@ __device__ __forceinline__ bool needs_exact_quotient(float q) {
   return b < 0x3C800008u || ((b & 0xFFFFFu) - 0x7FFFBu) < 11u;
 }
 
-// Quantize one block held as 8 words of bf16 pairs (element 2j in the low
-// half of word j).  dr[c] = (d, r) of E4M3 scale code c: d = val(c) * alpha,
-// r = 1/d (0 if infinite).
 // The block step on 16 binary32 values held as pairs p[j] = (x_j, x_{j+8})
-// with block max b: scale(s) and codes of the chosen candidate.
+// with block max b: scale(s) and codes of the chosen candidate.  tab[c] holds
+// the constants of E4M3 scale code c (ScaleEntry).
 template <bool FOUR_OVER_SIX, int RULE>
 __device__ __forceinline__ void quantize_pairs(const f2 p[8], float b, const BlockConsts& k,
-                                               const float2* dr, uint2& codes, uint32_t& scale) {
+                                               const ScaleEntry* tab, uint2& codes, uint32_t& scale) {
   float s6raw = __fmul_rn(b, k.inv6);
   float s4raw = FOUR_OVER_SIX ? __fmul_rn(b, k.inv4) : 0.0f;
   if (!k.fast_div || needs_exact_quotient(s6raw) || (FOUR_OVER_SIX && needs_exact_quotient(s4raw))) {
@@ -221,28 +245,22 @@ __device__ __forceinline__ void quantize_pairs(const f2 p[8], float b, const Blo
     if (FOUR_OVER_SIX) s4raw = __fdiv_rn(b, k.a4);
   }
   const uint32_t sc = cvt_e4m3x2(s4raw, s6raw);  // low byte: scale-6, high byte: scale-4
-  const float2 dr6 = dr[sc & 0xFFu];
   if (!FOUR_OVER_SIX) {
-    codes = candidate_codes(p, dr6.y);
+    codes = candidate_codes(p, load_rr(tab, sc & 0xFFu));
     scale = sc & 0xFFu;
     return;
   }
-  const float2 dr4 = dr[sc >> 8];
+  f2 rr6, nd6, rr4, nd4;
+  load_entry(tab, sc & 0xFFu, rr6, nd6);
+  load_entry(tab, sc >> 8, rr4, nd4);
   uint2 c6, c4;
-  const float E6 = candidate<RULE>(p, dr6.x, dr6.y, c6);
-  const float E4 = candidate<RULE>(p, dr4.x, dr4.y, c4);
+  const float E6 = candidate<RULE>(p, rr6, nd6, c6);
+  const float E4 = candidate<RULE>(p, rr4, nd4, c4);
   const bool pick4 = E4 < E6;  // ties keep scale 6
   codes = pick4 ? c4 : c6;
   scale = pick4 ? (sc >> 8) : (sc & 0xFFu);
 }
 
-// Three-input maximum that propagates NaN (one instruction on sm_100; the
-// compiler folds fabsf of an operand into it).
-__device__ __forceinline__ float max3_nan(float a, float b, float c) {
-  float d;
-  asm("max.NaN.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
-  return d;
-}
 
 // bf16 block (8 words of bf16 pairs, element 2j in the low half of word j) ->
 // binary32 pairs p[j] = (x_j, x_{j+8}); returns the block's max |x| bit
@@ -254,18 +272,18 @@ __device__ __forceinline__ uint32_t unpack_block(const uint4& lo, const uint4& h
     // bf16 -> binary32 as a mixed-precision add of -0 (exact for every bf16
     // value, signed zeros included), which runs on the FMA pipe instead of
     // taking integer shifts and masks
-    float a0, a1, b0, b1;
-    asm("{\n\t.reg .b16 l0, h0, l1, h1;\n\t"
-        "mov.b32 {l0, h0}, %4;\n\t"
-        "mov.b32 {l1, h1}, %5;\n\t"
-        "add.rn.f32.bf16 %0, l0, 0f80000000;\n\t"
-        "add.rn.f32.bf16 %1, l1, 0f80000000;\n\t"
-        "add.rn.f32.bf16 %2, h0, 0f80000000;\n\t"
-        "add.rn.f32.bf16 %3, h1, 0f80000000;\n\t}"
-        : "=f"(a0), "=f"(a1), "=f"(b0), "=f"(b1)
+    // (the pairs are formed inside the asm, so no register moves are needed)
+    asm("{\n\t.reg .b16 l0, h0, l1, h1;\n\t.reg .f32 a0, a1, b0, b1;\n\t"
+        "mov.b32 {l0, h0}, %2;\n\t"
+        "mov.b32 {l1, h1}, %3;\n\t"
+        "add.rn.f32.bf16 a0, l0, 0f80000000;\n\t"
+        "add.rn.f32.bf16 a1, l1, 0f80000000;\n\t"
+        "add.rn.f32.bf16 b0, h0, 0f80000000;\n\t"
+        "add.rn.f32.bf16 b1, h1, 0f80000000;\n\t"
+        "mov.b64 %0, {a0, a1};\n\t"
+        "mov.b64 %1, {b0, b1};\n\t}"
+        : "=l"(p[2 * i].v), "=l"(p[2 * i + 1].v)
         : "r"(w[i]), "r"(w[i + 4]));
-    p[2 * i] = make_f2(a0, a1);
-    p[2 * i + 1] = make_f2(b0, b1);
   }
   // max |x| of the 16 values (exact: a maximum of bf16 values), NaN kept
   const float m0 = max3_nan(fabsf(p[0].a()), fabsf(p[1].a()), fabsf(p[2].a()));
@@ -280,42 +298,40 @@ __device__ __forceinline__ uint32_t unpack_block(const uint4& lo, const uint4& h
 // Quantize one bf16 block; returns its max |x| bit pattern.
 template <bool FOUR_OVER_SIX, int RULE>
 __device__ __forceinline__ uint32_t quantize_block(const uint4& lo, const uint4& hi, const BlockConsts& k,
-                                                   const float2* dr, uint2& codes, uint32_t& scale) {
+                                                   const ScaleEntry* tab, uint2& codes, uint32_t& scale) {
   f2 p[8];
   const uint32_t bbits = unpack_block(lo, hi, p);
-  quantize_pairs<FOUR_OVER_SIX, RULE>(p, __uint_as_float(bbits << 16), k, dr, codes, scale);
+  quantize_pairs<FOUR_OVER_SIX, RULE>(p, __uint_as_float(bbits << 16), k, tab, codes, scale);
   return bbits;
 }
 
 // E2M1 codes (element i in nibble i of c.x for i < 8, of c.y for i >= 8) back
 // to binary32 pairs q[j] = (val(code j), val(code j+8)), exact via f16.
 __device__ __forceinline__ void decode_pairs(const uint2 c, f2 q[8]) {
-  float v[16];
-#pragma unroll
-  for (int b = 0; b < 4; ++b) {
-    asm("{\n\t.reg .b8 c;\n\t.reg .b32 h2;\n\t.reg .f16 h0, h1;\n\t"
-        "cvt.u8.u32 c, %2;\n\t"
-        "cvt.rn.f16x2.e2m1x2 h2, c;\n\t"
-        "mov.b32 {h0, h1}, h2;\n\t"
-        "cvt.f32.f16 %0, h0;\n\t"
-        "cvt.f32.f16 %1, h1;\n\t}"
-        : "=f"(v[2 * b]), "=f"(v[2 * b + 1])
-        : "r"((c.x >> (8 * b)) & 0xFFu));
-    asm("{\n\t.reg .b8 c;\n\t.reg .b32 h2;\n\t.reg .f16 h0, h1;\n\t"
-        "cvt.u8.u32 c, %2;\n\t"
-        "cvt.rn.f16x2.e2m1x2 h2, c;\n\t"
-        "mov.b32 {h0, h1}, h2;\n\t"
-        "cvt.f32.f16 %0, h0;\n\t"
-        "cvt.f32.f16 %1, h1;\n\t}"
-        : "=f"(v[8 + 2 * b]), "=f"(v[8 + 2 * b + 1])
-        : "r"((c.y >> (8 * b)) & 0xFFu));
-  }
-#pragma unroll
-  for (int j = 0; j < 8; ++j) q[j] = make_f2(v[j], v[j + 8]);
+  asm("{\n\t.reg .f32 qa<8>, qb<8>;\n\t.reg .b8 cx<4>, cy<4>;\n\t"
+      ".reg .b32 hx<4>, hy<4>;\n\t.reg .f16 fa<8>, fb<8>;\n\t"
+      "mov.b32 {cx0, cx1, cx2, cx3}, %8;\n\tmov.b32 {cy0, cy1, cy2, cy3}, %9;\n\t"
+      "cvt.rn.f16x2.e2m1x2 hx0, cx0;\n\tcvt.rn.f16x2.e2m1x2 hx1, cx1;\n\t"
+      "cvt.rn.f16x2.e2m1x2 hx2, cx2;\n\tcvt.rn.f16x2.e2m1x2 hx3, cx3;\n\t"
+      "cvt.rn.f16x2.e2m1x2 hy0, cy0;\n\tcvt.rn.f16x2.e2m1x2 hy1, cy1;\n\t"
+      "cvt.rn.f16x2.e2m1x2 hy2, cy2;\n\tcvt.rn.f16x2.e2m1x2 hy3, cy3;\n\t"
+      "mov.b32 {fa0, fa1}, hx0;\n\tmov.b32 {fa2, fa3}, hx1;\n\tmov.b32 {fa4, fa5}, hx2;\n\tmov.b32 {fa6, fa7}, hx3;\n\t"
+      "mov.b32 {fb0, fb1}, hy0;\n\tmov.b32 {fb2, fb3}, hy1;\n\tmov.b32 {fb4, fb5}, hy2;\n\tmov.b32 {fb6, fb7}, hy3;\n\t"
+      "cvt.f32.f16 qa0, fa0;\n\tcvt.f32.f16 qb0, fb0;\n\tmov.b64 %0, {qa0, qb0};\n\t"
+      "cvt.f32.f16 qa1, fa1;\n\tcvt.f32.f16 qb1, fb1;\n\tmov.b64 %1, {qa1, qb1};\n\t"
+      "cvt.f32.f16 qa2, fa2;\n\tcvt.f32.f16 qb2, fb2;\n\tmov.b64 %2, {qa2, qb2};\n\t"
+      "cvt.f32.f16 qa3, fa3;\n\tcvt.f32.f16 qb3, fb3;\n\tmov.b64 %3, {qa3, qb3};\n\t"
+      "cvt.f32.f16 qa4, fa4;\n\tcvt.f32.f16 qb4, fb4;\n\tmov.b64 %4, {qa4, qb4};\n\t"
+      "cvt.f32.f16 qa5, fa5;\n\tcvt.f32.f16 qb5, fb5;\n\tmov.b64 %5, {qa5, qb5};\n\t"
+      "cvt.f32.f16 qa6, fa6;\n\tcvt.f32.f16 qb6, fb6;\n\tmov.b64 %6, {qa6, qb6};\n\t"
+      "cvt.f32.f16 qa7, fa7;\n\tcvt.f32.f16 qb7, fb7;\n\tmov.b64 %7, {qa7, qb7};\n\t}"
+      : "=l"(q[0].v), "=l"(q[1].v), "=l"(q[2].v), "=l"(q[3].v), "=l"(q[4].v), "=l"(q[5].v), "=l"(q[6].v),
+        "=l"(q[7].v)
+      : "r"(c.x), "r"(c.y));
 }
 
-// Per-call constants and the (d, r) table of every E4M3 scale code for a
-// given alpha; the table needs 128 threads (thread t fills entry t).
+// Per-call constants and the table of every E4M3 scale code for a given
+// alpha; the table needs 128 threads (thread t fills entry t).
 __device__ __forceinline__ void make_block_consts(float alpha, BlockConsts& k) {
   k.a6 = __fmul_rn(alpha, 6.0f);
   k.a4 = __fmul_rn(alpha, 4.0f);
@@ -323,12 +339,14 @@ __device__ __forceinline__ void make_block_consts(float alpha, BlockConsts& k) {
   k.inv4 = __frcp_rn(k.a4);
   k.fast_div = k.inv6 >= 1.17549435e-38f && !isinf(k.inv4);
 }
-__device__ __forceinline__ void fill_scale_table(float alpha, float2* dr, uint32_t t) {
+__device__ __forceinline__ void fill_scale_table(float alpha, ScaleEntry* tab, uint32_t t) {
   if (t < 128) {
     float s, unused;
     e4m3x2_to_f32(t, s, unused);
     const float d = t == 0x7F ? 0.0f : __fmul_rn(s, alpha);  // 0x7F is NaN and never produced
-    dr[t] = make_float2(d, safe_recip(d));
+    const float r = safe_recip(d);
+    tab[t].rr = make_f2(r, r);
+    tab[t].nd = make_f2(-d, -d);
   }
 }
 

@@ -395,7 +395,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     // NVFP4 output: the block step's constants and (d, r) table for the
     // output alpha, in the staging area (which the NVFP4 output does not use)
     BlockConsts qk;
-    float2* q_dr = reinterpret_cast<float2*>(smem + OFF_STG);
+    ScaleEntry* q_dr = reinterpret_cast<ScaleEntry*>(smem + OFF_STG);
     bool q_ok = true;
     if (EPI > 0) {
       const float qa = __ldg(p.q_alpha);

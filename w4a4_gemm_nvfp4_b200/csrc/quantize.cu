@@ -42,8 +42,9 @@ namespace {
 
 constexpr int kAmaxThreads = 512;
 constexpr int kMaxPartials = 4096;
-constexpr int kArcRows = 4;          // rows per step of the augmented quantizer
-constexpr int64_t kArcMaxK = 16384;  // its shared memory: 2 bytes x K x (1 + kArcRows)
+constexpr int kArcMaxRows = 4;              // rows per step of the augmented quantizer, at most
+constexpr int64_t kArcMaxK = 16384;         // channels of x it takes, at most
+constexpr int64_t kArcSmemBudget = 98304;   // its shared memory: 2 bytes x K x (1 + 2 x rows per step)
 constexpr int kQuantThreads = 256;
 constexpr int kQuantWarps = kQuantThreads / 32;
 
@@ -117,6 +118,7 @@ struct QuantParams {
   const int32_t* perm = nullptr;  // channel order, K entries
   int64_t S = 0;                  // augmented channels
   int augment = 0;                // 0: residual of the first S reordered channels, 1: their copy
+  int arc_rows = 1;               // rows per step of the augmented quantizer
 };
 
 // Start of every quantize kernel: alpha (a caller-supplied static scale, or
@@ -125,7 +127,7 @@ struct QuantParams {
 // the (d, r) table of every E4M3 scale code.  Returns false when the kernel
 // must stop (non-finite tensor, invalid static alpha); that is uniform over
 // the grid.
-__device__ __forceinline__ bool quant_prologue(const QuantParams& p, BlockConsts& k, float2* s_dr) {
+__device__ __forceinline__ bool quant_prologue(const QuantParams& p, BlockConsts& k, ScaleEntry* s_dr) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   // launched as a programmatic dependent of the amax pass (dynamic alpha):
   // let the next kernel be scheduled, then wait for the amax pass to finish
@@ -162,120 +164,154 @@ __device__ __forceinline__ bool quant_prologue(const QuantParams& p, BlockConsts
     if (nonfinite) return false;
   }
   make_block_consts(alpha, k);
-  fill_scale_table(alpha, s_dr, threadIdx.x);  // (d, r) of every E4M3 scale code
+  fill_scale_table(alpha, s_dr, threadIdx.x);  // constants of every E4M3 scale code
   __syncthreads();
   return true;
 }
 
-// Warp tasks of the row-wise kernel: chunks of 32 consecutive 16-element
-// blocks (512 elements) of one row, lane i taking block i; the last chunk of a
-// row is partial when K % 512 != 0.  Tasks are numbered row-major over the
-// rows padded to a multiple of 128 and each warp takes one contiguous run of
-// them, so inside a row its lanes' pointers into x, the codes and the
-// swizzled scales all advance by constants (512 elements, 256 bytes, 4096
-// bytes: the next K group of atoms) and only a row change recomputes them.
-// Rows past `rows` only write their (zero) scale bytes.  Each warp loads its
-// next task's block while it quantizes the current one.
+// Warp tasks of the row-wise kernel: pairs of chunks of 32 consecutive
+// 16-element blocks (2 x 512 elements, 2 KB of x) of one row; lane i takes
+// block i of each chunk, first chunk 2j, then chunk 2j+1 (absent when a row
+// has an odd number of chunks; the last chunk of a row is partial when
+// K % 512 != 0).  Tasks are numbered row-major over the rows padded to a
+// multiple of 128, and the W warps of the grid take them in a sweep (warp g:
+// tasks g, g + W, g + 2W, ...), so at any moment they work on neighbouring
+// chunks and the grid reads x front to back as one stream (measured 93 % of
+// the copy bandwidth for the bare load/store loop, against 83-86 % when each
+// warp or CTA walks a region of its own).  A step of W tasks is a fixed number
+// of rows and chunk pairs, so the row and the lane's pointers into x and the
+// codes advance by precomputed increments (one of two, depending on whether
+// the pair index wrapped); the second chunk of a task is at fixed offsets from
+// the first, so the bookkeeping of a task is paid once per two blocks.  Each
+// lane loads its next block (the task's second one, or the next task's first)
+// while it quantizes the current one.  Rows past `rows` only write their
+// (zero) scale bytes.
 __device__ __forceinline__ void ld_block2(const uint16_t* p, uint4& lo, uint4& hi) {
   const uint4* q = reinterpret_cast<const uint4*>(p);
   lo = ld_stream(q);
   hi = ld_stream(q + 1);
 }
 
-__device__ __forceinline__ int64_t scale_row_offset(int64_t row, uint32_t kgroups) {
-  return ((row >> 7) * kgroups) * 512 + (row & 31) * 16 + ((row >> 5) & 3) * 4;
+__device__ __forceinline__ int64_t scale_row_offset(uint32_t row, uint32_t kgroups) {
+  return static_cast<int64_t>(row >> 7) * kgroups * 512 + (row & 31) * 16 + ((row >> 5) & 3) * 4;
 }
 
 template <bool FOUR_OVER_SIX, int RULE>
-// Four CTAs per SM: measured faster than five or six in both modes.
-__global__ void __launch_bounds__(kQuantThreads, 4)
+// Scale-6: four CTAs per SM (64 registers), measured faster than three, five
+// or six.  Four-Over-Six: three CTAs per SM (up to 85 registers), which keeps
+// its two candidates' state out of local memory; measured 2-3 % faster than
+// four with spills.
+__global__ void __launch_bounds__(kQuantThreads, FOUR_OVER_SIX ? 3 : 4)
     quantize_kernel(const QuantParams p) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   BlockConsts k;
-  __shared__ float2 s_dr[128];
+  __shared__ ScaleEntry s_dr[128];
   if (!quant_prologue(p, k, s_dr)) return;
 
-  // this warp's run of tasks [t, t_end): tasks split evenly over all warps
   const uint32_t nwarps = gridDim.x * kQuantWarps;
-  const uint32_t gw = blockIdx.x * kQuantWarps + warp;
-  const uint32_t base = p.ntasks / nwarps, extra = p.ntasks % nwarps;
-  uint32_t t = gw * base + min(gw, extra);
-  const uint32_t t_end = t + base + (gw < extra ? 1u : 0u);
-  if (t >= t_end) return;
+  uint32_t t = blockIdx.x * kQuantWarps + warp;  // < 2^31: t + nwarps does not wrap
+  if (t >= p.ntasks) return;
   const uint32_t cpr = p.chunks;                       // chunks per row
+  const uint32_t ppr = (cpr + 1) / 2;                  // chunk pairs (tasks) per row
   const uint32_t kbs = static_cast<uint32_t>(p.K / 16);
-  // lanes past the last block of a row (only in a partial last chunk)
+  // whether this lane has a block in chunk c of a row
   const bool lane_in_last = static_cast<uint32_t>(lane) < kbs - (cpr - 1) * 32;
-  int64_t row = t / cpr;
-  uint32_t chunk = t - static_cast<uint32_t>(row) * cpr;
+  auto has_block = [&](uint32_t c) { return c + 1 < cpr || (c + 1 == cpr && lane_in_last); };
+  const uint32_t rows = static_cast<uint32_t>(p.rows);  // < 2^31 (ntasks < 2^31)
+  // one sweep step = drow rows + dpair chunk pairs; the pointer increments for
+  // a step without and with a pair-index wrap (the next row's first pairs)
+  const uint32_t drow = nwarps / ppr, dpair = nwarps - drow * ppr;
   const int64_t half_k = p.K / 2;
-  const uint32_t lane_scale = static_cast<uint32_t>(lane >> 2) * 512 + (lane & 3);
-  // lane pointers of the current task
-  const uint16_t* xp = p.x + row * p.ldx + chunk * 512 + lane * 16;
-  uint8_t* cp = p.codes + row * half_k + chunk * 256 + lane * 8;
-  uint8_t* sp = p.scales + scale_row_offset(row, p.kgroups) + chunk * 4096 + lane_scale;
+  const int64_t dx = static_cast<int64_t>(drow) * p.ldx + dpair * 1024;
+  const int64_t dx_wrap = dx + p.ldx - static_cast<int64_t>(ppr) * 1024;
+  const int64_t dc = static_cast<int64_t>(drow) * half_k + dpair * 512;
+  const int64_t dc_wrap = dc + half_k - static_cast<int64_t>(ppr) * 512;
+  uint32_t row = t / ppr, pair = t - row * ppr;
+  const uint16_t* xp = p.x + static_cast<int64_t>(row) * p.ldx + pair * 1024 + lane * 16;
+  uint8_t* cp = p.codes + static_cast<int64_t>(row) * half_k + pair * 512 + lane * 8;
+  uint8_t* const sp = p.scales + static_cast<uint32_t>(lane >> 2) * 512 + (lane & 3);
 
-  uint4 lo = make_uint4(0, 0, 0, 0), hi = lo;
-  if (row < p.rows && (chunk + 1 < cpr || lane_in_last)) ld_block2(xp, lo, hi);
-  for (;;) {
-    const bool live = chunk + 1 < cpr || lane_in_last;
-    const bool real_row = row < p.rows;
-    uint8_t* const cur_cp = cp;
-    uint8_t* const cur_sp = sp;
-    // advance to the next task and start its load
-    if (++chunk < cpr) {
-      xp += 512;
-      cp += 256;
-      sp += 4096;
-    } else {
-      chunk = 0;
-      ++row;
-      xp = p.x + row * p.ldx + lane * 16;
-      cp = p.codes + row * half_k + lane * 8;
-      sp = p.scales + scale_row_offset(row, p.kgroups) + lane_scale;
-    }
-    const bool more = ++t < t_end;
-    uint4 nlo = make_uint4(0, 0, 0, 0), nhi = nlo;
-    if (more && row < p.rows && (chunk + 1 < cpr || lane_in_last)) ld_block2(xp, nlo, nhi);
-
-    if (live) {
-      uint32_t scale = 0;
-      if (real_row) {
-        uint2 codes;
-        const uint32_t bmax = quantize_block<FOUR_OVER_SIX, RULE>(lo, hi, k, s_dr, codes, scale);
-        if (p.alpha_in && bmax >= 0x7F80u) {
-          // Inf/NaN in this block (a static alpha skips the tensor check):
-          // the block is written as zeros and the call reports it
-          codes = make_uint2(0u, 0u);
-          scale = 0u;
-          p.ws->status = NVFP4_ERR_NONFINITE;
-        }
-        *reinterpret_cast<uint2*>(cur_cp) = codes;
+  // quantize one block (loaded in lo/hi) of row `r` at codes `c` and scale `s`
+  auto block = [&](const uint4& lo, const uint4& hi, uint32_t r, uint8_t* c, uint8_t* s) {
+    uint32_t scale = 0;
+    if (r < rows) {
+      uint2 codes;
+      const uint32_t bmax = quantize_block<FOUR_OVER_SIX, RULE>(lo, hi, k, s_dr, codes, scale);
+      if (p.alpha_in && bmax >= 0x7F80u) {
+        // Inf/NaN in this block (a static alpha skips the tensor check):
+        // the block is written as zeros and the call reports it
+        codes = make_uint2(0u, 0u);
+        scale = 0u;
+        p.ws->status = NVFP4_ERR_NONFINITE;
       }
-      *cur_sp = static_cast<uint8_t>(scale);
+      *reinterpret_cast<uint2*>(c) = codes;
     }
+    *s = static_cast<uint8_t>(scale);
+  };
+
+  // (a block register pair is only used when its block is quantized, and such
+  // a block was always loaded; they are zeroed once so that no copy of them
+  // is ever of an indeterminate value)
+  uint4 lo = make_uint4(0, 0, 0, 0), hi = lo, nlo = lo, nhi = lo;
+  if (row < rows && has_block(2 * pair)) ld_block2(xp, lo, hi);
+  for (;;) {
+    const uint32_t cur_row = row, c0 = 2 * pair;
+    const uint16_t* const cur_xp = xp;
+    uint8_t* const cur_cp = cp;
+    uint8_t* const cur_sp = sp + scale_row_offset(cur_row, p.kgroups) + c0 * 4096;
+    // first chunk of the pair, while the second one loads
+    const bool second = has_block(c0 + 1);
+    if (cur_row < rows && second) ld_block2(cur_xp + 512, nlo, nhi);
+    if (has_block(c0)) block(lo, hi, cur_row, cur_cp, cur_sp);
+    // advance to the next task
+    t += nwarps;
+    row += drow;
+    pair += dpair;
+    const bool wrap = pair >= ppr;
+    if (wrap) {
+      pair -= ppr;
+      ++row;
+    }
+    xp += wrap ? dx_wrap : dx;
+    cp += wrap ? dc_wrap : dc;
+    const bool more = t < p.ntasks;
+    // second chunk, while the next task's first chunk loads
+    if (more && row < rows && has_block(2 * pair)) ld_block2(xp, lo, hi);
+    if (second) block(nlo, nhi, cur_row, cur_cp + 256, cur_sp + 4096);
     if (!more) break;
-    lo = nlo;
-    hi = nhi;
   }
 }
 
 // Quantization of x^T: the NVFP4 operand of the [K, rows] matrix x^T, i.e.
 // 16-element blocks along rows (a column of x), as the weight-gradient and
-// input-gradient GEMMs of training need it.  A CTA loads a 128-row x 64-column
-// tile of x into shared memory (16-byte chunks, chunk index XOR-swizzled by
-// the 16-row group so the column reads below hit 32 distinct banks), then
-// thread t quantizes the two columns 2(t>>3), 2(t>>3)+1 over rows
-// 16(t&7) .. 16(t&7)+15 with the same block step as the row-wise kernel.
+// input-gradient GEMMs of training need it.  A CTA walks 128-row x 64-column
+// tiles of x (grid-stride).  Each tile is copied into shared memory with
+// 16-byte asynchronous copies (cp.async; chunks outside x are zero-filled),
+// chunk index XOR-swizzled by the 16-row group so the column reads below hit
+// 32 distinct banks; two tile buffers are used in turn, so the next tile's
+// copies are in flight while the current one is quantized.  Thread t
+// quantizes the two columns 2(t>>3), 2(t>>3)+1 over rows 16(t&7) ..
+// 16(t&7)+15 with the same block step as the row-wise kernel.
 // Output row kk of x^T, block mb: codes at kk*(rows/2) + 8*mb, scale in the
 // swizzled layout of a [K, rows] operand; rows kk in [K, ceil(K/128)*128)
 // get zero scales.
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool valid) {
+  // src-size 0 copies nothing and zero-fills the 16 bytes
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(valid ? 16 : 0)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
 template <bool FOUR_OVER_SIX, int RULE>
 __global__ void __launch_bounds__(kQuantThreads)
     quantize_t_kernel(const QuantParams p) {
   BlockConsts k;
-  __shared__ float2 s_dr[128];
-  __shared__ __align__(16) uint32_t tile[128 * 32];  // 128 rows x 128 bytes
+  __shared__ ScaleEntry s_dr[128];
+  __shared__ __align__(16) uint32_t tile[2][128 * 32];  // two buffers of 128 rows x 128 bytes
   if (!quant_prologue(p, k, s_dr)) return;
 
   const int64_t M = p.rows, K = p.K;
@@ -286,31 +322,46 @@ __global__ void __launch_bounds__(kQuantThreads)
   const int cp = threadIdx.x >> 3, mb = threadIdx.x & 7;
   const int64_t half_m = M / 2;
   const int64_t kgroups_t = M / 64;  // K groups of the transposed operand
-  for (uint32_t t = blockIdx.x; t < ntiles; t += gridDim.x) {
+  // issue the copies of tile `t` into buffer `b` (4 chunks of 16 bytes per thread)
+  auto load_tile = [&](uint32_t t, int b) {
     const int64_t m0 = static_cast<int64_t>(t % tiles_m) * 128;
     const int64_t k0 = static_cast<int64_t>(t / tiles_m) * 64;
-    // ---- load: 128 rows x 8 chunks of 16 bytes, 4 per thread ----
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const int q = threadIdx.x + i * kQuantThreads;
       const int r = q >> 3, ch = q & 7;
-      uint4 v = make_uint4(0, 0, 0, 0);
-      if (m0 + r < M && k0 + ch * 8 < K)
-        v = ld_stream(reinterpret_cast<const uint4*>(p.x + (m0 + r) * p.ldx + k0 + ch * 8));
-      *reinterpret_cast<uint4*>(&tile[r * 32 + ((ch ^ ((r >> 4) & 7)) << 2)]) = v;
+      const bool valid = m0 + r < M && k0 + ch * 8 < K;
+      const uint16_t* src = valid ? p.x + (m0 + r) * p.ldx + k0 + ch * 8 : p.x;
+      cp_async16(smem_u32(&tile[b][r * 32 + ((ch ^ ((r >> 4) & 7)) << 2)]), src, valid);
+    }
+    cp_async_commit();
+  };
+  uint32_t t = blockIdx.x;
+  if (t >= ntiles) return;
+  load_tile(t, 0);
+  for (int b = 0;; b ^= 1) {
+    const uint32_t next = t + gridDim.x;
+    if (next < ntiles) {
+      load_tile(next, b ^ 1);
+      cp_async_wait<1>();  // this tile's copies have landed (the next tile's may still fly)
+    } else {
+      cp_async_wait<0>();
     }
     __syncthreads();
+    const int64_t m0 = static_cast<int64_t>(t % tiles_m) * 128;
+    const int64_t k0 = static_cast<int64_t>(t / tiles_m) * 64;
     // ---- two column blocks per thread ----
     const int64_t mb_g = m0 / 16 + mb;
     if (mb_g * 16 < M) {
+      const uint32_t* tl = tile[b];
       uint32_t wl[8], wh[8];  // column 2cp / 2cp+1 as bf16 pairs (element 2i in the low half)
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         const int r0 = mb * 16 + 2 * i;
-        const uint32_t a = tile[r0 * 32 + (((cp >> 2) ^ mb) << 2) + (cp & 3)];
-        const uint32_t b = tile[(r0 + 1) * 32 + (((cp >> 2) ^ mb) << 2) + (cp & 3)];
-        wl[i] = __byte_perm(a, b, 0x5410);
-        wh[i] = __byte_perm(a, b, 0x7632);
+        const uint32_t a = tl[r0 * 32 + (((cp >> 2) ^ mb) << 2) + (cp & 3)];
+        const uint32_t c = tl[(r0 + 1) * 32 + (((cp >> 2) ^ mb) << 2) + (cp & 3)];
+        wl[i] = __byte_perm(a, c, 0x5410);
+        wh[i] = __byte_perm(a, c, 0x7632);
       }
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
@@ -334,7 +385,9 @@ __global__ void __launch_bounds__(kQuantThreads)
             static_cast<uint8_t>(scale);
       }
     }
-    __syncthreads();
+    if (next >= ntiles) break;
+    __syncthreads();  // every thread has read this buffer before it is refilled
+    t = next;
   }
 }
 
@@ -342,22 +395,25 @@ __global__ void __launch_bounds__(kQuantThreads)
 // taken in the order perm, the usual block step on them (primary stage), and
 // S appended channels -- the residual e = fma(-q, d, x) of the first S
 // reordered channels against the primary stage, quantized with the same block
-// step (augment 0), or a copy of them (augment 1, for the weight).  Each CTA
-// takes kArcRows rows at a time: the rows and the permutation sit in shared
-// memory (2 bytes per channel each), so the channel gather reads shared
-// memory only.
+// step (augment 0), or a copy of them (augment 1, for the weight).  The
+// permutation and the rows sit in shared memory (2 bytes per channel each),
+// so the channel gather reads shared memory only.  Each CTA takes
+// p.arc_rows rows per step (4 for K up to about 5K channels, fewer for wider
+// rows, so that two CTAs fit on an SM); two row buffers are used in turn,
+// filled with 16-byte asynchronous copies (cp.async), so the next step's
+// rows load while the current ones are quantized.
 // Output: the [rows, K + S] operand (codes and swizzled scales).
 template <bool FOUR_OVER_SIX, int RULE>
 __global__ void __launch_bounds__(kQuantThreads)
     quantize_arc_kernel(const QuantParams p) {
   BlockConsts k;
-  __shared__ float2 s_dr[128];
-  extern __shared__ __align__(16) uint16_t s_dyn[];  // [K] permutation, then [K] row
+  __shared__ ScaleEntry s_dr[128];
+  extern __shared__ __align__(16) uint16_t s_dyn[];  // [K] permutation, then 2 x [arc_rows][K] rows
   if (!quant_prologue(p, k, s_dr)) return;
 
   const int64_t K = p.K, KA = p.K + p.S;
+  const int R = p.arc_rows;
   uint16_t* s_perm = s_dyn;
-  uint16_t* s_rows = s_dyn + K;  // kArcRows rows
   for (int64_t i = threadIdx.x; i < K; i += kQuantThreads) {
     const int32_t c = p.perm[i];
     s_perm[i] = static_cast<uint16_t>(c >= 0 && c < K ? c : 0);  // out-of-range entries read channel 0
@@ -365,18 +421,33 @@ __global__ void __launch_bounds__(kQuantThreads)
   const int64_t rows_padded = (p.rows + 127) / 128 * 128;
   const int64_t half_ka = KA / 2, kgroups_a = KA / 64;
   const int nprim = static_cast<int>(K / 16), nres = static_cast<int>(p.S / 16);
-  // kArcRows consecutive rows per step (rows_padded is a multiple of 128)
-  for (int64_t row0 = static_cast<int64_t>(blockIdx.x) * kArcRows; row0 < rows_padded;
-       row0 += static_cast<int64_t>(gridDim.x) * kArcRows) {
-    __syncthreads();  // the permutation is staged / the previous rows are consumed
-    for (int rr = 0; rr < kArcRows; ++rr) {
+  // the copies of the R rows starting at row0 into buffer `buf`, one commit group
+  auto load_rows = [&](int64_t row0, int buf) {
+    const uint32_t dst0 = smem_u32(s_dyn + K + static_cast<int64_t>(buf) * R * K);
+    for (int rr = 0; rr < R; ++rr) {
       if (row0 + rr >= p.rows) break;
-      const uint4* src = reinterpret_cast<const uint4*>(p.x + (row0 + rr) * p.ldx);
-      uint4* dst = reinterpret_cast<uint4*>(s_rows + rr * K);
-      for (int64_t c = threadIdx.x; c < K / 8; c += kQuantThreads) dst[c] = ld_stream(src + c);
+      const uint16_t* src = p.x + (row0 + rr) * p.ldx;
+      const uint32_t dst = dst0 + static_cast<uint32_t>(rr * K) * 2;
+      for (int64_t c = threadIdx.x; c < K / 8; c += kQuantThreads)
+        cp_async16(dst + static_cast<uint32_t>(c) * 16, src + c * 8, true);
     }
-    __syncthreads();
-    for (int jr = threadIdx.x; jr < kArcRows * nprim; jr += kQuantThreads) {
+    cp_async_commit();
+  };
+  // R consecutive rows per step (rows_padded is a multiple of 128, R divides 128)
+  int64_t row0 = static_cast<int64_t>(blockIdx.x) * R;
+  if (row0 >= rows_padded) return;
+  load_rows(row0, 0);
+  for (int buf = 0;; buf ^= 1) {
+    const int64_t next0 = row0 + static_cast<int64_t>(gridDim.x) * R;
+    if (next0 < rows_padded) {
+      load_rows(next0, buf ^ 1);
+      cp_async_wait<1>();  // this step's rows have landed (the next step's may still fly)
+    } else {
+      cp_async_wait<0>();
+    }
+    __syncthreads();  // every thread's copies (and, the first time, the permutation) are visible
+    const uint16_t* s_rows = s_dyn + K + static_cast<int64_t>(buf) * R * K;
+    for (int jr = threadIdx.x; jr < R * nprim; jr += kQuantThreads) {
       const int rr = jr / nprim, j = jr - rr * nprim;
       const int64_t row = row0 + rr;
       const bool live = row < p.rows;
@@ -403,8 +474,7 @@ __global__ void __launch_bounds__(kQuantThreads)
             codes_a = codes;
             scale_a = scale;
           } else {
-            const float d = s_dr[scale].x;
-            const f2 nd = make_f2(-d, -d);
+            const f2 nd = s_dr[scale].nd;
             f2 q[8], e[8];
             decode_pairs(codes, q);
             float b = 0.0f;
@@ -425,25 +495,37 @@ __global__ void __launch_bounds__(kQuantThreads)
         p.scales[(atom_row + (ja >> 2)) * 512 + in_atom + (ja & 3)] = static_cast<uint8_t>(scale_a);
       }
     }
+    if (next0 >= rows_padded) break;
+    __syncthreads();  // the buffer just quantized is refilled at the top of the next step
+    row0 = next0;
   }
+}
+
+// Rows per step of the augmented quantizer for K channels: the most (up to 4,
+// a power of two so it divides the 128-row padding) whose permutation and two
+// row buffers fit the shared-memory budget.
+int arc_rows_per_step(int64_t K) {
+  int r = kArcMaxRows;
+  while (r > 1 && 2 * K * (1 + 2 * r) > kArcSmemBudget) r /= 2;
+  return r;
 }
 
 template <bool F, int R>
 cudaError_t launch_quantize_arc(int dev, int sms, const QuantParams& p, cudaStream_t s, bool pdl) {
-  const size_t smem = static_cast<size_t>(p.K) * 2 * (1 + kArcRows);
+  const size_t smem = static_cast<size_t>(p.K) * 2 * (1 + 2 * p.arc_rows);
   // the shared-memory opt-in is an attribute of the kernel in this context
   static PerContextCache<int> attr;
   int done = 0;
   cudaError_t e = per_context(attr, dev, [](int* v) {
     *v = 1;
     return cudaFuncSetAttribute(quantize_arc_kernel<F, R>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                static_cast<int>(kArcMaxK * 2 * (1 + kArcRows)));
+                                static_cast<int>(kArcSmemBudget));
   }, &done);
   if (e != cudaSuccess) return e;
   int occ = 0;
   e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, quantize_arc_kernel<F, R>, kQuantThreads, smem);
   if (e != cudaSuccess) return e;
-  const int64_t steps = (p.rows + 127) / 128 * 128 / kArcRows;
+  const int64_t steps = (p.rows + 127) / 128 * 128 / p.arc_rows;
   const int grid = static_cast<int>(std::max<int64_t>(
       1, std::min<int64_t>(steps, static_cast<int64_t>(sms) * std::max(1, occ))));
   return launch_kernel(quantize_arc_kernel<F, R>, dim3(grid), dim3(kQuantThreads), smem, s, pdl, p);
@@ -521,9 +603,10 @@ size_t nvfp4_quantize_workspace_bytes(int64_t rows, int64_t K) {
 namespace {
 
 // ------------------------------------------------------------ host side --
-// Warp tasks of the row-wise kernel: chunks of 32 blocks of 16 elements (the
-// last chunk of a row may be partial) over the rows padded to a multiple of 128.
-int64_t row_tasks(int64_t rows, int64_t K) { return (rows + 127) / 128 * 128 * ((K + 511) / 512); }
+// Warp tasks of the row-wise kernel: pairs of chunks of 32 blocks of 16
+// elements (the last pair of a row may hold one chunk, the last chunk may be
+// partial) over the rows padded to a multiple of 128.
+int64_t row_tasks(int64_t rows, int64_t K) { return (rows + 127) / 128 * 128 * (((K + 511) / 512 + 1) / 2); }
 
 // Checks shared by every quantize entry point: pointers, shape, row pitch,
 // mode, rule, alignment and the size limits of the kernels' index arithmetic.
@@ -666,6 +749,7 @@ nvfp4_status quantize_impl(const char* fn, QuantKind kind, const void* x, int64_
   p.perm = perm;
   p.S = S;
   p.augment = augment;
+  p.arc_rows = arc_rows_per_step(K);
   const int amax_grid = std::min(amax_grid_size(rows, K, ldx, sms), kMaxPartials);
   return launch_dynamic(kind, p, mode, rule, fp8_max, global_scale, partials, amax_grid, dev, sms,
                         static_cast<cudaStream_t>(stream));
