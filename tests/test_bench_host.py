@@ -78,3 +78,23 @@ def test_sampler_without_nvml_reports_why(monkeypatch):
 @pytest.mark.parametrize("world,flops,ms,expect", [(1, 2e12, 1.0, 2000.0), (4, 1e12, 2.0, 2000.0)])
 def test_job_throughput_counts_all_ranks_over_the_slowest(world, flops, ms, expect):
     assert bench.job_tflops(world, flops, ms) == pytest.approx(expect)
+
+
+def test_recorded_traffic_only_for_the_captured_kernel(monkeypatch):
+    """The GEMM's recorded DRAM traffic is reported only for the full-size
+    prefill workload and only while the kernel sources hash to the value
+    recorded with the capture."""
+    args = types.SimpleNamespace(workload="prefill", x_rows=0)
+    monkeypatch.setitem(bench.GEMM_PREFILL_TRAFFIC, "kernel_sources_sha1", bench.gemm_sources_sha1())
+    assert bench.recorded_traffic(args)["bytes"] == bench.GEMM_PREFILL_TRAFFIC["bytes"]
+    assert bench.recorded_traffic(types.SimpleNamespace(workload="prefill", x_rows=8192)) is None
+    assert bench.recorded_traffic(types.SimpleNamespace(workload="mlp8b", x_rows=0)) is None
+    monkeypatch.setitem(bench.GEMM_PREFILL_TRAFFIC, "kernel_sources_sha1", "0" * 40)
+    assert bench.recorded_traffic(args) is None
+
+
+def test_x_rows_replaces_only_the_activation_rows():
+    wl = bench.workload_of(types.SimpleNamespace(workload="prefill", x_rows=8192))
+    ref = bench.workloads.WORKLOADS["prefill"]
+    assert (wl.M, wl.N, wl.K) == (8192, ref.N, ref.K)
+    assert wl.x.seed == ref.x.seed and wl.w == ref.w
