@@ -43,8 +43,12 @@ namespace {
 constexpr int kAmaxThreads = 512;
 constexpr int kMaxPartials = 4096;
 constexpr int kArcMaxRows = 4;              // rows per step of the augmented quantizer, at most
+constexpr int kArcPrimThreads = 256;        // its threads for the primary blocks, at most
+constexpr int kArcMaxThreads = 640;         // its block size, at most
+constexpr int kArcBufs = 3;                 // its row buffers
+constexpr int64_t kArcSmemStep = 73728;     // shared memory it aims at: three CTAs per SM up to 5K channels
 constexpr int64_t kArcMaxK = 16384;         // channels of x it takes, at most
-constexpr int64_t kArcSmemBudget = 98304;   // its shared memory: 2 bytes x K x (1 + 2 x rows per step)
+constexpr int64_t kArcSmemBudget = 2 * 16384 * (1 + kArcBufs);  // its shared memory, at most: 2 bytes x K x (1 + 3 x rows per step)
 constexpr int kQuantThreads = 256;
 constexpr int kQuantWarps = kQuantThreads / 32;
 
@@ -119,12 +123,14 @@ struct QuantParams {
   int64_t S = 0;                  // augmented channels
   int augment = 0;                // 0: residual of the first S reordered channels, 1: their copy
   int arc_rows = 1;               // rows per step of the augmented quantizer
+  int arc_prim_threads = 128;     // its threads for the primary blocks; the rest take the appended ones
 };
 
 // Start of every quantize kernel: alpha (a caller-supplied static scale, or
 // the tensor amax reduced from the partials of the amax pass -- every CTA
 // reduces the same partials), the per-call constants of the block step and
-// the (d, r) table of every E4M3 scale code.  Returns false when the kernel
+// the (d, r) table of every E4M3 scale code.  The block size is a multiple of
+// 32 and at least 128 (the table has one entry per thread of the first 128).  Returns false when the kernel
 // must stop (non-finite tensor, invalid static alpha); that is uniform over
 // the grid.
 __device__ __forceinline__ bool quant_prologue(const QuantParams& p, BlockConsts& k, ScaleEntry* s_dr) {
@@ -144,16 +150,17 @@ __device__ __forceinline__ bool quant_prologue(const QuantParams& p, BlockConsts
     // the status word was cleared to NVFP4_OK before the launch; CTAs only
     // ever raise it (to NVFP4_ERR_NONFINITE), so their order does not matter
   } else {
-    __shared__ uint32_t s_red[kQuantWarps];
+    __shared__ uint32_t s_red[32];
     uint32_t m = 0;
-    for (int i = threadIdx.x; i < p.nparts; i += kQuantThreads) m = max(m, p.partials[i]);
+    for (int i = threadIdx.x; i < p.nparts; i += blockDim.x) m = max(m, p.partials[i]);
 #pragma unroll
     for (int o = 16; o; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
     if (lane == 0) s_red[warp] = m;
     __syncthreads();
     uint32_t amax_bits = 0;
 #pragma unroll
-    for (int w = 0; w < kQuantWarps; ++w) amax_bits = max(amax_bits, s_red[w]);
+    for (int w = 0; w < 32; ++w)
+      if (w < static_cast<int>(blockDim.x >> 5)) amax_bits = max(amax_bits, s_red[w]);
     const bool nonfinite = amax_bits >= 0x7F80u;
     alpha = amax_bits == 0 ? 1.0f : __fdiv_rn(__uint_as_float(amax_bits << 16), p.f6);
     if (blockIdx.x == 0 && threadIdx.x == 0) {
@@ -300,6 +307,24 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool v
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(valid ? 16 : 0)
                : "memory");
 }
+// Plain arrive (count 1) on a shared::cta mbarrier.
+__device__ __forceinline__ void mbar_arrive_local(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+// Bulk copy of `bytes` (a multiple of 16, both addresses 16-byte aligned) from
+// global to this CTA's shared memory, completing on the mbarrier `bar`.
+__device__ __forceinline__ void bulk_copy_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+               "l"(src), "r"(bytes), "r"(bar)
+               : "memory");
+}
+// 16-bit shared-memory load at a 32-bit shared address (zero-extended);
+// volatile, so it is not moved across the barriers that publish the rows
+__device__ __forceinline__ uint32_t ld_shared_u16(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared.u16 %0, [%1];" : "=r"(v) : "r"(addr));
+  return v;
+}
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 template <int N>
 __device__ __forceinline__ void cp_async_wait() {
@@ -396,80 +421,163 @@ __global__ void __launch_bounds__(kQuantThreads)
 // S appended channels -- the residual e = fma(-q, d, x) of the first S
 // reordered channels against the primary stage, quantized with the same block
 // step (augment 0), or a copy of them (augment 1, for the weight).  The
-// permutation and the rows sit in shared memory (2 bytes per channel each),
-// so the channel gather reads shared memory only.  Each CTA takes
-// p.arc_rows rows per step (4 for K up to about 5K channels, fewer for wider
-// rows, so that two CTAs fit on an SM); two row buffers are used in turn,
-// filled with 16-byte asynchronous copies (cp.async), so the next step's
-// rows load while the current ones are quantized.
+// permutation (as byte offsets into a row) and the rows sit in shared memory,
+// so the channel gather reads shared memory only.  Each CTA takes p.arc_rows
+// rows per step (2 for K up to about 5K channels, 1 for wider rows) through
+// kArcBufs row buffers: the CTA's last warp is the producer, which fills
+// buffer s % kArcBufs for step s with one bulk copy per row once every
+// consumer warp has released it (mbarriers full[] and consumed[]), so the
+// consumers run up to kArcBufs - 1 steps ahead of the slowest of them with no
+// CTA-wide barrier.  Of the consumer threads, the first P own the primary
+// block columns t, t + P, ...: a thread reads a column's 16 channel offsets
+// once per step and gathers that block from each of the step's rows with
+// them.  The remaining ones take the appended blocks (row, j < S/16) of the
+// step: each gathers block j again, repeats its primary step and quantizes
+// the residual (or copies the codes); kept apart from the primary threads,
+// this extra work does not make one warp of every step twice as long as the
+// others (a warp's time is that of its slowest lane).  Every wait is bounded:
+// one that sees no progress for 4 s records NVFP4_ERR_TIMEOUT, and the
+// producer lets the copies it issued land before the CTA exits.
 // Output: the [rows, K + S] operand (codes and swizzled scales).
 template <bool FOUR_OVER_SIX, int RULE>
-__global__ void __launch_bounds__(kQuantThreads)
+__global__ void __launch_bounds__(kArcMaxThreads)
     quantize_arc_kernel(const QuantParams p) {
   BlockConsts k;
   __shared__ ScaleEntry s_dr[128];
-  extern __shared__ __align__(16) uint16_t s_dyn[];  // [K] permutation, then 2 x [arc_rows][K] rows
+  extern __shared__ __align__(16) uint16_t s_dyn[];  // [K] channel byte offsets, then kArcBufs x [arc_rows][K] rows
   if (!quant_prologue(p, k, s_dr)) return;
 
   const int64_t K = p.K, KA = p.K + p.S;
   const int R = p.arc_rows;
-  uint16_t* s_perm = s_dyn;
-  for (int64_t i = threadIdx.x; i < K; i += kQuantThreads) {
+  const int T = static_cast<int>(blockDim.x), P = p.arc_prim_threads;
+  for (int64_t i = threadIdx.x; i < K; i += T) {
     const int32_t c = p.perm[i];
-    s_perm[i] = static_cast<uint16_t>(c >= 0 && c < K ? c : 0);  // out-of-range entries read channel 0
+    s_dyn[i] = static_cast<uint16_t>(2 * (c >= 0 && c < K ? c : 0));  // out-of-range entries read channel 0
   }
   const int64_t rows_padded = (p.rows + 127) / 128 * 128;
   const int64_t half_ka = KA / 2, kgroups_a = KA / 64;
   const int nprim = static_cast<int>(K / 16), nres = static_cast<int>(p.S / 16);
-  // the copies of the R rows starting at row0 into buffer `buf`, one commit group
-  auto load_rows = [&](int64_t row0, int buf) {
-    const uint32_t dst0 = smem_u32(s_dyn + K + static_cast<int64_t>(buf) * R * K);
-    for (int rr = 0; rr < R; ++rr) {
-      if (row0 + rr >= p.rows) break;
-      const uint16_t* src = p.x + (row0 + rr) * p.ldx;
-      const uint32_t dst = dst0 + static_cast<uint32_t>(rr * K) * 2;
-      for (int64_t c = threadIdx.x; c < K / 8; c += kQuantThreads)
-        cp_async16(dst + static_cast<uint32_t>(c) * 16, src + c * 8, true);
+  const uint32_t rows_base = smem_u32(s_dyn + K);
+  const uint32_t row_bytes = static_cast<uint32_t>(K) * 2, buf_bytes = row_bytes * R;
+  // Buffers: full[b] completes when buffer b holds its step's rows (the
+  // producer's arrival plus the copies' bytes); consumed[b] when every
+  // consumer warp is done with it.  Step s uses buffer s % kArcBufs; its
+  // waits are on phase s / kArcBufs of those barriers.
+  __shared__ __align__(8) uint64_t s_bar[2 * kArcBufs];
+  __shared__ int s_abort;
+  const uint32_t full0 = smem_u32(&s_bar[0]), consumed0 = smem_u32(&s_bar[kArcBufs]);
+  const int warp = static_cast<int>(threadIdx.x >> 5), lane = static_cast<int>(threadIdx.x & 31);
+  const int producer_warp = T / 32 - 1;
+  if (threadIdx.x == 0) {
+    for (int b = 0; b < kArcBufs; ++b) {
+      mbar_init(full0 + 8 * b, 1);
+      mbar_init(consumed0 + 8 * b, producer_warp);  // one arrival per consumer warp
     }
-    cp_async_commit();
+    s_abort = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();  // barriers initialised, channel offsets visible
+  volatile int* abort = &s_abort;
+  constexpr uint64_t kWaitNs = 4000000000ull;  // no progress for 4 s: report a timeout and stop
+  auto fail = [&](uint32_t where) {
+    if (!*abort) {
+      *abort = 1;
+      p.ws->detail = where;
+      p.ws->status = NVFP4_ERR_TIMEOUT;
+    }
   };
-  // R consecutive rows per step (rows_padded is a multiple of 128, R divides 128)
-  int64_t row0 = static_cast<int64_t>(blockIdx.x) * R;
-  if (row0 >= rows_padded) return;
-  load_rows(row0, 0);
-  for (int buf = 0;; buf ^= 1) {
-    const int64_t next0 = row0 + static_cast<int64_t>(gridDim.x) * R;
-    if (next0 < rows_padded) {
-      load_rows(next0, buf ^ 1);
-      cp_async_wait<1>();  // this step's rows have landed (the next step's may still fly)
-    } else {
-      cp_async_wait<0>();
+  const int64_t stride_rows = static_cast<int64_t>(gridDim.x) * R;
+  if (warp == producer_warp) {
+    // ------------------------------------------------------- producer ----
+    int s = 0;
+    for (int64_t row0 = static_cast<int64_t>(blockIdx.x) * R; row0 < rows_padded; row0 += stride_rows, ++s) {
+      const int b = s % kArcBufs;
+      if (s >= kArcBufs &&
+          !__all_sync(0xffffffffu, mbar_wait_bounded(consumed0 + 8 * b, (s / kArcBufs - 1) & 1, abort, kWaitNs))) {
+        if (lane == 0) fail(1);
+        break;
+      }
+      if (lane == 0) {
+        const int64_t left = p.rows - row0;
+        const int valid = left <= 0 ? 0 : (left < R ? static_cast<int>(left) : R);
+        mbar_expect_tx(full0 + 8 * b, static_cast<uint32_t>(valid) * row_bytes);
+        for (int rr = 0; rr < valid; ++rr)
+          bulk_copy_g2s(rows_base + b * buf_bytes + rr * row_bytes, p.x + (row0 + rr) * p.ldx, row_bytes,
+                        full0 + 8 * b);
+      }
+      __syncwarp();
     }
-    __syncthreads();  // every thread's copies (and, the first time, the permutation) are visible
-    const uint16_t* s_rows = s_dyn + K + static_cast<int64_t>(buf) * R * K;
-    for (int jr = threadIdx.x; jr < R * nprim; jr += kQuantThreads) {
-      const int rr = jr / nprim, j = jr - rr * nprim;
-      const int64_t row = row0 + rr;
-      const bool live = row < p.rows;
-      const uint16_t* s_row = s_rows + rr * K;
-      const int64_t atom_row = (row >> 7) * kgroups_a;
-      const int64_t in_atom = (row & 31) * 16 + ((row >> 5) & 3) * 4;
-      uint32_t scale = 0, scale_a = 0;
-      uint2 codes = make_uint2(0u, 0u), codes_a = codes;
-      if (live) {
-        // gather the block's 16 channels as bf16 pairs (element 2i low)
-        const uint4 pi0 = reinterpret_cast<const uint4*>(s_perm + 16 * j)[0];
-        const uint4 pi1 = reinterpret_cast<const uint4*>(s_perm + 16 * j)[1];
-        const uint32_t pw[8] = {pi0.x, pi0.y, pi0.z, pi0.w, pi1.x, pi1.y, pi1.z, pi1.w};
-        uint32_t w[8];
+    if (*abort && lane == 0) {
+      // let the copies already issued land before the CTA can exit
+      const volatile int no_abort = 0;
+      for (int k = s >= kArcBufs ? s - kArcBufs : 0; k < s; ++k)
+        mbar_wait_bounded(full0 + 8 * (k % kArcBufs), (k / kArcBufs) & 1, &no_abort, 100000000ull);
+    }
+    return;
+  }
+  // ---------------------------------------------------------- consumers ----
+  auto scale_at = [&](int64_t row, int col) -> uint8_t& {
+    return p.scales[(row >> 7) * kgroups_a * 512 + (row & 31) * 16 + ((row >> 5) & 3) * 4 + (col >> 2) * 512 +
+                    (col & 3)];
+  };
+  int s = 0;
+  for (int64_t row0 = static_cast<int64_t>(blockIdx.x) * R; row0 < rows_padded; row0 += stride_rows, ++s) {
+    const int b = s % kArcBufs;
+    if (!__all_sync(0xffffffffu, mbar_wait_bounded(full0 + 8 * b, (s / kArcBufs) & 1, abort, kWaitNs))) {
+      if (lane == 0) fail(2);
+      break;
+    }
+    const uint32_t s_buf = rows_base + static_cast<uint32_t>(b) * buf_bytes;  // shared address of the step's rows
+    // gather block j of buffer row rr (16 channels as bf16 pairs, element 2i low)
+    auto gather = [&](int rr, int j, f2 px[8]) {
+      const uint4 o0 = reinterpret_cast<const uint4*>(s_dyn + 16 * j)[0];
+      const uint4 o1 = reinterpret_cast<const uint4*>(s_dyn + 16 * j)[1];
+      const uint32_t ow[8] = {o0.x, o0.y, o0.z, o0.w, o1.x, o1.y, o1.z, o1.w};
+      const uint32_t s_row = s_buf + rr * row_bytes;
+      uint32_t w[8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
-          w[i] = static_cast<uint32_t>(s_row[pw[i] & 0xFFFFu]) | (static_cast<uint32_t>(s_row[pw[i] >> 16]) << 16);
-        f2 px[8];
-        const uint32_t bbits = unpack_block(make_uint4(w[0], w[1], w[2], w[3]),
-                                            make_uint4(w[4], w[5], w[6], w[7]), px);
-        quantize_pairs<FOUR_OVER_SIX, RULE>(px, __uint_as_float(bbits << 16), k, s_dr, codes, scale);
-        if (j < nres) {
+      for (int i = 0; i < 8; ++i)
+        w[i] = ld_shared_u16(s_row + (ow[i] & 0xFFFFu)) | (ld_shared_u16(s_row + (ow[i] >> 16)) << 16);
+      return unpack_block(make_uint4(w[0], w[1], w[2], w[3]), make_uint4(w[4], w[5], w[6], w[7]), px);
+    };
+    if (static_cast<int>(threadIdx.x) < P) {
+      // primary blocks
+      for (int j = threadIdx.x; j < nprim; j += P) {
+        const uint4 o0 = reinterpret_cast<const uint4*>(s_dyn + 16 * j)[0];
+        const uint4 o1 = reinterpret_cast<const uint4*>(s_dyn + 16 * j)[1];
+        const uint32_t ow[8] = {o0.x, o0.y, o0.z, o0.w, o1.x, o1.y, o1.z, o1.w};
+        for (int rr = 0; rr < R; ++rr) {
+          const int64_t row = row0 + rr;
+          uint32_t scale = 0;
+          if (row < p.rows) {
+            const uint32_t s_row = s_buf + rr * row_bytes;
+            uint32_t w[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              w[i] = ld_shared_u16(s_row + (ow[i] & 0xFFFFu)) | (ld_shared_u16(s_row + (ow[i] >> 16)) << 16);
+            f2 px[8];
+            const uint32_t bbits = unpack_block(make_uint4(w[0], w[1], w[2], w[3]),
+                                                make_uint4(w[4], w[5], w[6], w[7]), px);
+            uint2 codes;
+            quantize_pairs<FOUR_OVER_SIX, RULE>(px, __uint_as_float(bbits << 16), k, s_dr, codes, scale);
+            *reinterpret_cast<uint2*>(p.codes + row * half_ka + j * 8) = codes;
+          }
+          scale_at(row, j) = static_cast<uint8_t>(scale);
+        }
+      }
+    } else {
+      // appended blocks: units (rr, j) of this step, j < S/16
+      const int Tr = T - 32 - P;
+      for (int u = static_cast<int>(threadIdx.x) - P; u < R * nres; u += Tr) {
+        const int rr = u / nres, j = u - rr * nres;
+        const int64_t row = row0 + rr;
+        uint32_t scale_a = 0;
+        if (row < p.rows) {
+          f2 px[8];
+          const uint32_t bbits = gather(rr, j, px);
+          uint2 codes, codes_a;
+          uint32_t scale;
+          quantize_pairs<FOUR_OVER_SIX, RULE>(px, __uint_as_float(bbits << 16), k, s_dr, codes, scale);
           if (p.augment) {
             codes_a = codes;
             scale_a = scale;
@@ -477,42 +585,60 @@ __global__ void __launch_bounds__(kQuantThreads)
             const f2 nd = s_dr[scale].nd;
             f2 q[8], e[8];
             decode_pairs(codes, q);
-            float b = 0.0f;
+            float bmax = 0.0f;
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
               e[i] = fma2(q[i], nd, px[i]);
-              b = fmaxf(b, fmaxf(fabsf(e[i].a()), fabsf(e[i].b())));
+              bmax = fmaxf(bmax, fmaxf(fabsf(e[i].a()), fabsf(e[i].b())));
             }
-            quantize_pairs<FOUR_OVER_SIX, RULE>(e, b, k, s_dr, codes_a, scale_a);
+            quantize_pairs<FOUR_OVER_SIX, RULE>(e, bmax, k, s_dr, codes_a, scale_a);
           }
+          *reinterpret_cast<uint2*>(p.codes + row * half_ka + (nprim + j) * 8) = codes_a;
         }
-        *reinterpret_cast<uint2*>(p.codes + row * half_ka + j * 8) = codes;
-        if (j < nres) *reinterpret_cast<uint2*>(p.codes + row * half_ka + (nprim + j) * 8) = codes_a;
-      }
-      p.scales[(atom_row + (j >> 2)) * 512 + in_atom + (j & 3)] = static_cast<uint8_t>(scale);
-      if (j < nres) {
-        const int ja = nprim + j;
-        p.scales[(atom_row + (ja >> 2)) * 512 + in_atom + (ja & 3)] = static_cast<uint8_t>(scale_a);
+        scale_at(row, nprim + j) = static_cast<uint8_t>(scale_a);
       }
     }
-    if (next0 >= rows_padded) break;
-    __syncthreads();  // the buffer just quantized is refilled at the top of the next step
-    row0 = next0;
+    __syncwarp();
+    if (lane == 0) mbar_arrive_local(consumed0 + 8 * b);  // this warp is done with buffer b
   }
 }
 
+// Threads of the augmented quantizer for K channels: P for the primary blocks,
+// c block columns each (c >= 2 from 256 columns up, P <= 256, a multiple of
+// 32), so that a CTA stays small and several share an SM; then enough for the
+// step's R * S/16 appended blocks at about c * R / 2 each (two block steps
+// apiece, against c * R for a primary thread), within kArcMaxThreads; at
+// least 96 consumers in all; then the producer warp.
+int arc_prim_threads(int64_t K) {
+  const int64_t nprim = std::max<int64_t>(1, K / 16);
+  const int64_t cols = std::max<int64_t>((nprim + kArcPrimThreads - 1) / kArcPrimThreads, nprim >= 256 ? 2 : 1);
+  const int64_t t = (nprim + cols - 1) / cols;
+  return static_cast<int>((t + 31) / 32 * 32);
+}
+int arc_threads(int64_t K, int64_t S, int R) {
+  const int prim = arc_prim_threads(K);
+  const int64_t nprim = std::max<int64_t>(1, K / 16);
+  const int64_t cols = (nprim + prim - 1) / prim;
+  const int64_t units = R * (S / 16), per = std::max<int64_t>(1, cols * R / 2);
+  int64_t res = units == 0 ? 0 : ((units + per - 1) / per + 31) / 32 * 32;
+  res = std::min<int64_t>(res, kArcMaxThreads - 32 - prim);  // room for the producer warp
+  if (units > 0) res = std::max<int64_t>(res, 32);
+  return static_cast<int>(std::max<int64_t>(96, prim + res)) + 32;  // + the producer warp
+}
+
 // Rows per step of the augmented quantizer for K channels: the most (up to 4,
-// a power of two so it divides the 128-row padding) whose permutation and two
-// row buffers fit the shared-memory budget.
+// a power of two so it divides the 128-row padding) whose permutation and
+// kArcBufs row buffers fit kArcSmemStep (at least one row: K <= 16384 keeps
+// that within kArcSmemBudget).
 int arc_rows_per_step(int64_t K) {
   int r = kArcMaxRows;
-  while (r > 1 && 2 * K * (1 + 2 * r) > kArcSmemBudget) r /= 2;
+  while (r > 1 && 2 * K * (1 + kArcBufs * r) > kArcSmemStep) r /= 2;
   return r;
 }
 
 template <bool F, int R>
 cudaError_t launch_quantize_arc(int dev, int sms, const QuantParams& p, cudaStream_t s, bool pdl) {
-  const size_t smem = static_cast<size_t>(p.K) * 2 * (1 + 2 * p.arc_rows);
+  const size_t smem = static_cast<size_t>(p.K) * 2 * (1 + kArcBufs * p.arc_rows);
   // the shared-memory opt-in is an attribute of the kernel in this context
   static PerContextCache<int> attr;
   int done = 0;
@@ -522,13 +648,14 @@ cudaError_t launch_quantize_arc(int dev, int sms, const QuantParams& p, cudaStre
                                 static_cast<int>(kArcSmemBudget));
   }, &done);
   if (e != cudaSuccess) return e;
+  const int threads = arc_threads(p.K, p.S, p.arc_rows);
   int occ = 0;
-  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, quantize_arc_kernel<F, R>, kQuantThreads, smem);
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, quantize_arc_kernel<F, R>, threads, smem);
   if (e != cudaSuccess) return e;
   const int64_t steps = (p.rows + 127) / 128 * 128 / p.arc_rows;
   const int grid = static_cast<int>(std::max<int64_t>(
       1, std::min<int64_t>(steps, static_cast<int64_t>(sms) * std::max(1, occ))));
-  return launch_kernel(quantize_arc_kernel<F, R>, dim3(grid), dim3(kQuantThreads), smem, s, pdl, p);
+  return launch_kernel(quantize_arc_kernel<F, R>, dim3(grid), dim3(threads), smem, s, pdl, p);
 }
 
 cudaError_t launch_quantize_arc_kernel(int mode, int rule, int dev, int sms, const QuantParams& p,
@@ -749,7 +876,10 @@ nvfp4_status quantize_impl(const char* fn, QuantKind kind, const void* x, int64_
   p.perm = perm;
   p.S = S;
   p.augment = augment;
-  p.arc_rows = arc_rows_per_step(K);
+  if (kind == QuantKind::kAugmented) {
+    p.arc_rows = arc_rows_per_step(K);
+    p.arc_prim_threads = arc_prim_threads(K);
+  }
   const int amax_grid = std::min(amax_grid_size(rows, K, ldx, sms), kMaxPartials);
   return launch_dynamic(kind, p, mode, rule, fp8_max, global_scale, partials, amax_grid, dev, sms,
                         static_cast<cudaStream_t>(stream));
