@@ -293,6 +293,9 @@ def run_ours(args, world, rank, local):
     with ClockSampler(local) as clocks:
         steps_ms = timed_fused(args.steps)          # the headline: K whole steps
     assert nv.device_status(qx.workspace) == nv.OK and nv.device_status(gws) == nv.OK
+    # the breakdown, with its own clock samples (a long breakdown can run
+    # warmer, and so slower, than the headline steps)
+    bclocks = ClockSampler(local).__enter__()
     # the breakdown: the same step as two calls with an event between them
     _barrier(world)
     torch.cuda.synchronize()
@@ -344,17 +347,25 @@ def run_ours(args, world, rank, local):
     ms_qout = time_op(lambda: nv.gemm_quantized(qx, qw, y_alpha, "four_over_six", "mse", out=qy), args.steps)
     ms_arc_q = time_op(lambda: nv.quantize_arc(x, perm, S_ARC, nv.AUG_RESIDUAL, xm, xr, xF, out=qa), args.steps)
 
-    def arc_step():
-        nv.quantize_arc(x, perm, S_ARC, nv.AUG_RESIDUAL, xm, xr, xF, out=qa)
-        nv.gemm(qa, qw_arc, out_dtype=torch.bfloat16, out=y_arc, workspace=gws)
+    def arc_step():  # the augmented layer in one call, as the headline step is
+        nv.quantize_arc_gemm(x, perm, S_ARC, qw_arc, xm, xr, xF, out_dtype=torch.bfloat16, x_out=qa, out=y_arc,
+                             workspace=gws)
 
-    ms_arc_step = time_op(arc_step, args.steps)
+    # the augmented step against the plain step, alternated in one loop so
+    # that both see the same clocks
+    t_plain_pair, t_arc_pair = [], []
+    for i in range(args.steps):
+        t_plain_pair += time_op(fused_step, 1)
+        t_arc_pair += time_op(arc_step, 1)
+    ms_arc_step = t_arc_pair
     assert (nv.device_status(qy.workspace) == nv.OK and nv.device_status(qa.workspace) == nv.OK
             and nv.device_status(gws) == nv.OK)
+    ms_plain_pair = _max_over_ranks(world, statistics.mean(t_plain_pair), device)
     ms_qout = _max_over_ranks(world, statistics.mean(ms_qout), device)
     ms_arc_q = _max_over_ranks(world, statistics.mean(ms_arc_q), device)
     ms_arc_step = _max_over_ranks(world, statistics.mean(ms_arc_step), device)
     del qy, qa, qw_arc, y_arc
+    bclocks.__exit__(None, None, None)
 
     ms_step = _max_over_ranks(world, statistics.mean(steps_ms), device)
     ms_two_calls = _max_over_ranks(world, statistics.mean(a + b for a, b in zip(tq, tg)), device)
@@ -439,8 +450,10 @@ def run_ours(args, world, rank, local):
             "gemm_nvfp4_out_frac_fp4_peak": round(flops / (ms_qout * 1e-3) / 1e12 / fp4_peak, 4),
             "ms_quantize_arc_S128": round(ms_arc_q, 4),
             "ms_step_arc_S128": round(ms_arc_step, 4),
-            "arc_step_overhead_vs_step": round(ms_arc_step / ms_step - 1.0, 4),
+            "ms_step_beside_arc": round(ms_plain_pair, 4),
+            "arc_step_overhead_vs_step": round(ms_arc_step / ms_plain_pair - 1.0, 4),
         },
+        "clocks_breakdown": bclocks.summary(),
         "stats": {
             "what": "per-step CUDA-event times of this rank (rank 0), ms",
             "ms_per_step": spread(steps_ms),

@@ -300,6 +300,29 @@ NVFP4_API nvfp4_status nvfp4_quantize_gemm(const void* x, int64_t M, int64_t K, 
                                            int64_t ldy, int out_dtype, void* workspace, size_t workspace_bytes,
                                            void* stream);
 
+/* The augmented-channel W4A4 linear layer in one call (ARCQuant page, "방법론":
+ * reorder + dual quantization, then one NVFP4 GEMM over K + S): quantize x
+ * [M, K] as nvfp4_quantize_arc does with augment = 0 (into x_codes
+ * [M, (K+S)/2], x_scales nvfp4_scales_bytes(M, K + S), *x_global_scale, with
+ * x_workspace of nvfp4_quantize_workspace_bytes(M, K)), then
+ * Y [M, N] = X_aug . W_aug^T as nvfp4_gemm does over K + S, against a weight
+ * already quantized by nvfp4_quantize_arc with the same perm and S and
+ * augment = 1 (w_codes / w_scales / w_global, N rows, K + S columns).
+ * Enqueues the GEMM's status reset, the amax pass, the augmented quantize
+ * kernel and the GEMM kernel, each kernel a programmatic dependent of the one
+ * before it.  Results are those of the two calls made one after the other, bit
+ * for bit.  Arguments and requirements are those of nvfp4_quantize_arc and
+ * nvfp4_gemm (with K + S for the GEMM); every one is checked before anything
+ * is enqueued.  Device status: x_workspace as nvfp4_quantize_arc, workspace as
+ * nvfp4_gemm. */
+NVFP4_API nvfp4_status nvfp4_quantize_arc_gemm(const void* x, int64_t M, int64_t K, int64_t ldx,
+                                               const int32_t* perm, int64_t S, int mode, int rule, float fp8_max,
+                                               void* x_codes, void* x_scales, float* x_global_scale,
+                                               void* x_workspace, size_t x_workspace_bytes, const void* w_codes,
+                                               const void* w_scales, const float* w_global, int64_t N, void* y,
+                                               int64_t ldy, int out_dtype, void* workspace,
+                                               size_t workspace_bytes, void* stream);
+
 /* Synchronizes `stream`, then returns the status word the last call that used
  * `workspace` wrote (NVFP4_OK, NVFP4_ERR_INVALID_ARG, NVFP4_ERR_NONFINITE or
  * NVFP4_ERR_TIMEOUT), or

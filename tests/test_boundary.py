@@ -250,3 +250,34 @@ def test_quantize_gemm_without_gpu_fails_loudly():
     if torch.cuda.is_available():
         pytest.skip("a GPU is present")
     assert _qg() in (nv.ERR_CUDA, nv.ERR_UNSUPPORTED_DEVICE)
+
+
+def _qag(**kw):
+    args = dict(x=FAKE, M=64, K=512, ldx=512, perm=FAKE, S=128, mode=1, rule=2, fp8_max=256.0, x_codes=FAKE,
+                x_scales=FAKE, x_global_scale=FAKE, x_workspace=FAKE, x_workspace_bytes=1 << 20, w_codes=FAKE,
+                w_scales=FAKE, w_global=FAKE, N=256, y=FAKE, ldy=256, out_dtype=0, workspace=FAKE,
+                workspace_bytes=64, stream=None)
+    args.update(kw)
+    return nv.nvfp4_quantize_arc_gemm(*args.values())
+
+
+@pytest.mark.parametrize("bad", [
+    # the augmented quantize half
+    dict(x=None), dict(perm=None), dict(perm=FAKE + 2), dict(S=32), dict(S=576), dict(S=-64), dict(M=0),
+    dict(K=96), dict(K=16448, ldx=16448), dict(ldx=256), dict(mode=2), dict(rule=5), dict(fp8_max=100.0),
+    dict(x_workspace_bytes=16), dict(x_codes=None),
+    # the GEMM half (over K + S)
+    dict(w_codes=None), dict(w_global=None), dict(y=None), dict(N=0), dict(ldy=128), dict(out_dtype=3),
+    dict(workspace_bytes=4),
+])
+def test_quantize_arc_gemm_rejects_bad_arguments(bad):
+    assert _qag(**bad) == nv.ERR_INVALID_ARG
+    assert nv.last_error_message().startswith("nvfp4_quantize_arc_gemm")
+
+
+def test_quantize_arc_gemm_without_gpu_fails_loudly():
+    import torch
+
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    assert _qag() in (nv.ERR_CUDA, nv.ERR_UNSUPPORTED_DEVICE)

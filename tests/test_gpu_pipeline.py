@@ -75,3 +75,30 @@ def test_quantize_gemm_in_a_cuda_graph():
     qx_ref = nv.quantize(x, "four_over_six", "mse", 256.0)
     assert torch.equal(y, nv.gemm(qx_ref, qw, out_dtype=torch.bfloat16))
     del g
+
+
+@pytest.mark.parametrize("M,K,N,S,recipe", [(64, 512, 256, 64, ("four_over_six", "mse", 256.0)),
+                                           (300, 1024, 384, 128, ("six", "max", 448.0)),
+                                           (1000, 5120, 640, 128, ("four_over_six", "mae", 256.0))],
+                         ids=lambda v: str(v))
+def test_quantize_arc_gemm_equals_the_two_calls(M, K, N, S, recipe):
+    """nvfp4_quantize_arc_gemm: the augmented quantizer and the GEMM over K + S
+    in one call give the bytes and the Y of nvfp4_quantize_arc (residual)
+    followed by nvfp4_gemm, and the augmented operand is the oracle's."""
+    mode, rule, F = recipe
+    x = workloads.small_operand(M, K, seed=M + S).make().cuda()
+    w = workloads.small_operand(N, K, seed=M + S + 1, kind="normal").make().cuda()
+    perm = x.float().abs().amax(dim=0).argsort(descending=True).to(torch.int32)
+    qw = nv.quantize_arc(w, perm, S, nv.AUG_DUPLICATE, "six", "max", 448.0)
+    qx_ref = nv.quantize_arc(x, perm, S, nv.AUG_RESIDUAL, mode, rule, F)
+    y_ref = nv.gemm(qx_ref, qw, out_dtype=torch.bfloat16)
+    ws = torch.zeros(nv.nvfp4_gemm_workspace_bytes(), dtype=torch.uint8, device="cuda")
+    qx, y = nv.quantize_arc_gemm(x, perm, S, qw, mode, rule, F, out_dtype=torch.bfloat16, workspace=ws)
+    torch.cuda.synchronize()
+    assert nv.device_status(qx.workspace) == nv.OK and nv.device_status(ws) == nv.OK
+    assert torch.equal(qx.codes, qx_ref.codes) and torch.equal(qx.scales, qx_ref.scales)
+    assert torch.equal(qx.global_scale, qx_ref.global_scale)
+    assert torch.equal(y, y_ref)
+    codes, scales, alpha = oracle.quantize_arc(x.cpu(), perm.cpu().numpy(), S, oracle.AUG_RESIDUAL, MODE[mode],
+                                               RULE[rule], F)
+    assert np.array_equal(to_np(qx.codes), codes)

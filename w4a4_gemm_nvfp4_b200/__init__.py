@@ -17,7 +17,8 @@ B global scale per output-column segment (fused projections);
 output scale.
 ``quantize_gemm`` -- the linear layer in one call: quantize the activations,
 then the GEMM against a pre-quantized weight, each kernel starting as a
-programmatic dependent of the one before it.
+programmatic dependent of the one before it; ``quantize_arc_gemm`` the same
+with the augmented-channel quantizer and a GEMM over K + S.
 
 All of it runs in libnvfp4.so (CUDA, built in-tree by ``build.py``); this
 package is a ctypes binding around its C ABI (``include/nvfp4.h``).
@@ -29,4 +30,5 @@ from ._lib import (  # noqa: F401
     last_error_message, load, nvfp4_codes_bytes, nvfp4_gemm, nvfp4_gemm_workspace_bytes,
     nvfp4_get_device_status, nvfp4_quantize, nvfp4_quantize_noalloc, nvfp4_quantize_with_scale,
     nvfp4_quantize_workspace_bytes, nvfp4_scales_bytes,
-    quantize, quantize_t, nvfp4_quantize_t, quantize_gemm, nvfp4_quantize_gemm, quantize_arc, nvfp4_quantize_arc, AUG_RESIDUAL, AUG_DUPLICATE, status_string, testing_set_gemm_wait)
+    quantize, quantize_t, nvfp4_quantize_t, quantize_gemm, nvfp4_quantize_gemm, quantize_arc_gemm,
+    nvfp4_quantize_arc_gemm, quantize_arc, nvfp4_quantize_arc, AUG_RESIDUAL, AUG_DUPLICATE, status_string, testing_set_gemm_wait)

@@ -875,6 +875,33 @@ nvfp4_status nvfp4_quantize_gemm(const void* x, int64_t M, int64_t K, int64_t ld
   return gemm_enqueue(L, s, false, true);
 }
 
+nvfp4_status nvfp4_quantize_arc_gemm(const void* x, int64_t M, int64_t K, int64_t ldx, const int32_t* perm,
+                                     int64_t S, int mode, int rule, float fp8_max, void* x_codes, void* x_scales,
+                                     float* x_global_scale, void* x_workspace, size_t x_workspace_bytes,
+                                     const void* w_codes, const void* w_scales, const float* w_global, int64_t N,
+                                     void* y, int64_t ldy, int out_dtype, void* workspace, size_t workspace_bytes,
+                                     void* stream) {
+  const char* fn = "nvfp4_quantize_arc_gemm";
+  nvfp4_status st = quantize_arc_check(fn, x, M, K, ldx, perm, S, 0, mode, rule, fp8_max, x_codes, x_scales,
+                                       x_global_scale, x_workspace, x_workspace_bytes);
+  if (st != NVFP4_OK) return st;
+  GemmLaunch L;
+  const int64_t end = N;
+  if ((st = gemm_prepare(&L, fn, x_codes, x_scales, x_global_scale, w_codes, w_scales, w_global, &end, 1, M, N,
+                         K + S, y, ldy, out_dtype, workspace, workspace_bytes, 0, nullptr, nullptr, nullptr)) !=
+      NVFP4_OK)
+    return st;
+  // as in nvfp4_quantize_gemm: the status reset first, then the quantizer's
+  // kernels and the GEMM back to back, each a programmatic dependent
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemsetAsync(workspace, 0, sizeof(WorkspaceHeader), s);
+  if (e != cudaSuccess) return cuda_status(e, "cudaMemsetAsync(status)");
+  if ((st = quantize_arc_enqueue(fn, x, M, K, ldx, perm, S, 0, mode, rule, fp8_max, x_codes, x_scales,
+                                 x_global_scale, x_workspace, x_workspace_bytes, stream)) != NVFP4_OK)
+    return st;
+  return gemm_enqueue(L, s, false, true);
+}
+
 nvfp4_status nvfp4_gemm_segmented(const void* a_codes, const void* a_scales, const float* a_global,
                                   const void* b_codes, const void* b_scales, const float* b_globals,
                                   const int64_t* seg_ends, int nseg, int64_t M, int64_t N, int64_t K,

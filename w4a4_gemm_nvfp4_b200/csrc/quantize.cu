@@ -45,10 +45,10 @@ constexpr int kMaxPartials = 4096;
 constexpr int kArcMaxRows = 4;              // rows per step of the augmented quantizer, at most
 constexpr int kArcPrimThreads = 256;        // its threads for the primary blocks, at most
 constexpr int kArcMaxThreads = 640;         // its block size, at most
-constexpr int kArcBufs = 3;                 // its row buffers
+constexpr int kArcMaxBufs = 3;              // its row buffers: 3, or 2 for the widest rows
 constexpr int64_t kArcSmemStep = 73728;     // shared memory it aims at: three CTAs per SM up to 5K channels
 constexpr int64_t kArcMaxK = 16384;         // channels of x it takes, at most
-constexpr int64_t kArcSmemBudget = 2 * 16384 * (1 + kArcBufs);  // its shared memory, at most: 2 bytes x K x (1 + 3 x rows per step)
+constexpr int64_t kArcSmemBudget = 98304;   // its shared memory, at most: 2 bytes x K x (1 + buffers x rows per step)
 constexpr int kQuantThreads = 256;
 constexpr int kQuantWarps = kQuantThreads / 32;
 
@@ -124,6 +124,7 @@ struct QuantParams {
   int augment = 0;                // 0: residual of the first S reordered channels, 1: their copy
   int arc_rows = 1;               // rows per step of the augmented quantizer
   int arc_prim_threads = 128;     // its threads for the primary blocks; the rest take the appended ones
+  int arc_bufs = 3;               // its row buffers
 };
 
 // Start of every quantize kernel: alpha (a caller-supplied static scale, or
@@ -424,10 +425,11 @@ __global__ void __launch_bounds__(kQuantThreads)
 // permutation (as byte offsets into a row) and the rows sit in shared memory,
 // so the channel gather reads shared memory only.  Each CTA takes p.arc_rows
 // rows per step (2 for K up to about 5K channels, 1 for wider rows) through
-// kArcBufs row buffers: the CTA's last warp is the producer, which fills
-// buffer s % kArcBufs for step s with one bulk copy per row once every
+// p.arc_bufs row buffers (3; 2 above 9K channels, so that two CTAs still fit
+// on an SM): the CTA's last warp is the producer, which fills buffer
+// s % p.arc_bufs for step s with one bulk copy per row once every
 // consumer warp has released it (mbarriers full[] and consumed[]), so the
-// consumers run up to kArcBufs - 1 steps ahead of the slowest of them with no
+// consumers run up to p.arc_bufs - 1 steps ahead of the slowest of them with no
 // CTA-wide barrier.  Of the consumer threads, the first P own the primary
 // block columns t, t + P, ...: a thread reads a column's 16 channel offsets
 // once per step and gathers that block from each of the step's rows with
@@ -444,7 +446,7 @@ __global__ void __launch_bounds__(kArcMaxThreads)
     quantize_arc_kernel(const QuantParams p) {
   BlockConsts k;
   __shared__ ScaleEntry s_dr[128];
-  extern __shared__ __align__(16) uint16_t s_dyn[];  // [K] channel byte offsets, then kArcBufs x [arc_rows][K] rows
+  extern __shared__ __align__(16) uint16_t s_dyn[];  // [K] channel byte offsets, then arc_bufs x [arc_rows][K] rows
   if (!quant_prologue(p, k, s_dr)) return;
 
   const int64_t K = p.K, KA = p.K + p.S;
@@ -461,15 +463,16 @@ __global__ void __launch_bounds__(kArcMaxThreads)
   const uint32_t row_bytes = static_cast<uint32_t>(K) * 2, buf_bytes = row_bytes * R;
   // Buffers: full[b] completes when buffer b holds its step's rows (the
   // producer's arrival plus the copies' bytes); consumed[b] when every
-  // consumer warp is done with it.  Step s uses buffer s % kArcBufs; its
-  // waits are on phase s / kArcBufs of those barriers.
-  __shared__ __align__(8) uint64_t s_bar[2 * kArcBufs];
+  // consumer warp is done with it.  Step s uses buffer s % NB; its waits are
+  // on phase s / NB of those barriers.
+  const int NB = p.arc_bufs;
+  __shared__ __align__(8) uint64_t s_bar[2 * kArcMaxBufs];
   __shared__ int s_abort;
-  const uint32_t full0 = smem_u32(&s_bar[0]), consumed0 = smem_u32(&s_bar[kArcBufs]);
+  const uint32_t full0 = smem_u32(&s_bar[0]), consumed0 = smem_u32(&s_bar[kArcMaxBufs]);
   const int warp = static_cast<int>(threadIdx.x >> 5), lane = static_cast<int>(threadIdx.x & 31);
   const int producer_warp = T / 32 - 1;
   if (threadIdx.x == 0) {
-    for (int b = 0; b < kArcBufs; ++b) {
+    for (int b = 0; b < NB; ++b) {
       mbar_init(full0 + 8 * b, 1);
       mbar_init(consumed0 + 8 * b, producer_warp);  // one arrival per consumer warp
     }
@@ -491,9 +494,8 @@ __global__ void __launch_bounds__(kArcMaxThreads)
     // ------------------------------------------------------- producer ----
     int s = 0;
     for (int64_t row0 = static_cast<int64_t>(blockIdx.x) * R; row0 < rows_padded; row0 += stride_rows, ++s) {
-      const int b = s % kArcBufs;
-      if (s >= kArcBufs &&
-          !__all_sync(0xffffffffu, mbar_wait_bounded(consumed0 + 8 * b, (s / kArcBufs - 1) & 1, abort, kWaitNs))) {
+      const int b = s % NB;
+      if (s >= NB && !__all_sync(0xffffffffu, mbar_wait_bounded(consumed0 + 8 * b, (s / NB - 1) & 1, abort, kWaitNs))) {
         if (lane == 0) fail(1);
         break;
       }
@@ -510,8 +512,8 @@ __global__ void __launch_bounds__(kArcMaxThreads)
     if (*abort && lane == 0) {
       // let the copies already issued land before the CTA can exit
       const volatile int no_abort = 0;
-      for (int k = s >= kArcBufs ? s - kArcBufs : 0; k < s; ++k)
-        mbar_wait_bounded(full0 + 8 * (k % kArcBufs), (k / kArcBufs) & 1, &no_abort, 100000000ull);
+      for (int k = s >= NB ? s - NB : 0; k < s; ++k)
+        mbar_wait_bounded(full0 + 8 * (k % NB), (k / NB) & 1, &no_abort, 100000000ull);
     }
     return;
   }
@@ -522,8 +524,8 @@ __global__ void __launch_bounds__(kArcMaxThreads)
   };
   int s = 0;
   for (int64_t row0 = static_cast<int64_t>(blockIdx.x) * R; row0 < rows_padded; row0 += stride_rows, ++s) {
-    const int b = s % kArcBufs;
-    if (!__all_sync(0xffffffffu, mbar_wait_bounded(full0 + 8 * b, (s / kArcBufs) & 1, abort, kWaitNs))) {
+    const int b = s % NB;
+    if (!__all_sync(0xffffffffu, mbar_wait_bounded(full0 + 8 * b, (s / NB) & 1, abort, kWaitNs))) {
       if (lane == 0) fail(2);
       break;
     }
@@ -626,19 +628,21 @@ int arc_threads(int64_t K, int64_t S, int R) {
   return static_cast<int>(std::max<int64_t>(96, prim + res)) + 32;  // + the producer warp
 }
 
-// Rows per step of the augmented quantizer for K channels: the most (up to 4,
-// a power of two so it divides the 128-row padding) whose permutation and
-// kArcBufs row buffers fit kArcSmemStep (at least one row: K <= 16384 keeps
-// that within kArcSmemBudget).
+// Rows per step and row buffers of the augmented quantizer for K channels:
+// three buffers of the most rows (up to 4, a power of two so it divides the
+// 128-row padding) that fit kArcSmemStep with the permutation; above 9K
+// channels, where even one row per buffer does not, two buffers of one row
+// (within kArcSmemBudget for K <= 16384), so that two CTAs still share an SM.
 int arc_rows_per_step(int64_t K) {
   int r = kArcMaxRows;
-  while (r > 1 && 2 * K * (1 + kArcBufs * r) > kArcSmemStep) r /= 2;
+  while (r > 1 && 2 * K * (1 + kArcMaxBufs * r) > kArcSmemStep) r /= 2;
   return r;
 }
+int arc_buffers(int64_t K) { return 2 * K * (1 + kArcMaxBufs) > kArcSmemStep ? 2 : kArcMaxBufs; }
 
 template <bool F, int R>
 cudaError_t launch_quantize_arc(int dev, int sms, const QuantParams& p, cudaStream_t s, bool pdl) {
-  const size_t smem = static_cast<size_t>(p.K) * 2 * (1 + kArcBufs * p.arc_rows);
+  const size_t smem = static_cast<size_t>(p.K) * 2 * (1 + p.arc_bufs * p.arc_rows);
   // the shared-memory opt-in is an attribute of the kernel in this context
   static PerContextCache<int> attr;
   int done = 0;
@@ -879,6 +883,7 @@ nvfp4_status quantize_impl(const char* fn, QuantKind kind, const void* x, int64_
   if (kind == QuantKind::kAugmented) {
     p.arc_rows = arc_rows_per_step(K);
     p.arc_prim_threads = arc_prim_threads(K);
+    p.arc_bufs = arc_buffers(K);
   }
   const int amax_grid = std::min(amax_grid_size(rows, K, ldx, sms), kMaxPartials);
   return launch_dynamic(kind, p, mode, rule, fp8_max, global_scale, partials, amax_grid, dev, sms,
@@ -894,6 +899,22 @@ nvfp4_status quantize_rows_check(const char* fn, const void* x, int64_t rows, in
                                  const float* global_scale, const void* workspace, size_t workspace_bytes) {
   return check_quantize_call(fn, QuantKind::kRows, x, rows, K, ldx, mode, rule, fp8_max, codes, scales,
                              global_scale, workspace, workspace_bytes, nullptr, 0, 0);
+}
+
+nvfp4_status quantize_arc_check(const char* fn, const void* x, int64_t rows, int64_t K, int64_t ldx,
+                                const int32_t* perm, int64_t S, int augment, int mode, int rule, float fp8_max,
+                                const void* codes, const void* scales, const float* global_scale,
+                                const void* workspace, size_t workspace_bytes) {
+  return check_quantize_call(fn, QuantKind::kAugmented, x, rows, K, ldx, mode, rule, fp8_max, codes, scales,
+                             global_scale, workspace, workspace_bytes, perm, S, augment);
+}
+
+nvfp4_status quantize_arc_enqueue(const char* fn, const void* x, int64_t rows, int64_t K, int64_t ldx,
+                                  const int32_t* perm, int64_t S, int augment, int mode, int rule, float fp8_max,
+                                  void* codes, void* scales, float* global_scale, void* workspace,
+                                  size_t workspace_bytes, void* stream) {
+  return quantize_impl(fn, QuantKind::kAugmented, x, rows, K, ldx, mode, rule, fp8_max, codes, scales,
+                       global_scale, workspace, workspace_bytes, stream, perm, S, augment);
 }
 
 nvfp4_status quantize_rows_enqueue(const char* fn, const void* x, int64_t rows, int64_t K, int64_t ldx, int mode,
