@@ -346,6 +346,11 @@ def run_ours(args, world, rank, local):
     torch.cuda.synchronize()
     ms_qout = time_op(lambda: nv.gemm_quantized(qx, qw, y_alpha, "four_over_six", "mse", out=qy), args.steps)
     ms_arc_q = time_op(lambda: nv.quantize_arc(x, perm, S_ARC, nv.AUG_RESIDUAL, xm, xr, xF, out=qa), args.steps)
+    # the same with the activations' RMSNorm fused ahead (seeded gains near 1)
+    gains = (1.0 + 0.25 * torch.randn(K, generator=torch.Generator().manual_seed(7))).to(torch.bfloat16).to(device)
+    qn = nv.quantize_arc_rmsnorm(x, gains, 1e-6, perm, S_ARC, xm, xr, xF)
+    ms_arc_norm = time_op(lambda: nv.quantize_arc_rmsnorm(x, gains, 1e-6, perm, S_ARC, xm, xr, xF, out=qn),
+                          args.steps)
 
     def arc_step():  # the augmented layer in one call, as the headline step is
         nv.quantize_arc_gemm(x, perm, S_ARC, qw_arc, xm, xr, xF, out_dtype=torch.bfloat16, x_out=qa, out=y_arc,
@@ -359,12 +364,13 @@ def run_ours(args, world, rank, local):
         t_arc_pair += time_op(arc_step, 1)
     ms_arc_step = t_arc_pair
     assert (nv.device_status(qy.workspace) == nv.OK and nv.device_status(qa.workspace) == nv.OK
-            and nv.device_status(gws) == nv.OK)
+            and nv.device_status(qn.workspace) == nv.OK and nv.device_status(gws) == nv.OK)
     ms_plain_pair = _max_over_ranks(world, statistics.mean(t_plain_pair), device)
     ms_qout = _max_over_ranks(world, statistics.mean(ms_qout), device)
     ms_arc_q = _max_over_ranks(world, statistics.mean(ms_arc_q), device)
+    ms_arc_norm = _max_over_ranks(world, statistics.mean(ms_arc_norm), device)
     ms_arc_step = _max_over_ranks(world, statistics.mean(ms_arc_step), device)
-    del qy, qa, qw_arc, y_arc
+    del qy, qa, qn, qw_arc, y_arc
     bclocks.__exit__(None, None, None)
 
     ms_step = _max_over_ranks(world, statistics.mean(steps_ms), device)
@@ -373,20 +379,51 @@ def run_ours(args, world, rank, local):
     ms_gemm = _max_over_ranks(world, statistics.mean(tg), device)
     ms_quant6 = _max_over_ranks(world, statistics.mean(tq6), device)
 
-    # end to end through the public API with host buffers: pinned X in, Y out
-    y_host = torch.empty(M, N, dtype=torch.bfloat16, pin_memory=True)
-    e2e_steps = max(1, min(args.steps, 5))
+    # end to end through the public API with host buffers: every step copies
+    # its X in from pinned host memory and its Y back out.  Two steps are in
+    # flight, each with its own device X and Y: the copies in, the one-call
+    # layer and the copies out run on three streams, so one step's copies
+    # overlap the other's compute and the two copy directions overlap each
+    # other (PCIe is full duplex).
+    slots = 2
+    x_dev = [x] + [torch.empty_like(x) for _ in range(slots - 1)]
+    y_dev = [y] + [torch.empty_like(y) for _ in range(slots - 1)]
+    y_host = [torch.empty(M, N, dtype=torch.bfloat16, pin_memory=True) for _ in range(slots)]
+    s_in, s_out = torch.cuda.Stream(device), torch.cuda.Stream(device)
+    ev_in = [torch.cuda.Event() for _ in range(slots)]
+    ev_done = [torch.cuda.Event() for _ in range(slots)]
+    ev_out = [torch.cuda.Event() for _ in range(slots)]
+    e2e_steps = max(1, min(args.steps, 8))
     _barrier(world)
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    for _ in range(e2e_steps):
-        x.copy_(x_host, non_blocking=True)
-        fused_step()
-        y_host.copy_(y, non_blocking=True)
+    s_in.wait_stream(stream)
+    s_out.wait_stream(stream)
+    for i in range(e2e_steps):
+        k = i % slots
+        with torch.cuda.stream(s_in):
+            if i >= slots:
+                s_in.wait_event(ev_done[k])          # the slot's last compute has read its X
+            x_dev[k].copy_(x_host, non_blocking=True)
+            ev_in[k].record(s_in)
+        stream.wait_event(ev_in[k])
+        if i >= slots:
+            stream.wait_event(ev_out[k])             # the slot's last Y has been copied out
+        nv.quantize_gemm(x_dev[k], qw, xm, xr, xF, out_dtype=torch.bfloat16, x_out=qx, out=y_dev[k],
+                         workspace=gws)
+        ev_done[k].record(stream)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(ev_done[k])
+            y_host[k].copy_(y_dev[k], non_blocking=True)
+            ev_out[k].record(s_out)
+    stream.wait_stream(s_in)
+    stream.wait_stream(s_out)
     e1.record(stream)
     torch.cuda.synchronize()
+    assert nv.device_status(qx.workspace) == nv.OK and nv.device_status(gws) == nv.OK
     ms_e2e = _max_over_ranks(world, e0.elapsed_time(e1) / e2e_steps, device)
+    del x_dev, y_dev, y_host
 
     flops = 2.0 * M * N * K
     peaks = _peaks()
@@ -449,6 +486,7 @@ def run_ours(args, world, rank, local):
             "gemm_nvfp4_out_TFLOPs": round(flops / (ms_qout * 1e-3) / 1e12, 1),
             "gemm_nvfp4_out_frac_fp4_peak": round(flops / (ms_qout * 1e-3) / 1e12 / fp4_peak, 4),
             "ms_quantize_arc_S128": round(ms_arc_q, 4),
+            "ms_quantize_arc_rmsnorm_S128": round(ms_arc_norm, 4),
             "ms_step_arc_S128": round(ms_arc_step, 4),
             "ms_step_beside_arc": round(ms_plain_pair, 4),
             "arc_step_overhead_vs_step": round(ms_arc_step / ms_plain_pair - 1.0, 4),
@@ -468,6 +506,8 @@ def run_ours(args, world, rank, local):
             "h2d_bytes_per_step": M * K * 2,
             "d2h_bytes_per_step": M * N * 2,
             "ms_per_step": round(ms_e2e, 3),
+            "how": f"{e2e_steps} steps, two in flight: X in on one copy stream, the one-call layer, Y out on "
+                   "another (pinned host buffers)",
         },
         "gpu_launches": 3 * args.steps,
         "clocks": clocks.summary(),

@@ -160,6 +160,31 @@ NVFP4_API nvfp4_status nvfp4_quantize_arc(const void* x, int64_t rows, int64_t K
                                           float fp8_max, void* codes, void* scales, float* global_scale,
                                           void* workspace, size_t workspace_bytes, void* stream);
 
+/* nvfp4_quantize_arc with the RMSNorm of the activations fused ahead of it
+ * (ARCQuant page, "방법론", 커널 구현: the fused kernel normalizes, reorders
+ * and quantizes the primary and residual channels): the operand is that of
+ * nvfp4_quantize_arc (augment = 0) applied to the bf16 tensor
+ *   y[i, k] = bf16((x[i, k] * r_i) * gamma[k]),
+ *   r_i = 1 / sqrt(sum_k x[i, k]^2 / K + eps),
+ * every step one binary32 operation, the sum of squares taken as the
+ * contiguous pairwise tree over the row (zero-padded to a power of two), the
+ * square root and the divisions correctly rounded.  alpha is the amax of y.
+ * y is never written: a row pass computes r_i (kept in the workspace) and the
+ * amax partials, and the augmented quantizer normalizes the channels it
+ * gathers.
+ *   gamma   device bf16[K], 16-byte aligned
+ *   eps     a positive finite number
+ *   workspace  nvfp4_quantize_arc_rmsnorm_workspace_bytes(rows, K) bytes
+ * Other arguments and requirements as nvfp4_quantize_arc.  A non-finite y
+ * (from non-finite x, or a product past the bf16 range) sets
+ * NVFP4_ERR_NONFINITE as for nvfp4_quantize.  Two kernel launches. */
+NVFP4_API size_t nvfp4_quantize_arc_rmsnorm_workspace_bytes(int64_t rows, int64_t K);
+NVFP4_API nvfp4_status nvfp4_quantize_arc_rmsnorm(const void* x, int64_t rows, int64_t K, int64_t ldx,
+                                                  const void* gamma, float eps, const int32_t* perm, int64_t S,
+                                                  int mode, int rule, float fp8_max, void* codes, void* scales,
+                                                  float* global_scale, void* workspace, size_t workspace_bytes,
+                                                  void* stream);
+
 /* The NVFP4 operand of x^T: x is the same bf16 [rows, K] matrix as for
  * nvfp4_quantize, but the 16-element blocks run along rows (down a column of
  * x), so codes/scales describe the [K, rows] matrix x^T -- the layout the

@@ -85,6 +85,8 @@ def _load():
                 "or_quantize_arc": (ctypes.c_int, [u16p, i64, i64, i64, ctypes.POINTER(ctypes.c_int32), i64,
                                                    ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_float,
                                                    u8p, u8p, f32p]),
+                "or_rmsnorm_bf16": (ctypes.c_int, [u16p, i64, i64, i64, u16p, ctypes.c_float, u16p]),
+                "or_f32_to_bf16": (ctypes.c_uint16, [ctypes.c_float]),
                 "or_scales_swizzled_bytes": (i64, [i64, i64]),
                 "or_swizzle_scales": (None, [u8p, i64, i64, u8p]),
                 "or_unswizzle_scales": (None, [u8p, i64, i64, u8p]),
@@ -235,6 +237,35 @@ def quantize_arc(x, perm, S: int, augment: int, mode: int, rule: int, fp8_max: f
     if rc != 0:
         raise NonFiniteInput("tensor holds Inf or NaN")
     return codes, scales, float(np.float32(alpha.value))
+
+
+def rmsnorm(x, gamma, eps: float) -> np.ndarray:
+    """RMSNorm of each row of the bf16 tensor x [rows, K] with the bf16 gain
+    gamma [K] (ARCQuant page, 방법론, 커널 구현: normalization fused ahead of
+    the reorder and the dual quantization): y = bf16((x * r) * gamma) with
+    r = 1 / sqrt(pairwise_sum(x^2) / K + eps).  Returns the bf16 bit patterns
+    of y as a uint16 [rows, K] array."""
+    xb = as_bf16_bits(x)
+    gb = as_bf16_bits(gamma).reshape(-1)
+    rows, K = xb.shape
+    assert gb.shape == (K,)
+    y = np.zeros((rows, K), np.uint16)
+    rc = _load().or_rmsnorm_bf16(_ptr(xb, ctypes.c_uint16), rows, K, K, _ptr(np.ascontiguousarray(gb), ctypes.c_uint16),
+                                 float(np.float32(eps)), _ptr(y, ctypes.c_uint16))
+    assert rc == 0
+    return y
+
+
+def f32_to_bf16(v: float) -> int:
+    """bf16 bit pattern of the nearest bf16 to a binary32 value (ties to even)."""
+    return int(_load().or_f32_to_bf16(float(np.float32(v))))
+
+
+def quantize_arc_rmsnorm(x, gamma, eps: float, perm, S: int, mode: int, rule: int, fp8_max: float):
+    """The augmented quantization (residual channels) of rmsnorm(x, gamma,
+    eps): the normalized bf16 rows, reordered, quantized, with S residual
+    channels.  Returns (codes, canonical scales, alpha) like quantize_arc."""
+    return quantize_arc(rmsnorm(x, gamma, eps), perm, S, AUG_RESIDUAL, mode, rule, fp8_max)
 
 
 # ------------------------------------------------------------ scale layout --

@@ -49,6 +49,7 @@
  */
 #include <math.h>
 #include <stdint.h>
+#include <stdlib.h>
 #include <string.h>
 
 #define OR_MODE_SIX 0
@@ -269,6 +270,73 @@ int or_quantize_arc(const uint16_t* x, int64_t rows, int64_t K, int64_t ldx, con
     }
   }
   if (alpha_out) *alpha_out = alpha;
+  return 0;
+}
+
+/* ------------------------------------------------------------- RMSNorm --- */
+
+/* Round a binary32 to bf16: nearest, ties to the even bf16 significand;
+ * values past the bf16 range round to infinity; a NaN stays a (quiet) NaN.
+ * Adding 0x7FFF plus the last kept bit to the bit pattern and truncating is
+ * exactly that rounding on the magnitude (the carry moves into the exponent
+ * when the significand overflows). */
+uint16_t or_f32_to_bf16(float f) {
+  uint32_t u;
+  memcpy(&u, &f, 4);
+  if (isnan(f)) return (uint16_t)((u >> 16) | 0x40u);
+  u += 0x7FFFu + ((u >> 16) & 1u);
+  return (uint16_t)(u >> 16);
+}
+
+/* The contiguous pairwise tree over n terms, padded with zeros to the next
+ * power of two (adding +0 changes no partial sum): (t0+t1),(t2+t3),... then
+ * pairs of those, down to one value. */
+static float pairwise_sum(const float* t, int64_t n) {
+  int64_t p = 1;
+  while (p < n) p *= 2;
+  float* a = (float*)calloc((size_t)p, sizeof(float));
+  if (!a) return NAN;
+  memcpy(a, t, (size_t)n * sizeof(float));
+  for (int64_t m = p; m > 1; m /= 2)
+    for (int64_t i = 0; i < m / 2; ++i) a[i] = a[2 * i] + a[2 * i + 1];
+  const float sum = a[0];
+  free(a);
+  return sum;
+}
+
+/* RMSNorm of each row of a bf16 [rows, K] tensor with a bf16 gain gamma[K]
+ * ([ARC] "방법론", 커널 구현: the fused kernel normalizes the activations before
+ * reordering and quantizing them; the page gives no formula, so this is the
+ * standard RMSNorm):
+ *   ms = (sum_k x_k * x_k) / K    squares exact for finite bf16; the sum
+ *                                 is the contiguous pairwise tree; one IEEE
+ *                                 division by K
+ *   r  = 1 / sqrt(ms + eps)       an IEEE add, a correctly rounded square
+ *                                 root, then an IEEE division
+ *   y_k = bf16((x_k * r) * gamma_k)  two binary32 products, in that order,
+ *                                 rounded to bf16 (the normalized activation
+ *                                 is a bf16 tensor, as the quantizer input is)
+ * y is [rows, K] contiguous.  Returns 0 (eps is the caller's; a zero row with
+ * eps = 0 gives r = inf and NaN outputs). */
+int or_rmsnorm_bf16(const uint16_t* x, int64_t rows, int64_t K, int64_t ldx, const uint16_t* gamma,
+                    float eps, uint16_t* y) {
+  float* t = (float*)malloc((size_t)K * sizeof(float));
+  if (!t) return 1;
+  for (int64_t r = 0; r < rows; ++r) {
+    const uint16_t* row = x + r * ldx;
+    for (int64_t k = 0; k < K; ++k) {
+      const float v = bf16_to_f32(row[k]);
+      t[k] = v * v;
+    }
+    const float ms = pairwise_sum(t, K) / (float)K;
+    const float q = sqrtf(ms + eps);
+    const float rinv = 1.0f / q;
+    for (int64_t k = 0; k < K; ++k) {
+      const float xr = bf16_to_f32(row[k]) * rinv;
+      y[r * K + k] = or_f32_to_bf16(xr * bf16_to_f32(gamma[k]));
+    }
+  }
+  free(t);
   return 0;
 }
 

@@ -204,6 +204,140 @@ def block(x, alpha, rule, **reading):
     return (c4 if pick4 else c6), (s4 if pick4 else s6), pick4, e6, e4
 
 
+# ------------------------------------------------------------ RMSNorm --
+
+def sqrt32(q):
+    """Correctly rounded binary32 square root of a rational q >= 0 (ties to
+    even): the candidate from the float square root, then its neighbours
+    checked against q exactly (midpoint squared vs q)."""
+    q = Fraction(q)
+    assert q >= 0
+    if q == 0:
+        return Fraction(0)
+    guess = rn32(Fraction(math.sqrt(float(q))))
+    import struct
+
+    def step(v, d):
+        b = struct.unpack("<I", struct.pack("<f", float(v)))[0] + d
+        return Fraction(struct.unpack("<f", struct.pack("<I", b))[0])
+
+    v = guess
+    for _ in range(4):  # move to the binary32 value whose rounding interval holds sqrt(q)
+        lo, hi = (v + step(v, -1)) / 2, (v + step(v, 1)) / 2
+        if lo * lo > q:
+            v = step(v, -1)
+        elif hi * hi < q:
+            v = step(v, 1)
+        else:
+            break
+    lo, hi = (v + step(v, -1)) / 2, (v + step(v, 1)) / 2
+    assert lo * lo <= q <= hi * hi
+    if lo * lo == q or hi * hi == q:  # a tie: the even significand
+        other = step(v, -1) if lo * lo == q else step(v, 1)
+        bits = struct.unpack("<I", struct.pack("<f", float(v)))[0]
+        return v if bits % 2 == 0 else other
+    return v
+
+
+def bf16_rne(q):
+    """Nearest bf16 (8-bit significand, binary32's exponent range) of a
+    rational, ties to the even significand, overflow to +-INF; returned as a
+    Fraction (or +-INF)."""
+    q = Fraction(q)
+    if q == 0:
+        return Fraction(0)
+    neg = q < 0
+    a = -q if neg else q
+    e = max(_floor_log2(a), _MIN_EXP)
+    ulp = Fraction(2) ** (e - 7)
+    n = a / ulp
+    k = n.numerator // n.denominator
+    rem = n - k
+    if rem > Fraction(1, 2) or (rem == Fraction(1, 2) and k % 2 == 1):
+        k += 1
+    r = k * ulp
+    if r >= Fraction(2) ** 128:
+        return -INF if neg else INF
+    return -r if neg else r
+
+
+def pairwise_sum(t):
+    """Contiguous pairwise tree over len(t) terms zero-padded to a power of
+    two, each add rounded."""
+    a = list(t)
+    p = 1
+    while p < len(a):
+        p *= 2
+    a += [Fraction(0)] * (p - len(a))
+    while len(a) > 1:
+        a = [rn32(a[2 * i] + a[2 * i + 1]) for i in range(len(a) // 2)]
+    return a[0]
+
+
+def rmsnorm_row(x, gamma, eps, *, summation="pairwise", mean="divide", rsqrt="sqrt_then_divide",
+                order="x_r_then_gamma"):
+    """One row of RMSNorm with every step rounded to binary32, y rounded to
+    bf16.  x, gamma: lists of bf16 values as Fractions; eps a binary32 value.
+    The keywords select the reading of the steps the pages leave open; the
+    defaults are this library's:
+      summation  'pairwise' (contiguous tree) | 'sequential'
+      mean       'divide': fl(s / K)          | 'reciprocal': fl(s * fl(1/K))
+      rsqrt      'sqrt_then_divide': fl(1 / fl(sqrt(d)))
+                 | 'rsqrt': the correctly rounded 1/sqrt(d)
+      order      'x_r_then_gamma': fl(fl(x*r)*g) | 'r_gamma_first': fl(x*fl(r*g))"""
+    r = rms_scale(x, eps, summation=summation, mean=mean, rsqrt=rsqrt)
+    return [rms_out(v, r, g, order=order) for v, g in zip(x, gamma)]
+
+
+def rms_scale(x, eps, *, summation="pairwise", mean="divide", rsqrt="sqrt_then_divide"):
+    """The row's factor r = 1 / sqrt(mean(x^2) + eps) under the readings of
+    rmsnorm_row."""
+    K = len(x)
+    t = [rn32(v * v) for v in x]
+    s = pairwise_sum(t) if summation == "pairwise" else _seq(t)
+    ms = rn32(s / K) if mean == "divide" else rn32(s * rn32(Fraction(1, K)))
+    d = rn32(ms + eps)
+    return rn32(1 / sqrt32(d)) if rsqrt == "sqrt_then_divide" else _rsqrt32(d)
+
+
+def rms_out(v, r, g, *, order="x_r_then_gamma"):
+    """One output element bf16((v * r) * g) under the product-order reading."""
+    if order == "x_r_then_gamma":
+        return bf16_rne(rn32(rn32(v * r) * g))
+    return bf16_rne(rn32(v * rn32(r * g)))
+
+
+def _seq(t):
+    s = t[0]
+    for v in t[1:]:
+        s = rn32(s + v)
+    return s
+
+
+def _rsqrt32(d):
+    """Correctly rounded binary32 1/sqrt(d), d > 0: the binary32 value v whose
+    rounding interval holds 1/sqrt(d), i.e. lo <= 1/sqrt(d) <= hi, checked as
+    lo^2 * d <= 1 <= hi^2 * d."""
+    import struct
+
+    def step(v, k):
+        b = struct.unpack("<I", struct.pack("<f", float(v)))[0] + k
+        return Fraction(struct.unpack("<f", struct.pack("<I", b))[0])
+
+    v = rn32(Fraction(1 / math.sqrt(float(d))))
+    for _ in range(4):
+        lo, hi = (v + step(v, -1)) / 2, (v + step(v, 1)) / 2
+        if lo * lo * d > 1:
+            v = step(v, -1)
+        elif hi * hi * d < 1:
+            v = step(v, 1)
+        else:
+            break
+    lo, hi = (v + step(v, -1)) / 2, (v + step(v, 1)) / 2
+    assert lo * lo * d <= 1 <= hi * hi * d
+    return v
+
+
 def float_hex(q) -> str:
     """binary32 value as a C99 hex float (exact)."""
     return float(q).hex() if q not in (INF, -INF) else ("inf" if q > 0 else "-inf")

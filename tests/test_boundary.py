@@ -281,3 +281,35 @@ def test_quantize_arc_gemm_without_gpu_fails_loudly():
     if torch.cuda.is_available():
         pytest.skip("a GPU is present")
     assert _qag() in (nv.ERR_CUDA, nv.ERR_UNSUPPORTED_DEVICE)
+
+
+def _qar(**kw):
+    args = dict(x=FAKE, rows=64, K=512, ldx=512, gamma=FAKE, eps=1e-6, perm=FAKE, S=128, mode=1, rule=2,
+                fp8_max=256.0, codes=FAKE, scales=FAKE, global_scale=FAKE, workspace=FAKE,
+                workspace_bytes=1 << 20, stream=None)
+    args.update(kw)
+    return nv.nvfp4_quantize_arc_rmsnorm(*args.values())
+
+
+@pytest.mark.parametrize("bad", [
+    dict(gamma=None), dict(gamma=FAKE + 1), dict(gamma=FAKE + 8), dict(eps=0.0), dict(eps=-1e-6), dict(eps=float("inf")),
+    dict(eps=float("nan")), dict(x=None), dict(perm=None), dict(S=32), dict(S=576), dict(K=96),
+    dict(K=16448, ldx=16448), dict(mode=2), dict(fp8_max=100.0), dict(workspace=None),
+    dict(workspace_bytes=16), dict(rows=4096, workspace_bytes=16448 + 4 * 4096 - 1),
+])
+def test_quantize_arc_rmsnorm_rejects_bad_arguments(bad):
+    assert _qar(**bad) == nv.ERR_INVALID_ARG
+    assert nv.last_error_message().startswith("nvfp4_quantize_arc_rmsnorm")
+
+
+def test_quantize_arc_rmsnorm_workspace_holds_a_float_per_row():
+    assert (nv.nvfp4_quantize_arc_rmsnorm_workspace_bytes(4096, 512)
+            == nv.nvfp4_quantize_workspace_bytes(4096, 512) + 4 * 4096)
+
+
+def test_quantize_arc_rmsnorm_without_gpu_fails_loudly():
+    import torch
+
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    assert _qar() in (nv.ERR_CUDA, nv.ERR_UNSUPPORTED_DEVICE)

@@ -95,3 +95,89 @@ def test_augmented_gemm_matches_oracle_and_beats_plain():
     err_aug = np.abs(y - exact).mean()
     err_plain = np.abs(plain - exact).mean()
     assert err_aug < err_plain, (err_aug, err_plain)
+
+
+# ------------------------------------------------- RMSNorm fused ahead --
+
+def _gains(K, seed):
+    g = torch.Generator().manual_seed(seed)
+    return (1.0 + 0.25 * torch.randn(K, generator=g)).to(torch.bfloat16)
+
+
+def gpu_arc_rmsnorm(x_cpu, gamma, eps, perm, S, mode, rule, F, canary=0xA5):
+    rows, K = x_cpu.shape
+    KA = K + S
+    out = nv.NVFP4Tensor(
+        codes=torch.full((rows, KA // 2), canary, dtype=torch.uint8, device="cuda"),
+        scales=torch.full((nv.nvfp4_scales_bytes(rows, KA),), canary, dtype=torch.uint8, device="cuda"),
+        global_scale=torch.full((1,), -1.0, dtype=torch.float32, device="cuda"),
+        workspace=torch.full((nv.nvfp4_quantize_arc_rmsnorm_workspace_bytes(rows, K),), 0xFF, dtype=torch.uint8,
+                             device="cuda"),
+        rows=rows, K=KA)
+    nv.quantize_arc_rmsnorm(x_cpu.cuda(), gamma.cuda(), eps, torch.from_numpy(perm).cuda(), S, mode, rule, F,
+                            out=out)
+    return out, nv.device_status(out.workspace)
+
+
+@pytest.mark.parametrize("recipe", RECIPES, ids=lambda r: "-".join(map(str, r)))
+@pytest.mark.parametrize("shape,S", [((1, 64), 64), ((129, 256), 64), ((300, 512), 128), ((64, 1024), 0),
+                                     ((37, 5120), 128), ((5, 16384), 256)], ids=str)
+def test_quantize_arc_rmsnorm_matches_oracle(shape, S, recipe):
+    """Bit-exact with the oracle's RMSNorm (pinned in test_oracle_rmsnorm.py)
+    followed by its augmented quantization; every byte, padding included."""
+    rows, K = shape
+    mode, rule, F = recipe
+    x = workloads.small_operand(rows, K, seed=rows + K).make()
+    gamma = _gains(K, K)
+    perm = outlier_perm(x)
+    q, status = gpu_arc_rmsnorm(x, gamma, 1e-6, perm, S, mode, rule, F)
+    assert status == nv.OK
+    y = torch.from_numpy(oracle.rmsnorm(x, gamma, 1e-6).view(np.int16)).view(torch.bfloat16)
+    assert_arc_equal(q, y, perm, S, nv.AUG_RESIDUAL, mode, rule, F)
+
+
+def test_quantize_arc_rmsnorm_reading_pins():
+    """The rows of tests/golden/rmsnorm_pins.txt (each separates one reading of
+    the RMSNorm rounding order from its alternative) quantized on the GPU:
+    the operand equals the oracle's on the pinned normalized rows."""
+    import test_oracle_rmsnorm as tr
+
+    for case in tr.CASES:
+        x_bits, g_bits = tr._row_arrays(case)
+        x = torch.from_numpy(x_bits.view(np.int16)).view(torch.bfloat16)
+        gamma = torch.from_numpy(g_bits.view(np.int16)).view(torch.bfloat16)
+        perm = np.arange(case["K"], dtype=np.int32)
+        q, status = gpu_arc_rmsnorm(x, gamma, case["eps"], perm, 0, "six", "max", 448.0)
+        assert status == nv.OK
+        y = oracle.rmsnorm(x_bits, g_bits, case["eps"])
+        assert int(y[0, case["i"]]) == case["y"]
+        assert_arc_equal(q, torch.from_numpy(y.view(np.int16)).view(torch.bfloat16), perm, 0,
+                         nv.AUG_RESIDUAL, "six", "max", 448.0)
+
+
+def test_quantize_arc_rmsnorm_nonfinite_input_is_reported():
+    x = workloads.small_operand(8, 256, seed=3).make()
+    x[5, 17] = float("inf")
+    q, status = gpu_arc_rmsnorm(x, _gains(256, 1), 1e-6, np.arange(256, dtype=np.int32), 64, "six", "max", 448.0)
+    assert status == nv.ERR_NONFINITE
+    assert np.isnan(float(q.global_scale.cpu()[0]))
+
+
+def test_quantize_arc_rmsnorm_gemm_uses_the_normalized_activations():
+    """The augmented GEMM over K + S on the fused operand matches the fp64
+    oracle GEMM of the normalized activations against the duplicated weight."""
+    M, K, N, S = 256, 1024, 384, 128
+    x = workloads.small_operand(M, K, seed=11).make()
+    w = workloads.small_operand(N, K, seed=12, kind="normal").make()
+    gamma = _gains(K, 13)
+    perm = outlier_perm(x)
+    qx, status = gpu_arc_rmsnorm(x, gamma, 1e-5, perm, S, "four_over_six", "mse", 256.0)
+    assert status == nv.OK
+    qw = nv.quantize_arc(w.cuda(), torch.from_numpy(perm).cuda(), S, nv.AUG_DUPLICATE, "six", "max", 448.0)
+    y_gpu = nv.gemm(qx, qw, out_dtype=torch.float32)
+    yb = torch.from_numpy(oracle.rmsnorm(x, gamma, 1e-5).view(np.int16)).view(torch.bfloat16)
+    xc, xs, xa = oracle.quantize_arc(yb, perm, S, oracle.AUG_RESIDUAL, oracle.MODE_FOUR_OVER_SIX,
+                                     oracle.RULE_MSE, 256.0)
+    wc, ws_, wa = oracle.quantize_arc(w, perm, S, oracle.AUG_DUPLICATE, oracle.MODE_SIX, oracle.RULE_MAX, 448.0)
+    ref, guard = oracle.gemm_reference(xc[:64], xs[:64], xa, wc, ws_, wa)
+    assert_gemm_close(to_np(y_gpu)[:64], ref, guard, bf16=False)

@@ -9,7 +9,8 @@ replaces the amax pass.
 of the gradient GEMMs in training.
 ``quantize_arc`` -- ARCQuant augmented residual channels: channels in a
 calibration order plus S appended channels holding the residual of the first
-S (activations) or a copy of them (weights), for one GEMM over K + S.
+S (activations) or a copy of them (weights), for one GEMM over K + S;
+``quantize_arc_rmsnorm`` the same for activations with their RMSNorm fused in.
 ``gemm`` -- Y = A_hat @ B_hat^T on two NVFP4 operands (tcgen05 block-scaled FP4
 MMA, fp32 accumulation, bf16 or fp32 output); ``gemm_segmented`` applies one
 B global scale per output-column segment (fused projections);
@@ -31,4 +32,5 @@ from ._lib import (  # noqa: F401
     nvfp4_get_device_status, nvfp4_quantize, nvfp4_quantize_noalloc, nvfp4_quantize_with_scale,
     nvfp4_quantize_workspace_bytes, nvfp4_scales_bytes,
     quantize, quantize_t, nvfp4_quantize_t, quantize_gemm, nvfp4_quantize_gemm, quantize_arc_gemm,
-    nvfp4_quantize_arc_gemm, quantize_arc, nvfp4_quantize_arc, AUG_RESIDUAL, AUG_DUPLICATE, status_string, testing_set_gemm_wait)
+    nvfp4_quantize_arc_gemm, quantize_arc_rmsnorm, nvfp4_quantize_arc_rmsnorm,
+    nvfp4_quantize_arc_rmsnorm_workspace_bytes, quantize_arc, nvfp4_quantize_arc, AUG_RESIDUAL, AUG_DUPLICATE, status_string, testing_set_gemm_wait)

@@ -40,6 +40,9 @@ _SIGNATURES = {
                                               ctypes.c_float, _P, _P, _P, _P]),
     "nvfp4_quantize_arc": (ctypes.c_int, [_P, _I64, _I64, _I64, _P, _I64, ctypes.c_int, ctypes.c_int,
                                           ctypes.c_int, ctypes.c_float, _P, _P, _P, _P, ctypes.c_size_t, _P]),
+    "nvfp4_quantize_arc_rmsnorm_workspace_bytes": (ctypes.c_size_t, [_I64, _I64]),
+    "nvfp4_quantize_arc_rmsnorm": (ctypes.c_int, [_P, _I64, _I64, _I64, _P, ctypes.c_float, _P, _I64, ctypes.c_int,
+                                                  ctypes.c_int, ctypes.c_float, _P, _P, _P, _P, ctypes.c_size_t, _P]),
     "nvfp4_quantize_t": (ctypes.c_int, [_P, _I64, _I64, _I64, ctypes.c_int, ctypes.c_int,
                                         ctypes.c_float, _P, _P, _P, _P, ctypes.c_size_t, _P]),
     "nvfp4_quantize_with_scale": (ctypes.c_int, [_P, _I64, _I64, _I64, ctypes.c_int, ctypes.c_int,
@@ -164,6 +167,16 @@ def nvfp4_gemm_segmented(a_codes, a_scales, a_global, b_codes, b_scales, b_globa
     return load().nvfp4_gemm_segmented(a_codes, a_scales, a_global, b_codes, b_scales, b_globals,
                                        seg_ends, nseg, M, N, K, y, ldy, out_dtype, workspace,
                                        workspace_bytes, stream)
+
+
+def nvfp4_quantize_arc_rmsnorm_workspace_bytes(rows, K):
+    return load().nvfp4_quantize_arc_rmsnorm_workspace_bytes(rows, K)
+
+
+def nvfp4_quantize_arc_rmsnorm(x, rows, K, ldx, gamma, eps, perm, S, mode, rule, fp8_max, codes, scales,
+                               global_scale, workspace, workspace_bytes, stream=None):
+    return load().nvfp4_quantize_arc_rmsnorm(x, rows, K, ldx, gamma, eps, perm, S, mode, rule, fp8_max, codes,
+                                             scales, global_scale, workspace, workspace_bytes, stream)
 
 
 def nvfp4_quantize_gemm(x, M, K, ldx, mode, rule, fp8_max, x_codes, x_scales, x_global_scale, x_workspace,
@@ -379,6 +392,45 @@ def quantize_arc(x, perm, S: int, augment: int = AUG_RESIDUAL, mode: str = "six"
                             out.global_scale.data_ptr(), out.workspace.data_ptr(), out.workspace.numel(),
                             _stream_handle(stream))
     _check(st, "nvfp4_quantize_arc")
+    return out
+
+
+def quantize_arc_rmsnorm(x, gamma, eps: float, perm, S: int, mode: str = "six", rule: str = "max",
+                         fp8_max: float | None = None, out: NVFP4Tensor | None = None, stream=None) -> NVFP4Tensor:
+    """``quantize_arc`` (residual channels) of the RMSNorm of x: the rows of
+    the bf16 CUDA matrix x [rows, K] are normalized by their root mean square
+    (plus eps) and scaled by the bf16 gains ``gamma`` [K], rounded to bf16,
+    reordered by ``perm`` and quantized with S residual channels, all in the
+    library's two kernels (the normalized tensor is never written)."""
+    import torch
+
+    if x.dtype != torch.bfloat16 or x.dim() != 2 or not x.is_cuda:
+        raise ValueError("x must be a 2-D bfloat16 CUDA tensor")
+    if x.stride(1) != 1:
+        raise ValueError("x must have unit stride along K")
+    rows, K = x.shape
+    if perm.dtype != torch.int32 or perm.numel() != K or not perm.is_cuda or perm.device != x.device:
+        raise ValueError("perm must be an int32 tensor with K entries on x's device")
+    if gamma.dtype != torch.bfloat16 or gamma.numel() != K or not gamma.is_cuda or gamma.device != x.device:
+        raise ValueError("gamma must be a bfloat16 tensor with K entries on x's device")
+    gamma = gamma.contiguous()
+    F = DEFAULT_FP8_MAX[mode] if fp8_max is None else float(fp8_max)
+    KA = K + S
+    if out is None:
+        dev = x.device
+        out = NVFP4Tensor(
+            codes=torch.empty(rows, KA // 2, dtype=torch.uint8, device=dev),
+            scales=torch.empty(max(1, nvfp4_scales_bytes(rows, KA)), dtype=torch.uint8, device=dev),
+            global_scale=torch.empty(1, dtype=torch.float32, device=dev),
+            workspace=torch.empty(nvfp4_quantize_arc_rmsnorm_workspace_bytes(rows, K), dtype=torch.uint8,
+                                  device=dev),
+            rows=rows, K=KA)
+    _check_operand(out, "out", rows, KA, x.device, workspace=True)
+    st = nvfp4_quantize_arc_rmsnorm(x.data_ptr(), rows, K, _row_pitch(x), gamma.data_ptr(), float(eps),
+                                    perm.data_ptr(), S, MODES[mode], RULES[rule], F, out.codes.data_ptr(),
+                                    out.scales.data_ptr(), out.global_scale.data_ptr(), out.workspace.data_ptr(),
+                                    out.workspace.numel(), _stream_handle(stream))
+    _check(st, "nvfp4_quantize_arc_rmsnorm")
     return out
 
 

@@ -48,7 +48,9 @@ constexpr int kArcMaxThreads = 640;         // its block size, at most
 constexpr int kArcMaxBufs = 3;              // its row buffers: 3, or 2 for the widest rows
 constexpr int64_t kArcSmemStep = 73728;     // shared memory it aims at: three CTAs per SM up to 5K channels
 constexpr int64_t kArcMaxK = 16384;         // channels of x it takes, at most
-constexpr int64_t kArcSmemBudget = 98304;   // its shared memory, at most: 2 bytes x K x (1 + buffers x rows per step)
+// its shared memory, at most: 2 bytes x K x (lead arrays + buffers x rows per step), K <= 16384 (two
+// buffers of one row; the offsets and, with RMSNorm, the gains ahead of them)
+constexpr int64_t kArcSmemBudget = 2 * 16384 * 4;
 constexpr int kQuantThreads = 256;
 constexpr int kQuantWarps = kQuantThreads / 32;
 
@@ -125,6 +127,9 @@ struct QuantParams {
   int arc_rows = 1;               // rows per step of the augmented quantizer
   int arc_prim_threads = 128;     // its threads for the primary blocks; the rest take the appended ones
   int arc_bufs = 3;               // its row buffers
+  // RMSNorm ahead of the augmented quantizer only
+  const uint16_t* gamma = nullptr;  // bf16 gains, K entries
+  const float* rinv = nullptr;      // 1 / rms of each row, written by the RMS pass
 };
 
 // Start of every quantize kernel: alpha (a caller-supplied static scale, or
@@ -417,6 +422,136 @@ __global__ void __launch_bounds__(kQuantThreads)
   }
 }
 
+// ------------------------------------------------------------- RMS pass --
+// RMSNorm ahead of the augmented quantizer (ARCQuant page, 방법론, 커널
+// 구현: the fused kernel normalizes the activations before reordering and
+// quantizing them; the page gives no formula, so this is the standard RMSNorm,
+// each step one binary32 operation):
+//   r = 1 / sqrt(sum_k x_k^2 / K + eps),  y_k = bf16((x_k * r) * gamma_k)
+// with the sum of squares taken as the contiguous pairwise tree over the row
+// (zero-padded to a power of two P).  One warp per row, no block barrier: in
+// round q the warp reads 256 consecutive elements (lane l the 16-byte group
+// 32q + l, coalesced), each lane sums its group's squares as a pairwise tree,
+// and an xor butterfly over the lanes combines the groups (1, then 2, 4, ...
+// adjacent subtrees: the same tree, addition being commutative); the rounds'
+// sums, all lanes holding them, merge like a binary counter (each completed
+// subtree added to the equal-size one on its left).  Every lane ends with the
+// row's sum and computes r.  The pass writes r for every row and, like the
+// amax pass, each CTA's max |y| as a bf16 bit pattern.
+constexpr int kRmsThreads = 256;
+
+// two binary32 values -> a bf16 pair (lo in the low half), nearest, ties to even
+__device__ __forceinline__ uint32_t bf16x2_rn(float lo, float hi) {
+  uint32_t w;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(w) : "f"(hi), "f"(lo));
+  return w;
+}
+
+// the squares of the 8 bf16 values of one 16-byte group, summed as a pairwise tree
+__device__ __forceinline__ float sq_tree8(const uint4 v) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  float a[8];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float lo = __uint_as_float(w[i] << 16), hi = __uint_as_float(w[i] & 0xFFFF0000u);
+    a[2 * i] = __fmul_rn(lo, lo);
+    a[2 * i + 1] = __fmul_rn(hi, hi);
+  }
+  const float b0 = __fadd_rn(a[0], a[1]), b1 = __fadd_rn(a[2], a[3]);
+  const float b2 = __fadd_rn(a[4], a[5]), b3 = __fadd_rn(a[6], a[7]);
+  return __fadd_rn(__fadd_rn(b0, b1), __fadd_rn(b2, b3));
+}
+
+// max |y| of one 16-byte group of x and its gains, y = bf16((x * r) * gamma)
+__device__ __forceinline__ uint32_t rms_group_max(const uint4 xv, const uint4 gv, float r, uint32_t m) {
+  const uint32_t xs[4] = {xv.x, xv.y, xv.z, xv.w}, gs[4] = {gv.x, gv.y, gv.z, gv.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float y0 = __fmul_rn(__fmul_rn(__uint_as_float(xs[i] << 16), r), __uint_as_float(gs[i] << 16));
+    const float y1 = __fmul_rn(__fmul_rn(__uint_as_float(xs[i] & 0xFFFF0000u), r), __uint_as_float(gs[i] & 0xFFFF0000u));
+    const uint32_t yw = bf16x2_rn(y0, y1);
+    m = max(m, max(yw & 0x7FFFu, (yw >> 16) & 0x7FFFu));
+  }
+  return m;
+}
+
+__global__ void __launch_bounds__(kRmsThreads)
+    rms_amax_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t K, int64_t ldx,
+                    const uint16_t* __restrict__ gamma, float eps, float* __restrict__ rinv,
+                    uint32_t* __restrict__ partials) {
+  pdl_launch_dependents();  // the quantize kernel may be scheduled now; it waits for this grid's end
+  // rounds that hold elements; the zero-padded rest of the tree up to the next
+  // power of two adds exact zeros and is not computed
+  const int used = static_cast<int>((K + 255) / 256);  // 1 .. 64 (K <= 16384)
+  const int lane = static_cast<int>(threadIdx.x & 31), warp = static_cast<int>(threadIdx.x >> 5);
+  const int64_t nwarps = static_cast<int64_t>(gridDim.x) * (kRmsThreads / 32);
+  uint32_t m = 0;
+  for (int64_t r = static_cast<int64_t>(blockIdx.x) * (kRmsThreads / 32) + warp; r < rows; r += nwarps) {
+    const uint16_t* xr = x + r * ldx;
+    float stk[7];
+    float v = 0.0f;
+    for (int q = 0; q < used; ++q) {
+      const int64_t k = 256 * static_cast<int64_t>(q) + 8 * lane;  // K % 8 == 0: a group is inside or past the row
+      v = k < K ? sq_tree8(*reinterpret_cast<const uint4*>(xr + k)) : 0.0f;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) v = __fadd_rn(v, __shfl_xor_sync(0xffffffffu, v, o));
+      // merge with the completed round subtrees of equal size on the left
+#pragma unroll
+      for (int lvl = 0; lvl < 7; ++lvl) {
+        if (!((q >> lvl) & 1)) {
+          stk[lvl] = v;
+          break;
+        }
+        v = __fadd_rn(stk[lvl], v);
+      }
+    }
+    // the stack now holds one complete subtree per set bit of `used`, the
+    // lowest bit's the rightmost; the zero padding leaves each as the left
+    // operand of everything to its right
+    bool have = false;
+#pragma unroll
+    for (int lvl = 0; lvl < 7; ++lvl) {
+      if ((used >> lvl) & 1) {
+        v = have ? __fadd_rn(stk[lvl], v) : stk[lvl];
+        have = true;
+      }
+    }
+    const float ms = __fdiv_rn(v, static_cast<float>(K));
+    const float rr = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(ms, eps)));
+    if (lane == 0) rinv[r] = rr;
+    // the row's outputs and their max |y|, in the same coalesced order
+    for (int q = 0; q < used; ++q) {
+      const int64_t k = 256 * static_cast<int64_t>(q) + 8 * lane;
+      if (k < K)
+        m = rms_group_max(*reinterpret_cast<const uint4*>(xr + k), *reinterpret_cast<const uint4*>(gamma + k), rr, m);
+    }
+  }
+#pragma unroll
+  for (int o = 16; o; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
+  __shared__ uint32_t s_max[kRmsThreads / 32];
+  if (lane == 0) s_max[warp] = m;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    uint32_t mm = 0;
+    for (int w = 0; w < kRmsThreads / 32; ++w) mm = max(mm, s_max[w]);
+    partials[blockIdx.x] = mm;
+  }
+}
+
+// The RMSNorm of a gathered block: x (8 bf16 pairs, element 2i low) becomes
+// bf16((x * r) * gamma) with the block's gains gw (same layout), as the RMS
+// pass computes it; packed products are one RNE binary32 product per lane.
+__device__ __forceinline__ void rms_normalize(uint32_t w[8], const uint32_t gw[8], float r) {
+  const f2 rr = make_f2(r, r);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const f2 xv = make_f2(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xFFFF0000u));
+    const f2 gv = make_f2(__uint_as_float(gw[i] << 16), __uint_as_float(gw[i] & 0xFFFF0000u));
+    const f2 y = mul2(mul2(xv, rr), gv);
+    w[i] = bf16x2_rn(y.a(), y.b());
+  }
+}
+
 // Augmented quantization (ARCQuant page, 기술 요약 / 방법론): channels of x
 // taken in the order perm, the usual block step on them (primary stage), and
 // S appended channels -- the residual e = fma(-q, d, x) of the first S
@@ -441,12 +576,13 @@ __global__ void __launch_bounds__(kQuantThreads)
 // one that sees no progress for 4 s records NVFP4_ERR_TIMEOUT, and the
 // producer lets the copies it issued land before the CTA exits.
 // Output: the [rows, K + S] operand (codes and swizzled scales).
-template <bool FOUR_OVER_SIX, int RULE>
+template <bool FOUR_OVER_SIX, int RULE, bool NORM>
 __global__ void __launch_bounds__(kArcMaxThreads)
     quantize_arc_kernel(const QuantParams p) {
   BlockConsts k;
   __shared__ ScaleEntry s_dr[128];
-  extern __shared__ __align__(16) uint16_t s_dyn[];  // [K] channel byte offsets, then arc_bufs x [arc_rows][K] rows
+  // [K] channel byte offsets, with NORM [K] gains in channel order, then arc_bufs x [arc_rows][K] rows
+  extern __shared__ __align__(16) uint16_t s_dyn[];
   if (!quant_prologue(p, k, s_dr)) return;
 
   const int64_t K = p.K, KA = p.K + p.S;
@@ -454,12 +590,14 @@ __global__ void __launch_bounds__(kArcMaxThreads)
   const int T = static_cast<int>(blockDim.x), P = p.arc_prim_threads;
   for (int64_t i = threadIdx.x; i < K; i += T) {
     const int32_t c = p.perm[i];
-    s_dyn[i] = static_cast<uint16_t>(2 * (c >= 0 && c < K ? c : 0));  // out-of-range entries read channel 0
+    const int32_t cc = c >= 0 && c < K ? c : 0;  // out-of-range entries read channel 0
+    s_dyn[i] = static_cast<uint16_t>(2 * cc);
+    if (NORM) s_dyn[K + i] = p.gamma[cc];
   }
   const int64_t rows_padded = (p.rows + 127) / 128 * 128;
   const int64_t half_ka = KA / 2, kgroups_a = KA / 64;
   const int nprim = static_cast<int>(K / 16), nres = static_cast<int>(p.S / 16);
-  const uint32_t rows_base = smem_u32(s_dyn + K);
+  const uint32_t rows_base = smem_u32(s_dyn + (NORM ? 2 : 1) * K);
   const uint32_t row_bytes = static_cast<uint32_t>(K) * 2, buf_bytes = row_bytes * R;
   // Buffers: full[b] completes when buffer b holds its step's rows (the
   // producer's arrival plus the copies' bytes); consumed[b] when every
@@ -540,6 +678,12 @@ __global__ void __launch_bounds__(kArcMaxThreads)
 #pragma unroll
       for (int i = 0; i < 8; ++i)
         w[i] = ld_shared_u16(s_row + (ow[i] & 0xFFFFu)) | (ld_shared_u16(s_row + (ow[i] >> 16)) << 16);
+      if (NORM) {
+        const uint4 g0 = reinterpret_cast<const uint4*>(s_dyn + K + 16 * j)[0];
+        const uint4 g1 = reinterpret_cast<const uint4*>(s_dyn + K + 16 * j)[1];
+        const uint32_t gw[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+        rms_normalize(w, gw, __ldg(p.rinv + row0 + rr));
+      }
       return unpack_block(make_uint4(w[0], w[1], w[2], w[3]), make_uint4(w[4], w[5], w[6], w[7]), px);
     };
     if (static_cast<int>(threadIdx.x) < P) {
@@ -548,6 +692,13 @@ __global__ void __launch_bounds__(kArcMaxThreads)
         const uint4 o0 = reinterpret_cast<const uint4*>(s_dyn + 16 * j)[0];
         const uint4 o1 = reinterpret_cast<const uint4*>(s_dyn + 16 * j)[1];
         const uint32_t ow[8] = {o0.x, o0.y, o0.z, o0.w, o1.x, o1.y, o1.z, o1.w};
+        uint32_t gw[8];
+        if (NORM) {
+          const uint4 g0 = reinterpret_cast<const uint4*>(s_dyn + K + 16 * j)[0];
+          const uint4 g1 = reinterpret_cast<const uint4*>(s_dyn + K + 16 * j)[1];
+          gw[0] = g0.x, gw[1] = g0.y, gw[2] = g0.z, gw[3] = g0.w, gw[4] = g1.x, gw[5] = g1.y, gw[6] = g1.z,
+          gw[7] = g1.w;
+        }
         for (int rr = 0; rr < R; ++rr) {
           const int64_t row = row0 + rr;
           uint32_t scale = 0;
@@ -557,6 +708,7 @@ __global__ void __launch_bounds__(kArcMaxThreads)
 #pragma unroll
             for (int i = 0; i < 8; ++i)
               w[i] = ld_shared_u16(s_row + (ow[i] & 0xFFFFu)) | (ld_shared_u16(s_row + (ow[i] >> 16)) << 16);
+            if (NORM) rms_normalize(w, gw, __ldg(p.rinv + row));
             f2 px[8];
             const uint32_t bbits = unpack_block(make_uint4(w[0], w[1], w[2], w[3]),
                                                 make_uint4(w[4], w[5], w[6], w[7]), px);
@@ -628,46 +780,54 @@ int arc_threads(int64_t K, int64_t S, int R) {
   return static_cast<int>(std::max<int64_t>(96, prim + res)) + 32;  // + the producer warp
 }
 
-// Rows per step and row buffers of the augmented quantizer for K channels:
-// three buffers of the most rows (up to 4, a power of two so it divides the
-// 128-row padding) that fit kArcSmemStep with the permutation; above 9K
+// Rows per step and row buffers of the augmented quantizer for K channels,
+// with `lead` K-sized bf16 arrays ahead of the rows (the offsets; with RMSNorm
+// the gains too): three buffers of the most rows (up to 4, a power of two so
+// it divides the 128-row padding) that fit kArcSmemStep; above about 9K
 // channels, where even one row per buffer does not, two buffers of one row
 // (within kArcSmemBudget for K <= 16384), so that two CTAs still share an SM.
-int arc_rows_per_step(int64_t K) {
+int arc_rows_per_step(int64_t K, int lead) {
   int r = kArcMaxRows;
-  while (r > 1 && 2 * K * (1 + kArcMaxBufs * r) > kArcSmemStep) r /= 2;
+  while (r > 1 && 2 * K * (lead + kArcMaxBufs * r) > kArcSmemStep) r /= 2;
   return r;
 }
-int arc_buffers(int64_t K) { return 2 * K * (1 + kArcMaxBufs) > kArcSmemStep ? 2 : kArcMaxBufs; }
+int arc_buffers(int64_t K, int lead) { return 2 * K * (lead + kArcMaxBufs) > kArcSmemStep ? 2 : kArcMaxBufs; }
 
-template <bool F, int R>
+template <bool F, int R, bool NORM>
 cudaError_t launch_quantize_arc(int dev, int sms, const QuantParams& p, cudaStream_t s, bool pdl) {
-  const size_t smem = static_cast<size_t>(p.K) * 2 * (1 + p.arc_bufs * p.arc_rows);
+  const size_t smem = static_cast<size_t>(p.K) * 2 * ((NORM ? 2 : 1) + p.arc_bufs * p.arc_rows);
   // the shared-memory opt-in is an attribute of the kernel in this context
   static PerContextCache<int> attr;
   int done = 0;
   cudaError_t e = per_context(attr, dev, [](int* v) {
     *v = 1;
-    return cudaFuncSetAttribute(quantize_arc_kernel<F, R>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    return cudaFuncSetAttribute(quantize_arc_kernel<F, R, NORM>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 static_cast<int>(kArcSmemBudget));
   }, &done);
   if (e != cudaSuccess) return e;
   const int threads = arc_threads(p.K, p.S, p.arc_rows);
   int occ = 0;
-  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, quantize_arc_kernel<F, R>, threads, smem);
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, quantize_arc_kernel<F, R, NORM>, threads, smem);
   if (e != cudaSuccess) return e;
   const int64_t steps = (p.rows + 127) / 128 * 128 / p.arc_rows;
   const int grid = static_cast<int>(std::max<int64_t>(
       1, std::min<int64_t>(steps, static_cast<int64_t>(sms) * std::max(1, occ))));
-  return launch_kernel(quantize_arc_kernel<F, R>, dim3(grid), dim3(threads), smem, s, pdl, p);
+  return launch_kernel(quantize_arc_kernel<F, R, NORM>, dim3(grid), dim3(threads), smem, s, pdl, p);
+}
+
+template <bool NORM>
+cudaError_t launch_quantize_arc_norm(int mode, int rule, int dev, int sms, const QuantParams& p, cudaStream_t s,
+                                     bool pdl) {
+  if (mode == NVFP4_MODE_SIX) return launch_quantize_arc<false, kRuleMax, NORM>(dev, sms, p, s, pdl);
+  if (rule == NVFP4_RULE_MAX) return launch_quantize_arc<true, kRuleMax, NORM>(dev, sms, p, s, pdl);
+  if (rule == NVFP4_RULE_MAE) return launch_quantize_arc<true, kRuleMae, NORM>(dev, sms, p, s, pdl);
+  return launch_quantize_arc<true, kRuleMse, NORM>(dev, sms, p, s, pdl);
 }
 
 cudaError_t launch_quantize_arc_kernel(int mode, int rule, int dev, int sms, const QuantParams& p,
                                        cudaStream_t s, bool pdl) {
-  if (mode == NVFP4_MODE_SIX) return launch_quantize_arc<false, kRuleMax>(dev, sms, p, s, pdl);
-  if (rule == NVFP4_RULE_MAX) return launch_quantize_arc<true, kRuleMax>(dev, sms, p, s, pdl);
-  if (rule == NVFP4_RULE_MAE) return launch_quantize_arc<true, kRuleMae>(dev, sms, p, s, pdl);
-  return launch_quantize_arc<true, kRuleMse>(dev, sms, p, s, pdl);
+  return p.gamma ? launch_quantize_arc_norm<true>(mode, rule, dev, sms, p, s, pdl)
+                 : launch_quantize_arc_norm<false>(mode, rule, dev, sms, p, s, pdl);
 }
 
 template <bool F, int R>
@@ -727,6 +887,10 @@ size_t nvfp4_quantize_workspace_bytes(int64_t rows, int64_t K) {
   (void)rows;
   (void)K;
   return sizeof(WorkspaceHeader) + sizeof(uint32_t) * kMaxPartials;
+}
+
+size_t nvfp4_quantize_arc_rmsnorm_workspace_bytes(int64_t rows, int64_t K) {
+  return nvfp4_quantize_workspace_bytes(rows, K) + sizeof(float) * static_cast<size_t>(rows > 0 ? rows : 0);
 }
 
 }  // extern "C"
@@ -836,6 +1000,23 @@ nvfp4_status launch_dynamic(QuantKind kind, QuantParams p, int mode, int rule, f
   return NVFP4_OK;
 }
 
+// The RMS pass, then the augmented quantizer with RMSNorm as its
+// programmatic dependent.
+nvfp4_status launch_rms_dynamic(QuantParams p, int mode, int rule, float fp8_max, float* global_scale,
+                                uint32_t* partials, int grid, float eps, int dev, int sms, cudaStream_t s) {
+  rms_amax_kernel<<<grid, kRmsThreads, 0, s>>>(p.x, p.rows, p.K, p.ldx, p.gamma, eps, const_cast<float*>(p.rinv),
+                                              partials);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_status(e, "rms_amax_kernel launch");
+  p.global_scale = global_scale;
+  p.partials = partials;
+  p.nparts = grid;
+  p.f6 = fp8_max * 6.0f;
+  e = launch_quantize_arc_kernel(mode, rule, dev, sms, p, s, true);
+  if (e != cudaSuccess) return cuda_status(e, "quantize kernel launch");
+  return NVFP4_OK;
+}
+
 // nvfp4_quantize (row-wise blocks of x), nvfp4_quantize_t (blocks along the
 // rows of x, i.e. the operand of x^T) and nvfp4_quantize_arc (row-wise with
 // reordered and augmented channels), with the caller's workspace.
@@ -844,7 +1025,8 @@ nvfp4_status launch_dynamic(QuantKind kind, QuantParams p, int mode, int rule, f
 nvfp4_status check_quantize_call(const char* fn, QuantKind kind, const void* x, int64_t rows, int64_t K,
                                  int64_t ldx, int mode, int rule, float fp8_max, const void* codes,
                                  const void* scales, const float* global_scale, const void* workspace,
-                                 size_t workspace_bytes, const int32_t* perm, int64_t S, int augment) {
+                                 size_t workspace_bytes, const int32_t* perm, int64_t S, int augment,
+                                 const uint16_t* gamma = nullptr, float eps = 0.0f) {
   nvfp4_status st = check_quant_args(fn, kind == QuantKind::kTransposed, x, rows, K, ldx, mode, rule, codes,
                                      scales, global_scale);
   if (st != NVFP4_OK) return st;
@@ -859,6 +1041,13 @@ nvfp4_status check_quantize_call(const char* fn, QuantKind kind, const void* x, 
   }
   if (!workspace || !aligned16(workspace))
     return set_error(NVFP4_ERR_INVALID_ARG, "%s: workspace must be a non-null 16-byte aligned pointer", fn);
+  if (gamma) {
+    if (!aligned16(gamma)) return set_error(NVFP4_ERR_INVALID_ARG, "%s: gamma must be 16-byte aligned", fn);
+    if (!(eps > 0.0f) || isinf(eps))
+      return set_error(NVFP4_ERR_INVALID_ARG, "%s: eps must be a positive finite number", fn);
+    if (workspace_bytes < nvfp4_quantize_arc_rmsnorm_workspace_bytes(rows, K))
+      return set_error(NVFP4_ERR_INVALID_ARG, "%s: workspace too small", fn);
+  }
   if (workspace_bytes < nvfp4_quantize_workspace_bytes(rows, K))
     return set_error(NVFP4_ERR_INVALID_ARG, "%s: workspace too small", fn);
   return NVFP4_OK;
@@ -867,9 +1056,10 @@ nvfp4_status check_quantize_call(const char* fn, QuantKind kind, const void* x, 
 nvfp4_status quantize_impl(const char* fn, QuantKind kind, const void* x, int64_t rows, int64_t K,
                            int64_t ldx, int mode, int rule, float fp8_max, void* codes, void* scales,
                            float* global_scale, void* workspace, size_t workspace_bytes, void* stream,
-                           const int32_t* perm = nullptr, int64_t S = 0, int augment = 0) {
+                           const int32_t* perm = nullptr, int64_t S = 0, int augment = 0,
+                           const uint16_t* gamma = nullptr, float eps = 0.0f) {
   nvfp4_status st = check_quantize_call(fn, kind, x, rows, K, ldx, mode, rule, fp8_max, codes, scales,
-                                        global_scale, workspace, workspace_bytes, perm, S, augment);
+                                        global_scale, workspace, workspace_bytes, perm, S, augment, gamma, eps);
   if (st != NVFP4_OK) return st;
   int dev = 0, sms = 0;
   if ((st = check_device(&dev, &sms)) != NVFP4_OK) return st;
@@ -881,9 +1071,21 @@ nvfp4_status quantize_impl(const char* fn, QuantKind kind, const void* x, int64_
   p.S = S;
   p.augment = augment;
   if (kind == QuantKind::kAugmented) {
-    p.arc_rows = arc_rows_per_step(K);
+    const int lead = gamma ? 2 : 1;
+    p.arc_rows = arc_rows_per_step(K, lead);
     p.arc_prim_threads = arc_prim_threads(K);
-    p.arc_bufs = arc_buffers(K);
+    p.arc_bufs = arc_buffers(K, lead);
+  }
+  if (gamma) {
+    // RMSNorm ahead of the augmented quantizer: the RMS pass takes the amax
+    // pass's place and leaves 1/rms of every row after the partials
+    p.gamma = gamma;
+    p.rinv = reinterpret_cast<float*>(static_cast<char*>(workspace) + nvfp4_quantize_workspace_bytes(rows, K));
+    // one warp per row: enough CTAs for every row, at most eight per SM
+    const int64_t want = (rows + kRmsThreads / 32 - 1) / (kRmsThreads / 32);
+    const int grid = static_cast<int>(std::min<int64_t>(std::min<int64_t>(want, int64_t{sms} * 8), kMaxPartials));
+    return launch_rms_dynamic(p, mode, rule, fp8_max, global_scale, partials, grid, eps, dev, sms,
+                              static_cast<cudaStream_t>(stream));
   }
   const int amax_grid = std::min(amax_grid_size(rows, K, ldx, sms), kMaxPartials);
   return launch_dynamic(kind, p, mode, rule, fp8_max, global_scale, partials, amax_grid, dev, sms,
@@ -942,6 +1144,17 @@ nvfp4_status nvfp4_quantize_arc(const void* x, int64_t rows, int64_t K, int64_t 
                                 void* workspace, size_t workspace_bytes, void* stream) {
   return quantize_impl("nvfp4_quantize_arc", QuantKind::kAugmented, x, rows, K, ldx, mode, rule, fp8_max,
                        codes, scales, global_scale, workspace, workspace_bytes, stream, perm, S, augment);
+}
+
+nvfp4_status nvfp4_quantize_arc_rmsnorm(const void* x, int64_t rows, int64_t K, int64_t ldx, const void* gamma,
+                                        float eps, const int32_t* perm, int64_t S, int mode, int rule,
+                                        float fp8_max, void* codes, void* scales, float* global_scale,
+                                        void* workspace, size_t workspace_bytes, void* stream) {
+  const char* fn = "nvfp4_quantize_arc_rmsnorm";
+  if (!gamma) return set_error(NVFP4_ERR_INVALID_ARG, "%s: null pointer argument", fn);
+  return quantize_impl(fn, QuantKind::kAugmented, x, rows, K, ldx, mode, rule, fp8_max, codes, scales,
+                       global_scale, workspace, workspace_bytes, stream, perm, S, 0,
+                       static_cast<const uint16_t*>(gamma), eps);
 }
 
 nvfp4_status nvfp4_quantize_t(const void* x, int64_t rows, int64_t K, int64_t ldx, int mode,
