@@ -782,16 +782,28 @@ int arc_threads(int64_t K, int64_t S, int R) {
 
 // Rows per step and row buffers of the augmented quantizer for K channels,
 // with `lead` K-sized bf16 arrays ahead of the rows (the offsets; with RMSNorm
-// the gains too): three buffers of the most rows (up to 4, a power of two so
-// it divides the 128-row padding) that fit kArcSmemStep; above about 9K
-// channels, where even one row per buffer does not, two buffers of one row
-// (within kArcSmemBudget for K <= 16384), so that two CTAs still share an SM.
-int arc_rows_per_step(int64_t K, int lead) {
-  int r = kArcMaxRows;
-  while (r > 1 && 2 * K * (lead + kArcMaxBufs * r) > kArcSmemStep) r /= 2;
-  return r;
+// the gains too), within kArcSmemStep: three buffers of the most rows (up to 4,
+// a power of two so it divides the 128-row padding).  With RMSNorm, two rows in
+// two buffers are taken before one row in three, when three do not fit (the
+// gather's per-row costs are shared by the rows of a step).  Where even one row
+// per buffer does not fit (K above about 9K), two buffers of one row (within
+// kArcSmemBudget for K <= 16384), so that two CTAs still share an SM.
+void arc_layout(int64_t K, int lead, int* rows, int* bufs) {
+  for (int r = kArcMaxRows; r >= 1; r /= 2) {
+    if (2 * K * (lead + kArcMaxBufs * r) <= kArcSmemStep) {
+      *rows = r;
+      *bufs = kArcMaxBufs;
+      return;
+    }
+    if (lead > 1 && r > 1 && 2 * K * (lead + 2 * r) <= kArcSmemStep) {
+      *rows = r;
+      *bufs = 2;
+      return;
+    }
+  }
+  *rows = 1;
+  *bufs = 2;
 }
-int arc_buffers(int64_t K, int lead) { return 2 * K * (lead + kArcMaxBufs) > kArcSmemStep ? 2 : kArcMaxBufs; }
 
 template <bool F, int R, bool NORM>
 cudaError_t launch_quantize_arc(int dev, int sms, const QuantParams& p, cudaStream_t s, bool pdl) {
@@ -1071,10 +1083,8 @@ nvfp4_status quantize_impl(const char* fn, QuantKind kind, const void* x, int64_
   p.S = S;
   p.augment = augment;
   if (kind == QuantKind::kAugmented) {
-    const int lead = gamma ? 2 : 1;
-    p.arc_rows = arc_rows_per_step(K, lead);
+    arc_layout(K, gamma ? 2 : 1, &p.arc_rows, &p.arc_bufs);
     p.arc_prim_threads = arc_prim_threads(K);
-    p.arc_bufs = arc_buffers(K, lead);
   }
   if (gamma) {
     // RMSNorm ahead of the augmented quantizer: the RMS pass takes the amax
