@@ -348,6 +348,22 @@ NVFP4_API nvfp4_status nvfp4_quantize_arc_gemm(const void* x, int64_t M, int64_t
                                                int64_t ldy, int out_dtype, void* workspace,
                                                size_t workspace_bytes, void* stream);
 
+/* nvfp4_quantize_arc_gemm with the activations' RMSNorm fused ahead: x is
+ * quantized as nvfp4_quantize_arc_rmsnorm does (gamma, eps; x_workspace of
+ * nvfp4_quantize_arc_rmsnorm_workspace_bytes(M, K)), then the GEMM over K + S
+ * against the weight quantized by nvfp4_quantize_arc with the same perm and S
+ * and augment = 1.  Results are those of the two calls made one after the
+ * other, bit for bit; every argument is checked before anything is enqueued. */
+NVFP4_API nvfp4_status nvfp4_quantize_arc_rmsnorm_gemm(const void* x, int64_t M, int64_t K, int64_t ldx,
+                                                       const void* gamma, float eps, const int32_t* perm,
+                                                       int64_t S, int mode, int rule, float fp8_max,
+                                                       void* x_codes, void* x_scales, float* x_global_scale,
+                                                       void* x_workspace, size_t x_workspace_bytes,
+                                                       const void* w_codes, const void* w_scales,
+                                                       const float* w_global, int64_t N, void* y, int64_t ldy,
+                                                       int out_dtype, void* workspace, size_t workspace_bytes,
+                                                       void* stream);
+
 /* Synchronizes `stream`, then returns the status word the last call that used
  * `workspace` wrote (NVFP4_OK, NVFP4_ERR_INVALID_ARG, NVFP4_ERR_NONFINITE or
  * NVFP4_ERR_TIMEOUT), or

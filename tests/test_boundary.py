@@ -313,3 +313,30 @@ def test_quantize_arc_rmsnorm_without_gpu_fails_loudly():
     if torch.cuda.is_available():
         pytest.skip("a GPU is present")
     assert _qar() in (nv.ERR_CUDA, nv.ERR_UNSUPPORTED_DEVICE)
+
+
+def _qarg(**kw):
+    args = dict(x=FAKE, M=64, K=512, ldx=512, gamma=FAKE, eps=1e-6, perm=FAKE, S=128, mode=1, rule=2,
+                fp8_max=256.0, x_codes=FAKE, x_scales=FAKE, x_global_scale=FAKE, x_workspace=FAKE,
+                x_workspace_bytes=1 << 20, w_codes=FAKE, w_scales=FAKE, w_global=FAKE, N=256, y=FAKE, ldy=256,
+                out_dtype=0, workspace=FAKE, workspace_bytes=64, stream=None)
+    args.update(kw)
+    return nv.nvfp4_quantize_arc_rmsnorm_gemm(*args.values())
+
+
+@pytest.mark.parametrize("bad", [
+    dict(gamma=None), dict(gamma=FAKE + 8), dict(eps=0.0), dict(eps=float("nan")), dict(perm=None), dict(S=32),
+    dict(K=96), dict(x_workspace_bytes=16448), dict(w_codes=None), dict(N=0), dict(ldy=128), dict(out_dtype=3),
+    dict(workspace_bytes=4),
+])
+def test_quantize_arc_rmsnorm_gemm_rejects_bad_arguments(bad):
+    assert _qarg(**bad) == nv.ERR_INVALID_ARG
+    assert nv.last_error_message().startswith("nvfp4_quantize_arc_rmsnorm_gemm")
+
+
+def test_quantize_arc_rmsnorm_gemm_without_gpu_fails_loudly():
+    import torch
+
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    assert _qarg() in (nv.ERR_CUDA, nv.ERR_UNSUPPORTED_DEVICE)

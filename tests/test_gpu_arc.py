@@ -181,3 +181,41 @@ def test_quantize_arc_rmsnorm_gemm_uses_the_normalized_activations():
     wc, ws_, wa = oracle.quantize_arc(w, perm, S, oracle.AUG_DUPLICATE, oracle.MODE_SIX, oracle.RULE_MAX, 448.0)
     ref, guard = oracle.gemm_reference(xc[:64], xs[:64], xa, wc, ws_, wa)
     assert_gemm_close(to_np(y_gpu)[:64], ref, guard, bf16=False)
+
+
+@pytest.mark.parametrize("recipe", RECIPES[:2], ids=lambda r: "-".join(map(str, r)))
+def test_quantize_arc_rmsnorm_pitched_rows(recipe):
+    """x as a view with a row pitch above K (the RMS pass and the bulk row
+    copies both follow the pitch)."""
+    mode, rule, F = recipe
+    rows, K, S = 200, 1024, 128
+    wide = workloads.small_operand(rows, K + 64, seed=21).make()
+    x = wide[:, 32:32 + K]  # a 64-byte aligned column offset: 16-byte aligned rows
+    gamma = _gains(K, 22)
+    perm = outlier_perm(x)
+    out = nv.quantize_arc_rmsnorm(wide.cuda()[:, 32:32 + K], gamma.cuda(), 1e-6, torch.from_numpy(perm).cuda(), S,
+                                  mode, rule, F)
+    assert nv.device_status(out.workspace) == nv.OK
+    y = torch.from_numpy(oracle.rmsnorm(x.contiguous(), gamma, 1e-6).view(np.int16)).view(torch.bfloat16)
+    assert_arc_equal(out, y, perm, S, nv.AUG_RESIDUAL, mode, rule, F)
+
+
+def test_quantize_arc_rmsnorm_gemm_equals_the_two_calls():
+    """nvfp4_quantize_arc_rmsnorm_gemm: RMSNorm, augmented quantization and the
+    GEMM over K + S in one call, bit-equal to the two calls."""
+    M, K, N, S = 300, 2048, 384, 128
+    x = workloads.small_operand(M, K, seed=31).make().cuda()
+    w = workloads.small_operand(N, K, seed=32, kind="normal").make().cuda()
+    gamma = _gains(K, 33).cuda()
+    perm = torch.from_numpy(outlier_perm(x.cpu())).cuda()
+    qw = nv.quantize_arc(w, perm, S, nv.AUG_DUPLICATE, "six", "max", 448.0)
+    qx_ref = nv.quantize_arc_rmsnorm(x, gamma, 1e-6, perm, S, "four_over_six", "mse", 256.0)
+    y_ref = nv.gemm(qx_ref, qw, out_dtype=torch.bfloat16)
+    ws = torch.zeros(nv.nvfp4_gemm_workspace_bytes(), dtype=torch.uint8, device="cuda")
+    qx, y = nv.quantize_arc_gemm(x, perm, S, qw, "four_over_six", "mse", 256.0, out_dtype=torch.bfloat16,
+                                 workspace=ws, gamma=gamma, eps=1e-6)
+    torch.cuda.synchronize()
+    assert nv.device_status(qx.workspace) == nv.OK and nv.device_status(ws) == nv.OK
+    assert torch.equal(qx.codes, qx_ref.codes) and torch.equal(qx.scales, qx_ref.scales)
+    assert torch.equal(qx.global_scale, qx_ref.global_scale)
+    assert torch.equal(y, y_ref)

@@ -33,4 +33,4 @@ from ._lib import (  # noqa: F401
     nvfp4_quantize_workspace_bytes, nvfp4_scales_bytes,
     quantize, quantize_t, nvfp4_quantize_t, quantize_gemm, nvfp4_quantize_gemm, quantize_arc_gemm,
     nvfp4_quantize_arc_gemm, quantize_arc_rmsnorm, nvfp4_quantize_arc_rmsnorm,
-    nvfp4_quantize_arc_rmsnorm_workspace_bytes, quantize_arc, nvfp4_quantize_arc, AUG_RESIDUAL, AUG_DUPLICATE, status_string, testing_set_gemm_wait)
+    nvfp4_quantize_arc_rmsnorm_workspace_bytes, nvfp4_quantize_arc_rmsnorm_gemm, quantize_arc, nvfp4_quantize_arc, AUG_RESIDUAL, AUG_DUPLICATE, status_string, testing_set_gemm_wait)

@@ -59,6 +59,10 @@ _SIGNATURES = {
     "nvfp4_quantize_arc_gemm": (ctypes.c_int, [_P, _I64, _I64, _I64, _P, _I64, ctypes.c_int, ctypes.c_int,
                                                ctypes.c_float, _P, _P, _P, _P, ctypes.c_size_t, _P, _P, _P, _I64,
                                                _P, _I64, ctypes.c_int, _P, ctypes.c_size_t, _P]),
+    "nvfp4_quantize_arc_rmsnorm_gemm": (ctypes.c_int, [_P, _I64, _I64, _I64, _P, ctypes.c_float, _P, _I64,
+                                                       ctypes.c_int, ctypes.c_int, ctypes.c_float, _P, _P, _P, _P,
+                                                       ctypes.c_size_t, _P, _P, _P, _I64, _P, _I64, ctypes.c_int,
+                                                       _P, ctypes.c_size_t, _P]),
     "nvfp4_get_device_status": (ctypes.c_int, [_P, _P]),
     "nvfp4_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "nvfp4_last_error_message": (ctypes.c_char_p, []),
@@ -185,6 +189,15 @@ def nvfp4_quantize_gemm(x, M, K, ldx, mode, rule, fp8_max, x_codes, x_scales, x_
     return load().nvfp4_quantize_gemm(x, M, K, ldx, mode, rule, fp8_max, x_codes, x_scales, x_global_scale,
                                       x_workspace, x_workspace_bytes, w_codes, w_scales, w_global, N, y, ldy,
                                       out_dtype, workspace, workspace_bytes, stream)
+
+
+def nvfp4_quantize_arc_rmsnorm_gemm(x, M, K, ldx, gamma, eps, perm, S, mode, rule, fp8_max, x_codes, x_scales,
+                                    x_global_scale, x_workspace, x_workspace_bytes, w_codes, w_scales, w_global, N,
+                                    y, ldy, out_dtype, workspace, workspace_bytes, stream=None):
+    return load().nvfp4_quantize_arc_rmsnorm_gemm(x, M, K, ldx, gamma, eps, perm, S, mode, rule, fp8_max, x_codes,
+                                                  x_scales, x_global_scale, x_workspace, x_workspace_bytes,
+                                                  w_codes, w_scales, w_global, N, y, ldy, out_dtype, workspace,
+                                                  workspace_bytes, stream)
 
 
 def nvfp4_quantize_arc_gemm(x, M, K, ldx, perm, S, mode, rule, fp8_max, x_codes, x_scales, x_global_scale,
@@ -534,14 +547,15 @@ def quantize_gemm(x, w: NVFP4Tensor, mode: str = "six", rule: str = "max", fp8_m
 
 def quantize_arc_gemm(x, perm, S: int, w: NVFP4Tensor, mode: str = "six", rule: str = "max",
                       fp8_max: float | None = None, out_dtype=None, x_out: NVFP4Tensor | None = None, out=None,
-                      workspace=None, stream=None):
+                      workspace=None, stream=None, gamma=None, eps: float = 1e-6):
     """The augmented-channel W4A4 linear layer in one call: quantize the bf16
     CUDA activations x [M, K] with channel order ``perm`` and S residual
-    channels (as ``quantize_arc`` with AUG_RESIDUAL, into ``x_out``), then
-    Y = X_aug @ W_aug^T over K + S against ``w``, the weight quantized by
-    ``quantize_arc`` with the same perm and S and AUG_DUPLICATE.  The kernels
-    run as programmatic dependents of the kernel before them.  Returns
-    (x_out, Y)."""
+    channels (as ``quantize_arc`` with AUG_RESIDUAL, into ``x_out``; with
+    ``gamma``, as ``quantize_arc_rmsnorm``: RMSNorm with those bf16 gains and
+    ``eps`` fused ahead), then Y = X_aug @ W_aug^T over K + S against ``w``,
+    the weight quantized by ``quantize_arc`` with the same perm and S and
+    AUG_DUPLICATE.  The kernels run as programmatic dependents of the kernel
+    before them.  Returns (x_out, Y)."""
     import torch
 
     if x.dtype != torch.bfloat16 or x.dim() != 2 or not x.is_cuda:
@@ -558,12 +572,18 @@ def quantize_arc_gemm(x, perm, S: int, w: NVFP4Tensor, mode: str = "six", rule: 
     dev = x.device
     F = DEFAULT_FP8_MAX[mode] if fp8_max is None else float(fp8_max)
     out_dtype, code = _out_code(out_dtype, out)
+    if gamma is not None:
+        if gamma.dtype != torch.bfloat16 or gamma.numel() != K or not gamma.is_cuda or gamma.device != x.device:
+            raise ValueError("gamma must be a bfloat16 tensor with K entries on x's device")
+        gamma = gamma.contiguous()
     if x_out is None:
+        ws_bytes = (nvfp4_quantize_arc_rmsnorm_workspace_bytes(M, K) if gamma is not None
+                    else nvfp4_quantize_workspace_bytes(M, K))
         x_out = NVFP4Tensor(
             codes=torch.empty(M, KA // 2, dtype=torch.uint8, device=dev),
             scales=torch.empty(max(1, nvfp4_scales_bytes(M, KA)), dtype=torch.uint8, device=dev),
             global_scale=torch.empty(1, dtype=torch.float32, device=dev),
-            workspace=torch.empty(nvfp4_quantize_workspace_bytes(M, K), dtype=torch.uint8, device=dev),
+            workspace=torch.empty(ws_bytes, dtype=torch.uint8, device=dev),
             rows=M, K=KA)
     _check_operand(x_out, "x_out", M, KA, dev, workspace=True)
     _check_operand(w, "w", N, KA, dev)
@@ -573,6 +593,15 @@ def quantize_arc_gemm(x, perm, S: int, w: NVFP4Tensor, mode: str = "six", rule: 
         workspace = torch.empty(nvfp4_gemm_workspace_bytes(), dtype=torch.uint8, device=dev)
     _check_output(out, M, N, out_dtype, dev)
     _require(workspace, "workspace", torch.uint8, 0, dev)
+    if gamma is not None:
+        st = nvfp4_quantize_arc_rmsnorm_gemm(
+            x.data_ptr(), M, K, _row_pitch(x), gamma.data_ptr(), float(eps), perm.data_ptr(), S, MODES[mode],
+            RULES[rule], F, x_out.codes.data_ptr(), x_out.scales.data_ptr(), x_out.global_scale.data_ptr(),
+            x_out.workspace.data_ptr(), x_out.workspace.numel(), w.codes.data_ptr(), w.scales.data_ptr(),
+            w.global_scale.data_ptr(), N, out.data_ptr(), _row_pitch(out), code, workspace.data_ptr(),
+            workspace.numel(), _stream_handle(stream))
+        _check(st, "nvfp4_quantize_arc_rmsnorm_gemm")
+        return x_out, out
     st = nvfp4_quantize_arc_gemm(x.data_ptr(), M, K, _row_pitch(x), perm.data_ptr(), S, MODES[mode], RULES[rule],
                                  F, x_out.codes.data_ptr(), x_out.scales.data_ptr(), x_out.global_scale.data_ptr(),
                                  x_out.workspace.data_ptr(), x_out.workspace.numel(), w.codes.data_ptr(),

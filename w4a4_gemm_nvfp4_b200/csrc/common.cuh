@@ -33,15 +33,18 @@ nvfp4_status quantize_rows_check(const char* fn, const void* x, int64_t rows, in
 nvfp4_status quantize_rows_enqueue(const char* fn, const void* x, int64_t rows, int64_t K, int64_t ldx, int mode,
                                    int rule, float fp8_max, void* codes, void* scales, float* global_scale,
                                    void* workspace, size_t workspace_bytes, void* stream);
-// The same pair for nvfp4_quantize_arc.
+// The same pair for nvfp4_quantize_arc; with `gamma` non-null, for
+// nvfp4_quantize_arc_rmsnorm (augment 0, RMSNorm with gains gamma and eps).
 nvfp4_status quantize_arc_check(const char* fn, const void* x, int64_t rows, int64_t K, int64_t ldx,
                                 const int32_t* perm, int64_t S, int augment, int mode, int rule, float fp8_max,
                                 const void* codes, const void* scales, const float* global_scale,
-                                const void* workspace, size_t workspace_bytes);
+                                const void* workspace, size_t workspace_bytes, const void* gamma = nullptr,
+                                float eps = 0.0f);
 nvfp4_status quantize_arc_enqueue(const char* fn, const void* x, int64_t rows, int64_t K, int64_t ldx,
                                   const int32_t* perm, int64_t S, int augment, int mode, int rule, float fp8_max,
                                   void* codes, void* scales, float* global_scale, void* workspace,
-                                  size_t workspace_bytes, void* stream);
+                                  size_t workspace_bytes, void* stream, const void* gamma = nullptr,
+                                  float eps = 0.0f);
 
 // Launches `kernel` on `stream`, as a programmatic dependent of the previous
 // kernel on the stream when `pdl` is set (the kernel must then call

@@ -875,15 +875,20 @@ nvfp4_status nvfp4_quantize_gemm(const void* x, int64_t M, int64_t K, int64_t ld
   return gemm_enqueue(L, s, false, true);
 }
 
-nvfp4_status nvfp4_quantize_arc_gemm(const void* x, int64_t M, int64_t K, int64_t ldx, const int32_t* perm,
-                                     int64_t S, int mode, int rule, float fp8_max, void* x_codes, void* x_scales,
-                                     float* x_global_scale, void* x_workspace, size_t x_workspace_bytes,
-                                     const void* w_codes, const void* w_scales, const float* w_global, int64_t N,
-                                     void* y, int64_t ldy, int out_dtype, void* workspace, size_t workspace_bytes,
-                                     void* stream) {
-  const char* fn = "nvfp4_quantize_arc_gemm";
+}  // extern "C"
+
+namespace {
+
+// The augmented-channel layer in one call (with the activations' RMSNorm
+// fused ahead when gamma is non-null).
+nvfp4_status arc_gemm_impl(const char* fn, const void* x, int64_t M, int64_t K, int64_t ldx, const void* gamma,
+                           float eps, const int32_t* perm, int64_t S, int mode, int rule, float fp8_max,
+                           void* x_codes, void* x_scales, float* x_global_scale, void* x_workspace,
+                           size_t x_workspace_bytes, const void* w_codes, const void* w_scales,
+                           const float* w_global, int64_t N, void* y, int64_t ldy, int out_dtype, void* workspace,
+                           size_t workspace_bytes, void* stream) {
   nvfp4_status st = quantize_arc_check(fn, x, M, K, ldx, perm, S, 0, mode, rule, fp8_max, x_codes, x_scales,
-                                       x_global_scale, x_workspace, x_workspace_bytes);
+                                       x_global_scale, x_workspace, x_workspace_bytes, gamma, eps);
   if (st != NVFP4_OK) return st;
   GemmLaunch L;
   const int64_t end = N;
@@ -897,9 +902,38 @@ nvfp4_status nvfp4_quantize_arc_gemm(const void* x, int64_t M, int64_t K, int64_
   cudaError_t e = cudaMemsetAsync(workspace, 0, sizeof(WorkspaceHeader), s);
   if (e != cudaSuccess) return cuda_status(e, "cudaMemsetAsync(status)");
   if ((st = quantize_arc_enqueue(fn, x, M, K, ldx, perm, S, 0, mode, rule, fp8_max, x_codes, x_scales,
-                                 x_global_scale, x_workspace, x_workspace_bytes, stream)) != NVFP4_OK)
+                                 x_global_scale, x_workspace, x_workspace_bytes, stream, gamma, eps)) != NVFP4_OK)
     return st;
   return gemm_enqueue(L, s, false, true);
+}
+
+}  // namespace
+
+extern "C" {
+
+nvfp4_status nvfp4_quantize_arc_gemm(const void* x, int64_t M, int64_t K, int64_t ldx, const int32_t* perm,
+                                     int64_t S, int mode, int rule, float fp8_max, void* x_codes, void* x_scales,
+                                     float* x_global_scale, void* x_workspace, size_t x_workspace_bytes,
+                                     const void* w_codes, const void* w_scales, const float* w_global, int64_t N,
+                                     void* y, int64_t ldy, int out_dtype, void* workspace, size_t workspace_bytes,
+                                     void* stream) {
+  return arc_gemm_impl("nvfp4_quantize_arc_gemm", x, M, K, ldx, nullptr, 0.0f, perm, S, mode, rule, fp8_max,
+                       x_codes, x_scales, x_global_scale, x_workspace, x_workspace_bytes, w_codes, w_scales,
+                       w_global, N, y, ldy, out_dtype, workspace, workspace_bytes, stream);
+}
+
+nvfp4_status nvfp4_quantize_arc_rmsnorm_gemm(const void* x, int64_t M, int64_t K, int64_t ldx, const void* gamma,
+                                             float eps, const int32_t* perm, int64_t S, int mode, int rule,
+                                             float fp8_max, void* x_codes, void* x_scales, float* x_global_scale,
+                                             void* x_workspace, size_t x_workspace_bytes, const void* w_codes,
+                                             const void* w_scales, const float* w_global, int64_t N, void* y,
+                                             int64_t ldy, int out_dtype, void* workspace, size_t workspace_bytes,
+                                             void* stream) {
+  const char* fn = "nvfp4_quantize_arc_rmsnorm_gemm";
+  if (!gamma) return set_error(NVFP4_ERR_INVALID_ARG, "%s: null pointer argument", fn);
+  return arc_gemm_impl(fn, x, M, K, ldx, gamma, eps, perm, S, mode, rule, fp8_max, x_codes, x_scales,
+                       x_global_scale, x_workspace, x_workspace_bytes, w_codes, w_scales, w_global, N, y, ldy,
+                       out_dtype, workspace, workspace_bytes, stream);
 }
 
 nvfp4_status nvfp4_gemm_segmented(const void* a_codes, const void* a_scales, const float* a_global,

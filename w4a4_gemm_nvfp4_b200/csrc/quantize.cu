@@ -1116,17 +1116,19 @@ nvfp4_status quantize_rows_check(const char* fn, const void* x, int64_t rows, in
 nvfp4_status quantize_arc_check(const char* fn, const void* x, int64_t rows, int64_t K, int64_t ldx,
                                 const int32_t* perm, int64_t S, int augment, int mode, int rule, float fp8_max,
                                 const void* codes, const void* scales, const float* global_scale,
-                                const void* workspace, size_t workspace_bytes) {
+                                const void* workspace, size_t workspace_bytes, const void* gamma, float eps) {
   return check_quantize_call(fn, QuantKind::kAugmented, x, rows, K, ldx, mode, rule, fp8_max, codes, scales,
-                             global_scale, workspace, workspace_bytes, perm, S, augment);
+                             global_scale, workspace, workspace_bytes, perm, S, augment,
+                             static_cast<const uint16_t*>(gamma), eps);
 }
 
 nvfp4_status quantize_arc_enqueue(const char* fn, const void* x, int64_t rows, int64_t K, int64_t ldx,
                                   const int32_t* perm, int64_t S, int augment, int mode, int rule, float fp8_max,
                                   void* codes, void* scales, float* global_scale, void* workspace,
-                                  size_t workspace_bytes, void* stream) {
+                                  size_t workspace_bytes, void* stream, const void* gamma, float eps) {
   return quantize_impl(fn, QuantKind::kAugmented, x, rows, K, ldx, mode, rule, fp8_max, codes, scales,
-                       global_scale, workspace, workspace_bytes, stream, perm, S, augment);
+                       global_scale, workspace, workspace_bytes, stream, perm, S, augment,
+                       static_cast<const uint16_t*>(gamma), eps);
 }
 
 nvfp4_status quantize_rows_enqueue(const char* fn, const void* x, int64_t rows, int64_t K, int64_t ldx, int mode,
