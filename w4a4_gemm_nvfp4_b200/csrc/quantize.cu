@@ -67,6 +67,9 @@ __device__ __forceinline__ uint4 ld_stream(const uint4* p) {
 // every NaN pattern (> 0x7F80) compares above Inf (0x7F80) above any finite
 // value, so one unsigned max gives both amax and the non-finite flag.  Each
 // thread keeps eight 16-byte loads in flight; two 512-thread CTAs per SM.
+// The pass walks x from its end, so that its last reads -- the front of x,
+// where the quantize kernel starts -- are the ones still in L2 (measured: 4/6
+// amax + quantize 2 us faster on a 32768 x 5120 x).
 __global__ void __launch_bounds__(kAmaxThreads, 2)
     amax_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t K, int64_t ldx,
                 uint32_t* __restrict__ partials) {
@@ -80,15 +83,15 @@ __global__ void __launch_bounds__(kAmaxThreads, 2)
     for (; i + 7 * stride < n; i += 8 * stride) {
       uint4 a[8];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) a[u] = ld_stream(v + i + u * stride);
+      for (int u = 0; u < 8; ++u) a[u] = ld_stream(v + (n - 1 - (i + u * stride)));
 #pragma unroll
       for (int u = 0; u < 8; ++u) m = absmax4(a[u], m);
     }
-    for (; i < n; i += stride) m = absmax4(ld_stream(v + i), m);
+    for (; i < n; i += stride) m = absmax4(ld_stream(v + (n - 1 - i)), m);
   } else {
     const int64_t k8 = K / 8;
     for (int64_t r = blockIdx.x; r < rows; r += gridDim.x) {
-      const uint4* v = reinterpret_cast<const uint4*>(x + r * ldx);
+      const uint4* v = reinterpret_cast<const uint4*>(x + (rows - 1 - r) * ldx);
       for (int64_t c = threadIdx.x; c < k8; c += blockDim.x) m = absmax4(ld_stream(v + c), m);
     }
   }
