@@ -25,11 +25,16 @@
 //                    every CTA, then makes one HBM pass over x: each lane owns
 //                    one whole 16-element block (two 16-byte loads), so the
 //                    block max and both candidates' errors stay in registers
-//                    with no shuffles.  Blocks are taken in row-major order,
-//                    32 consecutive blocks (1 KB of x) per warp task, so the
-//                    grid sweeps x front to back; every lane writes its 8
-//                    code bytes and its scale byte at that block's place in
-//                    the swizzled scale layout.
+//                    with no shuffles.  A warp task is a pair of chunks of 32
+//                    consecutive blocks (2 x 1 KB of x) of one row, and the
+//                    warps of the grid take the tasks in a sweep, so x is read
+//                    front to back; every lane writes its 8 code bytes and its
+//                    scale byte at that block's place in the swizzled scale
+//                    layout.
+// The other entry points reuse the block step: quantize_t_kernel (blocks down
+// the columns of x, through shared-memory tiles), quantize_arc_kernel
+// (reordered channels plus appended residual or duplicated ones, with an
+// optional RMSNorm of the activations) and its RMS pass rms_amax_kernel.
 #include <cuda_fp16.h>
 
 #include <algorithm>
