@@ -438,14 +438,16 @@ __global__ void __launch_bounds__(kQuantThreads)
 //   r = 1 / sqrt(sum_k x_k^2 / K + eps),  y_k = bf16((x_k * r) * gamma_k)
 // with the sum of squares taken as the contiguous pairwise tree over the row
 // (zero-padded to a power of two P).  One warp per row, no block barrier: in
-// round q the warp reads 256 consecutive elements (lane l the 16-byte group
-// 32q + l, coalesced), each lane sums its group's squares as a pairwise tree,
-// and an xor butterfly over the lanes combines the groups (1, then 2, 4, ...
-// adjacent subtrees: the same tree, addition being commutative); the rounds'
+// round q the warp reads 1024 consecutive elements, lane l the four 16-byte
+// groups 128q + 4l .. 128q + 4l + 3 (64 contiguous bytes; the warp's four
+// loads cover 2 KB), sums its 32 squares as a pairwise tree, and an xor
+// butterfly over the lanes combines the lanes' adjacent subtrees (1, then 2,
+// 4, ... lanes: the same tree, addition being commutative).  The rounds'
 // sums, all lanes holding them, merge like a binary counter (each completed
-// subtree added to the equal-size one on its left).  Every lane ends with the
-// row's sum and computes r.  The pass writes r for every row and, like the
-// amax pass, each CTA's max |y| as a bf16 bit pattern.
+// subtree added to the equal-size one on its left); the zero padding past the
+// last round is not computed.  Every lane ends with the row's sum and computes
+// r.  The pass writes r for every row and, like the amax pass, each CTA's max
+// |y| as a bf16 bit pattern.
 constexpr int kRmsThreads = 256;
 
 // two binary32 values -> a bf16 pair (lo in the low half), nearest, ties to even
@@ -490,22 +492,29 @@ __global__ void __launch_bounds__(kRmsThreads)
   pdl_launch_dependents();  // the quantize kernel may be scheduled now; it waits for this grid's end
   // rounds that hold elements; the zero-padded rest of the tree up to the next
   // power of two adds exact zeros and is not computed
-  const int used = static_cast<int>((K + 255) / 256);  // 1 .. 64 (K <= 16384)
+  const int used = static_cast<int>((K + 1023) / 1024);  // 1 .. 16 (K <= 16384)
   const int lane = static_cast<int>(threadIdx.x & 31), warp = static_cast<int>(threadIdx.x >> 5);
   const int64_t nwarps = static_cast<int64_t>(gridDim.x) * (kRmsThreads / 32);
   uint32_t m = 0;
   for (int64_t r = static_cast<int64_t>(blockIdx.x) * (kRmsThreads / 32) + warp; r < rows; r += nwarps) {
     const uint16_t* xr = x + r * ldx;
-    float stk[7];
+    float stk[5];
     float v = 0.0f;
     for (int q = 0; q < used; ++q) {
-      const int64_t k = 256 * static_cast<int64_t>(q) + 8 * lane;  // K % 8 == 0: a group is inside or past the row
-      v = k < K ? sq_tree8(*reinterpret_cast<const uint4*>(xr + k)) : 0.0f;
+      // this lane's four groups (K % 8 == 0: a group is inside or past the row)
+      const int64_t k0 = 1024 * static_cast<int64_t>(q) + 32 * lane;
+      float g[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int64_t k = k0 + 8 * u;
+        g[u] = k < K ? sq_tree8(*reinterpret_cast<const uint4*>(xr + k)) : 0.0f;
+      }
+      v = __fadd_rn(__fadd_rn(g[0], g[1]), __fadd_rn(g[2], g[3]));
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) v = __fadd_rn(v, __shfl_xor_sync(0xffffffffu, v, o));
       // merge with the completed round subtrees of equal size on the left
 #pragma unroll
-      for (int lvl = 0; lvl < 7; ++lvl) {
+      for (int lvl = 0; lvl < 5; ++lvl) {
         if (!((q >> lvl) & 1)) {
           stk[lvl] = v;
           break;
@@ -518,7 +527,7 @@ __global__ void __launch_bounds__(kRmsThreads)
     // operand of everything to its right
     bool have = false;
 #pragma unroll
-    for (int lvl = 0; lvl < 7; ++lvl) {
+    for (int lvl = 0; lvl < 5; ++lvl) {
       if ((used >> lvl) & 1) {
         v = have ? __fadd_rn(stk[lvl], v) : stk[lvl];
         have = true;
@@ -527,11 +536,16 @@ __global__ void __launch_bounds__(kRmsThreads)
     const float ms = __fdiv_rn(v, static_cast<float>(K));
     const float rr = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(ms, eps)));
     if (lane == 0) rinv[r] = rr;
-    // the row's outputs and their max |y|, in the same coalesced order
+    // the row's outputs and their max |y|, read in the same order
     for (int q = 0; q < used; ++q) {
-      const int64_t k = 256 * static_cast<int64_t>(q) + 8 * lane;
-      if (k < K)
-        m = rms_group_max(*reinterpret_cast<const uint4*>(xr + k), *reinterpret_cast<const uint4*>(gamma + k), rr, m);
+      const int64_t k0 = 1024 * static_cast<int64_t>(q) + 32 * lane;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int64_t k = k0 + 8 * u;
+        if (k < K)
+          m = rms_group_max(*reinterpret_cast<const uint4*>(xr + k), *reinterpret_cast<const uint4*>(gamma + k), rr,
+                            m);
+      }
     }
   }
 #pragma unroll
