@@ -121,7 +121,8 @@ def gpu_arc_rmsnorm(x_cpu, gamma, eps, perm, S, mode, rule, F, canary=0xA5):
 
 @pytest.mark.parametrize("recipe", RECIPES, ids=lambda r: "-".join(map(str, r)))
 @pytest.mark.parametrize("shape,S", [((1, 64), 64), ((129, 256), 64), ((300, 512), 128), ((64, 1024), 0),
-                                     ((37, 5120), 128), ((5, 16384), 256)], ids=str)
+                                     ((33, 2112), 64), ((37, 5120), 128), ((9, 7168), 128), ((6, 8192), 0),
+                                     ((4, 8256), 64), ((5, 16384), 256)], ids=str)
 def test_quantize_arc_rmsnorm_matches_oracle(shape, S, recipe):
     """Bit-exact with the oracle's RMSNorm (pinned in test_oracle_rmsnorm.py)
     followed by its augmented quantization; every byte, padding included."""
@@ -134,6 +135,19 @@ def test_quantize_arc_rmsnorm_matches_oracle(shape, S, recipe):
     assert status == nv.OK
     y = torch.from_numpy(oracle.rmsnorm(x, gamma, 1e-6).view(np.int16)).view(torch.bfloat16)
     assert_arc_equal(q, y, perm, S, nv.AUG_RESIDUAL, mode, rule, F)
+
+
+def test_quantize_arc_rmsnorm_more_rows_than_warps():
+    """More rows than the RMS pass has warps in one wave at K = 5120 (each warp
+    takes several rows in turn)."""
+    rows, K, S = 2600, 5120, 128
+    x = workloads.small_operand(rows, K, seed=11).make()
+    gamma = _gains(K, 3)
+    perm = outlier_perm(x)
+    q, status = gpu_arc_rmsnorm(x, gamma, 1e-6, perm, S, "four_over_six", "mse", 256.0)
+    assert status == nv.OK
+    y = torch.from_numpy(oracle.rmsnorm(x, gamma, 1e-6).view(np.int16)).view(torch.bfloat16)
+    assert_arc_equal(q, y, perm, S, nv.AUG_RESIDUAL, "four_over_six", "mse", 256.0)
 
 
 def test_quantize_arc_rmsnorm_reading_pins():

@@ -449,6 +449,7 @@ __global__ void __launch_bounds__(kQuantThreads)
 // r.  The pass writes r for every row and, like the amax pass, each CTA's max
 // |y| as a bf16 bit pattern.
 constexpr int kRmsThreads = 256;
+constexpr int kRmsRegThreads = 128;
 
 // two binary32 values -> a bf16 pair (lo in the low half), nearest, ties to even
 __device__ __forceinline__ uint32_t bf16x2_rn(float lo, float hi) {
@@ -457,34 +458,109 @@ __device__ __forceinline__ uint32_t bf16x2_rn(float lo, float hi) {
   return w;
 }
 
-// the squares of the 8 bf16 values of one 16-byte group, summed as a pairwise tree
-__device__ __forceinline__ float sq_tree8(const uint4 v) {
-  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-  float a[8];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const float lo = __uint_as_float(w[i] << 16), hi = __uint_as_float(w[i] & 0xFFFF0000u);
-    a[2 * i] = __fmul_rn(lo, lo);
-    a[2 * i + 1] = __fmul_rn(hi, hi);
-  }
-  const float b0 = __fadd_rn(a[0], a[1]), b1 = __fadd_rn(a[2], a[3]);
-  const float b2 = __fadd_rn(a[4], a[5]), b3 = __fadd_rn(a[6], a[7]);
-  return __fadd_rn(__fadd_rn(b0, b1), __fadd_rn(b2, b3));
+// the squares of a bf16 pair, each rounded once to binary32 (the mixed-precision
+// fma computes x * x + (-0) exactly and rounds it: the binary32 product)
+__device__ __forceinline__ void sq_pair(uint32_t w, float& lo, float& hi) {
+  asm("{\n\t.reg .b16 l, h;\n\t"
+      "mov.b32 {l, h}, %2;\n\t"
+      "fma.rn.f32.bf16 %0, l, l, 0f80000000;\n\t"
+      "fma.rn.f32.bf16 %1, h, h, 0f80000000;\n\t}"
+      : "=f"(lo), "=f"(hi)
+      : "r"(w));
 }
 
-// max |y| of one 16-byte group of x and its gains, y = bf16((x * r) * gamma)
-__device__ __forceinline__ uint32_t rms_group_max(const uint4 xv, const uint4 gv, float r, uint32_t m) {
+// the squares of the 8 bf16 values of one 16-byte group, summed as a pairwise tree
+__device__ __forceinline__ float sq_tree8(const uint4 v) {
+  float a[8];
+  sq_pair(v.x, a[0], a[1]);
+  sq_pair(v.y, a[2], a[3]);
+  sq_pair(v.z, a[4], a[5]);
+  sq_pair(v.w, a[6], a[7]);
+  // first level in packed pairs: (a0 + a1, a2 + a3) and (a4 + a5, a6 + a7)
+  const f2 b01 = add2(make_f2(a[0], a[2]), make_f2(a[1], a[3]));
+  const f2 b23 = add2(make_f2(a[4], a[6]), make_f2(a[5], a[7]));
+  return __fadd_rn(__fadd_rn(b01.a(), b01.b()), __fadd_rn(b23.a(), b23.b()));
+}
+
+// max(m, |(x * r) * gamma|) over one 16-byte group of x and its gains, in
+// binary32 before the bf16 rounding: rounding to nearest is monotone and odd,
+// so the largest |bf16(y)| is bf16 of the largest |y| and the pass rounds once
+__device__ __forceinline__ float rms_group_max(const uint4 xv, const uint4 gv, f2 rr, float m) {
   const uint32_t xs[4] = {xv.x, xv.y, xv.z, xv.w}, gs[4] = {gv.x, gv.y, gv.z, gv.w};
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    const float y0 = __fmul_rn(__fmul_rn(__uint_as_float(xs[i] << 16), r), __uint_as_float(gs[i] << 16));
-    const float y1 = __fmul_rn(__fmul_rn(__uint_as_float(xs[i] & 0xFFFF0000u), r), __uint_as_float(gs[i] & 0xFFFF0000u));
-    const uint32_t yw = bf16x2_rn(y0, y1);
-    m = max(m, max(yw & 0x7FFFu, (yw >> 16) & 0x7FFFu));
+    const f2 xf = make_f2(__uint_as_float(xs[i] << 16), __uint_as_float(xs[i] & 0xFFFF0000u));
+    const f2 gf = make_f2(__uint_as_float(gs[i] << 16), __uint_as_float(gs[i] & 0xFFFF0000u));
+    const f2 y = mul2(mul2(xf, rr), gf);
+    m = max3_nan(m, fabsf(y.a()), fabsf(y.b()));
   }
   return m;
 }
 
+// one round: the sum of this lane's four groups (32 contiguous elements; s_u
+// the pairwise sum of group u) as a pairwise tree, combined over the warp by the xor butterfly (a 1024-element
+// subtree; zero groups past the row add exact zeros)
+__device__ __forceinline__ float rms_round(float s0, float s1, float s2, float s3) {
+  float v = __fadd_rn(__fadd_rn(s0, s1), __fadd_rn(s2, s3));
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) v = __fadd_rn(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+// round q's subtree into the binary counter: each completed subtree is added
+// to the equal-size one on its left (q < 16)
+__device__ __forceinline__ void rms_push(float (&stk)[5], int q, float v) {
+#pragma unroll
+  for (int lvl = 0; lvl < 5; ++lvl) {
+    if (!((q >> lvl) & 1)) {
+      stk[lvl] = v;
+      break;
+    }
+    v = __fadd_rn(stk[lvl], v);
+  }
+}
+
+// the row's sum after `used` rounds: the counter holds one complete subtree
+// per set bit of `used`, the lowest bit's the rightmost; the zero padding up
+// to the next power of two leaves each the left operand of all to its right
+__device__ __forceinline__ float rms_close(const float (&stk)[5], int used) {
+  float v = 0.0f;
+  bool have = false;
+#pragma unroll
+  for (int lvl = 0; lvl < 5; ++lvl) {
+    if ((used >> lvl) & 1) {
+      v = have ? __fadd_rn(stk[lvl], v) : stk[lvl];
+      have = true;
+    }
+  }
+  return v;
+}
+
+// r = 1 / sqrt(sum / K + eps), each step one rounding
+__device__ __forceinline__ float rms_rinv(float sum, int64_t K, float eps) {
+  return __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(__fdiv_rn(sum, static_cast<float>(K)), eps)));
+}
+
+// the CTA's max |bf16(y)| from each lane's binary32 max, as a bf16 bit
+// pattern (a NaN becomes 0x7FFF), into partials[blockIdx.x]
+template <int THREADS>
+__device__ __forceinline__ void rms_write_partial(float m, uint32_t* partials) {
+  const int lane = static_cast<int>(threadIdx.x & 31), warp = static_cast<int>(threadIdx.x >> 5);
+  uint32_t mb = bf16x2_rn(m, 0.0f) & 0x7FFFu;
+#pragma unroll
+  for (int o = 16; o; o >>= 1) mb = max(mb, __shfl_xor_sync(0xffffffffu, mb, o));
+  __shared__ uint32_t s_max[THREADS / 32];
+  if (lane == 0) s_max[warp] = mb;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    uint32_t mm = 0;
+    for (int w = 0; w < THREADS / 32; ++w) mm = max(mm, s_max[w]);
+    partials[blockIdx.x] = mm;
+  }
+}
+
+// The RMS pass for any K <= 16384: round by round, the y phase reading the row
+// again (from L2).
 __global__ void __launch_bounds__(kRmsThreads)
     rms_amax_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t K, int64_t ldx,
                     const uint16_t* __restrict__ gamma, float eps, float* __restrict__ rinv,
@@ -495,69 +571,78 @@ __global__ void __launch_bounds__(kRmsThreads)
   const int used = static_cast<int>((K + 1023) / 1024);  // 1 .. 16 (K <= 16384)
   const int lane = static_cast<int>(threadIdx.x & 31), warp = static_cast<int>(threadIdx.x >> 5);
   const int64_t nwarps = static_cast<int64_t>(gridDim.x) * (kRmsThreads / 32);
-  uint32_t m = 0;
+  float m = 0.0f;
   for (int64_t r = static_cast<int64_t>(blockIdx.x) * (kRmsThreads / 32) + warp; r < rows; r += nwarps) {
     const uint16_t* xr = x + r * ldx;
     float stk[5];
-    float v = 0.0f;
     for (int q = 0; q < used; ++q) {
       // this lane's four groups (K % 8 == 0: a group is inside or past the row)
-      const int64_t k0 = 1024 * static_cast<int64_t>(q) + 32 * lane;
       float g[4];
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
-        const int64_t k = k0 + 8 * u;
+        const int64_t k = 1024 * static_cast<int64_t>(q) + 32 * lane + 8 * u;
         g[u] = k < K ? sq_tree8(*reinterpret_cast<const uint4*>(xr + k)) : 0.0f;
       }
-      v = __fadd_rn(__fadd_rn(g[0], g[1]), __fadd_rn(g[2], g[3]));
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) v = __fadd_rn(v, __shfl_xor_sync(0xffffffffu, v, o));
-      // merge with the completed round subtrees of equal size on the left
-#pragma unroll
-      for (int lvl = 0; lvl < 5; ++lvl) {
-        if (!((q >> lvl) & 1)) {
-          stk[lvl] = v;
-          break;
-        }
-        v = __fadd_rn(stk[lvl], v);
-      }
+      rms_push(stk, q, rms_round(g[0], g[1], g[2], g[3]));
     }
-    // the stack now holds one complete subtree per set bit of `used`, the
-    // lowest bit's the rightmost; the zero padding leaves each as the left
-    // operand of everything to its right
-    bool have = false;
-#pragma unroll
-    for (int lvl = 0; lvl < 5; ++lvl) {
-      if ((used >> lvl) & 1) {
-        v = have ? __fadd_rn(stk[lvl], v) : stk[lvl];
-        have = true;
-      }
-    }
-    const float ms = __fdiv_rn(v, static_cast<float>(K));
-    const float rr = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(ms, eps)));
+    const float rr = rms_rinv(rms_close(stk, used), K, eps);
     if (lane == 0) rinv[r] = rr;
     // the row's outputs and their max |y|, read in the same order
+    const f2 rrr = make_f2(rr, rr);
     for (int q = 0; q < used; ++q) {
-      const int64_t k0 = 1024 * static_cast<int64_t>(q) + 32 * lane;
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
-        const int64_t k = k0 + 8 * u;
+        const int64_t k = 1024 * static_cast<int64_t>(q) + 32 * lane + 8 * u;
         if (k < K)
-          m = rms_group_max(*reinterpret_cast<const uint4*>(xr + k), *reinterpret_cast<const uint4*>(gamma + k), rr,
+          m = rms_group_max(*reinterpret_cast<const uint4*>(xr + k), *reinterpret_cast<const uint4*>(gamma + k), rrr,
                             m);
       }
     }
   }
+  rms_write_partial<kRmsThreads>(m, partials);
+}
+
+// The RMS pass with the row held in registers (K <= 1024 * NR): a warp issues
+// every load of its row before any arithmetic, so the whole row is in flight
+// at once, and the y phase works on the same registers.
+template <int NR>
+__global__ void __launch_bounds__(kRmsRegThreads)
+    rms_amax_reg_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t K, int64_t ldx,
+                        const uint16_t* __restrict__ gamma, float eps, float* __restrict__ rinv,
+                        uint32_t* __restrict__ partials) {
+  pdl_launch_dependents();
+  constexpr int kWarps = kRmsRegThreads / 32;
+  const int lane = static_cast<int>(threadIdx.x & 31), warp = static_cast<int>(threadIdx.x >> 5);
+  const int64_t nwarps = static_cast<int64_t>(gridDim.x) * kWarps;
+  float m = 0.0f;
+  for (int64_t r = static_cast<int64_t>(blockIdx.x) * kWarps + warp; r < rows; r += nwarps) {
+    const uint16_t* xr = x + r * ldx;
+    uint4 d[NR][4];
 #pragma unroll
-  for (int o = 16; o; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
-  __shared__ uint32_t s_max[kRmsThreads / 32];
-  if (lane == 0) s_max[warp] = m;
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    uint32_t mm = 0;
-    for (int w = 0; w < kRmsThreads / 32; ++w) mm = max(mm, s_max[w]);
-    partials[blockIdx.x] = mm;
+    for (int q = 0; q < NR; ++q) {
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int64_t k = 1024 * q + 32 * lane + 8 * u;
+        d[q][u] = k < K ? *reinterpret_cast<const uint4*>(xr + k) : make_uint4(0u, 0u, 0u, 0u);
+      }
+    }
+    float stk[5];
+#pragma unroll
+    for (int q = 0; q < NR; ++q)
+      rms_push(stk, q, rms_round(sq_tree8(d[q][0]), sq_tree8(d[q][1]), sq_tree8(d[q][2]), sq_tree8(d[q][3])));
+    const float rr = rms_rinv(rms_close(stk, NR), K, eps);
+    if (lane == 0) rinv[r] = rr;
+    const f2 rrr = make_f2(rr, rr);
+#pragma unroll
+    for (int q = 0; q < NR; ++q) {
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int64_t k = 1024 * q + 32 * lane + 8 * u;
+        if (k < K) m = rms_group_max(d[q][u], *reinterpret_cast<const uint4*>(gamma + k), rrr, m);
+      }
+    }
   }
+  rms_write_partial<kRmsRegThreads>(m, partials);
 }
 
 // The RMSNorm of a gathered block: x (8 bf16 pairs, element 2i low) becomes
@@ -1036,12 +1121,62 @@ nvfp4_status launch_dynamic(QuantKind kind, QuantParams p, int mode, int rule, f
 
 // The RMS pass, then the augmented quantizer with RMSNorm as its
 // programmatic dependent.
+// One wave of CTAs of `kernel` (threads each), at most one warp per row.
+template <typename Kernel>
+cudaError_t rms_grid(PerContextCache<int>& per_sm, Kernel kernel, int threads, int dev, int sms, int64_t rows,
+                     int* grid) {
+  int occ = 0;
+  const cudaError_t e = per_context(per_sm, dev, [kernel, threads](int* v) {
+    const cudaError_t r = cudaOccupancyMaxActiveBlocksPerMultiprocessor(v, kernel, threads, 0);
+    *v = std::max(1, *v);
+    return r;
+  }, &occ);
+  if (e != cudaSuccess) return e;
+  const int64_t want = (rows + threads / 32 - 1) / (threads / 32);
+  *grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(std::min<int64_t>(want, int64_t{sms} * occ),
+                                                                  kMaxPartials)));
+  return cudaSuccess;
+}
+
+template <int NR>
+cudaError_t launch_rms_reg(const QuantParams& p, uint32_t* partials, float eps, int dev, int sms, cudaStream_t s,
+                           int* grid) {
+  static PerContextCache<int> per_sm;
+  cudaError_t e = rms_grid(per_sm, rms_amax_reg_kernel<NR>, kRmsRegThreads, dev, sms, p.rows, grid);
+  if (e != cudaSuccess) return e;
+  rms_amax_reg_kernel<NR><<<*grid, kRmsRegThreads, 0, s>>>(p.x, p.rows, p.K, p.ldx, p.gamma, eps,
+                                                            const_cast<float*>(p.rinv), partials);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_rms_pass(const QuantParams& p, uint32_t* partials, float eps, int dev, int sms, cudaStream_t s,
+                            int* grid) {
+  // the row in registers up to K = 8192 (168 registers at 8 rounds), round by
+  // round above that
+  switch ((p.K + 1023) / 1024) {
+    case 1: return launch_rms_reg<1>(p, partials, eps, dev, sms, s, grid);
+    case 2: return launch_rms_reg<2>(p, partials, eps, dev, sms, s, grid);
+    case 3: return launch_rms_reg<3>(p, partials, eps, dev, sms, s, grid);
+    case 4: return launch_rms_reg<4>(p, partials, eps, dev, sms, s, grid);
+    case 5: return launch_rms_reg<5>(p, partials, eps, dev, sms, s, grid);
+    case 6: return launch_rms_reg<6>(p, partials, eps, dev, sms, s, grid);
+    case 7: return launch_rms_reg<7>(p, partials, eps, dev, sms, s, grid);
+    case 8: return launch_rms_reg<8>(p, partials, eps, dev, sms, s, grid);
+    default: break;
+  }
+  static PerContextCache<int> per_sm;
+  cudaError_t e = rms_grid(per_sm, rms_amax_kernel, kRmsThreads, dev, sms, p.rows, grid);
+  if (e != cudaSuccess) return e;
+  rms_amax_kernel<<<*grid, kRmsThreads, 0, s>>>(p.x, p.rows, p.K, p.ldx, p.gamma, eps, const_cast<float*>(p.rinv),
+                                               partials);
+  return cudaGetLastError();
+}
+
 nvfp4_status launch_rms_dynamic(QuantParams p, int mode, int rule, float fp8_max, float* global_scale,
-                                uint32_t* partials, int grid, float eps, int dev, int sms, cudaStream_t s) {
-  rms_amax_kernel<<<grid, kRmsThreads, 0, s>>>(p.x, p.rows, p.K, p.ldx, p.gamma, eps, const_cast<float*>(p.rinv),
-                                              partials);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return cuda_status(e, "rms_amax_kernel launch");
+                                uint32_t* partials, float eps, int dev, int sms, cudaStream_t s) {
+  int grid = 0;
+  cudaError_t e = launch_rms_pass(p, partials, eps, dev, sms, s, &grid);
+  if (e != cudaSuccess) return cuda_status(e, "RMS pass launch");
   p.global_scale = global_scale;
   p.partials = partials;
   p.nparts = grid;
@@ -1113,10 +1248,7 @@ nvfp4_status quantize_impl(const char* fn, QuantKind kind, const void* x, int64_
     // pass's place and leaves 1/rms of every row after the partials
     p.gamma = gamma;
     p.rinv = reinterpret_cast<float*>(static_cast<char*>(workspace) + nvfp4_quantize_workspace_bytes(rows, K));
-    // one warp per row: enough CTAs for every row, at most eight per SM
-    const int64_t want = (rows + kRmsThreads / 32 - 1) / (kRmsThreads / 32);
-    const int grid = static_cast<int>(std::min<int64_t>(std::min<int64_t>(want, int64_t{sms} * 8), kMaxPartials));
-    return launch_rms_dynamic(p, mode, rule, fp8_max, global_scale, partials, grid, eps, dev, sms,
+    return launch_rms_dynamic(p, mode, rule, fp8_max, global_scale, partials, eps, dev, sms,
                               static_cast<cudaStream_t>(stream));
   }
   const int amax_grid = std::min(amax_grid_size(rows, K, ldx, sms), kMaxPartials);
