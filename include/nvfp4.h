@@ -169,9 +169,9 @@ NVFP4_API nvfp4_status nvfp4_quantize_arc(const void* x, int64_t rows, int64_t K
  * every step one binary32 operation, the sum of squares taken as the
  * contiguous pairwise tree over the row (zero-padded to a power of two), the
  * square root and the divisions correctly rounded.  alpha is the amax of y.
- * y is never written: a row pass computes r_i (kept in the workspace) and the
- * amax partials, and the augmented quantizer normalizes the channels it
- * gathers.
+ * y is never written: a row pass computes r_i and the amax partials, and
+ * copies gamma into channel order (both kept in the workspace), and the
+ * augmented quantizer normalizes the channels it gathers.
  *   gamma   device bf16[K], 16-byte aligned
  *   eps     a positive finite number
  *   workspace  nvfp4_quantize_arc_rmsnorm_workspace_bytes(rows, K) bytes

@@ -302,9 +302,14 @@ def test_quantize_arc_rmsnorm_rejects_bad_arguments(bad):
     assert nv.last_error_message().startswith("nvfp4_quantize_arc_rmsnorm")
 
 
-def test_quantize_arc_rmsnorm_workspace_holds_a_float_per_row():
-    assert (nv.nvfp4_quantize_arc_rmsnorm_workspace_bytes(4096, 512)
-            == nv.nvfp4_quantize_workspace_bytes(4096, 512) + 4 * 4096)
+def test_quantize_arc_rmsnorm_workspace_holds_a_float_per_row_and_the_gains():
+    """The quantize workspace, then a float per row and a bf16 gain per channel,
+    each area rounded up to 16 bytes."""
+    def up16(n):
+        return (n + 15) // 16 * 16
+    for rows, K in ((4096, 512), (3, 64), (1, 5120), (77, 16384)):
+        assert (nv.nvfp4_quantize_arc_rmsnorm_workspace_bytes(rows, K)
+                == nv.nvfp4_quantize_workspace_bytes(rows, K) + up16(4 * rows) + up16(2 * K))
 
 
 def test_quantize_arc_rmsnorm_without_gpu_fails_loudly():

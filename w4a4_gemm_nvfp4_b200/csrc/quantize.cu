@@ -47,6 +47,7 @@ namespace {
 
 constexpr int kAmaxThreads = 512;
 constexpr int kMaxPartials = 4096;
+constexpr size_t align16(size_t n) { return (n + 15) & ~static_cast<size_t>(15); }
 constexpr int kArcMaxRows = 4;              // rows per step of the augmented quantizer, at most
 constexpr int kArcPrimThreads = 256;        // its threads for the primary blocks, at most
 constexpr int kArcMaxThreads = 640;         // its block size, at most
@@ -138,6 +139,7 @@ struct QuantParams {
   // RMSNorm ahead of the augmented quantizer only
   const uint16_t* gamma = nullptr;  // bf16 gains, K entries
   const float* rinv = nullptr;      // 1 / rms of each row, written by the RMS pass
+  const uint16_t* gperm = nullptr;  // the gains in channel order (gamma[perm[i]]), written by the RMS pass
 };
 
 // Start of every quantize kernel: alpha (a caller-supplied static scale, or
@@ -559,13 +561,25 @@ __device__ __forceinline__ void rms_write_partial(float m, uint32_t* partials) {
   }
 }
 
+// gperm[i] = gamma[perm[i]] over the grid's threads, for the augmented
+// quantizer's RMSNorm (an out-of-range channel reads channel 0, as there)
+__device__ __forceinline__ void rms_permute_gains(const uint16_t* gamma, const int32_t* perm, int64_t K,
+                                                  uint16_t* gperm) {
+  const int64_t n = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < K; i += n) {
+    const int32_t c = perm[i];
+    gperm[i] = gamma[c >= 0 && c < K ? c : 0];
+  }
+}
+
 // The RMS pass for any K <= 16384: round by round, the y phase reading the row
 // again (from L2).
 __global__ void __launch_bounds__(kRmsThreads)
     rms_amax_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t K, int64_t ldx,
-                    const uint16_t* __restrict__ gamma, float eps, float* __restrict__ rinv,
-                    uint32_t* __restrict__ partials) {
+                    const uint16_t* __restrict__ gamma, float eps, const int32_t* __restrict__ perm,
+                    float* __restrict__ rinv, uint16_t* __restrict__ gperm, uint32_t* __restrict__ partials) {
   pdl_launch_dependents();  // the quantize kernel may be scheduled now; it waits for this grid's end
+  rms_permute_gains(gamma, perm, K, gperm);
   // rounds that hold elements; the zero-padded rest of the tree up to the next
   // power of two adds exact zeros and is not computed
   const int used = static_cast<int>((K + 1023) / 1024);  // 1 .. 16 (K <= 16384)
@@ -606,11 +620,12 @@ __global__ void __launch_bounds__(kRmsThreads)
 // every load of its row before any arithmetic, so the whole row is in flight
 // at once, and the y phase works on the same registers.
 template <int NR>
-__global__ void __launch_bounds__(kRmsRegThreads)
+__global__ void __launch_bounds__(kRmsRegThreads, NR <= 2 ? 8 : NR <= 3 ? 5 : NR <= 6 ? 4 : 3)
     rms_amax_reg_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t K, int64_t ldx,
-                        const uint16_t* __restrict__ gamma, float eps, float* __restrict__ rinv,
-                        uint32_t* __restrict__ partials) {
+                        const uint16_t* __restrict__ gamma, float eps, const int32_t* __restrict__ perm,
+                        float* __restrict__ rinv, uint16_t* __restrict__ gperm, uint32_t* __restrict__ partials) {
   pdl_launch_dependents();
+  rms_permute_gains(gamma, perm, K, gperm);
   constexpr int kWarps = kRmsRegThreads / 32;
   const int lane = static_cast<int>(threadIdx.x & 31), warp = static_cast<int>(threadIdx.x >> 5);
   const int64_t nwarps = static_cast<int64_t>(gridDim.x) * kWarps;
@@ -645,16 +660,25 @@ __global__ void __launch_bounds__(kRmsRegThreads)
   rms_write_partial<kRmsRegThreads>(m, partials);
 }
 
+// A block's 16 gains in channel order (two 16-byte loads of gamma[perm[.]])
+// as binary32 pairs, gv[i] = (gain 2i, gain 2i + 1).
+__device__ __forceinline__ void rms_gains(const uint16_t* gperm, int j, f2 gv[8]) {
+  const uint4 g0 = __ldg(reinterpret_cast<const uint4*>(gperm + 16 * j));
+  const uint4 g1 = __ldg(reinterpret_cast<const uint4*>(gperm + 16 * j) + 1);
+  const uint32_t gw[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+#pragma unroll
+  for (int i = 0; i < 8; ++i) gv[i] = make_f2(__uint_as_float(gw[i] << 16), __uint_as_float(gw[i] & 0xFFFF0000u));
+}
+
 // The RMSNorm of a gathered block: x (8 bf16 pairs, element 2i low) becomes
-// bf16((x * r) * gamma) with the block's gains gw (same layout), as the RMS
+// bf16((x * r) * gamma) with the block's gains gv (from rms_gains), as the RMS
 // pass computes it; packed products are one RNE binary32 product per lane.
-__device__ __forceinline__ void rms_normalize(uint32_t w[8], const uint32_t gw[8], float r) {
+__device__ __forceinline__ void rms_normalize(uint32_t w[8], const f2 gv[8], float r) {
   const f2 rr = make_f2(r, r);
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     const f2 xv = make_f2(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xFFFF0000u));
-    const f2 gv = make_f2(__uint_as_float(gw[i] << 16), __uint_as_float(gw[i] & 0xFFFF0000u));
-    const f2 y = mul2(mul2(xv, rr), gv);
+    const f2 y = mul2(mul2(xv, rr), gv[i]);
     w[i] = bf16x2_rn(y.a(), y.b());
   }
 }
@@ -688,7 +712,7 @@ __global__ void __launch_bounds__(kArcMaxThreads)
     quantize_arc_kernel(const QuantParams p) {
   BlockConsts k;
   __shared__ ScaleEntry s_dr[128];
-  // [K] channel byte offsets, with NORM [K] gains in channel order, then arc_bufs x [arc_rows][K] rows
+  // [K] channel byte offsets, then arc_bufs x [arc_rows][K] rows
   extern __shared__ __align__(16) uint16_t s_dyn[];
   if (!quant_prologue(p, k, s_dr)) return;
 
@@ -699,12 +723,11 @@ __global__ void __launch_bounds__(kArcMaxThreads)
     const int32_t c = p.perm[i];
     const int32_t cc = c >= 0 && c < K ? c : 0;  // out-of-range entries read channel 0
     s_dyn[i] = static_cast<uint16_t>(2 * cc);
-    if (NORM) s_dyn[K + i] = p.gamma[cc];
   }
   const int64_t rows_padded = (p.rows + 127) / 128 * 128;
   const int64_t half_ka = KA / 2, kgroups_a = KA / 64;
   const int nprim = static_cast<int>(K / 16), nres = static_cast<int>(p.S / 16);
-  const uint32_t rows_base = smem_u32(s_dyn + (NORM ? 2 : 1) * K);
+  const uint32_t rows_base = smem_u32(s_dyn + K);
   const uint32_t row_bytes = static_cast<uint32_t>(K) * 2, buf_bytes = row_bytes * R;
   // Buffers: full[b] completes when buffer b holds its step's rows (the
   // producer's arrival plus the copies' bytes); consumed[b] when every
@@ -786,10 +809,9 @@ __global__ void __launch_bounds__(kArcMaxThreads)
       for (int i = 0; i < 8; ++i)
         w[i] = ld_shared_u16(s_row + (ow[i] & 0xFFFFu)) | (ld_shared_u16(s_row + (ow[i] >> 16)) << 16);
       if (NORM) {
-        const uint4 g0 = reinterpret_cast<const uint4*>(s_dyn + K + 16 * j)[0];
-        const uint4 g1 = reinterpret_cast<const uint4*>(s_dyn + K + 16 * j)[1];
-        const uint32_t gw[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
-        rms_normalize(w, gw, __ldg(p.rinv + row0 + rr));
+        f2 gv[8];
+        rms_gains(p.gperm, j, gv);
+        rms_normalize(w, gv, __ldg(p.rinv + row0 + rr));
       }
       return unpack_block(make_uint4(w[0], w[1], w[2], w[3]), make_uint4(w[4], w[5], w[6], w[7]), px);
     };
@@ -799,13 +821,6 @@ __global__ void __launch_bounds__(kArcMaxThreads)
         const uint4 o0 = reinterpret_cast<const uint4*>(s_dyn + 16 * j)[0];
         const uint4 o1 = reinterpret_cast<const uint4*>(s_dyn + 16 * j)[1];
         const uint32_t ow[8] = {o0.x, o0.y, o0.z, o0.w, o1.x, o1.y, o1.z, o1.w};
-        uint32_t gw[8];
-        if (NORM) {
-          const uint4 g0 = reinterpret_cast<const uint4*>(s_dyn + K + 16 * j)[0];
-          const uint4 g1 = reinterpret_cast<const uint4*>(s_dyn + K + 16 * j)[1];
-          gw[0] = g0.x, gw[1] = g0.y, gw[2] = g0.z, gw[3] = g0.w, gw[4] = g1.x, gw[5] = g1.y, gw[6] = g1.z,
-          gw[7] = g1.w;
-        }
         for (int rr = 0; rr < R; ++rr) {
           const int64_t row = row0 + rr;
           uint32_t scale = 0;
@@ -815,7 +830,13 @@ __global__ void __launch_bounds__(kArcMaxThreads)
 #pragma unroll
             for (int i = 0; i < 8; ++i)
               w[i] = ld_shared_u16(s_row + (ow[i] & 0xFFFFu)) | (ld_shared_u16(s_row + (ow[i] >> 16)) << 16);
-            if (NORM) rms_normalize(w, gw, __ldg(p.rinv + row));
+            if (NORM) {
+              // the column's gains, read (L1) and unpacked per row: holding them
+              // across the rows takes the registers of a third CTA per SM
+              f2 gv[8];
+              rms_gains(p.gperm, j, gv);
+              rms_normalize(w, gv, __ldg(p.rinv + row));
+            }
             f2 px[8];
             const uint32_t bbits = unpack_block(make_uint4(w[0], w[1], w[2], w[3]),
                                                 make_uint4(w[4], w[5], w[6], w[7]), px);
@@ -914,7 +935,7 @@ void arc_layout(int64_t K, int lead, int* rows, int* bufs) {
 
 template <bool F, int R, bool NORM>
 cudaError_t launch_quantize_arc(int dev, int sms, const QuantParams& p, cudaStream_t s, bool pdl) {
-  const size_t smem = static_cast<size_t>(p.K) * 2 * ((NORM ? 2 : 1) + p.arc_bufs * p.arc_rows);
+  const size_t smem = static_cast<size_t>(p.K) * 2 * (1 + p.arc_bufs * p.arc_rows);
   // the shared-memory opt-in is an attribute of the kernel in this context
   static PerContextCache<int> attr;
   int done = 0;
@@ -1009,7 +1030,9 @@ size_t nvfp4_quantize_workspace_bytes(int64_t rows, int64_t K) {
 }
 
 size_t nvfp4_quantize_arc_rmsnorm_workspace_bytes(int64_t rows, int64_t K) {
-  return nvfp4_quantize_workspace_bytes(rows, K) + sizeof(float) * static_cast<size_t>(rows > 0 ? rows : 0);
+  // the quantize workspace, then 1 / rms of each row, then the gains in channel order
+  return nvfp4_quantize_workspace_bytes(rows, K) + align16(sizeof(float) * static_cast<size_t>(rows > 0 ? rows : 0)) +
+         align16(sizeof(uint16_t) * static_cast<size_t>(K > 0 ? K : 0));
 }
 
 }  // extern "C"
@@ -1144,8 +1167,9 @@ cudaError_t launch_rms_reg(const QuantParams& p, uint32_t* partials, float eps, 
   static PerContextCache<int> per_sm;
   cudaError_t e = rms_grid(per_sm, rms_amax_reg_kernel<NR>, kRmsRegThreads, dev, sms, p.rows, grid);
   if (e != cudaSuccess) return e;
-  rms_amax_reg_kernel<NR><<<*grid, kRmsRegThreads, 0, s>>>(p.x, p.rows, p.K, p.ldx, p.gamma, eps,
-                                                            const_cast<float*>(p.rinv), partials);
+  rms_amax_reg_kernel<NR><<<*grid, kRmsRegThreads, 0, s>>>(p.x, p.rows, p.K, p.ldx, p.gamma, eps, p.perm,
+                                                            const_cast<float*>(p.rinv),
+                                                            const_cast<uint16_t*>(p.gperm), partials);
   return cudaGetLastError();
 }
 
@@ -1167,8 +1191,8 @@ cudaError_t launch_rms_pass(const QuantParams& p, uint32_t* partials, float eps,
   static PerContextCache<int> per_sm;
   cudaError_t e = rms_grid(per_sm, rms_amax_kernel, kRmsThreads, dev, sms, p.rows, grid);
   if (e != cudaSuccess) return e;
-  rms_amax_kernel<<<*grid, kRmsThreads, 0, s>>>(p.x, p.rows, p.K, p.ldx, p.gamma, eps, const_cast<float*>(p.rinv),
-                                               partials);
+  rms_amax_kernel<<<*grid, kRmsThreads, 0, s>>>(p.x, p.rows, p.K, p.ldx, p.gamma, eps, p.perm,
+                                               const_cast<float*>(p.rinv), const_cast<uint16_t*>(p.gperm), partials);
   return cudaGetLastError();
 }
 
@@ -1240,7 +1264,7 @@ nvfp4_status quantize_impl(const char* fn, QuantKind kind, const void* x, int64_
   p.S = S;
   p.augment = augment;
   if (kind == QuantKind::kAugmented) {
-    arc_layout(K, gamma ? 2 : 1, &p.arc_rows, &p.arc_bufs);
+    arc_layout(K, 1, &p.arc_rows, &p.arc_bufs);
     p.arc_prim_threads = arc_prim_threads(K);
   }
   if (gamma) {
@@ -1248,6 +1272,8 @@ nvfp4_status quantize_impl(const char* fn, QuantKind kind, const void* x, int64_
     // pass's place and leaves 1/rms of every row after the partials
     p.gamma = gamma;
     p.rinv = reinterpret_cast<float*>(static_cast<char*>(workspace) + nvfp4_quantize_workspace_bytes(rows, K));
+    p.gperm = reinterpret_cast<const uint16_t*>(static_cast<char*>(workspace) + nvfp4_quantize_workspace_bytes(rows, K) +
+                                                 align16(sizeof(float) * static_cast<size_t>(rows)));
     return launch_rms_dynamic(p, mode, rule, fp8_max, global_scale, partials, eps, dev, sms,
                               static_cast<cudaStream_t>(stream));
   }
