@@ -150,6 +150,78 @@ def test_quantize_arc_rmsnorm_more_rows_than_warps():
     assert_arc_equal(q, y, perm, S, nv.AUG_RESIDUAL, "four_over_six", "mse", 256.0)
 
 
+def _f32_rms_and_peak(x: torch.Tensor, gamma: torch.Tensor, eps: float):
+    """For choosing inputs only (expected values come from the oracle): each
+    row's r = 1 / sqrt(pairwise_sum(x^2) / K + eps) in binary32 numpy
+    arithmetic (the zero-padded pairwise tree, one rounding per step) and
+    T = max_k |x_k * gamma_k| (exact in binary32 for these values)."""
+    xf = x.float().numpy()
+    gf = gamma.float().numpy()
+    rows, K = xf.shape
+    n = 1 << (K - 1).bit_length()
+    a = np.zeros((rows, n), np.float32)
+    a[:, :K] = xf * xf
+    while a.shape[1] > 1:
+        a = a[:, 0::2] + a[:, 1::2]
+    r = np.float32(1.0) / np.sqrt(a[:, 0] / np.float32(K) + np.float32(eps))
+    T = np.abs(xf * gf[None, :]).max(axis=1)
+    return r, T
+
+
+def _bf16_of(v: float) -> int:
+    """bf16 bits of the nearest bf16 to the real number v >= 0 (ties to even)."""
+    from fractions import Fraction
+    import exact_binary32 as xb
+    return xb.bf16_rne(Fraction(v))
+
+
+@pytest.mark.parametrize("K,rows", [(256, 32768), (5120, 8192)], ids=str)
+def test_quantize_arc_rmsnorm_rows_whose_max_y_sits_on_a_bf16_boundary(K, rows):
+    """The RMS pass bounds a row's max |y| by P r (1 -+ 2^-20), P = max |x * gamma|,
+    and computes the row's y one by one only when the two bounds round to
+    different bf16 values.  Rows chosen so that they do (a few in ten thousand)
+    are quantized alone, so that each decides alpha, and compared with the
+    oracle bit for bit."""
+    x = workloads.small_operand(rows, K, seed=2 * K + 1).make()
+    gamma = _gains(K, K + 1)
+    r, T = _f32_rms_and_peak(x, gamma, 1e-6)
+    picked = []
+    for i in range(rows):
+        pr = float(T[i]) * float(r[i])
+        if _bf16_of(pr * (1 - 2.0 ** -20)) != _bf16_of(pr * (1 + 2.0 ** -20)):
+            picked.append(i)
+        if len(picked) == 6:
+            break
+    assert picked, "no row near a bf16 rounding boundary among the candidates"
+    perm = np.arange(K, dtype=np.int32)[::-1].copy()
+    for i in picked:
+        xi = x[i:i + 1].clone()
+        q, status = gpu_arc_rmsnorm(xi, gamma, 1e-6, perm, 64, "four_over_six", "mse", 256.0)
+        assert status == nv.OK
+        y = torch.from_numpy(oracle.rmsnorm(xi, gamma, 1e-6).view(np.int16)).view(torch.bfloat16)
+        assert_arc_equal(q, y, perm, 64, nv.AUG_RESIDUAL, "four_over_six", "mse", 256.0)
+
+
+@pytest.mark.parametrize("K", [256, 5120], ids=str)
+@pytest.mark.parametrize("case", ["large_gain", "tiny_rows"])
+def test_quantize_arc_rmsnorm_outside_the_bound_s_range(K, case):
+    """Where the RMS pass's bound on max |y| does not hold (a gain above 2^20,
+    or y near the bottom of the binary32 range) every y is computed; the result
+    is still the oracle's."""
+    rows = 64
+    x = workloads.small_operand(rows, K, seed=K + 5).make()
+    gamma = _gains(K, K + 2)
+    if case == "large_gain":
+        gamma[K // 3] = 2.0 ** 21
+    else:
+        x = (x.float() * 2.0 ** -120).to(torch.bfloat16)
+    perm = outlier_perm(x)
+    q, status = gpu_arc_rmsnorm(x, gamma, 1e-6, perm, 64, "four_over_six", "mae", 256.0)
+    assert status == nv.OK
+    y = torch.from_numpy(oracle.rmsnorm(x, gamma, 1e-6).view(np.int16)).view(torch.bfloat16)
+    assert_arc_equal(q, y, perm, 64, nv.AUG_RESIDUAL, "four_over_six", "mae", 256.0)
+
+
 def test_quantize_arc_rmsnorm_reading_pins():
     """The rows of tests/golden/rmsnorm_pins.txt (each separates one reading of
     the RMSNorm rounding order from its alternative) quantized on the GPU:

@@ -546,9 +546,8 @@ __device__ __forceinline__ float rms_rinv(float sum, int64_t K, float eps) {
 // the CTA's max |bf16(y)| from each lane's binary32 max, as a bf16 bit
 // pattern (a NaN becomes 0x7FFF), into partials[blockIdx.x]
 template <int THREADS>
-__device__ __forceinline__ void rms_write_partial(float m, uint32_t* partials) {
+__device__ __forceinline__ void rms_write_partial_bits(uint32_t mb, uint32_t* partials) {
   const int lane = static_cast<int>(threadIdx.x & 31), warp = static_cast<int>(threadIdx.x >> 5);
-  uint32_t mb = bf16x2_rn(m, 0.0f) & 0x7FFFu;
 #pragma unroll
   for (int o = 16; o; o >>= 1) mb = max(mb, __shfl_xor_sync(0xffffffffu, mb, o));
   __shared__ uint32_t s_max[THREADS / 32];
@@ -559,6 +558,10 @@ __device__ __forceinline__ void rms_write_partial(float m, uint32_t* partials) {
     for (int w = 0; w < THREADS / 32; ++w) mm = max(mm, s_max[w]);
     partials[blockIdx.x] = mm;
   }
+}
+template <int THREADS>
+__device__ __forceinline__ void rms_write_partial(float m, uint32_t* partials) {
+  rms_write_partial_bits<THREADS>(bf16x2_rn(m, 0.0f) & 0x7FFFu, partials);
 }
 
 // gperm[i] = gamma[perm[i]] over the grid's threads, for the augmented
@@ -616,6 +619,32 @@ __global__ void __launch_bounds__(kRmsThreads)
   rms_write_partial<kRmsThreads>(m, partials);
 }
 
+// max(m, |x * gamma|) over one 16-byte group: each product of two bf16 values
+// by one mixed-precision fma (exact: at most 16 significant bits, unless it
+// falls below the binary32 normal range)
+__device__ __forceinline__ float prod_group_max(const uint4 xv, const uint4 gv, float m) {
+  const uint32_t xs[4] = {xv.x, xv.y, xv.z, xv.w}, gs[4] = {gv.x, gv.y, gv.z, gv.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    float t0, t1;
+    asm("{\n\t.reg .b16 xl, xh, gl, gh;\n\t"
+        "mov.b32 {xl, xh}, %2;\n\t"
+        "mov.b32 {gl, gh}, %3;\n\t"
+        "fma.rn.f32.bf16 %0, xl, gl, 0f80000000;\n\t"
+        "fma.rn.f32.bf16 %1, xh, gh, 0f80000000;\n\t}"
+        : "=f"(t0), "=f"(t1)
+        : "r"(xs[i]), "r"(gs[i]));
+    m = max3_nan(m, fabsf(t0), fabsf(t1));
+  }
+  return m;
+}
+
+__device__ __forceinline__ float warp_max_nan(float v) {
+#pragma unroll
+  for (int o = 16; o; o >>= 1) v = max3_nan(v, __shfl_xor_sync(0xffffffffu, v, o), v);
+  return v;
+}
+
 // The RMS pass with the row held in registers (K <= 1024 * NR): a warp issues
 // every load of its row before any arithmetic, so the whole row is in flight
 // at once, and the y phase works on the same registers.
@@ -629,7 +658,14 @@ __global__ void __launch_bounds__(kRmsRegThreads, NR <= 2 ? 8 : NR <= 3 ? 5 : NR
   constexpr int kWarps = kRmsRegThreads / 32;
   const int lane = static_cast<int>(threadIdx.x & 31), warp = static_cast<int>(threadIdx.x >> 5);
   const int64_t nwarps = static_cast<int64_t>(gridDim.x) * kWarps;
-  float m = 0.0f;
+  // G = max |gamma| (NaN kept) bounds the error that underflow adds to the
+  // products below; the bound is only used while G <= 2^20
+  uint32_t gb = 0;  // max |gamma| as bf16 bits (a NaN compares above every number)
+  for (int64_t k = 8 * lane; k < K; k += 256) gb = absmax4(*reinterpret_cast<const uint4*>(gamma + k), gb);
+#pragma unroll
+  for (int o = 16; o; o >>= 1) gb = max(gb, __shfl_xor_sync(0xffffffffu, gb, o));
+  const bool gains_small = max(gb & 0xFFFFu, gb >> 16) <= 0x4980u;  // 2^20
+  uint32_t mb = 0;  // this lane's max |bf16(y)| as a bf16 bit pattern
   for (int64_t r = static_cast<int64_t>(blockIdx.x) * kWarps + warp; r < rows; r += nwarps) {
     const uint16_t* xr = x + r * ldx;
     uint4 d[NR][4];
@@ -641,23 +677,47 @@ __global__ void __launch_bounds__(kRmsRegThreads, NR <= 2 ? 8 : NR <= 3 ? 5 : NR
         d[q][u] = k < K ? *reinterpret_cast<const uint4*>(xr + k) : make_uint4(0u, 0u, 0u, 0u);
       }
     }
+    // the sum of squares and, from the same registers, P = max |x * gamma|
     float stk[5];
-#pragma unroll
-    for (int q = 0; q < NR; ++q)
-      rms_push(stk, q, rms_round(sq_tree8(d[q][0]), sq_tree8(d[q][1]), sq_tree8(d[q][2]), sq_tree8(d[q][3])));
-    const float rr = rms_rinv(rms_close(stk, NR), K, eps);
-    if (lane == 0) rinv[r] = rr;
-    const f2 rrr = make_f2(rr, rr);
+    float P = 0.0f;
 #pragma unroll
     for (int q = 0; q < NR; ++q) {
+      float g[4];
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
         const int64_t k = 1024 * q + 32 * lane + 8 * u;
-        if (k < K) m = rms_group_max(d[q][u], *reinterpret_cast<const uint4*>(gamma + k), rrr, m);
+        g[u] = sq_tree8(d[q][u]);
+        if (k < K) P = prod_group_max(d[q][u], *reinterpret_cast<const uint4*>(gamma + k), P);
       }
+      rms_push(stk, q, rms_round(g[0], g[1], g[2], g[3]));
+    }
+    const float rr = rms_rinv(rms_close(stk, NR), K, eps);
+    if (lane == 0) rinv[r] = rr;
+    // max |y| of the row, y = (x * r) * gamma with two roundings.  With
+    // P = max |x * gamma| (exact) and every y in the normal range, each |y| is
+    // within a factor (1 +- 2^-24)^2 of |x * gamma| * r, so max |y| lies in
+    // [lo, hi] = [P r (1 - 2^-20), P r (1 + 2^-20)] (rounded outward; the
+    // slack also covers what underflow can add while P r >= 2^-90 and
+    // G <= 2^20).  Rounding to bf16 is monotone: when lo and hi round to the
+    // same bf16 value, that is max |bf16(y)|; otherwise (about one row in a
+    // thousand) the row's y are computed one by one.
+    P = warp_max_nan(P);
+    const float plo = __fmul_rd(P, rr), phi = __fmul_ru(P, rr);
+    const uint32_t blo = bf16x2_rn(__fmul_rd(plo, 1.0f - 0x1p-20f), 0.0f) & 0x7FFFu;
+    const uint32_t bhi = bf16x2_rn(__fmul_ru(phi, 1.0f + 0x1p-20f), 0.0f) & 0x7FFFu;
+    if (gains_small && plo >= 0x1p-90f && P <= 0x1.fffffep127f && blo == bhi) {
+      mb = max(mb, blo);
+    } else {
+      // rare: the row read again (from L2), its y computed one by one
+      const f2 rrr = make_f2(rr, rr);
+      float m = 0.0f;
+#pragma unroll 1
+      for (int64_t k = 8 * lane; k < K; k += 256)
+        m = rms_group_max(*reinterpret_cast<const uint4*>(xr + k), *reinterpret_cast<const uint4*>(gamma + k), rrr, m);
+      mb = max(mb, bf16x2_rn(m, 0.0f) & 0x7FFFu);
     }
   }
-  rms_write_partial<kRmsRegThreads>(m, partials);
+  rms_write_partial_bits<kRmsRegThreads>(mb, partials);
 }
 
 // A block's 16 gains in channel order (two 16-byte loads of gamma[perm[.]])
