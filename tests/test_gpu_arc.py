@@ -270,16 +270,21 @@ def test_quantize_arc_rmsnorm_gemm_uses_the_normalized_activations():
 
 
 @pytest.mark.parametrize("recipe", RECIPES[:2], ids=lambda r: "-".join(map(str, r)))
-def test_quantize_arc_rmsnorm_pitched_rows(recipe):
+@pytest.mark.parametrize("offset", [32, 8], ids=["32-byte-aligned", "16-byte-aligned"])
+def test_quantize_arc_rmsnorm_pitched_rows(recipe, offset):
     """x as a view with a row pitch above K (the RMS pass and the bulk row
-    copies both follow the pitch)."""
+    copies both follow the pitch); with an 8-element column offset and gains
+    at a 16-byte (not 32-byte) boundary the RMS pass takes 128-bit loads."""
     mode, rule, F = recipe
     rows, K, S = 200, 1024, 128
-    wide = workloads.small_operand(rows, K + 64, seed=21).make()
-    x = wide[:, 32:32 + K]  # a 64-byte aligned column offset: 16-byte aligned rows
+    wide = workloads.small_operand(rows, K + 96, seed=21).make()  # a pitch of 70 x 32 bytes
+    x = wide[:, offset:offset + K]
     gamma = _gains(K, 22)
+    g_dev = torch.empty(K + 8, dtype=torch.bfloat16, device="cuda")
+    g_off = g_dev[8:] if offset == 8 else g_dev[:K]
+    g_off.copy_(gamma.cuda())
     perm = outlier_perm(x)
-    out = nv.quantize_arc_rmsnorm(wide.cuda()[:, 32:32 + K], gamma.cuda(), 1e-6, torch.from_numpy(perm).cuda(), S,
+    out = nv.quantize_arc_rmsnorm(wide.cuda()[:, offset:offset + K], g_off, 1e-6, torch.from_numpy(perm).cuda(), S,
                                   mode, rule, F)
     assert nv.device_status(out.workspace) == nv.OK
     y = torch.from_numpy(oracle.rmsnorm(x.contiguous(), gamma, 1e-6).view(np.int16)).view(torch.bfloat16)

@@ -645,10 +645,31 @@ __device__ __forceinline__ float warp_max_nan(float v) {
   return v;
 }
 
+// Two adjacent 16-byte groups (32 bytes at p): one 256-bit load when V8 (p
+// 32-byte aligned), else two 128-bit loads.  The 256-bit form halves the L1
+// sector lookups of the lane pattern below (lanes 64 bytes apart).  VOL keeps
+// a load in the loop for data that is the same every row (the gains), which
+// would otherwise be hoisted into registers the row needs.
+template <bool V8, bool VOL>
+__device__ __forceinline__ void ld_group_pair(const uint16_t* p, uint4& a, uint4& b) {
+  if constexpr (V8 && VOL) {
+    asm volatile("ld.global.v8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+                 : "=r"(a.x), "=r"(a.y), "=r"(a.z), "=r"(a.w), "=r"(b.x), "=r"(b.y), "=r"(b.z), "=r"(b.w)
+                 : "l"(p));
+  } else if constexpr (V8) {
+    asm("ld.global.v8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+        : "=r"(a.x), "=r"(a.y), "=r"(a.z), "=r"(a.w), "=r"(b.x), "=r"(b.y), "=r"(b.z), "=r"(b.w)
+        : "l"(p));
+  } else {
+    a = reinterpret_cast<const uint4*>(p)[0];
+    b = reinterpret_cast<const uint4*>(p)[1];
+  }
+}
+
 // The RMS pass with the row held in registers (K <= 1024 * NR): a warp issues
 // every load of its row before any arithmetic, so the whole row is in flight
 // at once, and the y phase works on the same registers.
-template <int NR>
+template <int NR, bool V8>
 __global__ void __launch_bounds__(kRmsRegThreads, NR <= 2 ? 8 : NR <= 3 ? 5 : NR <= 6 ? 4 : 3)
     rms_amax_reg_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t K, int64_t ldx,
                         const uint16_t* __restrict__ gamma, float eps, const int32_t* __restrict__ perm,
@@ -668,13 +689,19 @@ __global__ void __launch_bounds__(kRmsRegThreads, NR <= 2 ? 8 : NR <= 3 ? 5 : NR
   uint32_t mb = 0;  // this lane's max |bf16(y)| as a bf16 bit pattern
   for (int64_t r = static_cast<int64_t>(blockIdx.x) * kWarps + warp; r < rows; r += nwarps) {
     const uint16_t* xr = x + r * ldx;
+    // (K % 64 == 0: a pair of groups is inside the row or past it)
     uint4 d[NR][4];
 #pragma unroll
     for (int q = 0; q < NR; ++q) {
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int64_t k = 1024 * q + 32 * lane + 8 * u;
-        d[q][u] = k < K ? *reinterpret_cast<const uint4*>(xr + k) : make_uint4(0u, 0u, 0u, 0u);
+      for (int h = 0; h < 2; ++h) {
+        const int64_t k = 1024 * q + 32 * lane + 16 * h;
+        if (k < K) {
+          ld_group_pair<V8, false>(xr + k, d[q][2 * h], d[q][2 * h + 1]);
+        } else {
+          d[q][2 * h] = make_uint4(0u, 0u, 0u, 0u);
+          d[q][2 * h + 1] = make_uint4(0u, 0u, 0u, 0u);
+        }
       }
     }
     // the sum of squares and, from the same registers, P = max |x * gamma|
@@ -684,10 +711,15 @@ __global__ void __launch_bounds__(kRmsRegThreads, NR <= 2 ? 8 : NR <= 3 ? 5 : NR
     for (int q = 0; q < NR; ++q) {
       float g[4];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int64_t k = 1024 * q + 32 * lane + 8 * u;
-        g[u] = sq_tree8(d[q][u]);
-        if (k < K) P = prod_group_max(d[q][u], *reinterpret_cast<const uint4*>(gamma + k), P);
+      for (int h = 0; h < 2; ++h) {
+        const int64_t k = 1024 * q + 32 * lane + 16 * h;
+        g[2 * h] = sq_tree8(d[q][2 * h]);
+        g[2 * h + 1] = sq_tree8(d[q][2 * h + 1]);
+        if (k < K) {
+          uint4 ga, gb2;
+          ld_group_pair<V8, true>(gamma + k, ga, gb2);
+          P = prod_group_max(d[q][2 * h + 1], gb2, prod_group_max(d[q][2 * h], ga, P));
+        }
       }
       rms_push(stk, q, rms_round(g[0], g[1], g[2], g[3]));
     }
@@ -1221,16 +1253,25 @@ cudaError_t rms_grid(PerContextCache<int>& per_sm, Kernel kernel, int threads, i
   return cudaSuccess;
 }
 
-template <int NR>
-cudaError_t launch_rms_reg(const QuantParams& p, uint32_t* partials, float eps, int dev, int sms, cudaStream_t s,
-                           int* grid) {
+template <int NR, bool V8>
+cudaError_t launch_rms_reg_v(const QuantParams& p, uint32_t* partials, float eps, int dev, int sms, cudaStream_t s,
+                             int* grid) {
   static PerContextCache<int> per_sm;
-  cudaError_t e = rms_grid(per_sm, rms_amax_reg_kernel<NR>, kRmsRegThreads, dev, sms, p.rows, grid);
+  cudaError_t e = rms_grid(per_sm, rms_amax_reg_kernel<NR, V8>, kRmsRegThreads, dev, sms, p.rows, grid);
   if (e != cudaSuccess) return e;
-  rms_amax_reg_kernel<NR><<<*grid, kRmsRegThreads, 0, s>>>(p.x, p.rows, p.K, p.ldx, p.gamma, eps, p.perm,
+  rms_amax_reg_kernel<NR, V8><<<*grid, kRmsRegThreads, 0, s>>>(p.x, p.rows, p.K, p.ldx, p.gamma, eps, p.perm,
                                                             const_cast<float*>(p.rinv),
                                                             const_cast<uint16_t*>(p.gperm), partials);
   return cudaGetLastError();
+}
+// 256-bit loads where x's rows and the gains start on 32-byte boundaries
+template <int NR>
+cudaError_t launch_rms_reg(const QuantParams& p, uint32_t* partials, float eps, int dev, int sms, cudaStream_t s,
+                           int* grid) {
+  const bool v8 = reinterpret_cast<uintptr_t>(p.x) % 32 == 0 && p.ldx % 16 == 0 &&
+                  reinterpret_cast<uintptr_t>(p.gamma) % 32 == 0;
+  return v8 ? launch_rms_reg_v<NR, true>(p, partials, eps, dev, sms, s, grid)
+            : launch_rms_reg_v<NR, false>(p, partials, eps, dev, sms, s, grid);
 }
 
 cudaError_t launch_rms_pass(const QuantParams& p, uint32_t* partials, float eps, int dev, int sms, cudaStream_t s,
