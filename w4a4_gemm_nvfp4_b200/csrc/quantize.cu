@@ -209,17 +209,27 @@ __device__ __forceinline__ bool quant_prologue(const QuantParams& p, BlockConsts
 // lane loads its next block (the task's second one, or the next task's first)
 // while it quantizes the current one.  Rows past `rows` only write their
 // (zero) scale bytes.
+// A block's 32 bytes: one 256-bit load when V8 (p 32-byte aligned; the
+// sector then crosses from L2 once, where two non-allocating 128-bit loads
+// each fetch it), else two 128-bit loads.
+template <bool V8>
 __device__ __forceinline__ void ld_block2(const uint16_t* p, uint4& lo, uint4& hi) {
-  const uint4* q = reinterpret_cast<const uint4*>(p);
-  lo = ld_stream(q);
-  hi = ld_stream(q + 1);
+  if constexpr (V8) {
+    asm volatile("ld.global.nc.L1::no_allocate.v8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+                 : "=r"(lo.x), "=r"(lo.y), "=r"(lo.z), "=r"(lo.w), "=r"(hi.x), "=r"(hi.y), "=r"(hi.z), "=r"(hi.w)
+                 : "l"(p));
+  } else {
+    const uint4* q = reinterpret_cast<const uint4*>(p);
+    lo = ld_stream(q);
+    hi = ld_stream(q + 1);
+  }
 }
 
 __device__ __forceinline__ int64_t scale_row_offset(uint32_t row, uint32_t kgroups) {
   return static_cast<int64_t>(row >> 7) * kgroups * 512 + (row & 31) * 16 + ((row >> 5) & 3) * 4;
 }
 
-template <bool FOUR_OVER_SIX, int RULE>
+template <bool FOUR_OVER_SIX, int RULE, bool V8>
 // Scale-6: four CTAs per SM (64 registers), measured faster than three, five
 // or six.  Four-Over-Six: three CTAs per SM (up to 85 registers), which keeps
 // its two candidates' state out of local memory; measured 2-3 % faster than
@@ -276,7 +286,7 @@ __global__ void __launch_bounds__(kQuantThreads, FOUR_OVER_SIX ? 3 : 4)
   // a block was always loaded; they are zeroed once so that no copy of them
   // is ever of an indeterminate value)
   uint4 lo = make_uint4(0, 0, 0, 0), hi = lo, nlo = lo, nhi = lo;
-  if (row < rows && has_block(2 * pair)) ld_block2(xp, lo, hi);
+  if (row < rows && has_block(2 * pair)) ld_block2<V8>(xp, lo, hi);
   for (;;) {
     const uint32_t cur_row = row, c0 = 2 * pair;
     const uint16_t* const cur_xp = xp;
@@ -284,7 +294,7 @@ __global__ void __launch_bounds__(kQuantThreads, FOUR_OVER_SIX ? 3 : 4)
     uint8_t* const cur_sp = sp + scale_row_offset(cur_row, p.kgroups) + c0 * 4096;
     // first chunk of the pair, while the second one loads
     const bool second = has_block(c0 + 1);
-    if (cur_row < rows && second) ld_block2(cur_xp + 512, nlo, nhi);
+    if (cur_row < rows && second) ld_block2<V8>(cur_xp + 512, nlo, nhi);
     if (has_block(c0)) block(lo, hi, cur_row, cur_cp, cur_sp);
     // advance to the next task
     t += nwarps;
@@ -299,7 +309,7 @@ __global__ void __launch_bounds__(kQuantThreads, FOUR_OVER_SIX ? 3 : 4)
     cp += wrap ? dc_wrap : dc;
     const bool more = t < p.ntasks;
     // second chunk, while the next task's first chunk loads
-    if (more && row < rows && has_block(2 * pair)) ld_block2(xp, lo, hi);
+    if (more && row < rows && has_block(2 * pair)) ld_block2<V8>(xp, lo, hi);
     if (second) block(nlo, nhi, cur_row, cur_cp + 256, cur_sp + 4096);
     if (!more) break;
   }
@@ -1085,19 +1095,26 @@ cudaError_t launch_quantize_t_kernel(int mode, int rule, int dev, int sms, const
   return launch_quantize_t<true, kRuleMse>(dev, sms, p, s, pdl);
 }
 
-template <bool F, int R>
-cudaError_t launch_quantize(int dev, int sms, const QuantParams& p, cudaStream_t s, bool pdl) {
+template <bool F, int R, bool V8>
+cudaError_t launch_quantize_v(int dev, int sms, const QuantParams& p, cudaStream_t s, bool pdl) {
   static PerContextCache<int> per_sm;
   int occ = 0;
   cudaError_t e = per_context(per_sm, dev, [](int* v) {
-    const cudaError_t r = cudaOccupancyMaxActiveBlocksPerMultiprocessor(v, quantize_kernel<F, R>, kQuantThreads, 0);
+    const cudaError_t r =
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(v, quantize_kernel<F, R, V8>, kQuantThreads, 0);
     *v = std::max(1, *v);
     return r;
   }, &occ);
   if (e != cudaSuccess) return e;
   const int64_t want = (static_cast<int64_t>(p.ntasks) + kQuantWarps - 1) / kQuantWarps;
   const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(want, static_cast<int64_t>(sms) * occ)));
-  return launch_kernel(quantize_kernel<F, R>, dim3(grid), dim3(kQuantThreads), 0, s, pdl, p);
+  return launch_kernel(quantize_kernel<F, R, V8>, dim3(grid), dim3(kQuantThreads), 0, s, pdl, p);
+}
+// 256-bit block loads where every row of x starts on a 32-byte boundary
+template <bool F, int R>
+cudaError_t launch_quantize(int dev, int sms, const QuantParams& p, cudaStream_t s, bool pdl) {
+  const bool v8 = reinterpret_cast<uintptr_t>(p.x) % 32 == 0 && p.ldx % 16 == 0;
+  return v8 ? launch_quantize_v<F, R, true>(dev, sms, p, s, pdl) : launch_quantize_v<F, R, false>(dev, sms, p, s, pdl);
 }
 
 cudaError_t launch_quantize_kernel(int mode, int rule, int dev, int sms, const QuantParams& p, cudaStream_t s,
