@@ -202,12 +202,12 @@ def test_quantize_arc_rmsnorm_rows_whose_max_y_sits_on_a_bf16_boundary(K, rows):
         assert_arc_equal(q, y, perm, 64, nv.AUG_RESIDUAL, "four_over_six", "mse", 256.0)
 
 
-@pytest.mark.parametrize("K", [256, 5120], ids=str)
+@pytest.mark.parametrize("K", [256, 5120, 16384], ids=str)
 @pytest.mark.parametrize("case", ["large_gain", "tiny_rows"])
 def test_quantize_arc_rmsnorm_outside_the_bound_s_range(K, case):
     """Where the RMS pass's bound on max |y| does not hold (a gain above 2^20,
     or y near the bottom of the binary32 range) every y is computed; the result
-    is still the oracle's."""
+    is still the oracle's.  K = 16384 takes the round-by-round pass."""
     rows = 64
     x = workloads.small_operand(rows, K, seed=K + 5).make()
     gamma = _gains(K, K + 2)

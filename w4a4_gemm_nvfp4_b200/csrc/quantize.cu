@@ -585,50 +585,6 @@ __device__ __forceinline__ void rms_permute_gains(const uint16_t* gamma, const i
   }
 }
 
-// The RMS pass for any K <= 16384: round by round, the y phase reading the row
-// again (from L2).
-__global__ void __launch_bounds__(kRmsThreads)
-    rms_amax_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t K, int64_t ldx,
-                    const uint16_t* __restrict__ gamma, float eps, const int32_t* __restrict__ perm,
-                    float* __restrict__ rinv, uint16_t* __restrict__ gperm, uint32_t* __restrict__ partials) {
-  pdl_launch_dependents();  // the quantize kernel may be scheduled now; it waits for this grid's end
-  rms_permute_gains(gamma, perm, K, gperm);
-  // rounds that hold elements; the zero-padded rest of the tree up to the next
-  // power of two adds exact zeros and is not computed
-  const int used = static_cast<int>((K + 1023) / 1024);  // 1 .. 16 (K <= 16384)
-  const int lane = static_cast<int>(threadIdx.x & 31), warp = static_cast<int>(threadIdx.x >> 5);
-  const int64_t nwarps = static_cast<int64_t>(gridDim.x) * (kRmsThreads / 32);
-  float m = 0.0f;
-  for (int64_t r = static_cast<int64_t>(blockIdx.x) * (kRmsThreads / 32) + warp; r < rows; r += nwarps) {
-    const uint16_t* xr = x + r * ldx;
-    float stk[5];
-    for (int q = 0; q < used; ++q) {
-      // this lane's four groups (K % 8 == 0: a group is inside or past the row)
-      float g[4];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int64_t k = 1024 * static_cast<int64_t>(q) + 32 * lane + 8 * u;
-        g[u] = k < K ? sq_tree8(*reinterpret_cast<const uint4*>(xr + k)) : 0.0f;
-      }
-      rms_push(stk, q, rms_round(g[0], g[1], g[2], g[3]));
-    }
-    const float rr = rms_rinv(rms_close(stk, used), K, eps);
-    if (lane == 0) rinv[r] = rr;
-    // the row's outputs and their max |y|, read in the same order
-    const f2 rrr = make_f2(rr, rr);
-    for (int q = 0; q < used; ++q) {
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int64_t k = 1024 * static_cast<int64_t>(q) + 32 * lane + 8 * u;
-        if (k < K)
-          m = rms_group_max(*reinterpret_cast<const uint4*>(xr + k), *reinterpret_cast<const uint4*>(gamma + k), rrr,
-                            m);
-      }
-    }
-  }
-  rms_write_partial<kRmsThreads>(m, partials);
-}
-
 // max(m, |x * gamma|) over one 16-byte group: each product of two bf16 values
 // by one mixed-precision fma (exact: at most 16 significant bits, unless it
 // falls below the binary32 normal range)
@@ -676,6 +632,39 @@ __device__ __forceinline__ void ld_group_pair(const uint16_t* p, uint4& a, uint4
   }
 }
 
+// Whether max |gamma| <= 2^20 (NaN counts as not), over the warp: the bound
+// on a row's max |y| below is only used then.
+__device__ __forceinline__ bool rms_gains_small(const uint16_t* gamma, int64_t K, int lane) {
+  uint32_t gb = 0;  // max |gamma| as bf16 bits (a NaN compares above every number)
+  for (int64_t k = 8 * lane; k < K; k += 256) gb = absmax4(*reinterpret_cast<const uint4*>(gamma + k), gb);
+#pragma unroll
+  for (int o = 16; o; o >>= 1) gb = max(gb, __shfl_xor_sync(0xffffffffu, gb, o));
+  return max(gb & 0xFFFFu, gb >> 16) <= 0x4980u;  // 2^20
+}
+
+// max |bf16(y)| of row xr as a bf16 bit pattern, y = (x * r) * gamma with two
+// roundings, from P = max |x * gamma| over the row (exact) and r.  With every
+// y in the normal range, each |y| is within a factor (1 +- 2^-24)^2 of
+// |x * gamma| * r, so max |y| lies in [lo, hi] = [P r (1 - 2^-20), P r (1 + 2^-20)]
+// (rounded outward; the slack also covers what underflow can add while
+// P r >= 2^-90 and max |gamma| <= 2^20).  Rounding to bf16 is monotone and
+// odd: when lo and hi round to the same bf16 value, that is the answer;
+// otherwise (about one row in two thousand), or outside those ranges, the row
+// is read again and its y computed one by one.  Warp-uniform.
+__device__ __forceinline__ uint32_t rms_row_max_bits(float P, float rr, bool gains_small, const uint16_t* xr,
+                                                     const uint16_t* gamma, int64_t K, int lane) {
+  const float plo = __fmul_rd(P, rr), phi = __fmul_ru(P, rr);
+  const uint32_t blo = bf16x2_rn(__fmul_rd(plo, 1.0f - 0x1p-20f), 0.0f) & 0x7FFFu;
+  const uint32_t bhi = bf16x2_rn(__fmul_ru(phi, 1.0f + 0x1p-20f), 0.0f) & 0x7FFFu;
+  if (gains_small && plo >= 0x1p-90f && P <= 0x1.fffffep127f && blo == bhi) return blo;
+  const f2 rrr = make_f2(rr, rr);
+  float m = 0.0f;
+#pragma unroll 1
+  for (int64_t k = 8 * lane; k < K; k += 256)
+    m = rms_group_max(*reinterpret_cast<const uint4*>(xr + k), *reinterpret_cast<const uint4*>(gamma + k), rrr, m);
+  return bf16x2_rn(m, 0.0f) & 0x7FFFu;  // this lane's part; the partial takes the max over lanes
+}
+
 // The RMS pass with the row held in registers (K <= 1024 * NR): a warp issues
 // every load of its row before any arithmetic, so the whole row is in flight
 // at once, and the y phase works on the same registers.
@@ -689,13 +678,7 @@ __global__ void __launch_bounds__(kRmsRegThreads, NR <= 2 ? 8 : NR <= 3 ? 5 : NR
   constexpr int kWarps = kRmsRegThreads / 32;
   const int lane = static_cast<int>(threadIdx.x & 31), warp = static_cast<int>(threadIdx.x >> 5);
   const int64_t nwarps = static_cast<int64_t>(gridDim.x) * kWarps;
-  // G = max |gamma| (NaN kept) bounds the error that underflow adds to the
-  // products below; the bound is only used while G <= 2^20
-  uint32_t gb = 0;  // max |gamma| as bf16 bits (a NaN compares above every number)
-  for (int64_t k = 8 * lane; k < K; k += 256) gb = absmax4(*reinterpret_cast<const uint4*>(gamma + k), gb);
-#pragma unroll
-  for (int o = 16; o; o >>= 1) gb = max(gb, __shfl_xor_sync(0xffffffffu, gb, o));
-  const bool gains_small = max(gb & 0xFFFFu, gb >> 16) <= 0x4980u;  // 2^20
+  const bool gains_small = rms_gains_small(gamma, K, lane);
   uint32_t mb = 0;  // this lane's max |bf16(y)| as a bf16 bit pattern
   for (int64_t r = static_cast<int64_t>(blockIdx.x) * kWarps + warp; r < rows; r += nwarps) {
     const uint16_t* xr = x + r * ldx;
@@ -735,31 +718,56 @@ __global__ void __launch_bounds__(kRmsRegThreads, NR <= 2 ? 8 : NR <= 3 ? 5 : NR
     }
     const float rr = rms_rinv(rms_close(stk, NR), K, eps);
     if (lane == 0) rinv[r] = rr;
-    // max |y| of the row, y = (x * r) * gamma with two roundings.  With
-    // P = max |x * gamma| (exact) and every y in the normal range, each |y| is
-    // within a factor (1 +- 2^-24)^2 of |x * gamma| * r, so max |y| lies in
-    // [lo, hi] = [P r (1 - 2^-20), P r (1 + 2^-20)] (rounded outward; the
-    // slack also covers what underflow can add while P r >= 2^-90 and
-    // G <= 2^20).  Rounding to bf16 is monotone: when lo and hi round to the
-    // same bf16 value, that is max |bf16(y)|; otherwise (about one row in a
-    // thousand) the row's y are computed one by one.
-    P = warp_max_nan(P);
-    const float plo = __fmul_rd(P, rr), phi = __fmul_ru(P, rr);
-    const uint32_t blo = bf16x2_rn(__fmul_rd(plo, 1.0f - 0x1p-20f), 0.0f) & 0x7FFFu;
-    const uint32_t bhi = bf16x2_rn(__fmul_ru(phi, 1.0f + 0x1p-20f), 0.0f) & 0x7FFFu;
-    if (gains_small && plo >= 0x1p-90f && P <= 0x1.fffffep127f && blo == bhi) {
-      mb = max(mb, blo);
-    } else {
-      // rare: the row read again (from L2), its y computed one by one
-      const f2 rrr = make_f2(rr, rr);
-      float m = 0.0f;
-#pragma unroll 1
-      for (int64_t k = 8 * lane; k < K; k += 256)
-        m = rms_group_max(*reinterpret_cast<const uint4*>(xr + k), *reinterpret_cast<const uint4*>(gamma + k), rrr, m);
-      mb = max(mb, bf16x2_rn(m, 0.0f) & 0x7FFFu);
-    }
+    mb = max(mb, rms_row_max_bits(warp_max_nan(P), rr, gains_small, xr, gamma, K, lane));
   }
   rms_write_partial_bits<kRmsRegThreads>(mb, partials);
+}
+
+// The RMS pass for any K <= 16384, round by round: each round's loads, its
+// subtree of the sum and its part of P, then the next round.
+template <bool V8>
+__global__ void __launch_bounds__(kRmsThreads)
+    rms_amax_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t K, int64_t ldx,
+                    const uint16_t* __restrict__ gamma, float eps, const int32_t* __restrict__ perm,
+                    float* __restrict__ rinv, uint16_t* __restrict__ gperm, uint32_t* __restrict__ partials) {
+  pdl_launch_dependents();  // the quantize kernel may be scheduled now; it waits for this grid's end
+  rms_permute_gains(gamma, perm, K, gperm);
+  // rounds that hold elements; the zero-padded rest of the tree up to the next
+  // power of two adds exact zeros and is not computed
+  const int used = static_cast<int>((K + 1023) / 1024);  // 1 .. 16 (K <= 16384)
+  const int lane = static_cast<int>(threadIdx.x & 31), warp = static_cast<int>(threadIdx.x >> 5);
+  const int64_t nwarps = static_cast<int64_t>(gridDim.x) * (kRmsThreads / 32);
+  const bool gains_small = rms_gains_small(gamma, K, lane);
+  uint32_t mb = 0;
+  for (int64_t r = static_cast<int64_t>(blockIdx.x) * (kRmsThreads / 32) + warp; r < rows; r += nwarps) {
+    const uint16_t* xr = x + r * ldx;
+    float stk[5];
+    float P = 0.0f;
+    for (int q = 0; q < used; ++q) {
+      // this lane's two pairs of groups (K % 64 == 0: a pair is inside the row or past it)
+      float g[4];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int64_t k = 1024 * static_cast<int64_t>(q) + 32 * lane + 16 * h;
+        if (k < K) {
+          uint4 a, b, ga, gb;
+          ld_group_pair<V8, false>(xr + k, a, b);
+          ld_group_pair<V8, true>(gamma + k, ga, gb);
+          g[2 * h] = sq_tree8(a);
+          g[2 * h + 1] = sq_tree8(b);
+          P = prod_group_max(b, gb, prod_group_max(a, ga, P));
+        } else {
+          g[2 * h] = 0.0f;
+          g[2 * h + 1] = 0.0f;
+        }
+      }
+      rms_push(stk, q, rms_round(g[0], g[1], g[2], g[3]));
+    }
+    const float rr = rms_rinv(rms_close(stk, used), K, eps);
+    if (lane == 0) rinv[r] = rr;
+    mb = max(mb, rms_row_max_bits(warp_max_nan(P), rr, gains_small, xr, gamma, K, lane));
+  }
+  rms_write_partial_bits<kRmsThreads>(mb, partials);
 }
 
 // A block's 16 gains in channel order (two 16-byte loads of gamma[perm[.]])
@@ -1282,13 +1290,26 @@ cudaError_t launch_rms_reg_v(const QuantParams& p, uint32_t* partials, float eps
   return cudaGetLastError();
 }
 // 256-bit loads where x's rows and the gains start on 32-byte boundaries
+bool rms_aligned32(const QuantParams& p) {
+  return reinterpret_cast<uintptr_t>(p.x) % 32 == 0 && p.ldx % 16 == 0 &&
+         reinterpret_cast<uintptr_t>(p.gamma) % 32 == 0;
+}
 template <int NR>
 cudaError_t launch_rms_reg(const QuantParams& p, uint32_t* partials, float eps, int dev, int sms, cudaStream_t s,
                            int* grid) {
-  const bool v8 = reinterpret_cast<uintptr_t>(p.x) % 32 == 0 && p.ldx % 16 == 0 &&
-                  reinterpret_cast<uintptr_t>(p.gamma) % 32 == 0;
-  return v8 ? launch_rms_reg_v<NR, true>(p, partials, eps, dev, sms, s, grid)
-            : launch_rms_reg_v<NR, false>(p, partials, eps, dev, sms, s, grid);
+  return rms_aligned32(p) ? launch_rms_reg_v<NR, true>(p, partials, eps, dev, sms, s, grid)
+                          : launch_rms_reg_v<NR, false>(p, partials, eps, dev, sms, s, grid);
+}
+template <bool V8>
+cudaError_t launch_rms_stream(const QuantParams& p, uint32_t* partials, float eps, int dev, int sms, cudaStream_t s,
+                              int* grid) {
+  static PerContextCache<int> per_sm;
+  cudaError_t e = rms_grid(per_sm, rms_amax_kernel<V8>, kRmsThreads, dev, sms, p.rows, grid);
+  if (e != cudaSuccess) return e;
+  rms_amax_kernel<V8><<<*grid, kRmsThreads, 0, s>>>(p.x, p.rows, p.K, p.ldx, p.gamma, eps, p.perm,
+                                                   const_cast<float*>(p.rinv), const_cast<uint16_t*>(p.gperm),
+                                                   partials);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_rms_pass(const QuantParams& p, uint32_t* partials, float eps, int dev, int sms, cudaStream_t s,
@@ -1306,12 +1327,8 @@ cudaError_t launch_rms_pass(const QuantParams& p, uint32_t* partials, float eps,
     case 8: return launch_rms_reg<8>(p, partials, eps, dev, sms, s, grid);
     default: break;
   }
-  static PerContextCache<int> per_sm;
-  cudaError_t e = rms_grid(per_sm, rms_amax_kernel, kRmsThreads, dev, sms, p.rows, grid);
-  if (e != cudaSuccess) return e;
-  rms_amax_kernel<<<*grid, kRmsThreads, 0, s>>>(p.x, p.rows, p.K, p.ldx, p.gamma, eps, p.perm,
-                                               const_cast<float*>(p.rinv), const_cast<uint16_t*>(p.gperm), partials);
-  return cudaGetLastError();
+  return rms_aligned32(p) ? launch_rms_stream<true>(p, partials, eps, dev, sms, s, grid)
+                          : launch_rms_stream<false>(p, partials, eps, dev, sms, s, grid);
 }
 
 nvfp4_status launch_rms_dynamic(QuantParams p, int mode, int rule, float fp8_max, float* global_scale,
