@@ -743,6 +743,7 @@ __global__ void __launch_bounds__(kRmsThreads)
     const uint16_t* xr = x + r * ldx;
     float stk[5];
     float P = 0.0f;
+#pragma unroll 2  // two rounds' loads in flight (83.6 against 87.6 us on 8192 x 16384)
     for (int q = 0; q < used; ++q) {
       // this lane's two pairs of groups (K % 64 == 0: a pair is inside the row or past it)
       float g[4];
