@@ -23,7 +23,7 @@
 //                    pattern it saw to a partials array in the workspace.
 //   quantize_kernel  reduces the partials (a few KB, L2-resident) to alpha in
 //                    every CTA, then makes one HBM pass over x: each lane owns
-//                    one whole 16-element block (two 16-byte loads), so the
+//                    one whole 16-element block (one 32-byte load), so the
 //                    block max and both candidates' errors stay in registers
 //                    with no shuffles.  A warp task is a pair of chunks of 32
 //                    consecutive blocks (2 x 1 KB of x) of one row, and the
@@ -34,7 +34,8 @@
 // The other entry points reuse the block step: quantize_t_kernel (blocks down
 // the columns of x, through shared-memory tiles), quantize_arc_kernel
 // (reordered channels plus appended residual or duplicated ones, with an
-// optional RMSNorm of the activations) and its RMS pass rms_amax_kernel.
+// optional RMSNorm of the activations) and its RMS pass (rms_amax_reg_kernel
+// with the row in registers up to K = 8192, rms_amax_kernel above).
 #include <cuda_fp16.h>
 
 #include <algorithm>
