@@ -310,3 +310,53 @@ def test_quantize_arc_rmsnorm_gemm_equals_the_two_calls():
     assert torch.equal(qx.codes, qx_ref.codes) and torch.equal(qx.scales, qx_ref.scales)
     assert torch.equal(qx.global_scale, qx_ref.global_scale)
     assert torch.equal(y, y_ref)
+
+
+# ------------------------------------------------ full size, sampled rows --
+# The augmented quantizers on the 32768 x 5120 prefill activations with the
+# bench's recipe (4/6-MSE, fp8_max 256, S = 128, channels by descending column
+# amax).  alpha comes from the whole tensor: the oracle checks it from the
+# whole tensor's amax, and quantizes the sampled rows together with one extra
+# row that carries that amax, so that its alpha is the tensor's.
+
+def _amax_row(bits_u16: np.ndarray) -> np.ndarray:
+    """A row of zeros holding the largest |value| of the bf16 bit patterns."""
+    flat = bits_u16.reshape(-1)
+    mag = flat & 0x7FFF
+    row = np.zeros((1, bits_u16.shape[1]), np.uint16)
+    row[0, 0] = flat[int(np.argmax(mag))]
+    return row
+
+
+def _check_arc_sampled(q, y_bits: np.ndarray, perm, S, nsample=48, seed=3):
+    rows, K = y_bits.shape
+    mode, rule, F = "four_over_six", "mse", 256.0
+    idx = workloads.sample_rows(rows, nsample, seed).numpy()
+    sample = np.concatenate([y_bits[idx], _amax_row(y_bits)])
+    ys = torch.from_numpy(sample.view(np.int16)).view(torch.bfloat16)
+    oc, os_, oa = oracle.quantize_arc(ys, perm, S, nv.AUG_RESIDUAL, MODE[mode], RULE[rule], F)
+    amax, bad = oracle.amax(torch.from_numpy(y_bits.view(np.int16)).view(torch.bfloat16))
+    assert not bad and np.float32(oa) == np.float32(oracle.global_scale(amax, F))
+    assert float(q.global_scale.cpu()[0]) == np.float32(oa)
+    gc = to_np(q.codes[torch.from_numpy(idx).cuda()])
+    assert np.array_equal(gc, oc[:-1])
+    gs = oracle.unswizzle_scales(to_np(q.scales), rows, K + S)[idx]
+    assert np.array_equal(gs, os_[:-1])
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("rmsnorm", [False, True], ids=["plain", "rmsnorm"])
+def test_quantize_arc_prefill_full_size_sampled(rmsnorm):
+    x = workloads.WORKLOADS["prefill"].x.make()
+    K, S = x.shape[1], 128
+    perm = outlier_perm(x)
+    xd, pd = x.cuda(), torch.from_numpy(perm).cuda()
+    if rmsnorm:
+        gamma = _gains(K, 5)
+        q = nv.quantize_arc_rmsnorm(xd, gamma.cuda(), 1e-6, pd, S, "four_over_six", "mse", 256.0)
+        y_bits = oracle.rmsnorm(x, gamma, 1e-6)
+    else:
+        q = nv.quantize_arc(xd, pd, S, nv.AUG_RESIDUAL, "four_over_six", "mse", 256.0)
+        y_bits = oracle.as_bf16_bits(x)
+    assert nv.device_status(q.workspace) == nv.OK
+    _check_arc_sampled(q, y_bits, perm, S)
