@@ -227,6 +227,38 @@ def test_gemm_quantized_output_equals_gemm_then_quantize(M, N, K, recipe):
     assert np.array_equal(to_np(q.scales), oracle.swizzle_scales(os_, M, N))
 
 
+@pytest.mark.slow
+def test_prefill_nvfp4_output_and_static_alpha_full_size():
+    """The bench's prefill case (X 32768x5120 4/6-MSE, W 17408x5120 scale-6):
+    the GEMM writing Y as NVFP4 (4/6-MSE) equals the bf16 GEMM followed by the
+    static-alpha quantizer over the whole 32768x17408 output, and sampled rows
+    equal the oracle's row quantizer on that Y at the same alpha; X quantized
+    at a static alpha equal to its dynamic one reproduces the dynamic call."""
+    wl = workloads.WORKLOADS["prefill"]
+    x, w = wl.x.make(), wl.w.make()
+    xm, xr, xF = "four_over_six", "mse", 256.0
+    qx, st = gpu_quantize(x, xm, xr, xF, canary=0)
+    assert st == nv.OK
+    qs = nv.quantize(x.cuda(), xm, xr, global_scale=qx.global_scale.clone())
+    assert nv.device_status(qs.workspace) == nv.OK
+    assert torch.equal(qs.codes, qx.codes) and torch.equal(qs.scales, qx.scales)
+    wm, wr, wF = wl.w_recipe
+    qw, st = gpu_quantize(w, wm, wr, wF, canary=0)
+    assert st == nv.OK
+    y = nv.gemm(qx, qw, out_dtype=torch.bfloat16)
+    alpha = torch.tensor([float(y.float().abs().max()) / (6 * 256.0)], dtype=torch.float32, device="cuda")
+    q = nv.gemm_quantized(qx, qw, alpha, "four_over_six", "mse")
+    assert nv.device_status(q.workspace) == nv.OK
+    ref = nv.quantize(y, "four_over_six", "mse", global_scale=alpha)
+    assert torch.equal(q.codes, ref.codes) and torch.equal(q.scales, ref.scales)
+    M, N = y.shape
+    idx = workloads.sample_rows(M, 32, 2).numpy()
+    oc, os_ = oracle.quantize_rows(y[torch.from_numpy(idx).cuda()].cpu(), float(alpha.cpu()[0]), MODE["four_over_six"],
+                                   RULE["mse"])
+    assert np.array_equal(to_np(q.codes[torch.from_numpy(idx).cuda()]), oc)
+    assert np.array_equal(oracle.unswizzle_scales(to_np(q.scales), M, N)[idx], os_)
+
+
 @pytest.mark.skipif(torch.cuda.device_count() < 2, reason="needs two visible GPUs")
 def test_second_device_after_the_first():
     """Kernel attributes (the GEMM's and the augmented quantizer's shared-memory
