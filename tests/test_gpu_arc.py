@@ -360,3 +360,33 @@ def test_quantize_arc_prefill_full_size_sampled(rmsnorm):
         y_bits = oracle.as_bf16_bits(x)
     assert nv.device_status(q.workspace) == nv.OK
     _check_arc_sampled(q, y_bits, perm, S)
+
+
+@pytest.mark.slow
+def test_quantize_arc_gemm_prefill_full_size_sampled():
+    """The bench's augmented layer in one call on the prefill case: X
+    (32768x5120, 4/6-MSE) with 128 residual channels, W (17408x5120, scale-6)
+    with those channels duplicated, bf16 Y over K + 128.  W's operand equals the
+    oracle's in full; sampled rows of Y match the fp64 product of the oracle's
+    operands (X's rows quantized with the whole tensor's alpha)."""
+    wl = workloads.WORKLOADS["prefill"]
+    x, w = wl.x.make(), wl.w.make()
+    K, S = x.shape[1], 128
+    perm = outlier_perm(x)
+    pd = torch.from_numpy(perm).cuda()
+    wm, wr, wF = wl.w_recipe
+    qw = nv.quantize_arc(w.cuda(), pd, S, nv.AUG_DUPLICATE, wm, wr, wF)
+    assert nv.device_status(qw.workspace) == nv.OK
+    wc, ws, wa = oracle.quantize_arc(w, perm, S, nv.AUG_DUPLICATE, MODE[wm], RULE[wr], wF)
+    assert np.array_equal(to_np(qw.codes), wc)
+    qx, y = nv.quantize_arc_gemm(x.cuda(), pd, S, qw, "four_over_six", "mse", 256.0, out_dtype=torch.bfloat16)
+    assert nv.device_status(qx.workspace) == nv.OK
+    xb = oracle.as_bf16_bits(x)
+    idx = workloads.sample_rows(x.shape[0], 32, 4).numpy()
+    sample = np.concatenate([xb[idx], _amax_row(xb)])
+    xs_t = torch.from_numpy(sample.view(np.int16)).view(torch.bfloat16)
+    xc, xs, xa = oracle.quantize_arc(xs_t, perm, S, nv.AUG_RESIDUAL, MODE["four_over_six"], RULE["mse"], 256.0)
+    assert float(qx.global_scale.cpu()[0]) == np.float32(xa)
+    assert np.array_equal(to_np(qx.codes[torch.from_numpy(idx).cuda()]), xc[:-1])
+    ref, guard = oracle.gemm_reference(xc[:-1], xs[:-1], xa, wc, ws, wa)
+    assert_gemm_close(to_np(y[torch.from_numpy(idx).cuda()].float()), ref, guard, bf16=True)
