@@ -125,7 +125,8 @@ def test_tile_order_with_partial_last_group():
 @pytest.mark.parametrize("name", ["mlp8b", "attn27b", "prefill"])
 def test_pipeline_full_size_sampled(name):
     """quantize X (each recipe) and W on the GPU, GEMM, and compare sampled
-    rows of Y with the oracle's fp64 product of its own quantized operands."""
+    rows of Y with the oracle's fp64 product of its own quantized operands;
+    the one-call layer must give the same bytes as the two calls."""
     wl = workloads.WORKLOADS[name]
     x, w = wl.x.make(), wl.w.make()
     wm, wr, wF = wl.w_recipe
@@ -146,6 +147,11 @@ def test_pipeline_full_size_sampled(name):
         rows = torch.from_numpy(idx).cuda()
         assert_gemm_close(to_np(y32[rows]), ref, guard)
         assert_gemm_close(to_np(y[rows].float()), ref, guard, bf16=True)
+        # the one-call layer (the bench's timed step) gives the same bytes
+        ws1 = torch.zeros(nv.nvfp4_gemm_workspace_bytes(), dtype=torch.uint8, device="cuda")
+        qx1, y1 = nv.quantize_gemm(x.cuda(), qw, xm, xr, xF, out_dtype=torch.bfloat16, workspace=ws1)
+        assert nv.device_status(qx1.workspace) == nv.OK and nv.device_status(ws1) == nv.OK
+        assert torch.equal(qx1.codes, qx.codes) and torch.equal(y1, y)
 
 
 @pytest.mark.parametrize("ldy_pad", [3, 8, 130])
