@@ -554,10 +554,10 @@ __device__ __forceinline__ float rms_rinv(float sum, int64_t K, float eps) {
   return __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(__fdiv_rn(sum, static_cast<float>(K)), eps)));
 }
 
-// the CTA's max |bf16(y)| from each lane's binary32 max, as a bf16 bit
-// pattern (a NaN becomes 0x7FFF), into partials[blockIdx.x]
+// the CTA's max |bf16(y)| from each lane's (a bf16 bit pattern without its
+// sign; a NaN is 0x7FFF and compares above every number) into partials[blockIdx.x]
 template <int THREADS>
-__device__ __forceinline__ void rms_write_partial_bits(uint32_t mb, uint32_t* partials) {
+__device__ __forceinline__ void rms_write_partial(uint32_t mb, uint32_t* partials) {
   const int lane = static_cast<int>(threadIdx.x & 31), warp = static_cast<int>(threadIdx.x >> 5);
 #pragma unroll
   for (int o = 16; o; o >>= 1) mb = max(mb, __shfl_xor_sync(0xffffffffu, mb, o));
@@ -569,10 +569,6 @@ __device__ __forceinline__ void rms_write_partial_bits(uint32_t mb, uint32_t* pa
     for (int w = 0; w < THREADS / 32; ++w) mm = max(mm, s_max[w]);
     partials[blockIdx.x] = mm;
   }
-}
-template <int THREADS>
-__device__ __forceinline__ void rms_write_partial(float m, uint32_t* partials) {
-  rms_write_partial_bits<THREADS>(bf16x2_rn(m, 0.0f) & 0x7FFFu, partials);
 }
 
 // gperm[i] = gamma[perm[i]] over the grid's threads, for the augmented
@@ -721,7 +717,7 @@ __global__ void __launch_bounds__(kRmsRegThreads, NR <= 2 ? 8 : NR <= 3 ? 5 : NR
     if (lane == 0) rinv[r] = rr;
     mb = max(mb, rms_row_max_bits(warp_max_nan(P), rr, gains_small, xr, gamma, K, lane));
   }
-  rms_write_partial_bits<kRmsRegThreads>(mb, partials);
+  rms_write_partial<kRmsRegThreads>(mb, partials);
 }
 
 // The RMS pass for any K <= 16384, round by round: each round's loads, its
@@ -769,7 +765,7 @@ __global__ void __launch_bounds__(kRmsThreads)
     if (lane == 0) rinv[r] = rr;
     mb = max(mb, rms_row_max_bits(warp_max_nan(P), rr, gains_small, xr, gamma, K, lane));
   }
-  rms_write_partial_bits<kRmsThreads>(mb, partials);
+  rms_write_partial<kRmsThreads>(mb, partials);
 }
 
 // A block's 16 gains in channel order (two 16-byte loads of gamma[perm[.]])
