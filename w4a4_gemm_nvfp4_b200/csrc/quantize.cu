@@ -459,8 +459,9 @@ __global__ void __launch_bounds__(kQuantThreads)
 // sums, all lanes holding them, merge like a binary counter (each completed
 // subtree added to the equal-size one on its left); the zero padding past the
 // last round is not computed.  Every lane ends with the row's sum and computes
-// r.  The pass writes r for every row and, like the amax pass, each CTA's max
-// |y| as a bf16 bit pattern.
+// r.  The pass writes r for every row, the gains in channel order and, like
+// the amax pass, each CTA's max |bf16(y)| as a bit pattern (from the bound of
+// rms_row_max_bits, without computing y where the bound decides).
 constexpr int kRmsThreads = 256;
 constexpr int kRmsRegThreads = 128;
 
@@ -664,7 +665,7 @@ __device__ __forceinline__ uint32_t rms_row_max_bits(float P, float rr, bool gai
 
 // The RMS pass with the row held in registers (K <= 1024 * NR): a warp issues
 // every load of its row before any arithmetic, so the whole row is in flight
-// at once, and the y phase works on the same registers.
+// at once, and the sum of squares and P come from the same registers.
 template <int NR, bool V8>
 __global__ void __launch_bounds__(kRmsRegThreads, NR <= 2 ? 8 : NR <= 3 ? 5 : NR <= 6 ? 4 : 3)
     rms_amax_reg_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t K, int64_t ldx,
