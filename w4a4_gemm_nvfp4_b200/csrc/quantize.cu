@@ -55,8 +55,8 @@ constexpr int kArcMaxThreads = 640;         // its block size, at most
 constexpr int kArcMaxBufs = 3;              // its row buffers: 3, or 2 for the widest rows
 constexpr int64_t kArcSmemStep = 73728;     // shared memory it aims at: three CTAs per SM up to 5K channels
 constexpr int64_t kArcMaxK = 16384;         // channels of x it takes, at most
-// its shared memory, at most: 2 bytes x K x (lead arrays + buffers x rows per step), K <= 16384 (two
-// buffers of one row; the offsets and, with RMSNorm, the gains ahead of them)
+// its dynamic shared memory opt-in: 2 bytes x K x (1 + buffers x rows per step), the offsets
+// ahead of the row buffers, is at most 2 x 16384 x 3 (two buffers of one row)
 constexpr int64_t kArcSmemBudget = 2 * 16384 * 4;
 constexpr int kQuantThreads = 256;
 constexpr int kQuantWarps = kQuantThreads / 32;
@@ -1018,23 +1018,16 @@ int arc_threads(int64_t K, int64_t S, int R) {
 }
 
 // Rows per step and row buffers of the augmented quantizer for K channels,
-// with `lead` K-sized bf16 arrays ahead of the rows (the offsets; with RMSNorm
-// the gains too), within kArcSmemStep: three buffers of the most rows (up to 4,
-// a power of two so it divides the 128-row padding).  With RMSNorm, two rows in
-// two buffers are taken before one row in three, when three do not fit (the
-// gather's per-row costs are shared by the rows of a step).  Where even one row
-// per buffer does not fit (K above about 9K), two buffers of one row (within
-// kArcSmemBudget for K <= 16384), so that two CTAs still share an SM.
-void arc_layout(int64_t K, int lead, int* rows, int* bufs) {
+// with the K-entry channel offsets ahead of the rows, within kArcSmemStep:
+// three buffers of the most rows (up to 4, a power of two so it divides the
+// 128-row padding).  Where even one row per buffer does not fit (K above
+// about 9K), two buffers of one row (within kArcSmemBudget for K <= 16384), so
+// that two CTAs still share an SM.
+void arc_layout(int64_t K, int* rows, int* bufs) {
   for (int r = kArcMaxRows; r >= 1; r /= 2) {
-    if (2 * K * (lead + kArcMaxBufs * r) <= kArcSmemStep) {
+    if (2 * K * (1 + kArcMaxBufs * r) <= kArcSmemStep) {
       *rows = r;
       *bufs = kArcMaxBufs;
-      return;
-    }
-    if (lead > 1 && r > 1 && 2 * K * (lead + 2 * r) <= kArcSmemStep) {
-      *rows = r;
-      *bufs = 2;
       return;
     }
   }
@@ -1398,7 +1391,7 @@ nvfp4_status quantize_impl(const char* fn, QuantKind kind, const void* x, int64_
   p.S = S;
   p.augment = augment;
   if (kind == QuantKind::kAugmented) {
-    arc_layout(K, 1, &p.arc_rows, &p.arc_bufs);
+    arc_layout(K, &p.arc_rows, &p.arc_bufs);
     p.arc_prim_threads = arc_prim_threads(K);
   }
   if (gamma) {
